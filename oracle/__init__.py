@@ -1,0 +1,143 @@
+"""CPU oracle for the WCB1 block fixed-length BF16 exponent code.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference legs of ``bench.py`` may import this package. The
+product library (``lossless_weight_compression_b200``) never imports it, and
+the two share no code: the oracle is plain single-threaded C (``wc_oracle.c``)
+written from the stream definition, wrapped here with ctypes.
+
+Method source: "ENEC: A Lossless AI Model Compression Method Enabling Fast
+Inference on Ascend NPUs", Abstract (per-block fixed-length code, bit-width
+quantization, hierarchical halving packing, branch-free remap, prefix sum of
+block sizes). Each wrapper below names the step of ``wc_oracle.c`` it calls.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "wc_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+OK, INVALID_ARG, BUFFER_TOO_SMALL, CORRUPT = 0, 1, 2, 3
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``wc_oracle.c`` into ``liboracle.so`` with gcc (plain C99, -O2)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + ".tmp%d" % os.getpid()
+    subprocess.run(["gcc", "-std=c99", "-O2", "-Wall", "-Wextra", "-fPIC", "-shared",
+                    "-o", tmp, _SRC], check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB_PATH)
+        u8, u16, u64, uint = ctypes.c_uint8, ctypes.c_uint16, ctypes.c_uint64, ctypes.c_uint
+        vp = ctypes.c_void_p
+        L.oracle_exponent.argtypes, L.oracle_exponent.restype = [u16], u8
+        L.oracle_signman.argtypes, L.oracle_signman.restype = [u16], u8
+        L.oracle_merge.argtypes, L.oracle_merge.restype = [u8, u8], u16
+        L.oracle_bits.argtypes, L.oracle_bits.restype = [uint], uint
+        L.oracle_block_params.argtypes = [vp, u64, vp, vp]
+        L.oracle_block_params.restype = None
+        L.oracle_pack_octet.argtypes, L.oracle_pack_octet.restype = [vp, uint], u64
+        L.oracle_unpack_octet.argtypes = [u64, uint, vp]
+        L.oracle_unpack_octet.restype = None
+        L.oracle_bound.argtypes, L.oracle_bound.restype = [u64, ctypes.c_uint32], u64
+        L.oracle_compress.argtypes = [vp, u64, ctypes.c_uint32, vp, u64, vp]
+        L.oracle_compress.restype = ctypes.c_int
+        L.oracle_decompress.argtypes = [vp, u64, vp, u64, ctypes.c_uint32]
+        L.oracle_decompress.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data if a.size else 0
+
+
+# --- step 1: split / merge -------------------------------------------------
+def exponent(x: int) -> int:
+    return lib().oracle_exponent(x)
+
+
+def signman(x: int) -> int:
+    return lib().oracle_signman(x)
+
+
+def merge(e: int, s: int) -> int:
+    return lib().oracle_merge(e, s)
+
+
+# --- step 2: width quantization ----------------------------------------------
+def bits(d: int) -> int:
+    return lib().oracle_bits(d)
+
+
+def block_params(words: np.ndarray) -> tuple[int, int]:
+    """(base, w) of one block of BF16 bit patterns."""
+    words = np.ascontiguousarray(words, dtype=np.uint16)
+    base, w = ctypes.c_uint8(), ctypes.c_uint8()
+    lib().oracle_block_params(_ptr(words), words.size, ctypes.byref(base), ctypes.byref(w))
+    return base.value, w.value
+
+
+# --- step 4: hierarchical halving pack ---------------------------------------
+def pack_octet(values, w: int) -> int:
+    v = np.ascontiguousarray(values, dtype=np.uint8)
+    assert v.size == 8
+    return lib().oracle_pack_octet(_ptr(v), w)
+
+
+def unpack_octet(octet: int, w: int) -> list[int]:
+    v = np.zeros(8, dtype=np.uint8)
+    lib().oracle_unpack_octet(octet, w, _ptr(v))
+    return v.tolist()
+
+
+# --- whole streams -----------------------------------------------------------
+def bound(n: int, block: int) -> int:
+    return lib().oracle_bound(n, block)
+
+
+def compress(words: np.ndarray, block: int) -> np.ndarray:
+    """Encode BF16 bit patterns (uint16, any shape) into a WCB1 stream (uint8)."""
+    words = np.ascontiguousarray(words, dtype=np.uint16).reshape(-1)
+    cap = bound(words.size, block)
+    if cap == 0:
+        raise ValueError("oracle: invalid block size %r or n %d" % (block, words.size))
+    out = np.empty(cap, dtype=np.uint8)
+    nbytes = ctypes.c_uint64()
+    rc = lib().oracle_compress(_ptr(words), words.size, block, _ptr(out), cap,
+                               ctypes.byref(nbytes))
+    if rc != OK:
+        raise ValueError("oracle_compress failed with status %d" % rc)
+    return out[: nbytes.value].copy()
+
+
+def decompress_status(stream: np.ndarray, n: int, block: int) -> tuple[int, np.ndarray]:
+    """Decode; returns (status, words). Status CORRUPT for any invalid stream."""
+    stream = np.ascontiguousarray(stream, dtype=np.uint8).reshape(-1)
+    out = np.zeros(n, dtype=np.uint16)
+    rc = lib().oracle_decompress(_ptr(stream), stream.size, _ptr(out), n, block)
+    return rc, out
+
+
+def decompress(stream: np.ndarray, n: int, block: int) -> np.ndarray:
+    rc, out = decompress_status(stream, n, block)
+    if rc != OK:
+        raise ValueError("oracle_decompress failed with status %d" % rc)
+    return out

@@ -1,0 +1,339 @@
+/*
+ * wc_oracle.c -- plain, slow, single-threaded CPU oracle for the WCB1 stream
+ * (block fixed-length code of BF16 exponents, sign+mantissa bytes stored raw).
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the
+ * benchmark's CPU-baseline leg may load this file's library. The product path
+ * (libwcodec) never calls it, and this file shares no code, header, table or
+ * helper with the CUDA library: it is written separately from the stream
+ * definition so that the two can be compared byte for byte.
+ *
+ * Source of the method: "ENEC: A Lossless AI Model Compression Method Enabling
+ * Fast Inference on Ascend NPUs", Abstract. The abstract names the ingredients:
+ * blocks coded at one fixed length each, a per-block bit width ("bit-width
+ * quantization"), packing that combines values two, four, then eight at a time
+ * ("hierarchical halving bit-packing"), a branch-free integer remap of the
+ * values, and a prefix sum that places each block. It fixes no byte layout; the
+ * layout below is this project's reading, and every such reading is marked.
+ *
+ * Encoding steps, in the order the abstract lists them:
+ *   1. split each BF16 word into its exponent byte e = (x >> 7) & 0xFF and its
+ *      sign+mantissa byte s = sign << 7 | mantissa   (reading: bit positions)
+ *   2. bit-width quantization per block: lo = min e, hi = max e,
+ *      w = bits(hi - lo) in 0..8; w == 8 is the raw fallback with base 0,
+ *      otherwise base = lo                             (reading: remap = e - min)
+ *   3. branch-free remap v = e - base
+ *   4. hierarchical halving pack of each run of 8 values (an "octet") into
+ *      w bytes, element t at bits [t*w, (t+1)*w), little-endian
+ *   5. exclusive prefix sum of the block sizes ceil(L/8)*w -> block offsets
+ *   6. write the sections: 128-byte container header, u16 block headers,
+ *      u32 block offsets (16-byte units), mantissa plane, exponent plane;
+ *      every section starts on a 128-byte boundary and all padding is zero.
+ * Decoding is the exact inverse; its result is the input, bit for bit.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_INVALID_ARG 1
+#define ORC_BUFFER_TOO_SMALL 2
+#define ORC_CORRUPT 3
+
+#define ORC_MAGIC 0x31424357u /* the bytes "WCB1" read as a little-endian u32 */
+#define ORC_VERSION 1u
+#define ORC_HEADER_BYTES 128u
+#define ORC_MAX_ELEMS (1ull << 36)
+
+/* ------------------------------------------------------------------ */
+/* Little-endian byte access (the stream is defined byte by byte).     */
+/* ------------------------------------------------------------------ */
+static void put_le(uint8_t *p, uint64_t value, int nbytes)
+{
+    for (int k = 0; k < nbytes; k++)
+        p[k] = (uint8_t)(value >> (8 * k));
+}
+
+static uint64_t get_le(const uint8_t *p, int nbytes)
+{
+    uint64_t value = 0;
+    for (int k = 0; k < nbytes; k++)
+        value |= (uint64_t)p[k] << (8 * k);
+    return value;
+}
+
+static uint64_t round_up_128(uint64_t x) { return (x + 127u) / 128u * 128u; }
+
+static int block_size_allowed(uint32_t B)
+{
+    /* reading: B is a power of two from 128 to 4096 */
+    return B == 128 || B == 256 || B == 512 || B == 1024 || B == 2048 || B == 4096;
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 1: split and merge of one BF16 bit pattern.                    */
+/* ------------------------------------------------------------------ */
+uint8_t oracle_exponent(uint16_t x) { return (uint8_t)((x >> 7) & 0xFFu); }
+
+uint8_t oracle_signman(uint16_t x)
+{
+    uint8_t sign = (uint8_t)(x >> 15);      /* bit 15 */
+    uint8_t mantissa = (uint8_t)(x & 0x7Fu); /* bits 6..0 */
+    return (uint8_t)((sign << 7) | mantissa);
+}
+
+uint16_t oracle_merge(uint8_t e, uint8_t s)
+{
+    uint16_t sign = (uint16_t)(s >> 7);
+    uint16_t mantissa = (uint16_t)(s & 0x7Fu);
+    return (uint16_t)((sign << 15) | ((uint16_t)e << 7) | mantissa);
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 2: bit-width quantization of one block.                        */
+/* ------------------------------------------------------------------ */
+/* The number of bits needed to write d in binary (0 for d == 0). */
+unsigned oracle_bits(unsigned d)
+{
+    unsigned w = 0;
+    while (d != 0) {
+        w++;
+        d >>= 1;
+    }
+    return w;
+}
+
+/* For the L words of one block: its width w and base. */
+void oracle_block_params(const uint16_t *x, uint64_t L, uint8_t *base, uint8_t *w)
+{
+    unsigned lo = 255, hi = 0;
+    for (uint64_t i = 0; i < L; i++) {
+        unsigned e = oracle_exponent(x[i]);
+        if (e < lo) lo = e;
+        if (e > hi) hi = e;
+    }
+    if (L == 0) lo = hi = 0;
+    unsigned width = oracle_bits(hi - lo);
+    *w = (uint8_t)width;
+    *base = (uint8_t)(width == 8 ? 0 : lo); /* raw fallback: the exponent itself */
+}
+
+/* ------------------------------------------------------------------ */
+/* Step 4: hierarchical halving pack / unpack of one octet.            */
+/* ------------------------------------------------------------------ */
+static uint64_t low_mask(unsigned nbits)
+{
+    return nbits >= 64 ? ~0ull : ((1ull << nbits) - 1ull);
+}
+
+/* Pack 8 values of w bits: pairs, then quads, then the octet. */
+uint64_t oracle_pack_octet(const uint8_t v[8], unsigned w)
+{
+    uint64_t pair[4], quad[2];
+    for (int k = 0; k < 4; k++)
+        pair[k] = (uint64_t)v[2 * k] | ((uint64_t)v[2 * k + 1] << w);
+    for (int k = 0; k < 2; k++)
+        quad[k] = pair[2 * k] | (pair[2 * k + 1] << (2 * w));
+    return quad[0] | (quad[1] << (4 * w));
+}
+
+/* Undo the pack: the octet into quads, the quads into pairs, pairs into values. */
+void oracle_unpack_octet(uint64_t octet, unsigned w, uint8_t v[8])
+{
+    uint64_t quad[2], pair[4];
+    quad[0] = octet & low_mask(4 * w);
+    quad[1] = (4 * w >= 64 ? 0 : octet >> (4 * w)) & low_mask(4 * w);
+    for (int k = 0; k < 2; k++) {
+        pair[2 * k] = quad[k] & low_mask(2 * w);
+        pair[2 * k + 1] = (quad[k] >> (2 * w)) & low_mask(2 * w);
+    }
+    for (int k = 0; k < 4; k++) {
+        v[2 * k] = (uint8_t)(pair[k] & low_mask(w));
+        v[2 * k + 1] = (uint8_t)((pair[k] >> w) & low_mask(w));
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Section layout, a function of (n, B) alone.                         */
+/* ------------------------------------------------------------------ */
+typedef struct {
+    uint64_t nb, off_hdr, off_offs, off_man, off_exp;
+} layout_t;
+
+static layout_t layout_of(uint64_t n, uint32_t B)
+{
+    layout_t s;
+    s.nb = (n + B - 1) / B;
+    s.off_hdr = ORC_HEADER_BYTES;
+    s.off_offs = s.off_hdr + round_up_128(2 * s.nb);
+    s.off_man = s.off_offs + round_up_128(4 * s.nb);
+    s.off_exp = s.off_man + round_up_128(n);
+    return s;
+}
+
+static uint64_t block_len(uint64_t n, uint32_t B, uint64_t b)
+{
+    uint64_t start = b * (uint64_t)B;
+    return (n - start < B) ? n - start : B;
+}
+
+/* Largest possible stream: every block raw (w = 8). 0 for a bad B or n. */
+uint64_t oracle_bound(uint64_t n, uint32_t B)
+{
+    if (!block_size_allowed(B) || n > ORC_MAX_ELEMS) return 0;
+    layout_t s = layout_of(n, B);
+    uint64_t worst = 0;
+    for (uint64_t b = 0; b < s.nb; b++)
+        worst += (block_len(n, B, b) + 7) / 8 * 8;
+    return s.off_exp + worst;
+}
+
+/* ------------------------------------------------------------------ */
+/* Encoder.                                                            */
+/* ------------------------------------------------------------------ */
+int oracle_compress(const uint16_t *x, uint64_t n, uint32_t B, uint8_t *out,
+                    uint64_t out_capacity, uint64_t *out_bytes)
+{
+    if (!block_size_allowed(B) || n > ORC_MAX_ELEMS || out == NULL ||
+        out_bytes == NULL || (n > 0 && x == NULL))
+        return ORC_INVALID_ARG;
+    if (out_capacity < oracle_bound(n, B)) return ORC_BUFFER_TOO_SMALL;
+
+    layout_t s = layout_of(n, B);
+    uint8_t *base = (uint8_t *)malloc(s.nb ? s.nb : 1);
+    uint8_t *width = (uint8_t *)malloc(s.nb ? s.nb : 1);
+    uint64_t *start = (uint64_t *)malloc((s.nb ? s.nb : 1) * sizeof(uint64_t));
+    if (!base || !width || !start) {
+        free(base);
+        free(width);
+        free(start);
+        return ORC_INVALID_ARG;
+    }
+
+    /* Step 2: width and base of every block. */
+    for (uint64_t b = 0; b < s.nb; b++)
+        oracle_block_params(x + b * B, block_len(n, B, b), &base[b], &width[b]);
+
+    /* Step 5: exclusive prefix sum of the block sizes, one block after another. */
+    uint64_t running = 0;
+    for (uint64_t b = 0; b < s.nb; b++) {
+        start[b] = running;
+        running += (block_len(n, B, b) + 7) / 8 * width[b];
+    }
+    uint64_t E = running;
+    uint64_t total = s.off_exp + E;
+
+    /* Step 6: sections; everything not written below stays zero. */
+    memset(out, 0, total);
+    put_le(out + 0, ORC_MAGIC, 4);
+    put_le(out + 4, ORC_VERSION, 2);
+    put_le(out + 6, ORC_HEADER_BYTES, 2);
+    put_le(out + 8, B, 4);
+    put_le(out + 12, 0, 4);
+    put_le(out + 16, n, 8);
+    put_le(out + 24, s.nb, 8);
+    put_le(out + 32, s.off_hdr, 8);
+    put_le(out + 40, s.off_offs, 8);
+    put_le(out + 48, s.off_man, 8);
+    put_le(out + 56, s.off_exp, 8);
+    put_le(out + 64, E, 8);
+    put_le(out + 72, total, 8);
+
+    for (uint64_t b = 0; b < s.nb; b++) {
+        put_le(out + s.off_hdr + 2 * b, (uint64_t)base[b] | ((uint64_t)width[b] << 8), 2);
+        put_le(out + s.off_offs + 4 * b, start[b] / 16, 4);
+    }
+
+    /* Step 1 (mantissa half): the sign+mantissa bytes, in element order. */
+    for (uint64_t i = 0; i < n; i++)
+        out[s.off_man + i] = oracle_signman(x[i]);
+
+    /* Steps 3 and 4: remap, then pack each octet into w bytes. */
+    for (uint64_t b = 0; b < s.nb; b++) {
+        uint64_t L = block_len(n, B, b);
+        unsigned w = width[b];
+        for (uint64_t j = 0; j < (L + 7) / 8; j++) {
+            uint8_t v[8];
+            for (int t = 0; t < 8; t++) {
+                uint64_t k = 8 * j + (uint64_t)t;
+                v[t] = (uint8_t)(k < L ? oracle_exponent(x[b * B + k]) - base[b] : 0);
+            }
+            put_le(out + s.off_exp + start[b] + j * w, oracle_pack_octet(v, w), (int)w);
+        }
+    }
+
+    free(base);
+    free(width);
+    free(start);
+    *out_bytes = total;
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Decoder. Checks everything the stream definition fixes.             */
+/* ------------------------------------------------------------------ */
+static int all_zero(const uint8_t *p, uint64_t count)
+{
+    for (uint64_t k = 0; k < count; k++)
+        if (p[k] != 0) return 0;
+    return 1;
+}
+
+int oracle_decompress(const uint8_t *in, uint64_t in_bytes, uint16_t *out,
+                      uint64_t n, uint32_t B)
+{
+    if (!block_size_allowed(B) || n > ORC_MAX_ELEMS || in == NULL || (n > 0 && out == NULL))
+        return ORC_INVALID_ARG;
+    if (in_bytes < ORC_HEADER_BYTES) return ORC_CORRUPT;
+
+    layout_t s = layout_of(n, B);
+    if (get_le(in + 0, 4) != ORC_MAGIC || get_le(in + 4, 2) != ORC_VERSION ||
+        get_le(in + 6, 2) != ORC_HEADER_BYTES || get_le(in + 8, 4) != B ||
+        get_le(in + 12, 4) != 0 || get_le(in + 16, 8) != n ||
+        get_le(in + 24, 8) != s.nb || get_le(in + 32, 8) != s.off_hdr ||
+        get_le(in + 40, 8) != s.off_offs || get_le(in + 48, 8) != s.off_man ||
+        get_le(in + 56, 8) != s.off_exp || !all_zero(in + 80, 48))
+        return ORC_CORRUPT;
+    uint64_t E = get_le(in + 64, 8);
+    uint64_t total = get_le(in + 72, 8);
+    if (E > total || total != s.off_exp + E || total > in_bytes) return ORC_CORRUPT;
+
+    /* Padding between sections must be zero. */
+    if (!all_zero(in + s.off_hdr + 2 * s.nb, s.off_offs - s.off_hdr - 2 * s.nb) ||
+        !all_zero(in + s.off_offs + 4 * s.nb, s.off_man - s.off_offs - 4 * s.nb) ||
+        !all_zero(in + s.off_man + n, s.off_exp - s.off_man - n))
+        return ORC_CORRUPT;
+
+    /* Headers and offsets must agree with the prefix sum of the block sizes. */
+    uint64_t running = 0;
+    for (uint64_t b = 0; b < s.nb; b++) {
+        uint64_t h = get_le(in + s.off_hdr + 2 * b, 2);
+        unsigned base = (unsigned)(h & 0xFFu), w = (unsigned)(h >> 8);
+        if (w > 8 || (w == 8 && base != 0)) return ORC_CORRUPT;
+        if (get_le(in + s.off_offs + 4 * b, 4) * 16 != running) return ORC_CORRUPT;
+        running += (block_len(n, B, b) + 7) / 8 * w;
+    }
+    if (running != E) return ORC_CORRUPT;
+
+    for (uint64_t b = 0; b < s.nb; b++) {
+        uint64_t L = block_len(n, B, b);
+        uint64_t h = get_le(in + s.off_hdr + 2 * b, 2);
+        unsigned base = (unsigned)(h & 0xFFu), w = (unsigned)(h >> 8);
+        uint64_t first = get_le(in + s.off_offs + 4 * b, 4) * 16;
+        for (uint64_t j = 0; j < (L + 7) / 8; j++) {
+            uint8_t v[8];
+            oracle_unpack_octet(get_le(in + s.off_exp + first + j * w, (int)w), w, v);
+            for (int t = 0; t < 8; t++) {
+                uint64_t k = 8 * j + (uint64_t)t;
+                if (k >= L) {
+                    if (v[t] != 0) return ORC_CORRUPT; /* unused lanes are zero */
+                    continue;
+                }
+                unsigned e = base + v[t];
+                if (e > 255) return ORC_CORRUPT; /* no encoder writes such a value */
+                out[b * B + k] = oracle_merge((uint8_t)e, in[s.off_man + b * B + k]);
+            }
+        }
+    }
+    return ORC_OK;
+}

@@ -1,0 +1,50 @@
+"""Reader for the hand-derived stream fixtures in tests/golden/ (syntax in README.txt)."""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+
+GOLDEN_DIR = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _expand(tokens):
+    out = []
+    for tok in tokens:
+        if "*" in tok:
+            count, group = tok.split("*", 1)
+            out += [int(h, 16) for h in group.split(",")] * int(count)
+        else:
+            out.append(int(tok, 16))
+    return out
+
+
+def load(name: str):
+    """Returns (block, words uint16, expected stream uint8)."""
+    block = total = None
+    words, runs = [], []
+    with open(os.path.join(GOLDEN_DIR, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            key, _, rest = line.partition(" ")
+            if key == "block":
+                block = int(rest)
+            elif key == "words":
+                words += _expand(rest.split())
+            elif key == "total":
+                total = int(rest)
+            elif key == "at":
+                off, _, data = rest.partition(":")
+                runs.append((int(off), _expand(data.split())))
+            else:
+                raise ValueError("bad fixture line: %r" % line)
+    expected = np.zeros(total, dtype=np.uint8)
+    for off, data in runs:
+        expected[off:off + len(data)] = data
+    return block, np.array(words, dtype=np.uint16), expected
+
+
+def names():
+    return sorted(f for f in os.listdir(GOLDEN_DIR) if f.endswith(".txt") and f != "README.txt")
