@@ -1,0 +1,179 @@
+/*
+ * wcodec.h -- libwcodec: lossless compression of BF16 weight tensors with a
+ * block fixed-length exponent code, on NVIDIA B200 (sm_100a).
+ *
+ * The method: "ENEC: A Lossless AI Model Compression Method Enabling Fast
+ * Inference on Ascend NPUs", Abstract. A tensor is cut into blocks coded at one
+ * fixed length each; the length is a per-block bit width (bit-width
+ * quantization); values are packed two, four, then eight at a time
+ * (hierarchical halving bit-packing) after a branch-free integer remap; a
+ * prefix sum over block sizes places every block in the output. ZipServ
+ * ("ZipServ: Fast and Memory-Efficient LLM Inference with Hardware-Aware
+ * Lossless Compression", Abstract) is the reason the code is fixed-length:
+ * fixed-length blocks decode in constant time per element, in parallel.
+ *
+ * The stream ("WCB1"), as this library fixes it (little-endian throughout;
+ * sections start on 128-byte boundaries; all padding is zero):
+ *   [0, 128)       container header: magic "WCB1", version 1, header size,
+ *                  block size B, flags, n, nb, the four section offsets,
+ *                  exponent-plane bytes E, total bytes
+ *   off_hdr=128    u16 hdr[nb]   = base_b | w_b << 8
+ *   off_offs       u32 offs[nb]  = start of block b's payload, in 16-byte units
+ *   off_man        u8  s[n]      = sign << 7 | 7-bit mantissa of element i
+ *   off_exp        E bytes       = block b at 16*offs[b]; octet j at +j*w_b;
+ *                                  element t of an octet at bits [t*w, t*w+w)
+ * with e = (x >> 7) & 0xFF the exponent byte, w_b = bits(max e - min e) in
+ * 0..8 and base_b = min e (w_b < 8) or 0 (w_b == 8, the raw fallback).
+ *
+ * Conventions for every function below:
+ *  - Pointers named d_* are device pointers, h_* host pointers. The caller owns
+ *    every buffer. Device buffers must be 16-byte aligned.
+ *  - No function allocates memory or synchronizes the device. Work is enqueued
+ *    on `stream` (a cudaStream_t; 0 is the legacy default stream) and results
+ *    are visible once the caller synchronizes with it.
+ *  - The return value reports argument validation and launch errors only.
+ *    Errors found while the kernels run (a corrupt stream, a look-back that
+ *    timed out) are written to *d_status, an int32 in device memory that the
+ *    caller sets to 0 beforehand; the kernels only ever write a nonzero status
+ *    into it (the first error found is kept). d_status may be NULL, in which
+ *    case such errors are not reported.
+ *  - Block sizes B are powers of two from 128 to 4096; n <= 2^36.
+ */
+#ifndef WCODEC_H
+#define WCODEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WC_OK = 0,
+    WC_ERR_INVALID_ARG = 1,      /* bad pointer, alignment, B or n */
+    WC_ERR_BUFFER_TOO_SMALL = 2, /* output or workspace smaller than required */
+    WC_ERR_CORRUPT_STREAM = 3,   /* stream disagrees with the WCB1 definition */
+    WC_ERR_CUDA = 4,             /* a CUDA launch failed */
+    WC_ERR_TIMEOUT = 5           /* a bounded in-kernel wait ran out */
+} wc_status;
+
+#define WC_HEADER_BYTES 128u
+#define WC_MIN_BLOCK 128u
+#define WC_MAX_BLOCK 4096u
+#define WC_MAX_ELEMS (1ull << 36)
+
+/*
+ * Largest stream wc_compress can write for n elements at block size `block`:
+ * every block raw, 128 + A(2nb) + A(4nb) + A(n) + sum_b 8*ceil(L_b/8) bytes,
+ * A() rounding up to 128. Returns 0 if `block` or `n` is invalid.
+ * (Stream layout: ENEC Abstract for the ingredients; the byte layout is this
+ * library's.) Host-only, pure arithmetic.
+ */
+uint64_t wc_bound(uint64_t n, uint32_t block);
+
+/*
+ * Bytes of device workspace wc_compress needs for (n, block): the look-back
+ * state of each 8192-element tile of the single-pass encoder plus a ticket
+ * counter. Returns 0 if `block` or `n` is invalid. Host-only.
+ */
+uint64_t wc_workspace_size(uint64_t n, uint32_t block);
+
+/*
+ * Compress n BF16 words (d_in, read as 16-bit patterns: NaN payloads, -0 and
+ * denormals survive) into a WCB1 stream at d_out. Steps (ENEC Abstract):
+ * split each word into exponent and sign+mantissa bytes; per block, the bit
+ * width w = bits(max e - min e) and base; the remap e - base; hierarchical
+ * halving packing of each 8 values into w bytes; an exclusive prefix sum of
+ * block sizes, computed in one pass with a decoupled look-back over tiles.
+ *
+ *  d_in              n 16-bit words, device, 16-byte aligned
+ *  d_out             out_capacity bytes, device, 16-byte aligned;
+ *                    out_capacity >= wc_bound(n, block)
+ *  d_out_bytes       device u64: receives the stream's total size (0 on error)
+ *  d_workspace       workspace_bytes >= wc_workspace_size(n, block), device,
+ *                    16-byte aligned; the call clears it on `stream` first
+ *  d_status          nullable; WC_ERR_TIMEOUT if a look-back wait ran out
+ * Returns WC_ERR_INVALID_ARG, WC_ERR_BUFFER_TOO_SMALL or WC_ERR_CUDA
+ * without enqueuing work when the arguments are unusable. The stream is
+ * byte-for-byte the same on every run and every GPU.
+ */
+int wc_compress(const void *d_in, uint64_t n, uint32_t block,
+                void *d_out, uint64_t out_capacity, uint64_t *d_out_bytes,
+                void *d_workspace, uint64_t workspace_bytes,
+                int32_t *d_status, void *stream);
+
+/*
+ * Decompress the WCB1 stream d_stream (stream_bytes bytes, device, 16-byte
+ * aligned) into n BF16 words at d_out (device, 16-byte aligned), which the
+ * caller states together with `block` (wc_stream_info reads them from a host
+ * copy of the header). Each element is rebuilt as
+ *   x = (s & 0x80) << 8 | (base + v) << 7 | (s & 0x7F)
+ * from its mantissa byte s and its w-bit value v (ZipServ Abstract: a
+ * fixed-length code decodes in constant time, in parallel).
+ * The kernels check the container header against (n, block), every block's
+ * w <= 8 (and base 0 when w == 8), that offs is the prefix sum of the block
+ * sizes and that every read stays inside stream_bytes; a failed check writes
+ * WC_ERR_CORRUPT_STREAM to *d_status, and the output is then unspecified.
+ * No read or write ever leaves the given buffers.
+ * Returns WC_ERR_CORRUPT_STREAM at once if stream_bytes is smaller than the
+ * fixed sections that (n, block) imply.
+ */
+int wc_decompress(const void *d_stream, uint64_t stream_bytes, void *d_out,
+                  uint64_t n, uint32_t block, int32_t *d_status, void *stream);
+
+/*
+ * One tensor of a batched decode.
+ *   stream, stream_bytes: the WCB1 stream (device, 16-byte aligned)
+ *   out: n BF16 words (device, 16-byte aligned); block: its block size
+ */
+typedef struct {
+    const void *stream;
+    uint64_t stream_bytes;
+    void *out;
+    uint64_t n;
+    uint32_t block;
+    uint32_t reserved; /* must be 0 */
+} wc_batch_item;
+
+/*
+ * Decompress `count` independent streams in as few launches as possible (one
+ * launch per WC_BATCH_MAX items). h_items is a HOST array; its contents are
+ * passed to the kernel as launch parameters, so the call needs no device
+ * descriptor buffer and can be captured in a CUDA graph. Every check of
+ * wc_decompress applies to every item; d_status collects the first error.
+ */
+#define WC_BATCH_MAX 512u
+int wc_decompress_batch(const wc_batch_item *h_items, uint32_t count,
+                        int32_t *d_status, void *stream);
+
+/*
+ * Parse a host copy of a stream's first `header_bytes` (>= 128) bytes. Fills
+ * n, block and total_bytes (any may be NULL). Returns WC_ERR_CORRUPT_STREAM
+ * if the header is not a WCB1 version-1 header consistent with itself.
+ */
+int wc_stream_info(const void *h_header, uint64_t header_bytes,
+                   uint64_t *n, uint32_t *block, uint64_t *total_bytes);
+
+/* A static, human-readable name for a status code. */
+const char *wc_status_string(int status);
+
+/*
+ * Test hook for the bounded waits of wc_compress. Runs the same encoder,
+ * except that no thread block ever takes tile 0, so the look-back of every
+ * later tile waits on a flag that nothing sets. Each such wait gives up after
+ * timeout_ns nanoseconds (device global timer) and the call ends with
+ * WC_ERR_TIMEOUT in *d_status, leaving the device usable. Needs n large
+ * enough for at least two 8192-element tiles. Arguments as wc_compress.
+ */
+int wc_debug_compress_stalled(const void *d_in, uint64_t n, uint32_t block,
+                              void *d_out, uint64_t out_capacity,
+                              uint64_t *d_out_bytes, void *d_workspace,
+                              uint64_t workspace_bytes, int32_t *d_status,
+                              uint64_t timeout_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WCODEC_H */

@@ -1,0 +1,172 @@
+// wc_api.cu -- the extern "C" boundary of libwcodec: argument checks, layout
+// arithmetic and kernel launches. Declarations and their contracts are in
+// include/wcodec.h.
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/wcodec.h"
+#include "wc_internal.cuh"
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;  // bounded look-back wait: 1 s
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool args_ok(uint64_t n, uint32_t block) { return wc::block_ok(block) && n <= wc::kMaxElems; }
+
+int check_compress_args(const void* d_in, uint64_t n, uint32_t block, void* d_out,
+                        uint64_t out_capacity, uint64_t* d_out_bytes, void* d_workspace,
+                        uint64_t workspace_bytes) {
+    if (!args_ok(n, block) || d_out == nullptr || d_out_bytes == nullptr || d_workspace == nullptr ||
+        (n > 0 && d_in == nullptr))
+        return WC_ERR_INVALID_ARG;
+    if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) || !aligned16(d_workspace) ||
+        (reinterpret_cast<uintptr_t>(d_out_bytes) & 7u) != 0)
+        return WC_ERR_INVALID_ARG;
+    if (out_capacity < wc::bound_bytes(n, block) ||
+        workspace_bytes < wc::encode_workspace_bytes(n))
+        return WC_ERR_BUFFER_TOO_SMALL;
+    return WC_OK;
+}
+
+int check_decode_item(const wc_batch_item& it) {
+    if (!args_ok(it.n, it.block) || it.stream == nullptr || (it.n > 0 && it.out == nullptr) ||
+        it.reserved != 0)
+        return WC_ERR_INVALID_ARG;
+    if (!aligned16(it.stream) || (it.n > 0 && !aligned16(it.out))) return WC_ERR_INVALID_ARG;
+    // the fixed sections alone need off_exp bytes
+    if (it.stream_bytes < wc::make_layout(it.n, it.block).off_exp) return WC_ERR_CORRUPT_STREAM;
+    return WC_OK;
+}
+
+wc::DecodeItem to_item(const wc_batch_item& it) {
+    wc::DecodeItem d;
+    d.stream = static_cast<const uint8_t*>(it.stream);
+    d.stream_bytes = it.stream_bytes;
+    d.out = static_cast<uint16_t*>(it.out);
+    d.n = it.n;
+    d.block = it.block;
+    d.reserved = 0;
+    return d;
+}
+
+uint64_t get_le(const uint8_t* p, int nbytes) {
+    uint64_t v = 0;
+    for (int k = 0; k < nbytes; ++k) v |= uint64_t(p[k]) << (8 * k);
+    return v;
+}
+
+}  // namespace
+
+extern "C" {
+
+uint64_t wc_bound(uint64_t n, uint32_t block) {
+    return args_ok(n, block) ? wc::bound_bytes(n, block) : 0;
+}
+
+uint64_t wc_workspace_size(uint64_t n, uint32_t block) {
+    return args_ok(n, block) ? wc::encode_workspace_bytes(n) : 0;
+}
+
+static int compress_impl(const void* d_in, uint64_t n, uint32_t block, void* d_out,
+                         uint64_t out_capacity, uint64_t* d_out_bytes, void* d_workspace,
+                         uint64_t workspace_bytes, int32_t* d_status, uint64_t timeout_ns,
+                         uint32_t first_ticket, void* stream) {
+    const int rc = check_compress_args(d_in, n, block, d_out, out_capacity, d_out_bytes,
+                                       d_workspace, workspace_bytes);
+    if (rc != WC_OK) return rc;
+    const wc::Layout L = wc::make_layout(n, block);
+    const cudaError_t err = wc::launch_encode(
+        static_cast<const uint16_t*>(d_in), L, static_cast<uint8_t*>(d_out), d_out_bytes,
+        d_workspace, d_status, timeout_ns, first_ticket, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
+int wc_compress(const void* d_in, uint64_t n, uint32_t block, void* d_out, uint64_t out_capacity,
+                uint64_t* d_out_bytes, void* d_workspace, uint64_t workspace_bytes,
+                int32_t* d_status, void* stream) {
+    return compress_impl(d_in, n, block, d_out, out_capacity, d_out_bytes, d_workspace,
+                         workspace_bytes, d_status, kDefaultTimeoutNs, 0, stream);
+}
+
+int wc_debug_compress_stalled(const void* d_in, uint64_t n, uint32_t block, void* d_out,
+                              uint64_t out_capacity, uint64_t* d_out_bytes, void* d_workspace,
+                              uint64_t workspace_bytes, int32_t* d_status, uint64_t timeout_ns,
+                              void* stream) {
+    if (wc::num_tiles(n) < 2 || timeout_ns == 0 || timeout_ns > 10 * kDefaultTimeoutNs)
+        return WC_ERR_INVALID_ARG;
+    return compress_impl(d_in, n, block, d_out, out_capacity, d_out_bytes, d_workspace,
+                         workspace_bytes, d_status, timeout_ns, 1, stream);
+}
+
+int wc_decompress(const void* d_stream, uint64_t stream_bytes, void* d_out, uint64_t n,
+                  uint32_t block, int32_t* d_status, void* stream) {
+    wc_batch_item it;
+    it.stream = d_stream;
+    it.stream_bytes = stream_bytes;
+    it.out = d_out;
+    it.n = n;
+    it.block = block;
+    it.reserved = 0;
+    const int rc = check_decode_item(it);
+    if (rc != WC_OK) return rc;
+    const wc::DecodeItem d = to_item(it);
+    const cudaError_t err = wc::launch_decode(&d, 1, d_status, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
+int wc_decompress_batch(const wc_batch_item* h_items, uint32_t count, int32_t* d_status,
+                        void* stream) {
+    if (h_items == nullptr && count > 0) return WC_ERR_INVALID_ARG;
+    for (uint32_t i = 0; i < count; ++i) {  // validate everything before launching anything
+        const int rc = check_decode_item(h_items[i]);
+        if (rc != WC_OK) return rc;
+    }
+    wc::DecodeItem chunk[WC_BATCH_MAX];
+    for (uint32_t base = 0; base < count; base += WC_BATCH_MAX) {
+        const uint32_t c = (count - base < WC_BATCH_MAX) ? count - base : WC_BATCH_MAX;
+        for (uint32_t i = 0; i < c; ++i) chunk[i] = to_item(h_items[base + i]);
+        const cudaError_t err =
+            wc::launch_decode(chunk, c, d_status, static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return WC_ERR_CUDA;
+    }
+    return WC_OK;
+}
+
+int wc_stream_info(const void* h_header, uint64_t header_bytes, uint64_t* n, uint32_t* block,
+                   uint64_t* total_bytes) {
+    if (h_header == nullptr || header_bytes < WC_HEADER_BYTES) return WC_ERR_INVALID_ARG;
+    const uint8_t* p = static_cast<const uint8_t*>(h_header);
+    const uint64_t nn = get_le(p + 16, 8);
+    const uint32_t B = uint32_t(get_le(p + 8, 4));
+    if (get_le(p, 4) != wc::kMagic || get_le(p + 4, 2) != wc::kVersion ||
+        get_le(p + 6, 2) != wc::kHeaderBytes || get_le(p + 12, 4) != 0 || !args_ok(nn, B))
+        return WC_ERR_CORRUPT_STREAM;
+    const wc::Layout L = wc::make_layout(nn, B);
+    const uint64_t E = get_le(p + 64, 8), total = get_le(p + 72, 8);
+    if (get_le(p + 24, 8) != L.nb || get_le(p + 32, 8) != L.off_hdr ||
+        get_le(p + 40, 8) != L.off_offs || get_le(p + 48, 8) != L.off_man ||
+        get_le(p + 56, 8) != L.off_exp || E > nn + 8 || total != L.off_exp + E)
+        return WC_ERR_CORRUPT_STREAM;
+    for (int k = 80; k < 128; ++k)
+        if (p[k] != 0) return WC_ERR_CORRUPT_STREAM;
+    if (n) *n = nn;
+    if (block) *block = B;
+    if (total_bytes) *total_bytes = total;
+    return WC_OK;
+}
+
+const char* wc_status_string(int status) {
+    switch (status) {
+        case WC_OK: return "ok";
+        case WC_ERR_INVALID_ARG: return "invalid argument";
+        case WC_ERR_BUFFER_TOO_SMALL: return "buffer too small";
+        case WC_ERR_CORRUPT_STREAM: return "corrupt stream";
+        case WC_ERR_CUDA: return "CUDA error";
+        case WC_ERR_TIMEOUT: return "in-kernel wait timed out";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,247 @@
+"""ctypes binding of libwcodec (include/wcodec.h), plus torch-tensor helpers.
+
+The ``wc_*`` functions take the same arguments as the C functions (device
+pointers as ints, sizes, a cudaStream_t as an int); they only marshal
+arguments. Every step of compression and decompression runs in the library's
+CUDA kernels; there is no Python or CPU fallback, and loading fails loudly if
+``libwcodec.so`` has not been built (``python -m
+lossless_weight_compression_b200.build_lib``).
+
+The helpers below (``compress``, ``decompress``, ...) take torch tensors,
+allocate outputs with torch and call the same entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwcodec.so")
+
+WC_OK = 0
+WC_ERR_INVALID_ARG = 1
+WC_ERR_BUFFER_TOO_SMALL = 2
+WC_ERR_CORRUPT_STREAM = 3
+WC_ERR_CUDA = 4
+WC_ERR_TIMEOUT = 5
+WC_HEADER_BYTES = 128
+WC_BATCH_MAX = 512
+BLOCK_SIZES = (128, 256, 512, 1024, 2048, 4096)
+
+
+class WcodecError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__("%s: %s (status %d)" % (what, wc_status_string(status), status))
+        self.status = status
+
+
+class wc_batch_item(ctypes.Structure):
+    _fields_ = [
+        ("stream", ctypes.c_void_p),
+        ("stream_bytes", ctypes.c_uint64),
+        ("out", ctypes.c_void_p),
+        ("n", ctypes.c_uint64),
+        ("block", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libwcodec.so (once). Raises if it is missing: there is no fallback."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            "libwcodec.so is not built (%s); run `python -m lossless_weight_compression_b200."
+            "build_lib`" % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    u32, u64, vp, i = ctypes.c_uint32, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_int
+    L.wc_bound.argtypes, L.wc_bound.restype = [u64, u32], u64
+    L.wc_workspace_size.argtypes, L.wc_workspace_size.restype = [u64, u32], u64
+    L.wc_compress.argtypes = [vp, u64, u32, vp, u64, vp, vp, u64, vp, vp]
+    L.wc_compress.restype = i
+    L.wc_decompress.argtypes = [vp, u64, vp, u64, u32, vp, vp]
+    L.wc_decompress.restype = i
+    L.wc_decompress_batch.argtypes = [ctypes.POINTER(wc_batch_item), u32, vp, vp]
+    L.wc_decompress_batch.restype = i
+    L.wc_stream_info.argtypes = [vp, u64, ctypes.POINTER(u64), ctypes.POINTER(u32),
+                                 ctypes.POINTER(u64)]
+    L.wc_stream_info.restype = i
+    L.wc_status_string.argtypes, L.wc_status_string.restype = [i], ctypes.c_char_p
+    L.wc_debug_compress_stalled.argtypes = [vp, u64, u32, vp, u64, vp, vp, u64, vp, u64, vp]
+    L.wc_debug_compress_stalled.restype = i
+    _lib = L
+    return L
+
+
+# ---------------------------------------------------------------------------
+# The C functions, same names and arguments
+# ---------------------------------------------------------------------------
+def wc_bound(n: int, block: int) -> int:
+    return lib().wc_bound(n, block)
+
+
+def wc_workspace_size(n: int, block: int) -> int:
+    return lib().wc_workspace_size(n, block)
+
+
+def wc_compress(d_in, n, block, d_out, out_capacity, d_out_bytes, d_workspace, workspace_bytes,
+                d_status, stream) -> int:
+    return lib().wc_compress(d_in, n, block, d_out, out_capacity, d_out_bytes, d_workspace,
+                             workspace_bytes, d_status, stream)
+
+
+def wc_decompress(d_stream, stream_bytes, d_out, n, block, d_status, stream) -> int:
+    return lib().wc_decompress(d_stream, stream_bytes, d_out, n, block, d_status, stream)
+
+
+def wc_decompress_batch(items, count, d_status, stream) -> int:
+    return lib().wc_decompress_batch(items, count, d_status, stream)
+
+
+def wc_stream_info(h_header: bytes):
+    """Returns (status, n, block, total_bytes) parsed from a host copy of the header."""
+    n, blk, tot = ctypes.c_uint64(), ctypes.c_uint32(), ctypes.c_uint64()
+    buf = ctypes.create_string_buffer(bytes(h_header), len(h_header))
+    rc = lib().wc_stream_info(ctypes.cast(buf, ctypes.c_void_p), len(h_header), ctypes.byref(n),
+                              ctypes.byref(blk), ctypes.byref(tot))
+    return rc, n.value, blk.value, tot.value
+
+
+def wc_status_string(status: int) -> str:
+    return lib().wc_status_string(status).decode()
+
+
+def wc_debug_compress_stalled(d_in, n, block, d_out, out_capacity, d_out_bytes, d_workspace,
+                              workspace_bytes, d_status, timeout_ns, stream) -> int:
+    return lib().wc_debug_compress_stalled(d_in, n, block, d_out, out_capacity, d_out_bytes,
+                                           d_workspace, workspace_bytes, d_status, timeout_ns,
+                                           stream)
+
+
+# ---------------------------------------------------------------------------
+# torch helpers
+# ---------------------------------------------------------------------------
+def _stream_handle(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _check(rc: int, what: str):
+    if rc != WC_OK:
+        raise WcodecError(rc, what)
+
+
+def as_words(x: torch.Tensor) -> torch.Tensor:
+    """A 16-bit tensor (bf16 / int16 / uint16 / fp16) as contiguous flat int16 words."""
+    if x.element_size() != 2:
+        raise TypeError("wcodec compresses 16-bit words (BF16); got %s" % x.dtype)
+    return x.contiguous().view(-1).view(torch.int16)
+
+
+@dataclass
+class Compressed:
+    """A compressed tensor on the GPU: ``buffer`` holds ``wc_bound`` bytes of
+    which the first ``nbytes`` (a device int64) are the stream."""
+    buffer: torch.Tensor
+    nbytes: torch.Tensor
+    status: torch.Tensor
+    n: int
+    block: int
+    shape: tuple
+    dtype: torch.dtype
+
+    def size(self) -> int:
+        return int(self.nbytes.item())
+
+    def stream(self) -> torch.Tensor:
+        """The stream bytes (synchronises to read the size)."""
+        return self.buffer[: self.size()]
+
+
+def workspace_for(n: int, block: int, device) -> torch.Tensor:
+    ws = wc_workspace_size(n, block)
+    if ws == 0:
+        raise WcodecError(WC_ERR_INVALID_ARG, "workspace size")
+    return torch.empty((ws + 15) // 16 * 16, dtype=torch.uint8, device=device)
+
+
+def compress(x: torch.Tensor, block: int = 1024, *, workspace: torch.Tensor | None = None,
+             stream=None) -> Compressed:
+    """Compress a CUDA tensor of BF16 (any 16-bit dtype is read as bit patterns)."""
+    words = as_words(x)
+    n = words.numel()
+    cap = wc_bound(n, block)
+    if cap == 0:
+        raise WcodecError(WC_ERR_INVALID_ARG, "block size %r" % (block,))
+    dev = words.device
+    buf = torch.empty((cap + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+    nbytes = torch.zeros(1, dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = workspace_for(n, block, dev)
+    rc = wc_compress(words.data_ptr() if n else None, n, block, buf.data_ptr(), buf.numel(),
+                     nbytes.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                     status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_compress")
+    return Compressed(buf, nbytes, status, n, block, tuple(x.shape), x.dtype)
+
+
+def decompress(stream_bytes: torch.Tensor, n: int, block: int, *, out: torch.Tensor | None = None,
+               status: torch.Tensor | None = None, nbytes: int | None = None,
+               stream=None) -> torch.Tensor:
+    """Decode a stream (a uint8 CUDA tensor) into n BF16 values (``out`` if given)."""
+    if out is None:
+        out = torch.empty(n, dtype=torch.bfloat16, device=stream_bytes.device)
+    words = out.view(-1)
+    if words.numel() != n or not words.is_contiguous() or out.element_size() != 2:
+        raise ValueError("out must be a contiguous 16-bit tensor of %d elements" % n)
+    own_status = status is None
+    if own_status:
+        status = torch.zeros(1, dtype=torch.int32, device=stream_bytes.device)
+    size = stream_bytes.numel() if nbytes is None else nbytes
+    rc = wc_decompress(stream_bytes.data_ptr(), size, words.data_ptr() if n else None, n, block,
+                       status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_decompress")
+    return out
+
+
+def decompress_compressed(c: Compressed, out: torch.Tensor | None = None, status=None,
+                          stream=None) -> torch.Tensor:
+    """Decode a ``Compressed`` back into its original shape and dtype."""
+    if out is None:
+        out = torch.empty(c.shape, dtype=c.dtype, device=c.buffer.device)
+    return decompress(c.buffer, c.n, c.block, out=out, status=status, stream=stream)
+
+
+def make_batch(items) -> ctypes.Array:
+    """items: iterable of (stream uint8 tensor, stream_bytes, out tensor, n, block)."""
+    items = list(items)
+    arr = (wc_batch_item * max(1, len(items)))()
+    for k, (s, sb, o, n, b) in enumerate(items):
+        arr[k].stream = s.data_ptr()
+        arr[k].stream_bytes = sb
+        arr[k].out = o.data_ptr() if n else None
+        arr[k].n = n
+        arr[k].block = b
+        arr[k].reserved = 0
+    return arr, len(items)
+
+
+def decompress_batch(batch, status: torch.Tensor, stream=None):
+    """Decode a batch made by ``make_batch`` in one launch per 512 tensors."""
+    arr, count = batch
+    rc = wc_decompress_batch(arr, count, status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_decompress_batch")
+
+
+def stream_info(header: bytes):
+    rc, n, block, total = wc_stream_info(header)
+    _check(rc, "wc_stream_info")
+    return n, block, total

@@ -17,3 +17,20 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def wclib():
+    """The built libwcodec (compiled in-tree if missing or stale)."""
+    from lossless_weight_compression_b200 import build_lib, wcodec
+    build_lib.build()
+    wcodec.lib()
+    return wcodec
+
+
+@pytest.fixture(scope="session")
+def cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("GPU test run without a CUDA device")
+    return torch.device("cuda:0")

@@ -1,0 +1,120 @@
+"""The C-ABI library on the host: it loads, exports every function that
+include/wcodec.h declares, and its host-only arithmetic and argument checks
+behave as documented. No call here launches a kernel (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+BLOCKS = (128, 256, 512, 1024, 2048, 4096)
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)  # drop comments
+        names += re.findall(r"^[A-Za-z_][\w \*]*?\b(wc_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for f in ("wc_bound", "wc_workspace_size", "wc_compress", "wc_decompress",
+              "wc_decompress_batch", "wc_stream_info", "wc_status_string",
+              "wc_debug_compress_stalled"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol(wclib):
+    raw = ctypes.CDLL(wclib.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), name
+
+
+def test_bound_matches_oracle(wclib, orc):
+    rng = np.random.default_rng(0)
+    for B in BLOCKS:
+        for n in [0, 1, 7, 8, 9, B - 1, B, B + 1, 8191, 8192, 8193] + list(rng.integers(0, 10**7, 5)):
+            assert wclib.wc_bound(int(n), B) == orc.bound(int(n), B)
+    for bad in (0, 1, 64, 127, 129, 384, 8192, 2**31):
+        assert wclib.wc_bound(100, bad) == 0
+    assert wclib.wc_bound(2**36, 1024) > 0 and wclib.wc_bound(2**36 + 1, 1024) == 0
+
+
+def test_workspace_size(wclib):
+    for n, tiles in [(0, 0), (1, 1), (8192, 1), (8193, 2), (10**6, 123)]:
+        assert wclib.wc_workspace_size(n, 512) == 16 + 8 * tiles
+    assert wclib.wc_workspace_size(10, 100) == 0
+
+
+def test_stream_info_parses_oracle_headers(wclib, orc):
+    rng = np.random.default_rng(1)
+    for B in BLOCKS:
+        for n in (0, 1, 1000, 3 * B + 5):
+            words = rng.integers(0, 65536, n).astype(np.uint16)
+            s = orc.compress(words, B)
+            rc, nn, bb, tot = wclib.wc_stream_info(bytes(s[:128]))
+            assert (rc, nn, bb, tot) == (0, n, B, s.size)
+
+
+def test_stream_info_rejects_bad_headers(wclib, orc):
+    s = orc.compress(np.arange(5000, dtype=np.uint16), 256)
+    good = bytes(s[:128])
+    assert wclib.wc_stream_info(good)[0] == wclib.WC_OK
+    for off, val in [(0, 0), (4, 2), (6, 64), (8, 0x7F), (12, 1), (16, 0x99), (24, 3), (40, 1),
+                     (64, 0xFF), (72, 0), (100, 1)]:
+        b = bytearray(good)
+        b[off] = (b[off] + val) & 0xFF if val else (b[off] ^ 0xFF)
+        assert wclib.wc_stream_info(bytes(b))[0] == wclib.WC_ERR_CORRUPT_STREAM, off
+    assert wclib.wc_stream_info(good[:64])[0] == wclib.WC_ERR_INVALID_ARG
+
+
+def test_status_strings(wclib):
+    for code in range(6):
+        assert wclib.wc_status_string(code)
+    assert wclib.wc_status_string(99) == "unknown status"
+
+
+def test_argument_checks_before_any_launch(wclib):
+    """Invalid arguments are rejected on the host; these calls never reach CUDA."""
+    c = wclib
+    # null input with n > 0, null output, invalid block, misaligned pointers
+    assert c.wc_compress(None, 10, 128, 16, 10**6, 16, 16, 10**6, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_compress(16, 10, 128, None, 10**6, 16, 16, 10**6, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_compress(16, 10, 100, 16, 10**6, 16, 16, 10**6, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_compress(17, 10, 128, 16, 10**6, 16, 16, 10**6, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_compress(16, 10, 128, 16, 10, 16, 16, 10**6, None, None) == c.WC_ERR_BUFFER_TOO_SMALL
+    assert c.wc_compress(16, 10, 128, 16, 10**6, 16, 16, 8, None, None) == c.WC_ERR_BUFFER_TOO_SMALL
+    # decode: stream shorter than the fixed sections, null stream, misaligned output, bad block
+    assert c.wc_decompress(16, 100, 16, 10, 128, None, None) == c.WC_ERR_CORRUPT_STREAM
+    assert c.wc_decompress(None, 10**6, 16, 10, 128, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_decompress(16, 10**6, 18, 10, 128, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_decompress(16, 10**6, 16, 10, 3000, None, None) == c.WC_ERR_INVALID_ARG
+    # batch: every item is checked before anything is launched
+    arr, count = c.make_batch([])
+    items = (c.wc_batch_item * 2)()
+    items[0].stream, items[0].stream_bytes, items[0].out, items[0].n, items[0].block = 16, 10**6, 16, 10, 128
+    items[1].stream, items[1].stream_bytes, items[1].out, items[1].n, items[1].block = 16, 10**6, 16, 10, 99
+    assert c.wc_decompress_batch(items, 2, None, None) == c.WC_ERR_INVALID_ARG
+    items[1].block, items[1].reserved = 128, 1
+    assert c.wc_decompress_batch(items, 2, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_decompress_batch(None, 1, None, None) == c.WC_ERR_INVALID_ARG
+    # the stall test hook needs two tiles and a bounded timeout
+    assert c.wc_debug_compress_stalled(16, 100, 128, 16, 10**6, 16, 16, 10**6, None, 10**6,
+                                       None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_debug_compress_stalled(16, 10**5, 128, 16, 10**7, 16, 16, 10**6, None, 0,
+                                       None) == c.WC_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    from lossless_weight_compression_b200 import wcodec
+    monkeypatch.setattr(wcodec, "_lib", None)
+    monkeypatch.setattr(wcodec, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        wcodec.lib()
