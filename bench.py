@@ -43,6 +43,8 @@ FALLBACK_HBM_GBS = 6650.0
 WORKLOAD = ("llama3_8b_stack: 32 Llama-3-8B-shaped decoder layers + embedding + LM head "
             "(226 BF16 tensors, 8,029,995,008 elements, 16.06 GB), N(0, 0.02) with per-matrix "
             "std jitter U[0.7, 1.3], block 1024")
+LAYER_WORKLOAD = ("llama3_8b_layer: one Llama-3-8B-shaped decoder layer (7 BF16 tensors, "
+                  "218,103,808 elements, 436 MB), block 1024 -- a smaller case for profiling")
 
 
 def log(*a):
@@ -86,6 +88,11 @@ def barrier(dist, device):
             dist.barrier()
     if device.type == "cuda":
         torch.cuda.synchronize(device)
+
+
+def whole_job_gbs(world: int, bytes_per_rank: float, steps: int, max_seconds: float) -> float:
+    """Whole-job throughput: the bytes all ranks produced over the slowest rank's time."""
+    return world * bytes_per_rank * steps / max_seconds / 1e9
 
 
 def rank_seed_base(rank: int) -> int:
@@ -288,7 +295,11 @@ def run_wcodec(args):
     t0 = time.time()
     names, inputs = [], []
     hist = torch.zeros(256, dtype=torch.int64, device=dev)
-    for name, t in synth.stack_tensors(dev, rank_seed_base(rank)):
+    if args.workload == "stack":
+        tensors = synth.stack_tensors(dev, rank_seed_base(rank))
+    else:
+        tensors = synth.layer_tensors(0, dev, rank_seed_base(rank))
+    for name, t in tensors:
         words = t.view(-1).view(torch.int16)
         hist += torch.bincount(((words.to(torch.int32) >> 7) & 0xFF), minlength=256)
         names.append(name)
@@ -362,12 +373,14 @@ def run_wcodec(args):
     verified &= nb_again == sizes
 
     # ---- end to end: compressed streams from pinned host memory ---------------------
-    e2e = run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stream, dist,
-                  dev, n_total)
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stream, dist,
+                      dev, n_total)
 
     # ---- figures ---------------------------------------------------------------------
     bytes_out = 2 * n_total
-    value = world * bytes_out * args.steps / dec_total_s / 1e9
+    value = whole_job_gbs(world, bytes_out, args.steps, dec_total_s)
     moved = stream_total + bytes_out  # algorithmic bytes of one decode launch: read C, write 2n
     dec_launch_s = dec_total_s / args.steps
     achieved = moved / dec_launch_s / 1e9
@@ -394,12 +407,14 @@ def run_wcodec(args):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * dec_launch_s, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "u16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "block": BLOCK, "tensors": len(inputs),
+            "config": {"workload": WORKLOAD if args.workload == "stack" else LAYER_WORKLOAD,
+                       "block": BLOCK, "tensors": len(inputs),
                        "elements_per_gpu": n_total, "parallelism": "replicas: one stack per GPU",
-                       "l2": "inputs larger than L2 (16.06 GB BF16 in, %.2f GB stream per pass "
-                             "vs 126 MB L2); no flush" % (stream_total / 1e9),
-                       "step": "compress all 226 tensors (226 encoder launches) + decompress all "
-                               "(1 batched decoder launch); value times the decode phase"},
+                       "l2": "inputs larger than L2 (%.2f GB BF16 in, %.2f GB stream per pass "
+                             "vs 126 MB L2); no flush" % (bytes_out / 1e9, stream_total / 1e9),
+                       "step": "compress all %d tensors (one encoder launch each) + decompress "
+                               "all (1 batched decoder launch); value times the decode phase"
+                               % len(inputs)},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "peak_kind": peak_kind,
                          "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
@@ -410,7 +425,8 @@ def run_wcodec(args):
                             "exponent_entropy_bits": H, "entropy_bound_ratio": 16.0 / (8.0 + H),
                             "format_payload_bound_ratio": rho_fmt,
                             "ratio_over_format_bound": ratio / rho_fmt},
-            "encode": {"value": world * bytes_out * args.steps / enc_total_s / 1e9, "unit": "GB/s",
+            "encode": {"value": whole_job_gbs(world, bytes_out, args.steps, enc_total_s),
+                       "unit": "GB/s",
                        "ms_per_step": 1e3 * enc_total_s / args.steps,
                        "achieved_hbm_gbs": (bytes_out + stream_total) / (enc_total_s / args.steps) / 1e9},
             "e2e": e2e,
@@ -469,7 +485,7 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
     sec = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, dev)
     ok = status_host.item() == 0 and all(torch.equal(a, b) for a, b in zip(inputs, outs))
     world = dist.get_world_size() if dist is not None else 1
-    return {"value": world * 2 * n_total * steps / sec / 1e9, "unit": "GB/s",
+    return {"value": whole_job_gbs(world, 2 * n_total, steps, sec), "unit": "GB/s",
             "h2d_bytes_per_step": total, "d2h_bytes_per_step": 4, "steps": steps,
             "verified_bit_exact": bool(ok)}
 
@@ -480,8 +496,13 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("wcodec", "reference"), default="wcodec")
+    ap.add_argument("--workload", choices=("stack", "layer"), default="stack",
+                    help="stack: the 8B-shaped stack (the benchmark); layer: one decoder layer "
+                         "(a smaller case for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip timing the CPU oracle (for profiling runs)")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end (pinned host memory) measurement")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         log("note: fewer than 3 warm-up steps")
