@@ -104,6 +104,37 @@ int wc_compress(const void *d_in, uint64_t n, uint32_t block,
                 int32_t *d_status, void *stream);
 
 /*
+ * Allocation-free variant of wc_compress. The pages have no counterpart: this
+ * entry point exists for callers of the library, not for the method.
+ *
+ * Some callers cannot allocate device memory: an engine that reserves all of
+ * a GPU's memory for its own pools at start-up (KV caches, weight arenas),
+ * where a cudaMalloc fails or fragments the pool, or a latency-critical path
+ * that must not stall on the device-wide synchronisation cudaMalloc and
+ * cudaFree may imply. This call needs no workspace from them: the encoder's
+ * look-back state lives in a fixed array inside the library,
+ * WC_NOALLOC_SCRATCH_BYTES bytes of device memory that every GPU loading the
+ * library holds until the process exits. Inputs, outputs and their meaning are
+ * those of wc_compress.
+ *  - n may not exceed WC_NOALLOC_MAX_ELEMS (2^30); a larger n returns
+ *    WC_ERR_BUFFER_TOO_SMALL before anything is looked up or enqueued.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the one array and it keeps what the last call left;
+ *    every call clears the part it uses on `stream` before its kernel runs.
+ *    Calls that can overlap on the GPU (unordered streams, several host
+ *    threads) race on the array and can write wrong streams: serialise them.
+ *  - Neither the call nor its set-up allocates memory (no cudaMalloc,
+ *    cudaFree or allocating library routine).
+ */
+#define WC_NOALLOC_MAX_ELEMS (1ull << 30)
+#define WC_NOALLOC_SCRATCH_BYTES (16ull + 8ull * (WC_NOALLOC_MAX_ELEMS / 8192ull))
+int wc_compress_noalloc(const void *d_in, uint64_t n, uint32_t block,
+                        void *d_out, uint64_t out_capacity,
+                        uint64_t *d_out_bytes, int32_t *d_status, void *stream);
+
+/*
  * Decompress the WCB1 stream d_stream (stream_bytes bytes, device, 16-byte
  * aligned) into n BF16 words at d_out (device, 16-byte aligned), which the
  * caller states together with `block` (wc_stream_info reads them from a host

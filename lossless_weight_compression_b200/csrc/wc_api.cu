@@ -100,6 +100,29 @@ int wc_debug_compress_stalled(const void* d_in, uint64_t n, uint32_t block, void
                          workspace_bytes, d_status, timeout_ns, 1, stream);
 }
 
+int wc_compress_noalloc(const void* d_in, uint64_t n, uint32_t block, void* d_out,
+                        uint64_t out_capacity, uint64_t* d_out_bytes, int32_t* d_status,
+                        void* stream) {
+    // Size first: nothing is looked up or enqueued for a tensor the array cannot serve.
+    if (n > wc::noalloc_max_elems()) return WC_ERR_BUFFER_TOO_SMALL;
+    if (!wc::block_ok(block) || d_out == nullptr || d_out_bytes == nullptr ||
+        (n > 0 && d_in == nullptr))
+        return WC_ERR_INVALID_ARG;
+    if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) ||
+        (reinterpret_cast<uintptr_t>(d_out_bytes) & 7u) != 0)
+        return WC_ERR_INVALID_ARG;
+    if (out_capacity < wc::bound_bytes(n, block)) return WC_ERR_BUFFER_TOO_SMALL;
+    void* scratch = nullptr;
+    uint64_t scratch_bytes = 0;
+    if (wc::noalloc_scratch(&scratch, &scratch_bytes) != cudaSuccess) return WC_ERR_CUDA;
+    if (scratch_bytes < wc::encode_workspace_bytes(n)) return WC_ERR_BUFFER_TOO_SMALL;
+    const wc::Layout L = wc::make_layout(n, block);
+    const cudaError_t err = wc::launch_encode(
+        static_cast<const uint16_t*>(d_in), L, static_cast<uint8_t*>(d_out), d_out_bytes, scratch,
+        d_status, kDefaultTimeoutNs, 0, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
 int wc_decompress(const void* d_stream, uint64_t stream_bytes, void* d_out, uint64_t n,
                   uint32_t block, int32_t* d_status, void* stream) {
     wc_batch_item it;

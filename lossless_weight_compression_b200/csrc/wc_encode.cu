@@ -18,6 +18,8 @@
 // tile only ever waits on tiles that started before it; every wait is bounded
 // by a device-timer limit after which the tile reports WC_ERR_TIMEOUT and
 // marks its state word so that later tiles stop waiting too.
+#include <mutex>
+
 #include "wc_internal.cuh"
 
 namespace wc {
@@ -379,6 +381,55 @@ cudaError_t launch_encode(const uint16_t* in, const Layout& L, uint8_t* out, uin
     const unsigned grid = unsigned(ntiles ? ntiles : 1);
     encode_kernel<<<grid, kThreads, 0, stream>>>(a);
     return cudaGetLastError();
+}
+
+}  // namespace wc
+
+// ---------------------------------------------------------------------------
+// Allocation-free encoder entry (wc_compress_noalloc)
+// ---------------------------------------------------------------------------
+// Some callers cannot allocate device memory: an engine that reserves all of
+// a GPU's memory for its own pools at start-up (a cudaMalloc then fails or
+// fragments the pool), or a latency-critical path that must not stall on the
+// device-wide synchronisation cudaMalloc/cudaFree may imply. For them the
+// encoder's only scratch -- 16 bytes of control words plus one 8-byte
+// look-back word per 8192-element tile -- lives in this fixed array, which
+// every GPU that loads the library holds until the process exits. Its size
+// caps such calls at 2^30 elements.
+namespace wc {
+
+constexpr uint64_t kNoAllocMaxElems = 1ull << 30;
+constexpr uint64_t kNoAllocScratchBytes = 16 + 8 * ((kNoAllocMaxElems + kTile - 1) / kTile);
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices];  // device address of g_noalloc_scratch, per device
+}  // namespace
+
+uint64_t noalloc_max_elems() { return kNoAllocMaxElems; }
+
+// The array's device address on the current device. The first call on a device
+// looks it up with that device current; later calls reuse it. The name
+// g_noalloc_scratch in host code is only a host-side stand-in, never a device
+// address, so kernels always receive the looked-up pointer.
+cudaError_t noalloc_scratch(void** ptr, uint64_t* bytes) {
+    int dev = -1;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (err != cudaSuccess) return err;
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    *bytes = kNoAllocScratchBytes;
+    return cudaSuccess;
 }
 
 }  // namespace wc

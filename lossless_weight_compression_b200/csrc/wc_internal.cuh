@@ -130,4 +130,8 @@ inline uint64_t encode_workspace_bytes(uint64_t n) { return 16 + 8 * num_tiles(n
 cudaError_t launch_decode(const DecodeItem* items, uint32_t count, int32_t* status,
                           cudaStream_t stream);
 
+// The allocation-free encoder's fixed scratch array (wc_encode.cu).
+uint64_t noalloc_max_elems();
+cudaError_t noalloc_scratch(void** ptr, uint64_t* bytes);
+
 }  // namespace wc

@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
                                  ctypes.POINTER(u64)]
     L.wc_stream_info.restype = i
     L.wc_status_string.argtypes, L.wc_status_string.restype = [i], ctypes.c_char_p
+    L.wc_compress_noalloc.argtypes = [vp, u64, u32, vp, u64, vp, vp, vp]
+    L.wc_compress_noalloc.restype = i
     L.wc_debug_compress_stalled.argtypes = [vp, u64, u32, vp, u64, vp, vp, u64, vp, u64, vp]
     L.wc_debug_compress_stalled.restype = i
     _lib = L
@@ -95,6 +97,14 @@ def wc_compress(d_in, n, block, d_out, out_capacity, d_out_bytes, d_workspace, w
                 d_status, stream) -> int:
     return lib().wc_compress(d_in, n, block, d_out, out_capacity, d_out_bytes, d_workspace,
                              workspace_bytes, d_status, stream)
+
+
+def wc_compress_noalloc(d_in, n, block, d_out, out_capacity, d_out_bytes, d_status,
+                        stream) -> int:
+    """wc_compress without a workspace, for callers that cannot allocate device
+    memory; its scratch is a fixed array in the library (n <= 2^30)."""
+    return lib().wc_compress_noalloc(d_in, n, block, d_out, out_capacity, d_out_bytes, d_status,
+                                     stream)
 
 
 def wc_decompress(d_stream, stream_bytes, d_out, n, block, d_status, stream) -> int:
