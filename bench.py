@@ -178,8 +178,10 @@ def decode_kernel_digest() -> str:
 
 
 def ncu_traffic_per_elem():
-    """DRAM bytes per element of the decode kernel from the committed ncu summary,
-    or None if there is none or the kernel source changed since it was taken."""
+    """DRAM bytes per element of one decode launch, from the committed ncu
+    summary (dram__bytes_read.sum + dram__bytes_write.sum of one launch over
+    ``elements`` elements), or None if there is none or the decoder's source
+    changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")
     try:
         fields = dict(line.split(":", 1) for line in open(path) if ":" in line)
@@ -189,8 +191,8 @@ def ncu_traffic_per_elem():
     if fields.get("kernel_source_digest") != decode_kernel_digest():
         return None
     try:
-        return float(fields["dram_bytes_per_element"])
-    except (KeyError, ValueError):
+        return float(fields["dram_bytes_per_launch"]) / float(fields["elements"])
+    except (KeyError, ValueError, ZeroDivisionError):
         return None
 
 

@@ -8,74 +8,134 @@
 // byte 16*offs[b] + j*w_b of the exponent plane, lane t = i mod 8 at bits
 // [t*w_b, (t+1)*w_b); its mantissa byte is byte i of the mantissa plane.
 //
-// One thread block decodes one 8192-element tile of one tensor:
-//   1. 16-byte loads of the tile's mantissa bytes are issued first (their
-//      address depends on nothing in the stream);
-//   2. the tile's block headers and offsets are read and checked (w <= 8,
-//      base 0 when raw, offsets equal to the prefix sum of the block sizes,
-//      every byte inside the stream);
-//   3. the tile's exponent payload -- contiguous, starting 16-byte aligned --
-//      is staged in shared memory with 16-byte loads;
-//   4. each thread unpacks two octets per 16-element chunk by reversing the
-//      hierarchical halving (octet -> quads -> pairs -> values), adds the
-//      base, merges sign and mantissa, and writes 32 bytes of BF16 with
-//      16-byte stores.
+// The kernel is persistent and warp-specialised. Each thread block walks the
+// 8192-element tiles blockIdx.x, blockIdx.x + gridDim.x, ... of the batch
+// through a ring of kStages shared-memory stages guarded by mbarriers:
+//   producer warp   per tile: reads and checks the block headers and offsets
+//                   (w <= 8, base 0 when raw, offsets equal to the prefix sum
+//                   of the block sizes, every byte inside the stream), writes
+//                   per-block decode constants into the stage, and issues two
+//                   bulk asynchronous copies (cp.async.bulk) -- the tile's
+//                   mantissa bytes and its exponent payload, both contiguous
+//                   and 16-byte aligned -- that complete on the stage's
+//                   "full" barrier;
+//   8 consumer warps per tile: wait on "full", decode 16 elements per chunk
+//                   (2 chunks per thread) from shared memory by reversing the
+//                   hierarchical halving (octet -> quads -> pairs), add the
+//                   base, merge sign and mantissa, write 16-byte stores, and
+//                   release the stage on its "empty" barrier.
+// The decoding warps never wait on global-memory latency and never meet at a
+// block-wide barrier. Every mbarrier wait is bounded by the device timer; on
+// expiry the kernel reports WC_ERR_TIMEOUT and returns.
+//
 // A batch of tensors is one launch: the per-tensor descriptors travel as
-// launch parameters, and each thread block finds its tensor by a binary search
-// over the tensors' first tile indices.
+// launch parameters and the producer advances through them as its tiles do.
+#include <mutex>
+
 #include "wc_internal.cuh"
 
 namespace wc {
 namespace {
+
+constexpr int kConsumerWarps = kThreads / 32;  // 8
+constexpr int kProducerWarp = kConsumerWarps;
+constexpr int kDecodeThreads = kThreads + 32;  // 288
+constexpr int kStages = 4;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
 template <int MAXI>
 struct DecodeParams {
     int32_t* status;
     uint32_t count;
     uint32_t pad;
+    uint64_t total_tiles;
     uint64_t tile_begin[MAXI + 1];  // first global tile of each item; [count] = total
     DecodeItem item[MAXI];
 };
 
-// Eight w-bit values of one octet (lo/hi = its 64 bits; bits above 8w are
-// ignored) -> four words, each holding two finished BF16 values.
-//   quads: q0 = bits [0,4w), q1 = bits [4w,8w)
-//   pairs: p0 = q0 & m2, p1 = q0 >> 2w (taken from lo:hi), p2 = q1 & m2, p3 = q1 >> 2w
-//   pair -> two 16-bit lanes: (p & m1) | (p >> w & m1) << 16
-//   lane  -> BF16:  (v + base) << 7 | sign << 15 | mantissa
-struct OctetDecoder {
-    uint32_t w, m1, m1_hi, m2, m4, base7;
-    __device__ __forceinline__ OctetDecoder(uint32_t w_, uint32_t base) {
-        w = w_;
-        m1 = (1u << w) - 1u;
-        m1_hi = m1 << 16;
-        m2 = (1u << (2 * w)) - 1u;
-        m4 = (w == 8u) ? 0xFFFFFFFFu : ((1u << (4 * w)) - 1u);
-        base7 = base * 0x00800080u;  // base at bit 7 of both 16-bit lanes
-    }
-    __device__ __forceinline__ uint32_t lanes(uint32_t pair) const {
-        const uint32_t v = (pair & m1) | ((pair << (16 - w)) & m1_hi);
-        return v * 128u + base7;  // exponent field of both lanes: (v + base) << 7
-    }
-    // s4: the four sign+mantissa bytes of elements 0..3 (first) or 4..7
-    __device__ __forceinline__ uint4 decode(uint32_t lo, uint32_t hi, uint32_t s_lo4,
-                                            uint32_t s_hi4) const {
-        const uint32_t p0 = lo & m2;
-        const uint32_t p1 = __funnelshift_r(lo, hi, 2 * w) & m2;
-        const uint32_t q1 = __funnelshift_rc(lo, hi, 4 * w) & m4;
-        const uint32_t p2 = q1 & m2;
-        const uint32_t p3 = q1 >> (2 * w);
-        // sign+mantissa byte s replicated into both bytes of a lane: & 0x807F
-        // keeps the mantissa in bits 0..6 and moves the sign to bit 15.
-        uint4 r;
-        r.x = (prmt(s_lo4, 0u, 0x1100u) & 0x807F807Fu) | lanes(p0);
-        r.y = (prmt(s_lo4, 0u, 0x3322u) & 0x807F807Fu) | lanes(p1);
-        r.z = (prmt(s_hi4, 0u, 0x1100u) & 0x807F807Fu) | lanes(p2);
-        r.w = (prmt(s_hi4, 0u, 0x3322u) & 0x807F807Fu) | lanes(p3);
-        return r;
-    }
+struct __align__(16) StageInfo {
+    uint16_t* out;    // the tile's first output element
+    uint32_t tile_n;  // elements to decode (0: nothing, e.g. a corrupt tile)
+    uint32_t log2B;
 };
 
+// Per-block decode constants, computed once per block by the producer.
+//   t0 = {byte offset of the block's payload in the staged bytes, w, 2w, 4w}
+//   t1 = {M1 = m1 | m1 << 16, m2, m4, base * 0x00800080}, mk = 2^k - 1 (m4 = ~0 when 4w = 32)
+struct __align__(16) Stage {
+    uint8_t man[kTile];
+    uint8_t exp[kTile + 16];
+    uint4 t0[kMaxBlocksPerTile];
+    uint4 t1[kMaxBlocksPerTile];
+    StageInfo info;
+};
+
+struct DecodeSmem {
+    Stage stage[kStages];
+    unsigned long long full[kStages];
+    unsigned long long empty[kStages];
+    int abort;
+};
+
+// ---------------------------------------------------------------------------
+// mbarrier and bulk-copy helpers (PTX)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for the phase of `bar` with the given parity; false if the time limit
+// passed or another warp of the block gave up first.
+__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity,
+                                          volatile int* abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort || global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+// Bulk asynchronous copy global -> this block's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          unsigned long long* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// decoding of one octet
+// ---------------------------------------------------------------------------
 // 64 bits starting at byte q of the staged exponent bytes (q need not be aligned).
 __device__ __forceinline__ void fetch_octet(const uint32_t* s32, uint32_t q, uint32_t& lo,
                                             uint32_t& hi) {
@@ -85,11 +145,38 @@ __device__ __forceinline__ void fetch_octet(const uint32_t* s32, uint32_t q, uin
     hi = __funnelshift_r(x1, x2, r);
 }
 
+// A pair (2w bits, v0 | v1 << w) -> both 16-bit lanes' exponent fields (base + v) << 7.
+__device__ __forceinline__ uint32_t pair_lanes(uint32_t p, uint32_t sh, uint32_t M1,
+                                               uint32_t base7) {
+    return ((p | (p << sh)) & M1) * 128u + base7;
+}
+
+// Octet (lo:hi, bits above 8w ignored) + 8 sign+mantissa bytes -> 8 BF16 words.
+//   quads: bits [0,4w) and [4w,8w); pairs: the halves of each quad.
+// A sign+mantissa byte replicated into both bytes of a lane and masked with
+// 0x807F leaves the mantissa in bits 0..6 and the sign in bit 15.
+__device__ __forceinline__ uint4 decode_octet(uint32_t lo, uint32_t hi, uint32_t s03,
+                                              uint32_t s47, uint32_t w2, uint32_t w4,
+                                              uint32_t sh, uint4 t1) {
+    const uint32_t M1 = t1.x, m2 = t1.y, m4 = t1.z, base7 = t1.w;
+    const uint32_t p0 = lo & m2;
+    const uint32_t p1 = __funnelshift_r(lo, hi, w2) & m2;
+    const uint32_t q1 = __funnelshift_rc(lo, hi, w4) & m4;
+    const uint32_t p2 = q1 & m2;
+    const uint32_t p3 = q1 >> w2;
+    uint4 r;
+    r.x = (prmt(s03, 0u, 0x1100u) & 0x807F807Fu) | pair_lanes(p0, sh, M1, base7);
+    r.y = (prmt(s03, 0u, 0x3322u) & 0x807F807Fu) | pair_lanes(p1, sh, M1, base7);
+    r.z = (prmt(s47, 0u, 0x1100u) & 0x807F807Fu) | pair_lanes(p2, sh, M1, base7);
+    r.w = (prmt(s47, 0u, 0x3322u) & 0x807F807Fu) | pair_lanes(p3, sh, M1, base7);
+    return r;
+}
+
 __device__ __forceinline__ uint64_t ld_u64(const uint8_t* p) {
     return *reinterpret_cast<const uint64_t*>(p);
 }
 
-// Thread block 0 of each tensor checks the container header against (n, B).
+// The first tile of each tensor checks the container header against (n, B).
 __device__ void check_container(const DecodeItem& I, const Layout& L, int32_t* status) {
     const uint8_t* S = I.stream;
     bool bad = ld_u64(S) != (kMagic | (uint64_t(kVersion) << 32) | (uint64_t(kHeaderBytes) << 48));
@@ -106,135 +193,216 @@ __device__ void check_container(const DecodeItem& I, const Layout& L, int32_t* s
     if (bad) report(status, kStatusCorrupt);
 }
 
+// ---------------------------------------------------------------------------
+// producer: one warp
+// ---------------------------------------------------------------------------
 template <int MAXI>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeParams<MAXI> P) {
-    __shared__ __align__(16) uint8_t s_exp[kTile + 16];
-    __shared__ uint32_t s_hdr[kMaxBlocksPerTile];
-    __shared__ uint32_t s_off[kMaxBlocksPerTile];
-    __shared__ uint32_t s_blk[kMaxBlocksPerTile];  // base | w << 8 | staged byte offset << 16
-    __shared__ unsigned long long s_next, s_start;
-    __shared__ uint32_t s_len;
-    __shared__ int s_bad;
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const uint64_t gt = blockIdx.x;
-
-    int it = 0;
-    if (MAXI > 1) {  // the last item whose first tile is <= gt
-        int lo = 0, hi = int(P.count) - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (P.tile_begin[mid] <= gt) lo = mid; else hi = mid - 1;
+__device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem& sm, int lane) {
+    uint32_t it = 0;
+    DecodeItem I = P.item[0];
+    Layout L = make_layout(I.n, I.block);
+    for (uint64_t i = 0;; ++i) {
+        const uint64_t t = blockIdx.x + i * gridDim.x;
+        if (t >= P.total_tiles) break;
+        const int s = int(i % kStages);
+        const uint32_t round = uint32_t(i / kStages);
+        if (round > 0 && !mbar_wait(&sm.empty[s], (round & 1u) ^ 1u, &sm.abort)) {
+            if (lane == 0) {
+                report(P.status, kStatusTimeout);
+                sm.abort = 1;
+            }
+            return;
         }
-        it = lo;
-    }
-    const DecodeItem& I = P.item[it];
-    const uint64_t lt = gt - P.tile_begin[it];
-    const Layout L = make_layout(I.n, I.block);
-    const uint8_t* S = I.stream;
+        if (t >= P.tile_begin[it + 1]) {  // tiles only move forward: advance the item
+            while (t >= P.tile_begin[it + 1]) ++it;
+            I = P.item[it];
+            L = make_layout(I.n, I.block);
+        }
+        const uint64_t lt = t - P.tile_begin[it];
+        if (lt == 0 && lane == 0) check_container(I, L, P.status);
+        Stage& st = sm.stage[s];
 
-    if (lt == 0 && tid == 32) check_container(I, L, P.status);
-    if (L.n == 0) return;  // an empty tensor's tile only checks the header
-
-    const uint32_t log2B = L.log2_block, B = L.block;
-    const uint64_t tile_start = lt * kTile;
-    const uint32_t tile_n = uint32_t(min(uint64_t(kTile), L.n - tile_start));
-    const uint64_t b0 = tile_start >> log2B;
-    const uint32_t nblk = (tile_n + B - 1) >> log2B;
-
-    // 1. mantissa bytes (the mantissa section is padded to 128 bytes and the
-    //    host checked stream_bytes >= off_exp, so full 16-byte loads stay inside)
-    uint4 M[kChunksPerThread];
-#pragma unroll
-    for (int k = 0; k < kChunksPerThread; ++k) {
-        const uint32_t el = uint32_t(tid + k * kThreads) * kChunk;
-        if (el < tile_n) M[k] = ld_stream_v4(S + L.off_man + tile_start + el);
-    }
-    // 2. block headers and offsets of the tile, and where the next tile starts
-    if (tid < nblk) {
-        s_hdr[tid] = reinterpret_cast<const uint16_t*>(S + L.off_hdr)[b0 + tid];
-        s_off[tid] = reinterpret_cast<const uint32_t*>(S + L.off_offs)[b0 + tid];
-    } else if (tid == nblk) {
-        s_next = (b0 + nblk < L.nb) ? 16ull * reinterpret_cast<const uint32_t*>(S + L.off_offs)[b0 + nblk]
-                                    : ld_u64(S + 64);  // after the last block: E
-    }
-    __syncthreads();
-    if (warp == 0) {
+        uint32_t tile_n = 0, len16 = 0, man_bytes = 0;
+        uint64_t start = 0;
         bool bad = false;
-        unsigned long long start_j[2];
-        uint32_t blk[2];
+        if (L.n > 0) {
+            const uint32_t log2B = L.log2_block, B = L.block;
+            const uint64_t tile_start = lt * kTile;
+            tile_n = uint32_t(min(uint64_t(kTile), L.n - tile_start));
+            const uint64_t b0 = tile_start >> log2B;
+            const uint32_t nblk = (tile_n + B - 1) >> log2B;
+            const uint8_t* S = I.stream;
+            const uint16_t* hdr = reinterpret_cast<const uint16_t*>(S + L.off_hdr) + b0;
+            const uint32_t* offs = reinterpret_cast<const uint32_t*>(S + L.off_offs) + b0;
+            // lanes own blocks lane and lane + 32 (a tile holds at most 64 blocks)
+            uint32_t h[2] = {0, 0};
+            uint64_t sb[2] = {0, 0}, nx[2] = {0, 0};
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const uint32_t i = 2 * lane + j;
-            start_j[j] = 0;
-            blk[j] = 0;
-            if (i < nblk) {
-                const uint32_t h = s_hdr[i], w = h >> 8, base = h & 0xFFu;
-                bad |= w > 8u || (w == 8u && base != 0u);
-                const uint32_t len = min(B, tile_n - i * B);
-                const uint64_t size = uint64_t((len + 7) >> 3) * min(w, 8u);
-                start_j[j] = 16ull * s_off[i];
-                const uint64_t next = (i + 1 < nblk) ? 16ull * s_off[i + 1] : s_next;
-                bad |= start_j[j] + size != next;
-                blk[j] = h;
+            for (int j = 0; j < 2; ++j) {
+                const uint32_t b = lane + 32 * j;
+                if (b < nblk) {
+                    h[j] = hdr[b];
+                    sb[j] = 16ull * offs[b];
+                    nx[j] = (b + 1 < nblk || b0 + b + 1 < L.nb) ? 16ull * offs[b + 1]
+                                                                : ld_u64(S + 64);  // E
+                }
+            }
+            start = __shfl_sync(0xFFFFFFFFu, sb[0], 0);
+            const uint32_t last = nblk - 1;
+            const uint64_t end = __shfl_sync(0xFFFFFFFFu, last < 32 ? nx[0] : nx[1], last & 31);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const uint32_t b = lane + 32 * j;
+                if (b < nblk) {
+                    const uint32_t w = h[j] >> 8, base = h[j] & 0xFFu;
+                    const uint32_t len = min(B, tile_n - b * B);
+                    bad |= w > 8u || (w == 8u && base != 0u);
+                    bad |= sb[j] + uint64_t((len + 7) >> 3) * min(w, 8u) != nx[j];
+                }
+            }
+            bad |= end > I.stream_bytes - L.off_exp;
+            bad = __any_sync(0xFFFFFFFFu, bad);
+            if (!bad) {
+                // the offset chain holds, so end - start = the tile's payload <= kTile
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const uint32_t b = lane + 32 * j;
+                    if (b < nblk) {
+                        const uint32_t w = h[j] >> 8, base = h[j] & 0xFFu;
+                        const uint32_t m1 = (1u << w) - 1u;
+                        st.t0[b] = make_uint4(uint32_t(sb[j] - start), w, 2 * w, 4 * w);
+                        st.t1[b] = make_uint4(m1 | (m1 << 16), (1u << (2 * w)) - 1u,
+                                              w == 8u ? 0xFFFFFFFFu : (1u << (4 * w)) - 1u,
+                                              base * 0x00800080u);
+                    }
+                }
+                const uint32_t len = uint32_t(end - start);
+                len16 = len & ~15u;
+                const uint32_t rem = len - len16;  // only at the very end of a stream
+                if (lane < rem) st.exp[len16 + lane] = S[L.off_exp + start + len16 + lane];
+                man_bytes = (tile_n + 15u) & ~15u;  // inside the 128-byte padded plane
+                if (lane == 0)
+                    st.info = StageInfo{I.out + tile_start, tile_n, L.log2_block};
+            } else {
+                if (lane == 0) report(P.status, kStatusCorrupt);
             }
         }
-        const unsigned long long start = 16ull * s_off[0], end = s_next;
-        bad |= end > I.stream_bytes - L.off_exp;
-        bad = __any_sync(0xFFFFFFFFu, bad);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const uint32_t i = 2 * lane + j;
-            if (i < nblk && !bad) s_blk[i] = blk[j] | (uint32_t(start_j[j] - start) << 16);
+        if (L.n == 0 || bad) {
+            if (lane == 0) st.info = StageInfo{nullptr, 0u, 0u};
+            tile_n = 0;
         }
+        __syncwarp();
         if (lane == 0) {
-            s_start = start;
-            s_len = bad ? 0u : uint32_t(end - start);  // the offset chain bounds it by kTile
-            s_bad = bad;
+            if (tile_n == 0) {
+                mbar_arrive(&sm.full[s]);
+            } else {
+                mbar_arrive_expect_tx(&sm.full[s], man_bytes + len16);
+                const uint8_t* S = I.stream;
+                bulk_load(st.man, S + L.off_man + lt * kTile, man_bytes, &sm.full[s]);
+                if (len16) bulk_load(st.exp, S + L.off_exp + start, len16, &sm.full[s]);
+            }
         }
     }
-    __syncthreads();
-    if (s_bad) {
-        if (tid == 0) report(P.status, kStatusCorrupt);
-        return;
-    }
+}
 
-    // 3. stage the tile's exponent payload
-    {
-        const uint8_t* src = S + L.off_exp + s_start;
-        const uint32_t len = s_len;
-        for (uint32_t i = tid; i < len / 16; i += kThreads)
-            *reinterpret_cast<uint4*>(s_exp + 16 * i) = ld_stream_v4(src + 16 * i);
-        const uint32_t rem = len & 15u;
-        if (tid < rem) s_exp[len - rem + tid] = src[len - rem + tid];
-    }
-    __syncthreads();
-
-    // 4. decode 16 elements per chunk
-    const uint32_t* s32 = reinterpret_cast<const uint32_t*>(s_exp);
+// ---------------------------------------------------------------------------
+// consumers: eight warps
+// ---------------------------------------------------------------------------
+template <int MAXI>
+__device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem& sm, int tid, int lane) {
+    for (uint64_t i = 0;; ++i) {
+        const uint64_t t = blockIdx.x + i * gridDim.x;
+        if (t >= P.total_tiles) break;
+        const int s = int(i % kStages);
+        const uint32_t round = uint32_t(i / kStages);
+        if (!mbar_wait(&sm.full[s], round & 1u, &sm.abort)) {
+            if (lane == 0) {
+                report(P.status, kStatusTimeout);
+                sm.abort = 1;
+            }
+            return;
+        }
+        const Stage& st = sm.stage[s];
+        const StageInfo info = st.info;
+        const uint32_t* s32 = reinterpret_cast<const uint32_t*>(st.exp);
+        const uint32_t bmask = (1u << info.log2B) - 1u;
 #pragma unroll
-    for (int k = 0; k < kChunksPerThread; ++k) {
-        const uint32_t el = uint32_t(tid + k * kThreads) * kChunk;
-        if (el >= tile_n) continue;
-        const uint32_t blk = s_blk[el >> log2B];
-        const uint32_t w = (blk >> 8) & 0xFFu;
-        const OctetDecoder dec(w, blk & 0xFFu);
-        const uint32_t q = (blk >> 16) + ((el & (B - 1)) >> 3) * w;
-        uint32_t lo0, hi0, lo1, hi1;
-        fetch_octet(s32, q, lo0, hi0);
-        fetch_octet(s32, q + w, lo1, hi1);
-        const uint4 r0 = dec.decode(lo0, hi0, M[k].x, M[k].y);
-        const uint4 r1 = dec.decode(lo1, hi1, M[k].z, M[k].w);
-        uint16_t* dst = I.out + tile_start + el;
-        if (tile_n - el >= kChunk) {
-            st_stream_v4(dst, r0);
-            st_stream_v4(dst + 8, r1);
-        } else {
-            const uint32_t words[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-            const uint32_t nv = tile_n - el;
-            for (uint32_t i = 0; i < nv; ++i) dst[i] = uint16_t(words[i >> 1] >> (16 * (i & 1)));
+        for (int k = 0; k < kChunksPerThread; ++k) {
+            const uint32_t el = uint32_t(tid + k * kThreads) * kChunk;
+            if (el >= info.tile_n) continue;
+            const uint4 M = *reinterpret_cast<const uint4*>(st.man + el);
+            const uint32_t bl = el >> info.log2B;
+            const uint4 t0 = st.t0[bl], t1 = st.t1[bl];
+            const uint32_t w = t0.y, sh = 16u - w;
+            const uint32_t q = t0.x + ((el & bmask) >> 3) * w;
+            uint32_t lo0, hi0, lo1, hi1;
+            fetch_octet(s32, q, lo0, hi0);
+            fetch_octet(s32, q + w, lo1, hi1);
+            const uint4 r0 = decode_octet(lo0, hi0, M.x, M.y, t0.z, t0.w, sh, t1);
+            const uint4 r1 = decode_octet(lo1, hi1, M.z, M.w, t0.z, t0.w, sh, t1);
+            uint16_t* dst = info.out + el;
+            if (info.tile_n - el >= kChunk) {
+                st_stream_v4(dst, r0);
+                st_stream_v4(dst + 8, r1);
+            } else {
+                const uint32_t words[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+                const uint32_t nv = info.tile_n - el;
+                for (uint32_t e = 0; e < nv; ++e)
+                    dst[e] = uint16_t(words[e >> 1] >> (16 * (e & 1)));
+            }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[s]);
     }
+}
+
+template <int MAXI>
+__global__ void __launch_bounds__(kDecodeThreads)
+    decode_kernel(const __grid_constant__ DecodeParams<MAXI> P) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1);                // the producer's arrive (+ copied bytes)
+            mbar_init(&sm.empty[s], kConsumerWarps);  // one arrive per consumer warp
+        }
+        sm.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (warp == kProducerWarp)
+        produce<MAXI>(P, sm, lane);
+    else
+        consume<MAXI>(P, sm, tid, lane);
+}
+
+// Persistent grid: as many resident thread blocks as the SMs hold, never more
+// than there are tiles. Computed once per device and kernel instantiation.
+template <int MAXI>
+cudaError_t grid_for(uint64_t tiles, unsigned* grid) {
+    static std::mutex mu;
+    static int per_device[64];  // 0 = not yet known
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (per_device[dev] == 0) {
+        err = cudaFuncSetAttribute(decode_kernel<MAXI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   int(sizeof(DecodeSmem)));
+        if (err != cudaSuccess) return err;
+        int sms = 0, per_sm = 0;
+        err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (err != cudaSuccess) return err;
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<MAXI>,
+                                                            kDecodeThreads, sizeof(DecodeSmem));
+        if (err != cudaSuccess) return err;
+        per_device[dev] = (per_sm > 0 ? per_sm : 1) * sms;
+    }
+    const uint64_t cap = uint64_t(per_device[dev]);
+    *grid = unsigned(tiles < cap ? tiles : cap);
+    return cudaSuccess;
 }
 
 template <int MAXI>
@@ -253,8 +421,12 @@ cudaError_t launch_batch(const DecodeItem* items, uint32_t count, int32_t* statu
         tiles += nt ? nt : 1;  // an empty tensor still gets one tile to check its header
     }
     p.tile_begin[count] = tiles;
+    p.total_tiles = tiles;
     if (tiles == 0) return cudaSuccess;
-    decode_kernel<MAXI><<<unsigned(tiles), kThreads, 0, stream>>>(p);
+    unsigned grid = 0;
+    cudaError_t err = grid_for<MAXI>(tiles, &grid);
+    if (err != cudaSuccess) return err;
+    decode_kernel<MAXI><<<grid, kDecodeThreads, sizeof(DecodeSmem), stream>>>(p);
     return cudaGetLastError();
 }
 
