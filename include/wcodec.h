@@ -73,9 +73,10 @@ typedef enum {
 uint64_t wc_bound(uint64_t n, uint32_t block);
 
 /*
- * Bytes of device workspace wc_compress needs for (n, block): the look-back
- * state of each 8192-element tile of the single-pass encoder plus a ticket
- * counter. Returns 0 if `block` or `n` is invalid. Host-only.
+ * Bytes of device workspace wc_compress needs for (n, block): 16 bytes of
+ * control words (a tile ticket, an error flag) plus the 8-byte look-back
+ * state of each 8192-element tile of the single-pass encoder (one tile for
+ * n = 0). Returns 0 if `block` or `n` is invalid. Host-only.
  */
 uint64_t wc_workspace_size(uint64_t n, uint32_t block);
 
@@ -102,6 +103,45 @@ int wc_compress(const void *d_in, uint64_t n, uint32_t block,
                 void *d_out, uint64_t out_capacity, uint64_t *d_out_bytes,
                 void *d_workspace, uint64_t workspace_bytes,
                 int32_t *d_status, void *stream);
+
+/*
+ * One tensor of a batched compression.
+ *   in, n, block: the BF16 words (device, 16-byte aligned) and the block size
+ *   out, out_capacity: the stream buffer (device, 16-byte aligned),
+ *                      out_capacity >= wc_bound(n, block)
+ *   out_bytes: device u64 receiving the stream's size (0 on error), 8-byte aligned
+ */
+typedef struct {
+    const void *in;
+    uint64_t n;
+    uint32_t block;
+    uint32_t reserved; /* must be 0 */
+    void *out;
+    uint64_t out_capacity;
+    uint64_t *out_bytes;
+} wc_compress_item;
+
+/*
+ * Workspace bytes wc_compress_batch needs for these tensors (the look-back
+ * state of every tile of every tensor, in parts of up to WC_BATCH_MAX
+ * tensors). Returns 0 if an item has an invalid n or block. Host-only.
+ */
+uint64_t wc_compress_batch_workspace_size(const wc_compress_item *h_items, uint32_t count);
+
+/*
+ * Compress `count` independent tensors, each into its own WCB1 stream (every
+ * stream is the one wc_compress writes for that tensor), in one launch per
+ * WC_BATCH_MAX tensors. h_items is a HOST array passed to the kernel as launch
+ * parameters; d_workspace (device, 16-byte aligned) holds at least
+ * wc_compress_batch_workspace_size bytes and is cleared by the call on
+ * `stream`. Steps as wc_compress (ENEC Abstract); tiles of all tensors share
+ * one persistent grid, which removes per-tensor launch gaps for stacks of
+ * many small weight tensors. Every item is checked before anything is
+ * launched; errors as wc_compress.
+ */
+int wc_compress_batch(const wc_compress_item *h_items, uint32_t count,
+                      void *d_workspace, uint64_t workspace_bytes,
+                      int32_t *d_status, void *stream);
 
 /*
  * Allocation-free variant of wc_compress. The pages have no counterpart: this

@@ -25,9 +25,33 @@ int check_compress_args(const void* d_in, uint64_t n, uint32_t block, void* d_ou
         (reinterpret_cast<uintptr_t>(d_out_bytes) & 7u) != 0)
         return WC_ERR_INVALID_ARG;
     if (out_capacity < wc::bound_bytes(n, block) ||
-        workspace_bytes < wc::encode_workspace_bytes(n))
+        workspace_bytes < wc::encode_workspace_bytes(wc::encode_tiles(n)))
         return WC_ERR_BUFFER_TOO_SMALL;
     return WC_OK;
+}
+
+wc::EncodeItem to_encode_item(const void* d_in, uint64_t n, uint32_t block, void* d_out,
+                              uint64_t* d_out_bytes) {
+    wc::EncodeItem e;
+    e.in = static_cast<const uint16_t*>(d_in);
+    e.out = static_cast<uint8_t*>(d_out);
+    e.out_bytes = d_out_bytes;
+    e.n = n;
+    e.block = block;
+    e.reserved = 0;
+    return e;
+}
+
+// Workspace of a batch: one part per launch of up to WC_BATCH_MAX tensors.
+uint64_t batch_workspace_bytes(const wc_compress_item* items, uint32_t count) {
+    uint64_t total = 0;
+    for (uint32_t base = 0; base < count; base += WC_BATCH_MAX) {
+        const uint32_t c = (count - base < WC_BATCH_MAX) ? count - base : WC_BATCH_MAX;
+        uint64_t tiles = 0;
+        for (uint32_t i = 0; i < c; ++i) tiles += wc::encode_tiles(items[base + i].n);
+        total += (wc::encode_workspace_bytes(tiles) + 15) & ~uint64_t(15);
+    }
+    return total;
 }
 
 int check_decode_item(const wc_batch_item& it) {
@@ -66,7 +90,7 @@ uint64_t wc_bound(uint64_t n, uint32_t block) {
 }
 
 uint64_t wc_workspace_size(uint64_t n, uint32_t block) {
-    return args_ok(n, block) ? wc::encode_workspace_bytes(n) : 0;
+    return args_ok(n, block) ? wc::encode_workspace_bytes(wc::encode_tiles(n)) : 0;
 }
 
 static int compress_impl(const void* d_in, uint64_t n, uint32_t block, void* d_out,
@@ -76,10 +100,9 @@ static int compress_impl(const void* d_in, uint64_t n, uint32_t block, void* d_o
     const int rc = check_compress_args(d_in, n, block, d_out, out_capacity, d_out_bytes,
                                        d_workspace, workspace_bytes);
     if (rc != WC_OK) return rc;
-    const wc::Layout L = wc::make_layout(n, block);
-    const cudaError_t err = wc::launch_encode(
-        static_cast<const uint16_t*>(d_in), L, static_cast<uint8_t*>(d_out), d_out_bytes,
-        d_workspace, d_status, timeout_ns, first_ticket, static_cast<cudaStream_t>(stream));
+    const wc::EncodeItem item = to_encode_item(d_in, n, block, d_out, d_out_bytes);
+    const cudaError_t err = wc::launch_encode(&item, 1, d_workspace, d_status, timeout_ns,
+                                              first_ticket, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
@@ -115,12 +138,47 @@ int wc_compress_noalloc(const void* d_in, uint64_t n, uint32_t block, void* d_ou
     void* scratch = nullptr;
     uint64_t scratch_bytes = 0;
     if (wc::noalloc_scratch(&scratch, &scratch_bytes) != cudaSuccess) return WC_ERR_CUDA;
-    if (scratch_bytes < wc::encode_workspace_bytes(n)) return WC_ERR_BUFFER_TOO_SMALL;
-    const wc::Layout L = wc::make_layout(n, block);
-    const cudaError_t err = wc::launch_encode(
-        static_cast<const uint16_t*>(d_in), L, static_cast<uint8_t*>(d_out), d_out_bytes, scratch,
-        d_status, kDefaultTimeoutNs, 0, static_cast<cudaStream_t>(stream));
+    if (scratch_bytes < wc::encode_workspace_bytes(wc::encode_tiles(n)))
+        return WC_ERR_BUFFER_TOO_SMALL;
+    const wc::EncodeItem item = to_encode_item(d_in, n, block, d_out, d_out_bytes);
+    const cudaError_t err = wc::launch_encode(&item, 1, scratch, d_status, kDefaultTimeoutNs, 0,
+                                              static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
+uint64_t wc_compress_batch_workspace_size(const wc_compress_item* h_items, uint32_t count) {
+    if (h_items == nullptr && count > 0) return 0;
+    for (uint32_t i = 0; i < count; ++i)
+        if (!args_ok(h_items[i].n, h_items[i].block)) return 0;
+    return batch_workspace_bytes(h_items, count);
+}
+
+int wc_compress_batch(const wc_compress_item* h_items, uint32_t count, void* d_workspace,
+                      uint64_t workspace_bytes, int32_t* d_status, void* stream) {
+    if (h_items == nullptr && count > 0) return WC_ERR_INVALID_ARG;
+    if (count == 0) return WC_OK;
+    for (uint32_t i = 0; i < count; ++i) {  // check everything before launching anything
+        const wc_compress_item& it = h_items[i];
+        if (it.reserved != 0) return WC_ERR_INVALID_ARG;
+        const int rc = check_compress_args(it.in, it.n, it.block, it.out, it.out_capacity,
+                                           it.out_bytes, d_workspace, UINT64_MAX);
+        if (rc != WC_OK) return rc;
+    }
+    if (workspace_bytes < batch_workspace_bytes(h_items, count)) return WC_ERR_BUFFER_TOO_SMALL;
+    wc::EncodeItem chunk[WC_BATCH_MAX];
+    uint8_t* ws = static_cast<uint8_t*>(d_workspace);
+    for (uint32_t base = 0; base < count; base += WC_BATCH_MAX) {
+        const uint32_t c = (count - base < WC_BATCH_MAX) ? count - base : WC_BATCH_MAX;
+        for (uint32_t i = 0; i < c; ++i) {
+            const wc_compress_item& it = h_items[base + i];
+            chunk[i] = to_encode_item(it.in, it.n, it.block, it.out, it.out_bytes);
+        }
+        const cudaError_t err = wc::launch_encode(chunk, c, ws, d_status, kDefaultTimeoutNs, 0,
+                                                  static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return WC_ERR_CUDA;
+        ws += batch_workspace_bytes(h_items + base, c);
+    }
+    return WC_OK;
 }
 
 int wc_decompress(const void* d_stream, uint64_t stream_bytes, void* d_out, uint64_t n,

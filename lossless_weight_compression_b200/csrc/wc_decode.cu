@@ -41,7 +41,6 @@ constexpr int kConsumerWarps = kThreads / 32;  // 8
 constexpr int kProducerWarp = kConsumerWarps;
 constexpr int kDecodeThreads = kThreads + 32;  // 288
 constexpr int kStages = 4;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
 template <int MAXI>
 struct DecodeParams {
@@ -76,62 +75,6 @@ struct DecodeSmem {
     unsigned long long empty[kStages];
     int abort;
 };
-
-// ---------------------------------------------------------------------------
-// mbarrier and bulk-copy helpers (PTX)
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(unsigned long long* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
-                 : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return done != 0;
-}
-
-// Wait for the phase of `bar` with the given parity; false if the time limit
-// passed or another warp of the block gave up first.
-__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity,
-                                          volatile int* abort) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (*abort || global_timer_ns() - t0 > kWaitLimitNs) return false;
-    }
-    return true;
-}
-
-// Bulk asynchronous copy global -> this block's shared memory, completing on `bar`.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          unsigned long long* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_addr(dst)),
-        "l"(src), "r"(bytes), "r"(smem_addr(bar))
-        : "memory");
-}
 
 // ---------------------------------------------------------------------------
 // decoding of one octet
@@ -201,15 +144,21 @@ __device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem& sm, int lane) {
     uint32_t it = 0;
     DecodeItem I = P.item[0];
     Layout L = make_layout(I.n, I.block);
+    int issued_round[kStages];  // last round whose bulk copies were issued, per stage
+    for (int s = 0; s < kStages; ++s) issued_round[s] = -1;
     for (uint64_t i = 0;; ++i) {
         const uint64_t t = blockIdx.x + i * gridDim.x;
         if (t >= P.total_tiles) break;
         const int s = int(i % kStages);
         const uint32_t round = uint32_t(i / kStages);
-        if (round > 0 && !mbar_wait(&sm.empty[s], (round & 1u) ^ 1u, &sm.abort)) {
+        if (round > 0 && !mbar_wait(&sm.empty[s], (round & 1u) ^ 1u, &sm.abort, 256)) {
             if (lane == 0) {
                 report(P.status, kStatusTimeout);
                 sm.abort = 1;
+                // wait (bounded) for this warp's copies still in flight into shared memory
+                for (int k = 0; k < kStages; ++k)
+                    if (issued_round[k] >= 0)
+                        mbar_wait(&sm.full[k], uint32_t(issued_round[k]) & 1u, nullptr);
             }
             return;
         }
@@ -300,6 +249,7 @@ __device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem& sm, int lane) {
                 const uint8_t* S = I.stream;
                 bulk_load(st.man, S + L.off_man + lt * kTile, man_bytes, &sm.full[s]);
                 if (len16) bulk_load(st.exp, S + L.off_exp + start, len16, &sm.full[s]);
+                issued_round[s] = int(round);
             }
         }
     }

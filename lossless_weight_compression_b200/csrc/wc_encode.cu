@@ -1,23 +1,41 @@
 // wc_encode.cu -- single-pass WCB1 encoder for sm_100a.
 //
-// One thread block encodes one 8192-element tile (whole blocks of B elements)
-// and runs every step of the encoding of "ENEC: A Lossless AI Model
-// Compression Method Enabling Fast Inference on Ascend NPUs", Abstract:
+// Every step of the encoding of "ENEC: A Lossless AI Model Compression Method
+// Enabling Fast Inference on Ascend NPUs", Abstract, runs in one pass over
+// 8192-element tiles (whole blocks of B elements):
 //   split      each BF16 word -> exponent byte e, sign+mantissa byte s
-//              (s goes straight to the mantissa plane with 16-byte stores)
 //   width      per block lo = min e, hi = max e, w = bits(hi - lo); raw
 //              fallback (base 0) when w == 8, else base = lo
-//   scan       exclusive prefix sum of the block sizes ceil(L/8)*w: inside
-//              the tile by a warp scan, across tiles by a decoupled look-back
+//   scan       exclusive prefix sum of the block sizes ceil(L/8)*w: inside a
+//              tile by a warp scan, across tiles by a decoupled look-back
 //              (Merrill & Garland, "Single-pass Parallel Prefix Scan with
 //              Decoupled Look-back", 2016) over per-tile state words
 //   remap+pack v = e - base, packed by hierarchical halving (pairs, quads,
-//              octets) into w bytes per octet, staged in shared memory and
-//              written with 16-byte stores
-// The input is read once. Tiles take their index from an atomic ticket, so a
-// tile only ever waits on tiles that started before it; every wait is bounded
-// by a device-timer limit after which the tile reports WC_ERR_TIMEOUT and
-// marks its state word so that later tiles stop waiting too.
+//              octets) into w bytes per octet
+// The input is read once.
+//
+// The kernel is persistent and warp-specialised; each thread block runs
+//   a producer warp   takes the next tile from an atomic ticket (so a tile
+//                     only ever waits on tiles that started before it), finds
+//                     its tensor, and bulk-copies (cp.async.bulk) the tile's
+//                     16 KB of input into one of two input stages;
+//   8 worker warps    split (the mantissa bytes go straight to global memory
+//                     with coalesced 16-byte stores: their position needs no
+//                     prefix), reduce per-block min/max, compute widths and
+//                     the tile-local scan, publish the tile's byte count at
+//                     once, and pack the exponent payload into one of six
+//                     output stages -- none of this waits on other tiles;
+//   4 store warps     take alternate tiles; each runs the look-back over a
+//                     256-tile window per round trip (wide enough to keep up
+//                     with the rate at which tiles start), publishes the
+//                     inclusive prefix, writes the block headers and offsets,
+//                     bulk-stores the exponent payload at its offset and, for
+//                     a tensor's last tile, the container header and padding.
+//                     Several store warps keep look-back latency off the
+//                     workers' critical path.
+// Stages are handed over with mbarriers; every wait is bounded by the device
+// timer, and a tile whose look-back gives up marks its state word so that
+// later tiles stop waiting too (WC_ERR_TIMEOUT).
 #include <mutex>
 
 #include "wc_internal.cuh"
@@ -25,22 +43,62 @@
 namespace wc {
 namespace {
 
+constexpr int kWorkerWarps = kThreads / 32;  // 8
+constexpr int kProducerWarp = kWorkerWarps;
+constexpr int kStoreWarps = 4;                // tile i goes to store warp i % 4
+constexpr int kFirstStoreWarp = kWorkerWarps + 1;
+constexpr int kEncodeThreads = kThreads + 32 + 32 * kStoreWarps;  // 416
+constexpr int kInStages = 4;
+constexpr int kOutStages = 5;
+constexpr int kWindowRows = 8;  // look-back window: 8 x 32 tiles per round trip
+
 constexpr unsigned long long kFlagAggregate = 1ull << 62;  // value = this tile's bytes
 constexpr unsigned long long kFlagPrefix = 2ull << 62;     // value = bytes up to and incl. this tile
 constexpr unsigned long long kFlagError = 3ull << 62;      // the tile gave up
 constexpr unsigned long long kValueMask = (1ull << 62) - 1;
 
-struct EncodeArgs {
-    const uint16_t* in;
-    uint8_t* out;
-    uint64_t* out_bytes;
+template <int MAXI>
+struct EncodeParams {
     int32_t* status;
-    uint32_t* control;          // [0] ticket counter, [1] internal error flag
-    unsigned long long* state;  // one look-back word per tile
-    Layout L;
-    uint64_t ntiles;
+    uint32_t* control;          // [0] ticket counter, [1] error flag
+    unsigned long long* state;  // one look-back word per tile of the batch
     uint64_t timeout_ns;
+    uint64_t total_tiles;
+    uint32_t count;
     uint32_t first_ticket;
+    uint64_t tile_begin[MAXI + 1];  // first tile of each tensor; [count] = total
+    EncodeItem item[MAXI];
+};
+
+struct __align__(16) InInfo {
+    uint64_t t, lt;  // batch tile index, tile index within its tensor
+    uint32_t item, tile_n, end, pad;
+};
+
+struct __align__(16) InStage {
+    uint16_t words[kTile];
+    InInfo info;
+};
+
+struct __align__(16) OutInfo {
+    uint64_t t, lt;
+    uint32_t item, tile_n, nblk, total, end, pad[3];
+};
+
+struct __align__(16) OutStage {
+    uint8_t exp[kTile + 16];
+    uint32_t blk[kMaxBlocksPerTile];  // base | w << 8 | tile-local payload offset << 16
+    OutInfo info;
+};
+
+struct EncodeSmem {
+    InStage in[kInStages];
+    OutStage out[kOutStages];
+    unsigned long long in_full[kInStages], in_empty[kInStages];
+    unsigned long long out_full[kOutStages], out_empty[kOutStages];
+    int lo[2][kMaxBlocksPerTile], hi[2][kMaxBlocksPerTile];  // per-block min/max, by tile parity
+    int abort;        // some warp gave up: every wait of the block stops
+    int worker_stop;  // written by workers only, before their agreement barrier
 };
 
 __device__ __forceinline__ unsigned long long load_state(const unsigned long long* p) {
@@ -59,177 +117,321 @@ __device__ __forceinline__ uint32_t load_flag(const uint32_t* p) {
     return v;
 }
 
-// Two BF16 words in one u32 -> exponent bytes at bits 0-7 / 16-23 and
-// sign+mantissa bytes at bits 0-7 / 16-23 (sign to bit 7, mantissa bits 6..0).
-__device__ __forceinline__ void split_pair(uint32_t x, uint32_t& e2, uint32_t& s2) {
-    e2 = (x >> 7) & 0x00FF00FFu;
-    s2 = ((x >> 8) & 0x00800080u) | (x & 0x007F007Fu);
+__device__ __forceinline__ uint32_t log2_of(uint32_t B) { return uint32_t(__ffs(int(B))) - 1u; }
+
+// Four BF16 words (two u32) -> their four sign+mantissa bytes and their four
+// exponent bytes, in element order. lo/hi gather the words' low and high
+// bytes; s = hi's bit 7 (the sign) over lo's bits 6..0 (the mantissa);
+// e = hi's bits 6..0 above lo's bit 7 (the exponent, bits 14..7 of the word).
+__device__ __forceinline__ void split_quad(uint32_t x01, uint32_t x23, uint32_t& s4,
+                                           uint32_t& e4) {
+    const uint32_t lo = prmt(x01, x23, 0x6420u), hi = prmt(x01, x23, 0x7531u);
+    s4 = (hi & 0x80808080u) | (lo & 0x7F7F7F7Fu);
+    e4 = ((hi << 1) & 0xFEFEFEFEu) | ((lo >> 7) & 0x01010101u);
 }
 
-__device__ __forceinline__ uint32_t min_byte(uint32_t a) {
-    a = __vminu4(a, a >> 16);
-    a = __vminu4(a, a >> 8);
-    return a & 0xFFu;
+// Per 16-bit lane minimum / maximum (native on sm_90 and later).
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
-__device__ __forceinline__ uint32_t max_byte(uint32_t a) {
-    a = __vmaxu4(a, a >> 16);
-    a = __vmaxu4(a, a >> 8);
-    return a & 0xFFu;
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
-// Hierarchical halving: four w-bit values (bytes of v) -> pairs -> one quad of 4w bits.
-__device__ __forceinline__ uint32_t pack_quad(uint32_t v, uint32_t w) {
-    uint32_t pairs = (v & 0x00FF00FFu) | (((v >> 8) & 0x00FF00FFu) << w);
-    return (pairs & 0xFFFFu) | ((pairs >> 16) << (2 * w));
+// Hierarchical halving with a compile-time width W: four W-bit values (the
+// bytes of v) -> two pairs of 2W bits -> one quad of 4W bits.
+template <uint32_t W>
+__device__ __forceinline__ uint32_t pack_quad(uint32_t v) {
+    const uint32_t pairs = (v & 0x00FF00FFu) | (((v >> 8) & 0x00FF00FFu) << W);
+    return (pairs & 0xFFFFu) | ((pairs >> 16) << (2 * W));
 }
 
-// ... and two quads -> the octet, element t at bits [t*w, t*w + w).
-__device__ __forceinline__ uint64_t pack_octet(uint32_t v_lo, uint32_t v_hi, uint32_t w) {
-    return uint64_t(pack_quad(v_lo, w)) | (uint64_t(pack_quad(v_hi, w)) << (4 * w));
-}
-
-__device__ void write_container(uint8_t* out, const Layout& L, uint64_t E, int tid) {
-    if (tid < 16) {
-        uint64_t v = 0;
-        switch (tid) {
-            case 0: v = kMagic | (uint64_t(kVersion) << 32) | (uint64_t(kHeaderBytes) << 48); break;
-            case 1: v = L.block; break;  // flags (bytes 12..15) = 0
-            case 2: v = L.n; break;
-            case 3: v = L.nb; break;
-            case 4: v = L.off_hdr; break;
-            case 5: v = L.off_offs; break;
-            case 6: v = L.off_man; break;
-            case 7: v = L.off_exp; break;
-            case 8: v = E; break;
-            case 9: v = L.off_exp + E; break;
-            default: v = 0; break;
-        }
-        reinterpret_cast<uint64_t*>(out)[tid] = v;
-    }
-}
-
-// Zero the padding that follows the header, offset and mantissa sections.
-__device__ void write_padding(uint8_t* out, const Layout& L, int tid) {
-    const uint64_t a0 = L.off_hdr + 2 * L.nb, a1 = L.off_offs + 4 * L.nb, a2 = L.off_man + L.n;
-    for (uint64_t i = a0 + tid; i < L.off_offs; i += kThreads) out[i] = 0;
-    for (uint64_t i = a1 + tid; i < L.off_man; i += kThreads) out[i] = 0;
-    for (uint64_t i = a2 + tid; i < L.off_exp; i += kThreads) out[i] = 0;
-}
-
-__global__ void __launch_bounds__(kThreads) encode_kernel(const EncodeArgs a) {
-    __shared__ __align__(16) uint8_t s_stage[kTile + 16];
-    __shared__ int s_lo[kMaxBlocksPerTile], s_hi[kMaxBlocksPerTile];
-    __shared__ uint32_t s_blk[kMaxBlocksPerTile];  // base | w << 8 | tile-local byte offset << 16
-    __shared__ unsigned long long s_tile, s_prefix;
-    __shared__ uint32_t s_total;
-    __shared__ int s_abort;
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const Layout L = a.L;
-
-    if (L.n == 0) {  // empty tensor: the header alone
-        if (blockIdx.x == 0) {
-            write_container(a.out, L, 0, tid);
-            if (tid == 0) *a.out_bytes = kHeaderBytes;
-        }
+// A 16-element chunk at width W: four quads -> two octets -> the chunk's 2W
+// bytes (element t at bits [t*W, t*W + W)), stored little-endian at dst. dst
+// is a multiple of 2W bytes past a 16-byte boundary, so the widest aligned
+// store follows from W: one 16-byte store at W = 8, 8 bytes at W = 4, 4 at
+// W = 2, three 4-byte stores at W = 6, 2-byte stores for odd W.
+template <uint32_t W>
+__device__ __forceinline__ void pack_chunk(const uint32_t V[4], uint8_t* dst) {
+    if constexpr (W == 0) {
         return;
-    }
-
-    if (tid == 0) {
-        s_tile = uint64_t(atomicAdd(&a.control[0], 1u)) + a.first_ticket;
-        s_abort = load_flag(&a.control[1]) != 0;
-    }
-    if (tid < kMaxBlocksPerTile) {
-        s_lo[tid] = 255;
-        s_hi[tid] = 0;
-    }
-    __syncthreads();
-    const uint64_t t = s_tile;
-    if (t >= a.ntiles) return;
-    if (s_abort) {  // an earlier tile failed: mark this one so that nobody waits on it
-        if (tid == 0) {
-            store_state(&a.state[t], kFlagError);
-            if (t == a.ntiles - 1) *a.out_bytes = 0;
-        }
-        return;
-    }
-
-    const uint32_t log2B = L.log2_block, B = L.block;
-    const uint64_t tile_start = t * kTile;
-    const uint32_t tile_n = uint32_t(min(uint64_t(kTile), L.n - tile_start));
-    const uint32_t nblk = (tile_n + B - 1) >> log2B;
-    const uint32_t group = min(B / kChunk, 32u);  // chunks of one block inside a warp
-
-    // ---- split, mantissa plane, per-block min/max --------------------------------
-    uint32_t E[kChunksPerThread][4];
-    uint32_t nval[kChunksPerThread];
+    } else {
+        uint32_t F[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int k = 0; k < kChunksPerThread; ++k) {
-        const uint32_t el = uint32_t(tid + k * kThreads) * kChunk;
-        const uint32_t nv = el < tile_n ? min(uint32_t(kChunk), tile_n - el) : 0u;
-        nval[k] = nv;
-        const uint16_t* src = a.in + tile_start + el;
-        uint32_t x[8];
-        if (nv == kChunk) {
-            const uint4 u = ld_stream_v4(src), v = ld_stream_v4(src + 8);
-            x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
-            x[4] = v.x; x[5] = v.y; x[6] = v.z; x[7] = v.w;
+        for (uint32_t j = 0; j < 4; ++j) {
+            const uint32_t q = pack_quad<W>(V[j]);
+            constexpr uint32_t kBits = 4 * W;
+            const uint32_t pos = j * kBits, word = pos / 32, off = pos % 32;
+            F[word] |= q << off;
+            if (off != 0 && off + kBits > 32) F[word + 1] |= q >> (32 - off);
+        }
+        if constexpr (W == 8) {
+            *reinterpret_cast<uint4*>(dst) = make_uint4(F[0], F[1], F[2], F[3]);
+        } else if constexpr (W == 4) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(F[0], F[1]);
+        } else if constexpr (W == 2) {
+            *reinterpret_cast<uint32_t*>(dst) = F[0];
+        } else if constexpr (W == 6) {
+            uint32_t* d = reinterpret_cast<uint32_t*>(dst);
+            d[0] = F[0];
+            d[1] = F[1];
+            d[2] = F[2];
         } else {
-            // ragged end of the tensor: lanes past the end repeat the first
-            // element, which leaves min and max unchanged
-            const uint32_t first = nv ? src[0] : 0u;
+            uint16_t* d = reinterpret_cast<uint16_t*>(dst);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t h0 = (2u * i < nv) ? src[2 * i] : first;
-                const uint32_t h1 = (2u * i + 1 < nv) ? src[2 * i + 1] : first;
-                x[i] = h0 | (h1 << 16);
+            for (uint32_t m = 0; m < W; ++m) d[m] = uint16_t(F[m / 2] >> (16 * (m % 2)));
+        }
+    }
+}
+
+__device__ __forceinline__ void pack_chunk_w(uint32_t w, const uint32_t V[4], uint8_t* dst) {
+    switch (w) {
+        case 1: pack_chunk<1>(V, dst); break;
+        case 2: pack_chunk<2>(V, dst); break;
+        case 3: pack_chunk<3>(V, dst); break;
+        case 4: pack_chunk<4>(V, dst); break;
+        case 5: pack_chunk<5>(V, dst); break;
+        case 6: pack_chunk<6>(V, dst); break;
+        case 7: pack_chunk<7>(V, dst); break;
+        case 8: pack_chunk<8>(V, dst); break;
+        default: break;  // w = 0: no exponent bytes
+    }
+}
+
+// The ragged end of a tensor: the chunk's first nbytes bytes only, one at a
+// time (lanes past the end already hold 0).
+__device__ void pack_chunk_tail(uint32_t w, const uint32_t V[4], uint8_t* dst, uint32_t nbytes) {
+    for (uint32_t i = 0; i < nbytes; ++i) {
+        uint32_t byte = 0;
+        for (uint32_t bit = 0; bit < 8; ++bit) {  // bit 8i+bit of the chunk's field
+            const uint32_t pos = 8 * i + bit, t = pos / w, within = pos % w;
+            const uint32_t v = (V[t / 4] >> (8 * (t % 4))) & 0xFFu;
+            byte |= ((v >> within) & 1u) << bit;
+        }
+        dst[i] = uint8_t(byte);
+    }
+}
+
+template <int MAXI>
+__device__ __forceinline__ uint32_t find_item(const EncodeParams<MAXI>& P, uint64_t t) {
+    if (MAXI == 1) return 0;
+    int lo = 0, hi = int(P.count) - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.tile_begin[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return uint32_t(lo);
+}
+
+// The 8 worker warps meet on hardware barrier 1 (the other warps never use
+// it). A worker never leaves its loop between two of these barriers: the only
+// waits that can fail come first in an iteration, and the warps agree on the
+// outcome at the first barrier of that iteration.
+__device__ __forceinline__ void workers_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+}
+
+__device__ __forceinline__ void give_up(EncodeSmem& sm, int32_t* status, int lane) {
+    if (lane == 0) {
+        report(status, kStatusTimeout);
+        sm.abort = 1;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// producer warp
+// ---------------------------------------------------------------------------
+template <int MAXI>
+__device__ void encode_produce(const EncodeParams<MAXI>& P, EncodeSmem& sm, int lane) {
+    int issued_round[kInStages];  // last round whose bulk copy was issued, per stage
+    for (int s = 0; s < kInStages; ++s) issued_round[s] = -1;
+    // The next tile's ticket is taken while the current tile's copy is in flight,
+    // so the atomic's round trip stays off the stage's critical path.
+    uint64_t t_next = 0;
+    if (lane == 0) t_next = uint64_t(atomicAdd(&P.control[0], 1u)) + P.first_ticket;
+    t_next = __shfl_sync(0xFFFFFFFFu, t_next, 0);
+    for (uint32_t i = 0;; ++i) {
+        const int s = int(i % kInStages);
+        const uint32_t round = i / kInStages;
+        if (round > 0 && !mbar_wait(&sm.in_empty[s], (round & 1u) ^ 1u, &sm.abort, 256)) {
+            give_up(sm, P.status, lane);
+            break;
+        }
+        InStage& st = sm.in[s];
+        const uint64_t t = t_next;
+        if (t >= P.total_tiles) {
+            if (lane == 0) {
+                st.info.end = 1;
+                mbar_arrive(&sm.in_full[s]);
+            }
+            return;
+        }
+        const uint32_t it = find_item(P, t);
+        const EncodeItem& I = P.item[it];
+        const uint64_t lt = t - P.tile_begin[it];
+        const uint64_t first = lt * kTile;
+        const uint32_t tile_n = I.n ? uint32_t(min(uint64_t(kTile), I.n - first)) : 0u;
+        const uint32_t b16 = (2u * tile_n) & ~15u;  // bytes the bulk copy can move
+        const uint32_t rem = tile_n - b16 / 2u;     // trailing elements (< 8) loaded plainly
+        if (uint32_t(lane) < rem) st.words[b16 / 2 + lane] = I.in[first + b16 / 2 + lane];
+        if (lane == 0) st.info = InInfo{t, lt, it, tile_n, 0u, 0u};
+        __syncwarp();
+        if (lane == 0) {
+            if (b16) {
+                mbar_arrive_expect_tx(&sm.in_full[s], b16);
+                bulk_load(st.words, I.in + first, b16, &sm.in_full[s]);
+                issued_round[s] = int(round);
+            } else {
+                mbar_arrive(&sm.in_full[s]);
+            }
+            t_next = uint64_t(atomicAdd(&P.control[0], 1u)) + P.first_ticket;
+        }
+        t_next = __shfl_sync(0xFFFFFFFFu, t_next, 0);
+    }
+    // Giving up: wait (bounded) for this warp's copies still in flight into shared memory.
+    if (lane == 0)
+        for (int s = 0; s < kInStages; ++s)
+            if (issued_round[s] >= 0) mbar_wait(&sm.in_full[s], uint32_t(issued_round[s]) & 1u, nullptr);
+}
+
+// ---------------------------------------------------------------------------
+// worker warps
+// ---------------------------------------------------------------------------
+template <int MAXI>
+__device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem& sm, int tid, int lane,
+                            int warp) {
+    for (uint32_t i = 0;; ++i) {
+        const int s = int(i % kInStages), o = int(i % kOutStages);
+        const uint32_t rin = i / kInStages, rout = i / kOutStages;
+        if (!mbar_wait(&sm.in_full[s], rin & 1u, &sm.abort) ||
+            (rout > 0 && !mbar_wait(&sm.out_empty[o], (rout & 1u) ^ 1u, &sm.abort))) {
+            give_up(sm, P.status, lane);
+            if (lane == 0) sm.worker_stop = 1;
+        }
+        // Agree: either every worker goes on or every worker stops. worker_stop
+        // is only ever written above, before this barrier, so all read the same.
+        workers_sync();
+        if (sm.worker_stop) return;
+        const InStage& in = sm.in[s];
+        OutStage& out = sm.out[o];
+        const InInfo info = in.info;
+        int* lo_of = sm.lo[i & 1];
+        int* hi_of = sm.hi[i & 1];
+        if (info.end) {  // pass the end on to every store warp (the next 4 stages)
+            for (uint32_t q = 0; q < kStoreWarps; ++q) {
+                const uint32_t iq = i + q;
+                const int oq = int(iq % kOutStages);
+                const uint32_t rq = iq / kOutStages;
+                if (q > 0 && rq > 0 && !mbar_wait(&sm.out_empty[oq], (rq & 1u) ^ 1u, &sm.abort)) {
+                    give_up(sm, P.status, lane);
+                    return;
+                }
+                if (tid == 0) sm.out[oq].info.end = 1;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.out_full[oq]);
+            }
+            return;
+        }
+        const EncodeItem& I = P.item[info.item];
+        const uint32_t B = I.block, log2B = log2_of(B), tile_n = info.tile_n;
+        const uint32_t group = min(B / kChunk, 32u);  // chunks of one block inside a warp
+        const uint64_t man_base = make_layout(I.n, B).off_man + info.lt * kTile;
+
+        // ---- read the input, release the input stage --------------------------------
+        uint32_t x[kChunksPerThread][8];
+        uint32_t nval[kChunksPerThread];
+#pragma unroll
+        for (int k = 0; k < kChunksPerThread; ++k) {
+            const uint32_t el = uint32_t(tid + k * kThreads) * kChunk;
+            const uint32_t nv = el < tile_n ? min(uint32_t(kChunk), tile_n - el) : 0u;
+            nval[k] = nv;
+            if (nv) {
+                const uint4 a = *reinterpret_cast<const uint4*>(in.words + el);
+                const uint4 b = *reinterpret_cast<const uint4*>(in.words + el + 8);
+                x[k][0] = a.x; x[k][1] = a.y; x[k][2] = a.z; x[k][3] = a.w;
+                x[k][4] = b.x; x[k][5] = b.y; x[k][6] = b.z; x[k][7] = b.w;
+                if (nv < kChunk) {
+                    // lanes past the end repeat the first element: min and max stay put
+                    const uint32_t first = x[k][0] & 0xFFFFu;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t lo = (2u * j < nv) ? (x[k][j] & 0xFFFFu) : first;
+                        const uint32_t hi = (2u * j + 1 < nv) ? (x[k][j] >> 16) : first;
+                        x[k][j] = lo | (hi << 16);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) x[k][j] = 0;
             }
         }
-        uint32_t S[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t e_a, s_a, e_b, s_b;
-            split_pair(x[2 * i], e_a, s_a);
-            split_pair(x[2 * i + 1], e_b, s_b);
-            E[k][i] = prmt(e_a, e_b, 0x6420u);
-            S[i] = prmt(s_a, s_b, 0x6420u);
-        }
-        uint8_t* man = a.out + L.off_man + tile_start + el;
-        if (nv == kChunk) {
-            st_stream_v4(man, make_uint4(S[0], S[1], S[2], S[3]));
-        } else {
-            for (uint32_t i = 0; i < nv; ++i) man[i] = uint8_t(S[i >> 2] >> (8 * (i & 3)));
-        }
-        uint32_t lo = 255u, hi = 0u;
-        if (nv) {
-            lo = min_byte(__vminu4(__vminu4(E[k][0], E[k][1]), __vminu4(E[k][2], E[k][3])));
-            hi = max_byte(__vmaxu4(__vmaxu4(E[k][0], E[k][1]), __vmaxu4(E[k][2], E[k][3])));
-        }
-        for (uint32_t off = 1; off < group; off <<= 1) {
-            lo = min(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, off));
-            hi = max(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, off));
-        }
-        if ((lane & (group - 1)) == 0 && nv) {
-            atomicMin(&s_lo[el >> log2B], int(lo));
-            atomicMax(&s_hi[el >> log2B], int(hi));
-        }
-    }
-    __syncthreads();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.in_empty[s]);
 
-    // ---- warp 0: widths, sizes, tile-local scan, look-back -----------------------
-    if (warp == 0) {
+        // ---- split: mantissa bytes to global memory, exponents kept; per-block min/max
+        // The exponent is the top byte of a word's 15-bit magnitude, so the
+        // minimum and maximum exponent are those of the smallest and largest
+        // magnitude, found with 16-bit lane min/max on the sign-cleared words.
+        uint32_t E[kChunksPerThread][4];
+#pragma unroll
+        for (int k = 0; k < kChunksPerThread; ++k) {
+            const uint32_t el = uint32_t(tid + k * kThreads) * kChunk;
+            const uint32_t nv = nval[k];
+            uint32_t S[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) split_quad(x[k][2 * j], x[k][2 * j + 1], S[j], E[k][j]);
+            if (nv < kChunk) {  // mantissa bytes past the end are the plane's zero padding
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int valid = int(nv) - 4 * j;
+                    if (valid < 4) S[j] &= valid <= 0 ? 0u : (0xFFFFFFFFu >> (32 - 8 * valid));
+                }
+            }
+            if (nv)
+                st_stream_v4(I.out + man_base + el, make_uint4(S[0], S[1], S[2], S[3]));
+            // key = largest magnitude << 16 | (0x7FFF - smallest magnitude): one
+            // 16-bit lane maximum reduces both across the lanes of a block
+            uint32_t key = 0u;
+            if (nv) {
+                uint32_t mn = x[k][0] & 0x7FFF7FFFu, mx = mn;
+#pragma unroll
+                for (int j = 1; j < 8; ++j) {
+                    const uint32_t m = x[k][j] & 0x7FFF7FFFu;
+                    mn = min_u16x2(mn, m);
+                    mx = max_u16x2(mx, m);
+                }
+                key = (max(mx & 0xFFFFu, mx >> 16) << 16) | (0x7FFFu - min(mn & 0xFFFFu, mn >> 16));
+            }
+            for (uint32_t off = 1; off < group; off <<= 1)
+                key = max_u16x2(key, __shfl_xor_sync(0xFFFFFFFFu, key, off));
+            const uint32_t lo = (0x7FFFu - (key & 0xFFFFu)) >> 7, hi = key >> (16 + 7);
+            if ((lane & (group - 1)) == 0 && nv) {
+                atomicMin(&lo_of[el >> log2B], int(lo));
+                atomicMax(&hi_of[el >> log2B], int(hi));
+            }
+        }
+        workers_sync();  // all per-block min/max are in
+
+        // ---- every worker warp: widths, sizes and the tile-local scan (each warp
+        //      needs the offsets of its own blocks; computing them in every warp
+        //      saves a barrier); worker warp 0 also publishes the tile --------------
+        const uint32_t nblk = (tile_n + B - 1) >> log2B;
         uint32_t sz[2], hdr[2];
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-            const uint32_t i = 2 * lane + j;
+            const uint32_t b = 2 * lane + j;
             sz[j] = 0;
             hdr[j] = 0;
-            if (i < nblk) {
-                const uint32_t lo = s_lo[i], hi = s_hi[i], d = hi - lo;
+            if (b < nblk) {
+                const uint32_t lo = lo_of[b], hi = hi_of[b], d = hi - lo;
                 const uint32_t w = d ? 32u - __clz(d) : 0u;
                 const uint32_t base = (w == 8u) ? 0u : lo;
-                const uint32_t len = min(B, tile_n - i * B);
+                const uint32_t len = min(B, tile_n - b * B);
                 sz[j] = ((len + 7) >> 3) * w;
                 hdr[j] = base | (w << 8);
             }
@@ -242,145 +444,332 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(const EncodeArgs a) {
             if (lane >= off) incl += y;
         }
         const uint32_t excl = incl - pair;
-        if (2 * lane < nblk) s_blk[2 * lane] = hdr[0] | (excl << 16);
-        if (2 * lane + 1 < nblk) s_blk[2 * lane + 1] = hdr[1] | ((excl + sz[0]) << 16);
-        const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        // block b's entry lives in lane b/2, slot b&1
+        const uint32_t blk_a = hdr[0] | (excl << 16), blk_b = hdr[1] | ((excl + sz[0]) << 16);
+        if (warp == 0) {
+            if (2 * lane < nblk) out.blk[2 * lane] = blk_a;
+            if (2 * lane + 1 < nblk) out.blk[2 * lane + 1] = blk_b;
+            const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+            if (lane == 0) {
+                out.info = OutInfo{info.t, info.lt, info.item, tile_n, nblk, total, 0u, {0u, 0u, 0u}};
+                // the first tile of a tensor knows its prefix (0); others publish their size
+                store_state(&P.state[info.t], (info.lt == 0 ? kFlagPrefix : kFlagAggregate) | total);
+            }
+        }
+        // the other parity's min/max were read by every warp in the previous tile,
+        // before this tile's first barrier: reset them for the next tile
+        if (warp == 1) {
+            int* lo_next = sm.lo[(i + 1) & 1];
+            int* hi_next = sm.hi[(i + 1) & 1];
+            lo_next[lane] = 255;
+            lo_next[lane + 32] = 255;
+            hi_next[lane] = 0;
+            hi_next[lane + 32] = 0;
+        }
+
+        // ---- remap and pack into the stage -----------------------------------------
+#pragma unroll
+        for (int k = 0; k < kChunksPerThread; ++k) {
+            const uint32_t nv = nval[k];
+            const uint32_t el = uint32_t(tid + k * kThreads) * kChunk;
+            // block el/B's entry sits in lane (el/B)/2 (every lane takes part in the shuffles)
+            const uint32_t bl = (el >> log2B) & (kMaxBlocksPerTile - 1);
+            const uint32_t ea = __shfl_sync(0xFFFFFFFFu, blk_a, bl >> 1);
+            const uint32_t eb = __shfl_sync(0xFFFFFFFFu, blk_b, bl >> 1);
+            if (nv == 0) continue;
+            const uint32_t blk = (bl & 1u) ? eb : ea;
+            const uint32_t base = blk & 0xFFu, w = (blk >> 8) & 0xFFu;
+            const uint32_t dst = (blk >> 16) + ((el & (B - 1)) >> 3) * w;
+            uint32_t V[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) V[j] = E[k][j] - base * 0x01010101u;  // e >= base: no borrows
+            if (nv < kChunk) {  // lanes past the end pack as 0
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int valid = int(nv) - 4 * j;
+                    if (valid < 4) V[j] &= valid <= 0 ? 0u : (0xFFFFFFFFu >> (32 - 8 * valid));
+                }
+            }
+            if (nv == kChunk)
+                pack_chunk_w(w, V, out.exp + dst);
+            else
+                pack_chunk_tail(w, V, out.exp + dst, (nv > 8 ? 2u : 1u) * w);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.out_full[o]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// store warp
+// ---------------------------------------------------------------------------
+// Decoupled look-back for tile t (index lt in its tensor): the bytes of all
+// earlier tiles of the tensor. While the nearest predecessors are plain
+// aggregates it reads 8 x 32 state words per round trip; while it waits on an
+// unpublished predecessor it polls only the 32 nearest, backing off.
+template <int MAXI>
+__device__ int lookback(const EncodeParams<MAXI>& P, uint64_t t, uint64_t lt, int lane,
+                        volatile int* abort, unsigned long long* prefix_out) {
+    const long long first = (long long)(t - lt);  // the tensor's first tile: always a prefix
+    long long top = (long long)t - 1;             // nearest tile not yet accounted for
+    unsigned long long acc = 0;
+    int rows = 1;
+    uint32_t backoff = 32;
+    const uint64_t t0 = __shfl_sync(0xFFFFFFFFu, global_timer_ns(), 0);
+    while (true) {
+        unsigned long long v[kWindowRows];
+#pragma unroll
+        for (int k = 0; k < kWindowRows; ++k) {
+            const long long idx = top - (32 * k + lane);
+            v[k] = (k < rows && idx >= first) ? load_state(&P.state[idx]) : kFlagPrefix;
+        }
+        // nearest tile (smallest distance 32k + lane) that is not a plain aggregate
+        int found = -1;
+        uint32_t fflag = 0;
+#pragma unroll
+        for (int k = 0; k < kWindowRows; ++k) {
+            const unsigned b = __ballot_sync(0xFFFFFFFFu, k < rows && uint32_t(v[k] >> 62) != 1u);
+            if (found < 0 && b) {
+                const int l = __ffs(int(b)) - 1;
+                found = 32 * k + l;
+                fflag = __shfl_sync(0xFFFFFFFFu, uint32_t(v[k] >> 62), l);
+            }
+        }
+        // everything nearer than `found` is an aggregate: account for it now
+        const int upto = found < 0 ? 32 * rows : (fflag == 2u ? found + 1 : found);
+        unsigned long long sum = 0;
+#pragma unroll
+        for (int k = 0; k < kWindowRows; ++k)
+            if (32 * k + lane < upto) sum += v[k] & kValueMask;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
+        acc += sum;
+        top -= upto;
+        if (fflag == 2u && found >= 0) {
+            *prefix_out = acc;
+            return 0;
+        }
+        if (found < 0) {  // a full window of aggregates: read further back, wider
+            rows = kWindowRows;
+            continue;
+        }
+        if (fflag == 3u) return kStatusCorrupt;  // a predecessor gave up (already reported)
+        // the nearest unaccounted predecessor has not published yet: wait, bounded
+        const int stop = __shfl_sync(
+            0xFFFFFFFFu,
+            int(*abort || load_flag(&P.control[1]) != 0 || global_timer_ns() - t0 > P.timeout_ns),
+            0);
+        if (stop) return kStatusTimeout;
+        __nanosleep(backoff);
+        backoff = min(backoff * 2u, 1024u);
+        rows = 1;
+    }
+}
+
+__device__ void write_container(uint8_t* out, const Layout& L, uint64_t E, int lane) {
+    if (lane < 16) {
+        uint64_t v = 0;
+        switch (lane) {
+            case 0: v = kMagic | (uint64_t(kVersion) << 32) | (uint64_t(kHeaderBytes) << 48); break;
+            case 1: v = L.block; break;  // flags (bytes 12..15) = 0
+            case 2: v = L.n; break;
+            case 3: v = L.nb; break;
+            case 4: v = L.off_hdr; break;
+            case 5: v = L.off_offs; break;
+            case 6: v = L.off_man; break;
+            case 7: v = L.off_exp; break;
+            case 8: v = E; break;
+            case 9: v = L.off_exp + E; break;
+            default: v = 0; break;
+        }
+        reinterpret_cast<uint64_t*>(out)[lane] = v;
+    }
+}
+
+// Zero the padding after the header, offset and mantissa sections. The bytes
+// [n, round16(n)) of the mantissa plane were stored as zeros by the last tile.
+__device__ void write_padding(uint8_t* out, const Layout& L, int lane) {
+    const uint64_t a0 = L.off_hdr + 2 * L.nb, a1 = L.off_offs + 4 * L.nb;
+    const uint64_t a2 = L.off_man + ((L.n + 15) & ~uint64_t(15));
+    for (uint64_t i = a0 + lane; i < L.off_offs; i += 32) out[i] = 0;
+    for (uint64_t i = a1 + lane; i < L.off_man; i += 32) out[i] = 0;
+    for (uint64_t i = a2 + lane; i < L.off_exp; i += 32) out[i] = 0;
+}
+
+template <int MAXI>
+__device__ void encode_store(const EncodeParams<MAXI>& P, EncodeSmem& sm, int lane, int which) {
+    for (uint32_t i = uint32_t(which);; i += kStoreWarps) {
+        const int o = int(i % kOutStages);
+        const uint32_t round = i / kOutStages;
+        if (!mbar_wait(&sm.out_full[o], round & 1u, &sm.abort, 1024)) {
+            give_up(sm, P.status, lane);
+            break;
+        }
+        const OutStage& st = sm.out[o];
+        const OutInfo info = st.info;
+        if (info.end) break;
+        const EncodeItem& I = P.item[info.item];
+        const Layout L = make_layout(I.n, I.block);
+        const uint64_t first = info.lt * kTile;
+        const bool last_tile = info.lt + 1 == encode_tiles(I.n);
 
         unsigned long long prefix = 0;
-        bool failed = false, timed_out = false;
-        if (t == 0) {
-            if (lane == 0) store_state(&a.state[0], kFlagPrefix | total);
+        int rc = 0;
+        if (info.lt > 0 && load_flag(&P.control[1]) == 0) {
+            rc = lookback(P, info.t, info.lt, lane, &sm.abort, &prefix);
+        } else if (info.lt > 0) {
+            rc = kStatusCorrupt;  // an earlier failure: stop here without waiting
+        }
+        if (rc == 0) {
+            if (lane == 0 && info.lt > 0)
+                store_state(&P.state[info.t], kFlagPrefix | (prefix + info.total));
+            const uint64_t b0 = first >> L.log2_block;
+            for (uint32_t b = lane; b < info.nblk; b += 32) {
+                const uint32_t blk = st.blk[b];
+                reinterpret_cast<uint16_t*>(I.out + L.off_hdr)[b0 + b] = uint16_t(blk & 0xFFFFu);
+                reinterpret_cast<uint32_t*>(I.out + L.off_offs)[b0 + b] =
+                    uint32_t((prefix + (blk >> 16)) >> 4);
+            }
+            const uint32_t t16 = info.total & ~15u, rem = info.total - t16;
+            uint8_t* dst = I.out + L.off_exp + prefix;  // 16-byte aligned: earlier tiles are full
+            if (lane == 0 && t16) bulk_store(dst, st.exp, t16);
+            if (uint32_t(lane) < rem) dst[t16 + lane] = st.exp[t16 + lane];
+            if (last_tile) {
+                const uint64_t E = prefix + info.total;
+                write_container(I.out, L, E, lane);
+                write_padding(I.out, L, lane);
+                if (lane == 0) *I.out_bytes = L.off_exp + E;
+            }
         } else {
-            if (lane == 0) store_state(&a.state[t], kFlagAggregate | total);
-            long long top = (long long)t - 1;
-            const uint64_t t0 = __shfl_sync(0xFFFFFFFFu, global_timer_ns(), 0);
-            while (true) {
-                const long long idx = top - lane;
-                const unsigned long long s = idx >= 0 ? load_state(&a.state[idx]) : kFlagPrefix;
-                const uint32_t flag = uint32_t(s >> 62);
-                const unsigned not_agg = __ballot_sync(0xFFFFFFFFu, flag != 1u);
-                if (not_agg == 0u) {  // 32 aggregates: add them all, look further back
-                    unsigned long long v = s & kValueMask;
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-                    prefix += v;
-                    top -= 32;
-                    continue;
-                }
-                const int first = __ffs(not_agg) - 1;
-                const uint32_t fflag = __shfl_sync(0xFFFFFFFFu, flag, first);
-                if (fflag == 2u) {  // an inclusive prefix: add it and the aggregates after it
-                    unsigned long long v = (lane <= first) ? (s & kValueMask) : 0ull;
-#pragma unroll
-                    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-                    prefix += v;
-                    break;
-                }
-                if (fflag == 3u) {  // a predecessor gave up
-                    failed = true;
-                    break;
-                }
-                // the nearest unfinished predecessor has not published yet: wait, bounded
-                const bool expired = __shfl_sync(
-                    0xFFFFFFFFu, int(global_timer_ns() - t0 > a.timeout_ns), 0);
-                if (expired) {
-                    failed = timed_out = true;
-                    break;
-                }
-                __nanosleep(64);
+            if (lane == 0) {
+                store_state(&P.state[info.t], kFlagError);
+                atomicExch(&P.control[1], 1u);
+                if (rc == kStatusTimeout) report(P.status, kStatusTimeout);
+                if (last_tile) *I.out_bytes = 0;
             }
-            if (!failed && lane == 0) store_state(&a.state[t], kFlagPrefix | (prefix + total));
         }
+        // The stage is free once the bulk store has read it.
         if (lane == 0) {
-            s_prefix = prefix;
-            s_total = total;
-            s_abort = failed;
-            if (failed) {
-                store_state(&a.state[t], kFlagError);
-                atomicExch(&a.control[1], 1u);
-                if (timed_out) report(a.status, kStatusTimeout);
-                if (t == a.ntiles - 1) *a.out_bytes = 0;
-            }
+            bulk_commit();
+            bulk_wait_read<0>();
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.out_empty[o]);
+    }
+    if (lane == 0) bulk_wait_all();
+}
+
+template <int MAXI>
+__global__ void __launch_bounds__(kEncodeThreads)
+    encode_kernel(const __grid_constant__ EncodeParams<MAXI> P) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    EncodeSmem& sm = *reinterpret_cast<EncodeSmem*>(smem_raw);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        for (int s = 0; s < kInStages; ++s) {
+            mbar_init(&sm.in_full[s], 1);
+            mbar_init(&sm.in_empty[s], kWorkerWarps);
+        }
+        for (int o = 0; o < kOutStages; ++o) {
+            mbar_init(&sm.out_full[o], kWorkerWarps);
+            mbar_init(&sm.out_empty[o], 1);
+        }
+        sm.abort = 0;
+        sm.worker_stop = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (tid < 2 * kMaxBlocksPerTile) {
+        sm.lo[tid >> 6][tid & 63] = 255;
+        sm.hi[tid >> 6][tid & 63] = 0;
     }
     __syncthreads();
-    if (s_abort) return;
-    const unsigned long long prefix = s_prefix;
-    const uint32_t total = s_total;
+    if (warp == kProducerWarp)
+        encode_produce<MAXI>(P, sm, lane);
+    else if (warp >= kFirstStoreWarp)
+        encode_store<MAXI>(P, sm, lane, warp - kFirstStoreWarp);
+    else
+        encode_work<MAXI>(P, sm, tid, lane, warp);
+}
 
-    // ---- block headers and offsets -----------------------------------------------
-    if (tid < nblk) {
-        const uint32_t blk = s_blk[tid];
-        const uint64_t b = (tile_start >> log2B) + tid;
-        reinterpret_cast<uint16_t*>(a.out + L.off_hdr)[b] = uint16_t(blk & 0xFFFFu);
-        reinterpret_cast<uint32_t*>(a.out + L.off_offs)[b] = uint32_t((prefix + (blk >> 16)) >> 4);
+template <int MAXI>
+cudaError_t encode_grid(uint64_t tiles, unsigned* grid) {
+    static std::mutex mu;
+    static int per_device[64];
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (per_device[dev] == 0) {
+        err = cudaFuncSetAttribute(encode_kernel<MAXI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   int(sizeof(EncodeSmem)));
+        if (err != cudaSuccess) return err;
+        int sms = 0, per_sm = 0;
+        err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (err != cudaSuccess) return err;
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_kernel<MAXI>,
+                                                            kEncodeThreads, sizeof(EncodeSmem));
+        if (err != cudaSuccess) return err;
+        per_device[dev] = (per_sm > 0 ? per_sm : 1) * sms;
     }
+    const uint64_t cap = uint64_t(per_device[dev]);
+    *grid = unsigned(tiles < cap ? tiles : cap);
+    return cudaSuccess;
+}
 
-    // ---- remap and pack into the staging buffer ----------------------------------
-#pragma unroll
-    for (int k = 0; k < kChunksPerThread; ++k) {
-        const uint32_t nv = nval[k];
-        if (nv == 0) continue;
-        const uint32_t el = uint32_t(tid + k * kThreads) * kChunk;
-        const uint32_t blk = s_blk[el >> log2B];
-        const uint32_t base = blk & 0xFFu, w = (blk >> 8) & 0xFFu;
-        const uint32_t dst = (blk >> 16) + ((el & (B - 1)) >> 3) * w;
-        uint32_t V[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            V[i] = E[k][i] - base * 0x01010101u;  // e >= base in every byte: no borrows
-            const int valid = int(nv) - 4 * i;    // lanes past the end pack as 0
-            if (valid < 4) V[i] &= valid <= 0 ? 0u : (0xFFFFFFFFu >> (32 - 8 * valid));
-        }
-        const uint64_t o0 = pack_octet(V[0], V[1], w);
-        const uint64_t o1 = pack_octet(V[2], V[3], w);
-        const uint32_t nbytes = (nv > 8 ? 2u : 1u) * w;
-        for (uint32_t i = 0; i < nbytes; ++i) {
-            const uint64_t o = i < w ? o0 : o1;
-            const uint32_t sh = 8 * (i < w ? i : i - w);
-            s_stage[dst + i] = uint8_t(o >> sh);
-        }
+template <int MAXI>
+cudaError_t encode_batch(const EncodeItem* items, uint32_t count, uint8_t* workspace,
+                         int32_t* status, uint64_t timeout_ns, uint32_t first_ticket,
+                         cudaStream_t stream) {
+    static_assert(sizeof(EncodeParams<MAXI>) <= 32000, "launch parameters exceed the limit");
+    EncodeParams<MAXI> p;
+    p.status = status;
+    p.control = reinterpret_cast<uint32_t*>(workspace);
+    p.state = reinterpret_cast<unsigned long long*>(workspace + 16);
+    p.timeout_ns = timeout_ns;
+    p.count = count;
+    p.first_ticket = first_ticket;
+    uint64_t tiles = 0;
+    for (uint32_t i = 0; i < count; ++i) {
+        p.tile_begin[i] = tiles;
+        p.item[i] = items[i];
+        tiles += encode_tiles(items[i].n);
     }
-    __syncthreads();
-
-    // ---- the tile's exponent payload: 16-byte stores (the start is 16-aligned) ----
-    uint8_t* dst = a.out + L.off_exp + prefix;
-    for (uint32_t i = tid; i < total / 16; i += kThreads)
-        st_stream_v4(dst + 16 * i, *reinterpret_cast<const uint4*>(s_stage + 16 * i));
-    const uint32_t rem = total & 15u;
-    if (tid < rem) dst[total - rem + tid] = s_stage[total - rem + tid];
-
-    // ---- the last tile knows E: container header, padding, total size -----------
-    if (t == a.ntiles - 1) {
-        const uint64_t E = prefix + total;
-        write_container(a.out, L, E, tid);
-        write_padding(a.out, L, tid);
-        if (tid == 0) *a.out_bytes = L.off_exp + E;
-    }
+    p.tile_begin[count] = tiles;
+    p.total_tiles = tiles;
+    if (tiles == 0) return cudaSuccess;
+    if (tiles >= (1ull << 31)) return cudaErrorInvalidValue;  // the ticket is 32-bit
+    cudaError_t err = cudaMemsetAsync(workspace, 0, encode_workspace_bytes(tiles), stream);
+    if (err != cudaSuccess) return err;
+    unsigned grid = 0;
+    err = encode_grid<MAXI>(tiles, &grid);
+    if (err != cudaSuccess) return err;
+    encode_kernel<MAXI><<<grid, kEncodeThreads, sizeof(EncodeSmem), stream>>>(p);
+    return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_encode(const uint16_t* in, const Layout& L, uint8_t* out, uint64_t* out_bytes,
-                          void* workspace, int32_t* status, uint64_t timeout_ns,
-                          uint32_t first_ticket, cudaStream_t stream) {
-    const uint64_t ntiles = num_tiles(L.n);
-    cudaError_t err = cudaMemsetAsync(workspace, 0, encode_workspace_bytes(L.n), stream);
-    if (err != cudaSuccess) return err;
-    EncodeArgs a;
-    a.in = in;
-    a.out = out;
-    a.out_bytes = out_bytes;
-    a.status = status;
-    a.control = static_cast<uint32_t*>(workspace);
-    a.state = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + 16);
-    a.L = L;
-    a.ntiles = ntiles;
-    a.timeout_ns = timeout_ns;
-    a.first_ticket = first_ticket;
-    const unsigned grid = unsigned(ntiles ? ntiles : 1);
-    encode_kernel<<<grid, kThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+constexpr uint32_t kEncodeBatchMax = 512;
+
+cudaError_t launch_encode(const EncodeItem* items, uint32_t count, void* workspace,
+                          int32_t* status, uint64_t timeout_ns, uint32_t first_ticket,
+                          cudaStream_t stream) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (count == 1) return encode_batch<1>(items, 1, ws, status, timeout_ns, first_ticket, stream);
+    // Larger batches go out in launches of up to 512 tensors; each launch has
+    // its own part of the workspace, so they can follow each other on the stream.
+    for (uint32_t i = 0; i < count; i += kEncodeBatchMax) {
+        const uint32_t c = min(kEncodeBatchMax, count - i);
+        const cudaError_t err =
+            encode_batch<kEncodeBatchMax>(items + i, c, ws, status, timeout_ns, first_ticket, stream);
+        if (err != cudaSuccess) return err;
+        uint64_t tiles = 0;
+        for (uint32_t j = 0; j < c; ++j) tiles += encode_tiles(items[i + j].n);
+        ws += (encode_workspace_bytes(tiles) + 15) & ~uint64_t(15);
+    }
+    return cudaSuccess;
 }
 
 }  // namespace wc

@@ -43,9 +43,13 @@ __host__ __device__ inline bool block_ok(uint32_t B) {
 }
 
 __host__ __device__ inline uint32_t log2_pow2(uint32_t B) {
+#ifdef __CUDA_ARCH__
+    return uint32_t(__ffs(int(B))) - 1u;
+#else
     uint32_t k = 0;
     while ((1u << k) < B) ++k;
     return k;
+#endif
 }
 
 __host__ __device__ inline Layout make_layout(uint64_t n, uint32_t B) {
@@ -107,6 +111,102 @@ __device__ __forceinline__ void report(int32_t* status, int32_t code) {
     if (status != nullptr) atomicCAS(reinterpret_cast<int*>(status), 0, code);
 }
 
+// Every in-kernel wait on another warp or block gives up after this long.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+
+// ---------------------------------------------------------------------------
+// mbarrier and bulk-copy helpers (PTX)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// Test the phase with the given parity; the thread may sleep up to ~20 us in
+// the instruction waiting for it (woken early when the phase completes).
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for the phase of `bar` with the given parity; false if kWaitLimitNs
+// passed or (abort != nullptr) another warp of the block gave up first.
+// Warps off the critical path pass max_sleep_ns > 0: between polls they sleep,
+// doubling from 32 ns up to that cap, and leave the issue slots to others.
+__device__ __forceinline__ bool mbar_wait(unsigned long long* bar, uint32_t parity,
+                                          volatile int* abort, uint32_t max_sleep_ns = 0) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    uint32_t sleep = 32;
+    while (!mbar_try_wait(bar, parity)) {
+        if ((abort != nullptr && *abort) || global_timer_ns() - t0 > kWaitLimitNs) return false;
+        if (max_sleep_ns) {
+            __nanosleep(sleep);
+            sleep = min(sleep * 2u, max_sleep_ns);
+        }
+    }
+    return true;
+}
+
+// Bulk asynchronous copy global -> this block's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          unsigned long long* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Bulk asynchronous copy of this block's shared memory -> global, tracked by
+// the issuing thread's bulk async-groups.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+                 "r"(smem_addr(src)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Wait until at most N of this thread's committed bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until all of this thread's committed bulk groups have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Make this thread's generic-proxy writes to shared memory visible to bulk copies.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Launchers (defined in wc_encode.cu / wc_decode.cu)
 // ---------------------------------------------------------------------------
@@ -119,13 +219,28 @@ struct DecodeItem {
     uint32_t reserved;
 };
 
-cudaError_t launch_encode(const uint16_t* in, const Layout& L, uint8_t* out, uint64_t* out_bytes,
-                          void* workspace, int32_t* status, uint64_t timeout_ns,
-                          uint32_t first_ticket, cudaStream_t stream);
+struct EncodeItem {
+    const uint16_t* in;
+    uint8_t* out;
+    uint64_t* out_bytes;
+    uint64_t n;
+    uint32_t block;
+    uint32_t reserved;
+};
+
+// Tiles of one tensor in the encoder's look-back state (an empty tensor still
+// takes one, which writes its header).
+__host__ __device__ inline uint64_t encode_tiles(uint64_t n) { return n ? num_tiles(n) : 1; }
 
 // Bytes of workspace the encoder needs: a 16-byte control word (ticket,
 // internal error flag) and one 8-byte look-back state per tile.
-inline uint64_t encode_workspace_bytes(uint64_t n) { return 16 + 8 * num_tiles(n); }
+inline uint64_t encode_workspace_bytes(uint64_t tiles) { return 16 + 8 * tiles; }
+
+// One launch for `count` tensors (the launcher splits larger batches); the
+// workspace must hold encode_workspace_bytes(sum of encode_tiles) bytes.
+cudaError_t launch_encode(const EncodeItem* items, uint32_t count, void* workspace,
+                          int32_t* status, uint64_t timeout_ns, uint32_t first_ticket,
+                          cudaStream_t stream);
 
 cudaError_t launch_decode(const DecodeItem* items, uint32_t count, int32_t* status,
                           cudaStream_t stream);

@@ -37,6 +37,18 @@ class WcodecError(RuntimeError):
         self.status = status
 
 
+class wc_compress_item(ctypes.Structure):
+    _fields_ = [
+        ("in_", ctypes.c_void_p),
+        ("n", ctypes.c_uint64),
+        ("block", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32),
+        ("out", ctypes.c_void_p),
+        ("out_capacity", ctypes.c_uint64),
+        ("out_bytes", ctypes.c_void_p),
+    ]
+
+
 class wc_batch_item(ctypes.Structure):
     _fields_ = [
         ("stream", ctypes.c_void_p),
@@ -74,6 +86,10 @@ def lib() -> ctypes.CDLL:
                                  ctypes.POINTER(u64)]
     L.wc_stream_info.restype = i
     L.wc_status_string.argtypes, L.wc_status_string.restype = [i], ctypes.c_char_p
+    L.wc_compress_batch_workspace_size.argtypes = [ctypes.POINTER(wc_compress_item), u32]
+    L.wc_compress_batch_workspace_size.restype = u64
+    L.wc_compress_batch.argtypes = [ctypes.POINTER(wc_compress_item), u32, vp, u64, vp, vp]
+    L.wc_compress_batch.restype = i
     L.wc_compress_noalloc.argtypes = [vp, u64, u32, vp, u64, vp, vp, vp]
     L.wc_compress_noalloc.restype = i
     L.wc_debug_compress_stalled.argtypes = [vp, u64, u32, vp, u64, vp, vp, u64, vp, u64, vp]
@@ -97,6 +113,14 @@ def wc_compress(d_in, n, block, d_out, out_capacity, d_out_bytes, d_workspace, w
                 d_status, stream) -> int:
     return lib().wc_compress(d_in, n, block, d_out, out_capacity, d_out_bytes, d_workspace,
                              workspace_bytes, d_status, stream)
+
+
+def wc_compress_batch_workspace_size(items, count) -> int:
+    return lib().wc_compress_batch_workspace_size(items, count)
+
+
+def wc_compress_batch(items, count, d_workspace, workspace_bytes, d_status, stream) -> int:
+    return lib().wc_compress_batch(items, count, d_workspace, workspace_bytes, d_status, stream)
 
 
 def wc_compress_noalloc(d_in, n, block, d_out, out_capacity, d_out_bytes, d_status,
@@ -228,6 +252,46 @@ def decompress_compressed(c: Compressed, out: torch.Tensor | None = None, status
     if out is None:
         out = torch.empty(c.shape, dtype=c.dtype, device=c.buffer.device)
     return decompress(c.buffer, c.n, c.block, out=out, status=status, stream=stream)
+
+
+class CompressBatch:
+    """Reusable buffers and descriptors for compressing a fixed list of tensors
+    in one call: ``run()`` enqueues one encoder launch per 512 tensors."""
+
+    def __init__(self, tensors, block=1024):
+        self.words = [as_words(t) for t in tensors]
+        dev = self.words[0].device if self.words else torch.device("cuda")
+        k = len(self.words)
+        self.blocks = list(block) if isinstance(block, (list, tuple)) else [block] * k
+        self.buffers = [torch.empty((wc_bound(w.numel(), b) + 15) // 16 * 16,
+                                    dtype=torch.uint8, device=dev)
+                        for w, b in zip(self.words, self.blocks)]
+        self.nbytes = torch.zeros(max(1, k), dtype=torch.int64, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.items = (wc_compress_item * max(1, k))()
+        for j, w in enumerate(self.words):
+            it = self.items[j]
+            it.in_ = w.data_ptr() if w.numel() else None
+            it.n = w.numel()
+            it.block = self.blocks[j]
+            it.reserved = 0
+            it.out = self.buffers[j].data_ptr()
+            it.out_capacity = self.buffers[j].numel()
+            it.out_bytes = self.nbytes[j:].data_ptr()
+        ws = wc_compress_batch_workspace_size(self.items, k)
+        if k and ws == 0:
+            raise WcodecError(WC_ERR_INVALID_ARG, "wc_compress_batch_workspace_size")
+        self.workspace = torch.empty(max(16, (ws + 15) // 16 * 16), dtype=torch.uint8, device=dev)
+        self.count = k
+
+    def run(self, stream=None):
+        rc = wc_compress_batch(self.items, self.count, self.workspace.data_ptr(),
+                               self.workspace.numel(), self.status.data_ptr(),
+                               _stream_handle(stream))
+        _check(rc, "wc_compress_batch")
+
+    def sizes(self) -> list[int]:
+        return self.nbytes[: self.count].cpu().tolist()
 
 
 def make_batch(items) -> ctypes.Array:

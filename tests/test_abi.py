@@ -26,6 +26,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for f in ("wc_bound", "wc_workspace_size", "wc_compress", "wc_decompress",
+              "wc_compress_batch", "wc_compress_batch_workspace_size",
               "wc_decompress_batch", "wc_stream_info", "wc_status_string",
               "wc_debug_compress_stalled"):
         assert f in names
@@ -48,7 +49,7 @@ def test_bound_matches_oracle(wclib, orc):
 
 
 def test_workspace_size(wclib):
-    for n, tiles in [(0, 0), (1, 1), (8192, 1), (8193, 2), (10**6, 123)]:
+    for n, tiles in [(0, 1), (1, 1), (8192, 1), (8193, 2), (10**6, 123)]:
         assert wclib.wc_workspace_size(n, 512) == 16 + 8 * tiles
     assert wclib.wc_workspace_size(10, 100) == 0
 
@@ -105,6 +106,21 @@ def test_argument_checks_before_any_launch(wclib):
     items[1].block, items[1].reserved = 128, 1
     assert c.wc_decompress_batch(items, 2, None, None) == c.WC_ERR_INVALID_ARG
     assert c.wc_decompress_batch(None, 1, None, None) == c.WC_ERR_INVALID_ARG
+    # batched compression: every item is checked before anything is launched
+    citems = (c.wc_compress_item * 2)()
+    for j in range(2):
+        citems[j].in_, citems[j].n, citems[j].block = 16, 10, 128
+        citems[j].out, citems[j].out_capacity, citems[j].out_bytes = 16, 10**6, 16
+    citems[1].block = 100
+    assert c.wc_compress_batch(citems, 2, 16, 10**6, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_compress_batch_workspace_size(citems, 2) == 0
+    citems[1].block, citems[1].reserved = 128, 7
+    assert c.wc_compress_batch(citems, 2, 16, 10**6, None, None) == c.WC_ERR_INVALID_ARG
+    citems[1].reserved = 0
+    assert c.wc_compress_batch_workspace_size(citems, 2) == 2 * 8 + 16
+    assert c.wc_compress_batch(citems, 2, 16, 8, None, None) == c.WC_ERR_BUFFER_TOO_SMALL
+    citems[1].out_capacity = 10
+    assert c.wc_compress_batch(citems, 2, 16, 10**6, None, None) == c.WC_ERR_BUFFER_TOO_SMALL
     # the stall test hook needs two tiles and a bounded timeout
     assert c.wc_debug_compress_stalled(16, 100, 128, 16, 10**6, 16, 16, 10**6, None, 10**6,
                                        None) == c.WC_ERR_INVALID_ARG

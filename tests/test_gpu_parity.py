@@ -168,3 +168,55 @@ def test_many_item_batch_spans_launches(wclib, cuda):
     torch.cuda.synchronize()
     assert status.item() == 0
     assert all(torch.equal(a, b) for a, b in pairs)
+
+
+def test_batch_compress_matches_oracle(orc, wclib, cuda):
+    """One wc_compress_batch call over tensors of mixed sizes and block sizes
+    (including an empty one): every stream equals the oracle's."""
+    rng = np.random.default_rng(12)
+    shapes = [(0, 256), (1, 128), (8191, 512), (8193, 4096), (100_003, 128), (1 << 20, 1024),
+              (3 * 8192 + 5, 2048), (65536, 256)]
+    words = [random_words(rng, n, "mixed") for n, _ in shapes]
+    tensors = [to_gpu_words(w, cuda) for w in words]
+    batch = wclib.CompressBatch(tensors, block=[B for _, B in shapes])
+    batch.run()
+    torch.cuda.synchronize()
+    assert batch.status.item() == 0
+    for j, ((n, B), w) in enumerate(zip(shapes, words)):
+        got = batch.buffers[j][: batch.sizes()[j]].cpu().numpy()
+        assert np.array_equal(got, orc.compress(w, B)), (n, B)
+
+
+def test_batch_compress_spans_launches(orc, wclib, cuda):
+    """More tensors than one launch takes: each launch has its own workspace part."""
+    rng = np.random.default_rng(13)
+    words = [random_words(rng, int(rng.integers(0, 20000)), "gauss") for _ in range(700)]
+    batch = wclib.CompressBatch([to_gpu_words(w, cuda) for w in words], block=128)
+    batch.run()
+    torch.cuda.synchronize()
+    assert batch.status.item() == 0
+    sizes = batch.sizes()
+    for j in range(0, 700, 7):
+        got = batch.buffers[j][: sizes[j]].cpu().numpy()
+        assert np.array_equal(got, orc.compress(words[j], 128))
+
+
+def test_stack_shaped_batch_round_trip(wclib, cuda):
+    """A batch shaped like one decoder layer plus a ragged tensor, compressed in
+    one call and decoded in one call, gives back every tensor bit for bit."""
+    from lossless_weight_compression_b200 import synth
+    tensors = [t.view(-1).view(torch.int16) for _, t in synth.layer_tensors(3, cuda)]
+    tensors.append(to_gpu_words(random_words(np.random.default_rng(14), 123_457, "mixed"), cuda))
+    batch = wclib.CompressBatch(tensors, block=1024)
+    batch.run()
+    torch.cuda.synchronize()
+    assert batch.status.item() == 0
+    sizes = batch.sizes()
+    outs = [torch.empty_like(t) for t in tensors]
+    status = torch.zeros(1, dtype=torch.int32, device=cuda)
+    wclib.decompress_batch(wclib.make_batch(
+        [(batch.buffers[j], sizes[j], outs[j], t.numel(), 1024) for j, t in enumerate(tensors)]),
+        status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert all(torch.equal(a, b) for a, b in zip(tensors, outs))
