@@ -71,7 +71,8 @@ struct EncodeParams {
 };
 
 struct __align__(16) InInfo {
-    uint64_t t, lt;  // batch tile index, tile index within its tensor
+    uint64_t t, lt;    // batch tile index, tile index within its tensor
+    uint64_t man_off;  // byte offset of the tile's mantissa bytes in its stream
     uint32_t item, tile_n, end, pad;
 };
 
@@ -279,7 +280,8 @@ __device__ void encode_produce(const EncodeParams<MAXI>& P, EncodeSmem& sm, int 
         const uint32_t b16 = (2u * tile_n) & ~15u;  // bytes the bulk copy can move
         const uint32_t rem = tile_n - b16 / 2u;     // trailing elements (< 8) loaded plainly
         if (uint32_t(lane) < rem) st.words[b16 / 2 + lane] = I.in[first + b16 / 2 + lane];
-        if (lane == 0) st.info = InInfo{t, lt, it, tile_n, 0u, 0u};
+        if (lane == 0)
+            st.info = InInfo{t, lt, make_layout(I.n, I.block).off_man + first, it, tile_n, 0u, 0u};
         __syncwarp();
         if (lane == 0) {
             if (b16) {
@@ -340,7 +342,7 @@ __device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem& sm, int tid
         const EncodeItem& I = P.item[info.item];
         const uint32_t B = I.block, log2B = log2_of(B), tile_n = info.tile_n;
         const uint32_t group = min(B / kChunk, 32u);  // chunks of one block inside a warp
-        const uint64_t man_base = make_layout(I.n, B).off_man + info.lt * kTile;
+        const uint64_t man_base = info.man_off;
 
         // ---- read the input, release the input stage --------------------------------
         uint32_t x[kChunksPerThread][8];
@@ -407,8 +409,13 @@ __device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem& sm, int tid
                 }
                 key = (max(mx & 0xFFFFu, mx >> 16) << 16) | (0x7FFFu - min(mn & 0xFFFFu, mn >> 16));
             }
-            for (uint32_t off = 1; off < group; off <<= 1)
-                key = max_u16x2(key, __shfl_xor_sync(0xFFFFFFFFu, key, off));
+            if (group == 32) {  // B >= 512: the warp's 32 chunks are one block
+                key = (__reduce_max_sync(0xFFFFFFFFu, key >> 16) << 16) |
+                      __reduce_max_sync(0xFFFFFFFFu, key & 0xFFFFu);
+            } else {
+                for (uint32_t off = 1; off < group; off <<= 1)
+                    key = max_u16x2(key, __shfl_xor_sync(0xFFFFFFFFu, key, off));
+            }
             const uint32_t lo = (0x7FFFu - (key & 0xFFFFu)) >> 7, hi = key >> (16 + 7);
             if ((lane & (group - 1)) == 0 && nv) {
                 atomicMin(&lo_of[el >> log2B], int(lo));
