@@ -171,7 +171,7 @@ def hbm_peak():
 
 def decode_kernel_digest() -> str:
     h = hashlib.sha256()
-    for name in ("wc_decode.cu", "wc_internal.cuh"):
+    for name in ("wc_decode.cu", "wc_decode_core.cuh", "wc_internal.cuh"):
         with open(os.path.join(ROOT, "lossless_weight_compression_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -484,15 +484,137 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
             "verified_bit_exact": bool(ok)}
 
 
+# ---------------------------------------------------------------------------
+# next row: fused decode + matrix-vector products over the stack's linear weights
+# ---------------------------------------------------------------------------
+def run_gemv(args):
+    """One fused wc_gemv_batch launch over the 225 linear weight matrices of the
+    8B-shaped stack (32 layers x 7 + LM head; the embedding is a lookup, not a
+    product), n_vec activation vectors, against torch's BF16 matmul (cuBLAS) on
+    the same matrices, replayed from a CUDA graph."""
+    import torch
+
+    from lossless_weight_compression_b200 import build_lib, synth, wcodec
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    build_lib.build()
+    wc = wcodec.lib()
+    stream = torch.cuda.current_stream(dev)
+    nv = args.n_vec
+    if args.gemv_layers is None:
+        mats = [(name, t) for name, t in synth.stack_tensors(dev, rank_seed_base(rank))
+                if name != "embed_tokens"]
+    else:  # a smaller case for profiling: the first layers only
+        mats = [m for l in range(args.gemv_layers)
+                for m in synth.layer_tensors(l, dev, rank_seed_base(rank))]
+    weights = sum(t.numel() for _, t in mats)
+    enc = wcodec.CompressBatch([t for _, t in mats], block=BLOCK)
+    enc.run()
+    torch.cuda.synchronize(dev)
+    sizes = enc.sizes()
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    xs = [torch.randn((nv, t.shape[1]), generator=g, device=dev).to(torch.bfloat16) for _, t in mats]
+    ys = [torch.empty((nv, t.shape[0]), dtype=torch.float32, device=dev) for _, t in mats]
+    batch = wcodec.make_gemv_batch([(enc.buffers[k], sizes[k], xs[k], ys[k], t.shape[0], t.shape[1],
+                                     BLOCK) for k, (_, t) in enumerate(mats)])
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def fused():
+        rc = wc.wc_gemv_batch(batch[0], batch[1], nv, status.data_ptr(), stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError("wc_gemv_batch: %s" % wc.wc_status_string(rc))
+
+    # torch / cuBLAS on the uncompressed BF16 weights, all matrices in one graph
+    ts = [t for _, t in mats]
+    outs = [torch.empty((nv, t.shape[0]), dtype=torch.bfloat16, device=dev) for t in ts]
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(2):
+            for k, t in enumerate(ts):
+                torch.matmul(xs[k], t.T, out=outs[k])
+    stream.wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for k, t in enumerate(ts):
+            torch.matmul(xs[k], t.T, out=outs[k])
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        barrier(dist, dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        barrier(dist, dev)
+        return max_over_ranks(e0.elapsed_time(e1) / 1e3 / steps, dist, dev)
+
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        t_fused = timed(fused, args.steps)
+        t_blas = timed(graph.replay, args.steps)
+    torch.cuda.synchronize(dev)
+    # verification against the decoded weights in FP64 (outside the timed region)
+    ok = status.item() == 0
+    for k, t in enumerate(ts):
+        ref = xs[k].double() @ t.double().T
+        bound = (t.shape[1] - 1) * 2.0 ** -24 * (xs[k].double().abs() @ t.double().abs().T)
+        ok &= bool(((ys[k].double() - ref).abs() <= bound).all())
+    stream_bytes = sum(sizes)
+    x_bytes = sum(x.numel() * 2 for x in xs)
+    y_bytes = sum(y.numel() * 4 for y in ys)
+    moved = stream_bytes + x_bytes + y_bytes  # algorithmic bytes of the launch
+    peak, peak_kind = hbm_peak()
+    clk = clocks.summary()
+    line = {
+        "metric": "fused decode+GEMV weights/s (effective BF16 GB/s)",
+        "value": world * 2 * weights / t_fused / 1e9, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * t_fused, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u16 weights, f32 accumulate", "data": "synthetic",
+        "config": {"workload": "gemv over %d linear weight matrices of the 8B-shaped stack "
+                               "(%d weights), n_vec=%d, block %d" % (len(mats), weights, nv, BLOCK),
+                   "l2": "weights larger than L2; no flush"},
+        "roofline": {"bound": "hbm", "achieved": moved / t_fused / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": moved / t_fused / 1e9 / peak, "peak_kind": peak_kind,
+                     "kernel": "gemv_kernel<256,%d> (one launch per step)" % nv,
+                     "algorithmic_bytes_per_launch": moved, "traffic": None},
+        "cublas_bf16": {"ms_per_step": 1e3 * t_blas,
+                        "achieved_gbs": (2 * weights + x_bytes + 2 * sum(o.numel() for o in outs))
+                        / t_blas / 1e9,
+                        "speedup_of_fused": t_blas / t_fused},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "verified_within_fp32_bound": ok,
+    }
+    del graph
+    if dist is not None:
+        barrier(dist, dev)
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0 if ok else 1
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("wcodec", "reference"), default="wcodec")
-    ap.add_argument("--workload", choices=("stack", "layer"), default="stack",
+    ap.add_argument("--workload", choices=("stack", "layer", "gemv"), default="stack",
                     help="stack: the 8B-shaped stack (the benchmark); layer: one decoder layer "
-                         "(a smaller case for profiling)")
+                         "(a smaller case for profiling); gemv: fused decode + matrix-vector "
+                         "products over the stack's linear weights")
+    ap.add_argument("--n-vec", type=int, default=1, choices=(1, 2, 4),
+                    help="activation vectors per product (gemv workload)")
+    ap.add_argument("--gemv-layers", type=int, default=None,
+                    help="gemv workload on the first K decoder layers only (a smaller case)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip timing the CPU oracle (for profiling runs)")
     ap.add_argument("--no-e2e", action="store_true",
@@ -502,6 +624,8 @@ def main(argv=None):
         log("note: fewer than 3 warm-up steps")
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "gemv":
+        return run_gemv(args)
     return run_wcodec(args)
 
 

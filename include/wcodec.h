@@ -219,6 +219,39 @@ int wc_decompress_batch(const wc_batch_item *h_items, uint32_t count,
                         int32_t *d_status, void *stream);
 
 /*
+ * Fused decompression and matrix-vector products: for j < n_vec,
+ *   y[j][r] = sum_c W[r][c] * x[j][c]
+ * where W (rows x cols, row-major BF16) is given only as its WCB1 stream
+ * (n = rows*cols, block size `block`): the weights are decoded on chip and
+ * never written to memory ("ZipServ: Fast and Memory-Efficient LLM Inference
+ * with Hardware-Aware Lossless Compression", Abstract: load compressed, compute
+ * decompressed). x is n_vec x cols BF16 (device, 16-byte aligned, row-major),
+ * y is n_vec x rows FP32 (device, 4-byte aligned, row-major); n_vec is 1, 2
+ * or 4; cols must be a multiple of `block`. Products of two BF16 values are
+ * exact in FP32 and are summed in FP32 in a fixed order, so the result is the
+ * same on every run; it differs from the exact sum by at most
+ * (cols-1) * 2^-24 * sum_c |W[r][c] * x[j][c]| (the standard bound of an FP32
+ * sum). The stream is checked as by wc_decompress (errors to *d_status).
+ */
+typedef struct {
+    const void *stream;
+    uint64_t stream_bytes;
+    const void *x;
+    float *y;
+    uint32_t rows, cols, block;
+    uint32_t reserved; /* must be 0 */
+} wc_gemv_item;
+
+int wc_gemv(const void *d_stream, uint64_t stream_bytes, uint32_t rows, uint32_t cols,
+            uint32_t block, const void *d_x, uint32_t n_vec, float *d_y,
+            int32_t *d_status, void *stream);
+
+/* wc_gemv over `count` independent matrices (one launch per 256); h_items is a
+ * HOST array passed as launch parameters. */
+int wc_gemv_batch(const wc_gemv_item *h_items, uint32_t count, uint32_t n_vec,
+                  int32_t *d_status, void *stream);
+
+/*
  * Parse a host copy of a stream's first `header_bytes` (>= 128) bytes. Fills
  * n, block and total_bytes (any may be NULL). Returns WC_ERR_CORRUPT_STREAM
  * if the header is not a WCB1 version-1 header consistent with itself.

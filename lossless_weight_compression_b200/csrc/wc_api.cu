@@ -215,6 +215,65 @@ int wc_decompress_batch(const wc_batch_item* h_items, uint32_t count, int32_t* d
     return WC_OK;
 }
 
+static int check_gemv_item(const wc_gemv_item& it, uint32_t n_vec) {
+    if (n_vec != 1 && n_vec != 2 && n_vec != 4) return WC_ERR_INVALID_ARG;
+    if (!wc::block_ok(it.block) || it.reserved != 0 || it.stream == nullptr ||
+        (it.rows > 0 && (it.x == nullptr || it.y == nullptr)) || it.cols == 0 ||
+        it.cols % it.block != 0 || uint64_t(it.rows) * it.cols > wc::kMaxElems)
+        return WC_ERR_INVALID_ARG;
+    if (!aligned16(it.stream) || !aligned16(it.x) || (reinterpret_cast<uintptr_t>(it.y) & 3u) != 0)
+        return WC_ERR_INVALID_ARG;
+    if (it.stream_bytes < wc::make_layout(uint64_t(it.rows) * it.cols, it.block).off_exp)
+        return WC_ERR_CORRUPT_STREAM;
+    return WC_OK;
+}
+
+static wc::GemvItem to_gemv_item(const wc_gemv_item& it) {
+    wc::GemvItem g;
+    g.stream = static_cast<const uint8_t*>(it.stream);
+    g.stream_bytes = it.stream_bytes;
+    g.x = static_cast<const uint16_t*>(it.x);
+    g.y = it.y;
+    g.rows = it.rows;
+    g.cols = it.cols;
+    g.block = it.block;
+    g.reserved = 0;
+    return g;
+}
+
+int wc_gemv(const void* d_stream, uint64_t stream_bytes, uint32_t rows, uint32_t cols,
+            uint32_t block, const void* d_x, uint32_t n_vec, float* d_y, int32_t* d_status,
+            void* stream) {
+    wc_gemv_item it;
+    it.stream = d_stream;
+    it.stream_bytes = stream_bytes;
+    it.x = d_x;
+    it.y = d_y;
+    it.rows = rows;
+    it.cols = cols;
+    it.block = block;
+    it.reserved = 0;
+    return wc_gemv_batch(&it, 1, n_vec, d_status, stream);
+}
+
+int wc_gemv_batch(const wc_gemv_item* h_items, uint32_t count, uint32_t n_vec, int32_t* d_status,
+                  void* stream) {
+    if (h_items == nullptr && count > 0) return WC_ERR_INVALID_ARG;
+    for (uint32_t i = 0; i < count; ++i) {  // check everything before launching anything
+        const int rc = check_gemv_item(h_items[i], n_vec);
+        if (rc != WC_OK) return rc;
+    }
+    wc::GemvItem chunk[256];
+    for (uint32_t base = 0; base < count; base += 256) {
+        const uint32_t c = (count - base < 256) ? count - base : 256;
+        for (uint32_t i = 0; i < c; ++i) chunk[i] = to_gemv_item(h_items[base + i]);
+        const cudaError_t err =
+            wc::launch_gemv(chunk, c, n_vec, d_status, static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return WC_ERR_CUDA;
+    }
+    return WC_OK;
+}
+
 int wc_stream_info(const void* h_header, uint64_t header_bytes, uint64_t* n, uint32_t* block,
                    uint64_t* total_bytes) {
     if (h_header == nullptr || header_bytes < WC_HEADER_BYTES) return WC_ERR_INVALID_ARG;

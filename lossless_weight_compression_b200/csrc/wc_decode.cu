@@ -32,7 +32,7 @@
 // launch parameters and the producer advances through them as its tiles do.
 #include <mutex>
 
-#include "wc_internal.cuh"
+#include "wc_decode_core.cuh"
 
 namespace wc {
 namespace {
@@ -77,66 +77,6 @@ struct DecodeSmem {
 };
 
 // ---------------------------------------------------------------------------
-// decoding of one octet
-// ---------------------------------------------------------------------------
-// 64 bits starting at byte q of the staged exponent bytes (q need not be aligned).
-__device__ __forceinline__ void fetch_octet(const uint32_t* s32, uint32_t q, uint32_t& lo,
-                                            uint32_t& hi) {
-    const uint32_t a = q >> 2, r = (q & 3u) * 8u;
-    const uint32_t x0 = s32[a], x1 = s32[a + 1], x2 = s32[a + 2];
-    lo = __funnelshift_r(x0, x1, r);
-    hi = __funnelshift_r(x1, x2, r);
-}
-
-// A pair (2w bits, v0 | v1 << w) -> both 16-bit lanes' exponent fields (base + v) << 7.
-__device__ __forceinline__ uint32_t pair_lanes(uint32_t p, uint32_t sh, uint32_t M1,
-                                               uint32_t base7) {
-    return ((p | (p << sh)) & M1) * 128u + base7;
-}
-
-// Octet (lo:hi, bits above 8w ignored) + 8 sign+mantissa bytes -> 8 BF16 words.
-//   quads: bits [0,4w) and [4w,8w); pairs: the halves of each quad.
-// A sign+mantissa byte replicated into both bytes of a lane and masked with
-// 0x807F leaves the mantissa in bits 0..6 and the sign in bit 15.
-__device__ __forceinline__ uint4 decode_octet(uint32_t lo, uint32_t hi, uint32_t s03,
-                                              uint32_t s47, uint32_t w2, uint32_t w4,
-                                              uint32_t sh, uint4 t1) {
-    const uint32_t M1 = t1.x, m2 = t1.y, m4 = t1.z, base7 = t1.w;
-    const uint32_t p0 = lo & m2;
-    const uint32_t p1 = __funnelshift_r(lo, hi, w2) & m2;
-    const uint32_t q1 = __funnelshift_rc(lo, hi, w4) & m4;
-    const uint32_t p2 = q1 & m2;
-    const uint32_t p3 = q1 >> w2;
-    uint4 r;
-    r.x = (prmt(s03, 0u, 0x1100u) & 0x807F807Fu) | pair_lanes(p0, sh, M1, base7);
-    r.y = (prmt(s03, 0u, 0x3322u) & 0x807F807Fu) | pair_lanes(p1, sh, M1, base7);
-    r.z = (prmt(s47, 0u, 0x1100u) & 0x807F807Fu) | pair_lanes(p2, sh, M1, base7);
-    r.w = (prmt(s47, 0u, 0x3322u) & 0x807F807Fu) | pair_lanes(p3, sh, M1, base7);
-    return r;
-}
-
-__device__ __forceinline__ uint64_t ld_u64(const uint8_t* p) {
-    return *reinterpret_cast<const uint64_t*>(p);
-}
-
-// The first tile of each tensor checks the container header against (n, B).
-__device__ void check_container(const DecodeItem& I, const Layout& L, int32_t* status) {
-    const uint8_t* S = I.stream;
-    bool bad = ld_u64(S) != (kMagic | (uint64_t(kVersion) << 32) | (uint64_t(kHeaderBytes) << 48));
-    bad |= ld_u64(S + 8) != uint64_t(L.block);  // block size, flags = 0
-    bad |= ld_u64(S + 16) != L.n;
-    bad |= ld_u64(S + 24) != L.nb;
-    bad |= ld_u64(S + 32) != L.off_hdr;
-    bad |= ld_u64(S + 40) != L.off_offs;
-    bad |= ld_u64(S + 48) != L.off_man;
-    bad |= ld_u64(S + 56) != L.off_exp;
-    const uint64_t E = ld_u64(S + 64), total = ld_u64(S + 72);
-    bad |= E > L.n + 8 || total != L.off_exp + E || total > I.stream_bytes;
-    for (int k = 80; k < 128; k += 8) bad |= ld_u64(S + k) != 0;
-    if (bad) report(status, kStatusCorrupt);
-}
-
-// ---------------------------------------------------------------------------
 // producer: one warp
 // ---------------------------------------------------------------------------
 template <int MAXI>
@@ -175,60 +115,12 @@ __device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem& sm, int lane) {
         uint64_t start = 0;
         bool bad = false;
         if (L.n > 0) {
-            const uint32_t log2B = L.log2_block, B = L.block;
             const uint64_t tile_start = lt * kTile;
             tile_n = uint32_t(min(uint64_t(kTile), L.n - tile_start));
-            const uint64_t b0 = tile_start >> log2B;
-            const uint32_t nblk = (tile_n + B - 1) >> log2B;
-            const uint8_t* S = I.stream;
-            const uint16_t* hdr = reinterpret_cast<const uint16_t*>(S + L.off_hdr) + b0;
-            const uint32_t* offs = reinterpret_cast<const uint32_t*>(S + L.off_offs) + b0;
-            // lanes own blocks lane and lane + 32 (a tile holds at most 64 blocks)
-            uint32_t h[2] = {0, 0};
-            uint64_t sb[2] = {0, 0}, nx[2] = {0, 0};
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const uint32_t b = lane + 32 * j;
-                if (b < nblk) {
-                    h[j] = hdr[b];
-                    sb[j] = 16ull * offs[b];
-                    nx[j] = (b + 1 < nblk || b0 + b + 1 < L.nb) ? 16ull * offs[b + 1]
-                                                                : ld_u64(S + 64);  // E
-                }
-            }
-            start = __shfl_sync(0xFFFFFFFFu, sb[0], 0);
-            const uint32_t last = nblk - 1;
-            const uint64_t end = __shfl_sync(0xFFFFFFFFu, last < 32 ? nx[0] : nx[1], last & 31);
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const uint32_t b = lane + 32 * j;
-                if (b < nblk) {
-                    const uint32_t w = h[j] >> 8, base = h[j] & 0xFFu;
-                    const uint32_t len = min(B, tile_n - b * B);
-                    bad |= w > 8u || (w == 8u && base != 0u);
-                    bad |= sb[j] + uint64_t((len + 7) >> 3) * min(w, 8u) != nx[j];
-                }
-            }
-            bad |= end > I.stream_bytes - L.off_exp;
-            bad = __any_sync(0xFFFFFFFFu, bad);
+            const TileMeta meta = load_tile_meta(I.stream, L, tile_start, tile_n, lane);
+            bad = !commit_tile_meta(meta, I.stream, L, I.stream_bytes, tile_n, st.t0, st.t1,
+                                    st.exp, start, len16, lane);
             if (!bad) {
-                // the offset chain holds, so end - start = the tile's payload <= kTile
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const uint32_t b = lane + 32 * j;
-                    if (b < nblk) {
-                        const uint32_t w = h[j] >> 8, base = h[j] & 0xFFu;
-                        const uint32_t m1 = (1u << w) - 1u;
-                        st.t0[b] = make_uint4(uint32_t(sb[j] - start), w, 2 * w, 4 * w);
-                        st.t1[b] = make_uint4(m1 | (m1 << 16), (1u << (2 * w)) - 1u,
-                                              w == 8u ? 0xFFFFFFFFu : (1u << (4 * w)) - 1u,
-                                              base * 0x00800080u);
-                    }
-                }
-                const uint32_t len = uint32_t(end - start);
-                len16 = len & ~15u;
-                const uint32_t rem = len - len16;  // only at the very end of a stream
-                if (lane < rem) st.exp[len16 + lane] = S[L.off_exp + start + len16 + lane];
                 man_bytes = (tile_n + 15u) & ~15u;  // inside the 128-byte padded plane
                 if (lane == 0)
                     st.info = StageInfo{I.out + tile_start, tile_n, L.log2_block};

@@ -245,6 +245,18 @@ cudaError_t launch_encode(const EncodeItem* items, uint32_t count, void* workspa
 cudaError_t launch_decode(const DecodeItem* items, uint32_t count, int32_t* status,
                           cudaStream_t stream);
 
+struct GemvItem {
+    const uint8_t* stream;  // WCB1 stream of W (rows x cols, row-major BF16)
+    uint64_t stream_bytes;
+    const uint16_t* x;      // n_vec x cols BF16
+    float* y;               // n_vec x rows FP32
+    uint32_t rows, cols, block, reserved;
+};
+
+// Fused decode + matrix-vector products for n_vec in {1, 2, 4} (wc_gemv.cu).
+cudaError_t launch_gemv(const GemvItem* items, uint32_t count, uint32_t n_vec, int32_t* status,
+                        cudaStream_t stream);
+
 // The allocation-free encoder's fixed scratch array (wc_encode.cu).
 uint64_t noalloc_max_elems();
 cudaError_t noalloc_scratch(void** ptr, uint64_t* bytes);

@@ -49,6 +49,19 @@ class wc_compress_item(ctypes.Structure):
     ]
 
 
+class wc_gemv_item(ctypes.Structure):
+    _fields_ = [
+        ("stream", ctypes.c_void_p),
+        ("stream_bytes", ctypes.c_uint64),
+        ("x", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+        ("rows", ctypes.c_uint32),
+        ("cols", ctypes.c_uint32),
+        ("block", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32),
+    ]
+
+
 class wc_batch_item(ctypes.Structure):
     _fields_ = [
         ("stream", ctypes.c_void_p),
@@ -90,6 +103,10 @@ def lib() -> ctypes.CDLL:
     L.wc_compress_batch_workspace_size.restype = u64
     L.wc_compress_batch.argtypes = [ctypes.POINTER(wc_compress_item), u32, vp, u64, vp, vp]
     L.wc_compress_batch.restype = i
+    L.wc_gemv.argtypes = [vp, u64, u32, u32, u32, vp, u32, vp, vp, vp]
+    L.wc_gemv.restype = i
+    L.wc_gemv_batch.argtypes = [ctypes.POINTER(wc_gemv_item), u32, u32, vp, vp]
+    L.wc_gemv_batch.restype = i
     L.wc_compress_noalloc.argtypes = [vp, u64, u32, vp, u64, vp, vp, vp]
     L.wc_compress_noalloc.restype = i
     L.wc_debug_compress_stalled.argtypes = [vp, u64, u32, vp, u64, vp, vp, u64, vp, u64, vp]
@@ -137,6 +154,15 @@ def wc_decompress(d_stream, stream_bytes, d_out, n, block, d_status, stream) -> 
 
 def wc_decompress_batch(items, count, d_status, stream) -> int:
     return lib().wc_decompress_batch(items, count, d_status, stream)
+
+
+def wc_gemv(d_stream, stream_bytes, rows, cols, block, d_x, n_vec, d_y, d_status, stream) -> int:
+    return lib().wc_gemv(d_stream, stream_bytes, rows, cols, block, d_x, n_vec, d_y, d_status,
+                         stream)
+
+
+def wc_gemv_batch(items, count, n_vec, d_status, stream) -> int:
+    return lib().wc_gemv_batch(items, count, n_vec, d_status, stream)
 
 
 def wc_stream_info(h_header: bytes):
@@ -319,3 +345,40 @@ def stream_info(header: bytes):
     rc, n, block, total = wc_stream_info(header)
     _check(rc, "wc_stream_info")
     return n, block, total
+
+
+def gemv(stream_bytes: torch.Tensor, rows: int, cols: int, block: int, x: torch.Tensor, *,
+         nbytes: int | None = None, y: torch.Tensor | None = None,
+         status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = x @ W.T with W (rows x cols BF16) given as its stream; x is (n_vec, cols)
+    with n_vec in {1, 2, 4}; returns FP32 (n_vec, rows)."""
+    xw = as_words(x).view(-1, cols)
+    n_vec = xw.shape[0]
+    if y is None:
+        y = torch.empty((n_vec, rows), dtype=torch.float32, device=stream_bytes.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=stream_bytes.device)
+    rc = wc_gemv(stream_bytes.data_ptr(), stream_bytes.numel() if nbytes is None else nbytes,
+                 rows, cols, block, xw.data_ptr(), n_vec, y.data_ptr(), status.data_ptr(),
+                 _stream_handle(stream))
+    _check(rc, "wc_gemv")
+    return y
+
+
+def make_gemv_batch(items) -> tuple:
+    """items: iterable of (stream uint8 tensor, stream_bytes, x (n_vec, cols), y (n_vec, rows), rows, cols, block)."""
+    items = list(items)
+    arr = (wc_gemv_item * max(1, len(items)))()
+    for k, (s, sb, x, y, rows, cols, b) in enumerate(items):
+        arr[k].stream = s.data_ptr()
+        arr[k].stream_bytes = sb
+        arr[k].x = x.data_ptr()
+        arr[k].y = y.data_ptr()
+        arr[k].rows, arr[k].cols, arr[k].block, arr[k].reserved = rows, cols, b, 0
+    return arr, len(items)
+
+
+def gemv_batch(batch, n_vec: int, status: torch.Tensor, stream=None):
+    arr, count = batch
+    rc = wc_gemv_batch(arr, count, n_vec, status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_gemv_batch")

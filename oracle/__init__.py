@@ -141,3 +141,21 @@ def decompress(stream: np.ndarray, n: int, block: int) -> np.ndarray:
     if rc != OK:
         raise ValueError("oracle_decompress failed with status %d" % rc)
     return out
+
+
+# --- fused decode + matrix-vector products (GEMV) -----------------------------
+def bf16_to_f64(words: np.ndarray) -> np.ndarray:
+    """BF16 bit patterns -> float64 values (a BF16 is the top half of an FP32)."""
+    return (np.asarray(words, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def gemv(stream: np.ndarray, rows: int, cols: int, block: int, x_words: np.ndarray):
+    """y[j][r] = sum_c W[r][c] * x[j][c] in float64, W decoded from the stream by the
+    C oracle; also returns sum_c |W[r][c] * x[j][c]| for the error bound. The
+    definition written out: decode, then one float64 matrix product."""
+    W = bf16_to_f64(decompress(stream, rows * cols, block)).reshape(rows, cols)
+    x = bf16_to_f64(np.asarray(x_words, dtype=np.uint16).reshape(-1, cols))
+    with np.errstate(invalid="ignore", over="ignore"):
+        y = x @ W.T
+        absum = np.abs(x) @ np.abs(W).T
+    return y, absum

@@ -27,7 +27,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for f in ("wc_bound", "wc_workspace_size", "wc_compress", "wc_decompress",
               "wc_compress_batch", "wc_compress_batch_workspace_size",
-              "wc_decompress_batch", "wc_stream_info", "wc_status_string",
+              "wc_decompress_batch", "wc_stream_info", "wc_status_string", "wc_gemv",
+              "wc_gemv_batch",
               "wc_debug_compress_stalled"):
         assert f in names
 
@@ -121,6 +122,11 @@ def test_argument_checks_before_any_launch(wclib):
     assert c.wc_compress_batch(citems, 2, 16, 8, None, None) == c.WC_ERR_BUFFER_TOO_SMALL
     citems[1].out_capacity = 10
     assert c.wc_compress_batch(citems, 2, 16, 10**6, None, None) == c.WC_ERR_BUFFER_TOO_SMALL
+    # fused decode-GEMV: shapes and vector counts are checked on the host
+    assert c.wc_gemv(16, 10**6, 4, 1000, 128, 16, 1, 16, None, None) == c.WC_ERR_INVALID_ARG  # cols % B
+    assert c.wc_gemv(16, 10**6, 4, 1024, 128, 16, 3, 16, None, None) == c.WC_ERR_INVALID_ARG  # n_vec
+    assert c.wc_gemv(16, 10**6, 4, 1024, 128, 17, 1, 16, None, None) == c.WC_ERR_INVALID_ARG  # x align
+    assert c.wc_gemv(16, 100, 4, 1024, 128, 16, 1, 16, None, None) == c.WC_ERR_CORRUPT_STREAM
     # the stall test hook needs two tiles and a bounded timeout
     assert c.wc_debug_compress_stalled(16, 100, 128, 16, 10**6, 16, 16, 10**6, None, 10**6,
                                        None) == c.WC_ERR_INVALID_ARG
