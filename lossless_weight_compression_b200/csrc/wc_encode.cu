@@ -45,11 +45,11 @@ namespace {
 
 constexpr int kWorkerWarps = kThreads / 32;  // 8
 constexpr int kProducerWarp = kWorkerWarps;
-constexpr int kStoreWarps = 4;                // tile i goes to store warp i % 4
+constexpr int kStoreWarps = 2;                // tile i goes to store warp i % 2
 constexpr int kFirstStoreWarp = kWorkerWarps + 1;
-constexpr int kEncodeThreads = kThreads + 32 + 32 * kStoreWarps;  // 416
-constexpr int kInStages = 4;
-constexpr int kOutStages = 5;
+constexpr int kEncodeThreads = kThreads + 32 + 32 * kStoreWarps;  // 352
+constexpr int kInStages = 2;
+constexpr int kOutStages = 4;
 constexpr int kWindowRows = 8;  // look-back window: 8 x 32 tiles per round trip
 
 constexpr unsigned long long kFlagAggregate = 1ull << 62;  // value = this tile's bytes
@@ -97,7 +97,7 @@ struct EncodeSmem {
     OutStage out[kOutStages];
     unsigned long long in_full[kInStages], in_empty[kInStages];
     unsigned long long out_full[kOutStages], out_empty[kOutStages];
-    int lo[2][kMaxBlocksPerTile], hi[2][kMaxBlocksPerTile];  // per-block min/max, by tile parity
+    int lo[3][kMaxBlocksPerTile], hi[3][kMaxBlocksPerTile];  // per-block min/max, tile i uses i % 3
     int abort;        // some warp gave up: every wait of the block stops
     int worker_stop;  // written by workers only, before their agreement barrier
 };
@@ -230,9 +230,9 @@ __device__ __forceinline__ uint32_t find_item(const EncodeParams<MAXI>& P, uint6
 }
 
 // The 8 worker warps meet on hardware barrier 1 (the other warps never use
-// it). A worker never leaves its loop between two of these barriers: the only
-// waits that can fail come first in an iteration, and the warps agree on the
-// outcome at the first barrier of that iteration.
+// it), once per tile. Every worker reaches it on every path through an
+// iteration -- a failed wait or the end of the work included -- and only then
+// decides to leave, so no worker can wait there for one that has left.
 __device__ __forceinline__ void workers_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
 }
@@ -310,37 +310,34 @@ __device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem& sm, int tid
     for (uint32_t i = 0;; ++i) {
         const int s = int(i % kInStages), o = int(i % kOutStages);
         const uint32_t rin = i / kInStages, rout = i / kOutStages;
-        if (!mbar_wait(&sm.in_full[s], rin & 1u, &sm.abort) ||
-            (rout > 0 && !mbar_wait(&sm.out_empty[o], (rout & 1u) ^ 1u, &sm.abort))) {
+        const bool ok = mbar_wait(&sm.in_full[s], rin & 1u, &sm.abort) &&
+                        (rout == 0 || mbar_wait(&sm.out_empty[o], (rout & 1u) ^ 1u, &sm.abort));
+        if (!ok) {
             give_up(sm, P.status, lane);
             if (lane == 0) sm.worker_stop = 1;
         }
-        // Agree: either every worker goes on or every worker stops. worker_stop
-        // is only ever written above, before this barrier, so all read the same.
-        workers_sync();
-        if (sm.worker_stop) return;
         const InStage& in = sm.in[s];
         OutStage& out = sm.out[o];
-        const InInfo info = in.info;
-        int* lo_of = sm.lo[i & 1];
-        int* hi_of = sm.hi[i & 1];
-        if (info.end) {  // pass the end on to every store warp (the next 4 stages)
+        InInfo info = in.info;
+        if (!ok) info.end = 0, info.tile_n = 0;
+        int* lo_of = sm.lo[i % 3];
+        int* hi_of = sm.hi[i % 3];
+        if (info.end) {  // pass the end on to every store warp (the next kStoreWarps stages)
             for (uint32_t q = 0; q < kStoreWarps; ++q) {
                 const uint32_t iq = i + q;
                 const int oq = int(iq % kOutStages);
                 const uint32_t rq = iq / kOutStages;
                 if (q > 0 && rq > 0 && !mbar_wait(&sm.out_empty[oq], (rq & 1u) ^ 1u, &sm.abort)) {
                     give_up(sm, P.status, lane);
-                    return;
+                    break;
                 }
                 if (tid == 0) sm.out[oq].info.end = 1;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.out_full[oq]);
             }
-            return;
         }
         const EncodeItem& I = P.item[info.item];
-        const uint32_t B = I.block, log2B = log2_of(B), tile_n = info.tile_n;
+        const uint32_t B = I.block, log2B = log2_of(B), tile_n = info.end ? 0u : info.tile_n;
         const uint32_t group = min(B / kChunk, 32u);  // chunks of one block inside a warp
         const uint64_t man_base = info.man_off;
 
@@ -373,7 +370,7 @@ __device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem& sm, int tid
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.in_empty[s]);
+        if (ok && !info.end && lane == 0) mbar_arrive(&sm.in_empty[s]);
 
         // ---- split: mantissa bytes to global memory, exponents kept; per-block min/max
         // The exponent is the top byte of a word's 15-bit magnitude, so the
@@ -422,7 +419,11 @@ __device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem& sm, int tid
                 atomicMax(&hi_of[el >> log2B], int(hi));
             }
         }
-        workers_sync();  // all per-block min/max are in
+        // The one barrier of the tile: all per-block min/max are in, and the workers
+        // agree whether to go on. worker_stop is written only before this barrier
+        // and every worker reaches it on every path, so all read the same value.
+        workers_sync();
+        if (sm.worker_stop || info.end) return;
 
         // ---- every worker warp: widths, sizes and the tile-local scan (each warp
         //      needs the offsets of its own blocks; computing them in every warp
@@ -463,11 +464,13 @@ __device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem& sm, int tid
                 store_state(&P.state[info.t], (info.lt == 0 ? kFlagPrefix : kFlagAggregate) | total);
             }
         }
-        // the other parity's min/max were read by every warp in the previous tile,
-        // before this tile's first barrier: reset them for the next tile
+        // Tile i - 1's min/max (buffer (i + 2) % 3) were read by every warp before
+        // this tile's barrier; reset them now. The next tile to use that buffer,
+        // i + 2, adds to it only after the barrier of tile i + 1, which this warp
+        // reaches after the reset.
         if (warp == 1) {
-            int* lo_next = sm.lo[(i + 1) & 1];
-            int* hi_next = sm.hi[(i + 1) & 1];
+            int* lo_next = sm.lo[(i + 2) % 3];
+            int* hi_next = sm.hi[(i + 2) % 3];
             lo_next[lane] = 255;
             lo_next[lane + 32] = 255;
             hi_next[lane] = 0;
@@ -668,7 +671,7 @@ __device__ void encode_store(const EncodeParams<MAXI>& P, EncodeSmem& sm, int la
 }
 
 template <int MAXI>
-__global__ void __launch_bounds__(kEncodeThreads)
+__global__ void __launch_bounds__(kEncodeThreads, 3)
     encode_kernel(const __grid_constant__ EncodeParams<MAXI> P) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     EncodeSmem& sm = *reinterpret_cast<EncodeSmem*>(smem_raw);
@@ -686,7 +689,7 @@ __global__ void __launch_bounds__(kEncodeThreads)
         sm.worker_stop = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (tid < 2 * kMaxBlocksPerTile) {
+    if (tid < 3 * kMaxBlocksPerTile) {
         sm.lo[tid >> 6][tid & 63] = 255;
         sm.hi[tid >> 6][tid & 63] = 0;
     }
