@@ -479,9 +479,39 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
     sec = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, dev)
     ok = status_host.item() == 0 and all(torch.equal(a, b) for a, b in zip(inputs, outs))
     world = dist.get_world_size() if dist is not None else 1
-    return {"value": whole_job_gbs(world, 2 * n_total, steps, sec), "unit": "GB/s",
-            "h2d_bytes_per_step": total, "d2h_bytes_per_step": 4, "steps": steps,
-            "verified_bit_exact": bool(ok)}
+    result = {"value": whole_job_gbs(world, 2 * n_total, steps, sec), "unit": "GB/s",
+              "h2d_bytes_per_step": total, "d2h_bytes_per_step": 4, "steps": steps,
+              "verified_bit_exact": bool(ok)}
+    del host, views
+    # context: the same weights moved uncompressed (BF16, pinned host -> device), no decode
+    try:
+        raw = torch.empty(2 * n_total, dtype=torch.uint8, pin_memory=True)
+    except RuntimeError:
+        return result
+    raw_views, off = [], 0
+    for w in inputs:
+        nbytes = 2 * w.numel()
+        raw_views.append(raw[off:off + nbytes])
+        raw_views[-1].copy_(w.view(torch.uint8))
+        off += nbytes
+
+    def raw_step():
+        for k, w in enumerate(inputs):
+            outs[k].view(torch.uint8).copy_(raw_views[k], non_blocking=True)
+
+    raw_step()
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    e0.record(stream)
+    for _ in range(steps):
+        raw_step()
+    e1.record(stream)
+    barrier(dist, dev)
+    raw_sec = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, dev)
+    result["bf16_h2d_only"] = {"value": whole_job_gbs(world, 2 * n_total, steps, raw_sec),
+                               "unit": "GB/s", "h2d_bytes_per_step": 2 * n_total,
+                               "speedup_of_compressed_path": raw_sec / sec}
+    return result
 
 
 # ---------------------------------------------------------------------------

@@ -166,7 +166,6 @@ __device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem& sm, int tid, in
         }
         const Stage& st = sm.stage[s];
         const StageInfo info = st.info;
-        const uint32_t* s32 = reinterpret_cast<const uint32_t*>(st.exp);
         const uint32_t bmask = (1u << info.log2B) - 1u;
 #pragma unroll
         for (int k = 0; k < kChunksPerThread; ++k) {
@@ -175,13 +174,9 @@ __device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem& sm, int tid, in
             const uint4 M = *reinterpret_cast<const uint4*>(st.man + el);
             const uint32_t bl = el >> info.log2B;
             const uint4 t0 = st.t0[bl], t1 = st.t1[bl];
-            const uint32_t w = t0.y, sh = 16u - w;
-            const uint32_t q = t0.x + ((el & bmask) >> 3) * w;
-            uint32_t lo0, hi0, lo1, hi1;
-            fetch_octet(s32, q, lo0, hi0);
-            fetch_octet(s32, q + w, lo1, hi1);
-            const uint4 r0 = decode_octet(lo0, hi0, M.x, M.y, t0.z, t0.w, sh, t1);
-            const uint4 r1 = decode_octet(lo1, hi1, M.z, M.w, t0.z, t0.w, sh, t1);
+            const uint32_t q = t0.x + ((el & bmask) >> 3) * t0.y;
+            uint4 r0, r1;
+            decode_chunk(st.exp, q, M, t0, t1, r0, r1);
             uint16_t* dst = info.out + el;
             if (info.tile_n - el >= kChunk) {
                 st_stream_v4(dst, r0);

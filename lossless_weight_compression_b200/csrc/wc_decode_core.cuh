@@ -45,6 +45,45 @@ __device__ __forceinline__ uint4 decode_octet(uint32_t lo, uint32_t hi, uint32_t
     return r;
 }
 
+// The common case w = 4, as one chunk of 16 elements: its two octets are the 8
+// bytes at q (8-byte aligned: q = payload offset + 4 * (element offset in the
+// block / 8)), element t in nibble t. Low nibbles give the even elements, high
+// nibbles the odd ones; a byte permute then places elements 2k and 2k+1 in
+// the two 16-bit lanes of a word, using the permute's sign-replicating
+// selectors on bytes below 0x80 as zero bytes. Same result as decode_octet.
+__device__ __forceinline__ void decode_chunk_w4(const uint8_t* exp_stage, uint32_t q, uint4 M,
+                                                uint32_t base7, uint4& r0, uint4& r1) {
+    const uint2 F = *reinterpret_cast<const uint2*>(exp_stage + q);
+    const uint32_t e0 = F.x & 0x0F0F0F0Fu, o0 = (F.x >> 4) & 0x0F0F0F0Fu;  // elements 0..7
+    const uint32_t e1 = F.y & 0x0F0F0F0Fu, o1 = (F.y >> 4) & 0x0F0F0F0Fu;  // elements 8..15
+    r0.x = (prmt(M.x, 0u, 0x1100u) & 0x807F807Fu) | (prmt(e0, o0, 0xC480u) * 128u + base7);
+    r0.y = (prmt(M.x, 0u, 0x3322u) & 0x807F807Fu) | (prmt(e0, o0, 0xD591u) * 128u + base7);
+    r0.z = (prmt(M.y, 0u, 0x1100u) & 0x807F807Fu) | (prmt(e0, o0, 0xE6A2u) * 128u + base7);
+    r0.w = (prmt(M.y, 0u, 0x3322u) & 0x807F807Fu) | (prmt(e0, o0, 0xF7B3u) * 128u + base7);
+    r1.x = (prmt(M.z, 0u, 0x1100u) & 0x807F807Fu) | (prmt(e1, o1, 0xC480u) * 128u + base7);
+    r1.y = (prmt(M.z, 0u, 0x3322u) & 0x807F807Fu) | (prmt(e1, o1, 0xD591u) * 128u + base7);
+    r1.z = (prmt(M.w, 0u, 0x1100u) & 0x807F807Fu) | (prmt(e1, o1, 0xE6A2u) * 128u + base7);
+    r1.w = (prmt(M.w, 0u, 0x3322u) & 0x807F807Fu) | (prmt(e1, o1, 0xF7B3u) * 128u + base7);
+}
+
+// One chunk of 16 elements at any width: the w = 4 path above, else two octets
+// through decode_octet.
+__device__ __forceinline__ void decode_chunk(const uint8_t* exp_stage, uint32_t q, uint4 M,
+                                            uint4 t0, uint4 t1, uint4& r0, uint4& r1) {
+    const uint32_t w = t0.y;
+    if (w == 4u) {
+        decode_chunk_w4(exp_stage, q, M, t1.w, r0, r1);
+    } else {
+        const uint32_t* s32 = reinterpret_cast<const uint32_t*>(exp_stage);
+        const uint32_t sh = 16u - w;
+        uint32_t lo0, hi0, lo1, hi1;
+        fetch_octet(s32, q, lo0, hi0);
+        fetch_octet(s32, q + w, lo1, hi1);
+        r0 = decode_octet(lo0, hi0, M.x, M.y, t0.z, t0.w, sh, t1);
+        r1 = decode_octet(lo1, hi1, M.z, M.w, t0.z, t0.w, sh, t1);
+    }
+}
+
 __device__ __forceinline__ uint64_t ld_u64(const uint8_t* p) {
     return *reinterpret_cast<const uint64_t*>(p);
 }

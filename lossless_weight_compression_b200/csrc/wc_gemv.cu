@@ -255,7 +255,6 @@ __device__ void gemv_consume(GemvSmem<NV>& sm, int32_t* status, int tid, int lan
         const GemvStage& st = sm.stage[s];
         const GemvInfo info = st.info;
         if (info.nrows == 0) return;
-        const uint32_t* s32 = reinterpret_cast<const uint32_t*>(st.exp);
         const uint32_t bmask = (1u << info.log2B) - 1u;
 #pragma unroll
         for (int k = 0; k < kChunksPerThread; ++k) {
@@ -263,13 +262,9 @@ __device__ void gemv_consume(GemvSmem<NV>& sm, int32_t* status, int tid, int lan
             if (el >= info.len) continue;
             const uint4 M = *reinterpret_cast<const uint4*>(st.man + el);
             const uint4 t0 = st.t0[el >> info.log2B], t1 = st.t1[el >> info.log2B];
-            const uint32_t w = t0.y, sh = 16u - w;
-            const uint32_t q = t0.x + ((el & bmask) >> 3) * w;
-            uint32_t lo0, hi0, lo1, hi1;
-            fetch_octet(s32, q, lo0, hi0);
-            fetch_octet(s32, q + w, lo1, hi1);
-            const uint4 w0 = decode_octet(lo0, hi0, M.x, M.y, t0.z, t0.w, sh, t1);
-            const uint4 w1 = decode_octet(lo1, hi1, M.z, M.w, t0.z, t0.w, sh, t1);
+            const uint32_t q = t0.x + ((el & bmask) >> 3) * t0.y;
+            uint4 w0, w1;
+            decode_chunk(st.exp, q, M, t0, t1, w0, w1);
             const uint32_t row = __umulhi(el, info.magic);  // el / cols
             const uint32_t col = el - row * info.cols;
 #pragma unroll
