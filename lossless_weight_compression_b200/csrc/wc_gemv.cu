@@ -12,7 +12,7 @@
 // block metadata (loading the next tile's while the current one is staged) and
 // bulk-copies its mantissa bytes and exponent payload into a 3-stage mbarrier
 // ring; eight consumer warps decode 16 weights per chunk and accumulate
-// products in FP32. cols must be a multiple of the block size, so every row is
+// products in FP32 with mixed-precision FMAs (BF16 x BF16 + FP32). cols must be a multiple of the block size, so every row is
 // whole blocks. Work is cut into units a thread block owns whole: for
 // cols <= 8192 a unit is one tile of floor(8192 / cols) rows, for wider rows a
 // unit is one row, cut into tiles of up to 8192 weights. When a unit ends,
@@ -213,19 +213,25 @@ __device__ void gemv_produce(const GemvParams<MAXI>& P, GemvSmem<NV>& sm, int la
 // ---------------------------------------------------------------------------
 // consumer warps
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float lo_f32(uint32_t pair) { return __uint_as_float(pair << 16); }
-__device__ __forceinline__ float hi_f32(uint32_t pair) { return __uint_as_float(pair & 0xFFFF0000u); }
+// acc + a * b for two BF16 values and an FP32 accumulator, one rounding (the
+// product of two BF16 values is exact in FP32).
+__device__ __forceinline__ float fma_bf16(uint32_t a, uint32_t b, float acc) {
+    float d;
+    asm("fma.rn.f32.bf16 %0, %1, %2, %3;" : "=f"(d) : "h"(uint16_t(a)), "h"(uint16_t(b)), "f"(acc));
+    return d;
+}
 
-// acc + sum over 8 weights (4 BF16 pairs in w) times 8 x values (4 pairs in v)
+// acc + sum over 8 weights (4 BF16 pairs in w) times 8 x values (4 pairs in v),
+// in element order.
 __device__ __forceinline__ float dot8(uint4 w, uint4 v, float acc) {
-    acc = fmaf(lo_f32(w.x), lo_f32(v.x), acc);
-    acc = fmaf(hi_f32(w.x), hi_f32(v.x), acc);
-    acc = fmaf(lo_f32(w.y), lo_f32(v.y), acc);
-    acc = fmaf(hi_f32(w.y), hi_f32(v.y), acc);
-    acc = fmaf(lo_f32(w.z), lo_f32(v.z), acc);
-    acc = fmaf(hi_f32(w.z), hi_f32(v.z), acc);
-    acc = fmaf(lo_f32(w.w), lo_f32(v.w), acc);
-    acc = fmaf(hi_f32(w.w), hi_f32(v.w), acc);
+    acc = fma_bf16(w.x, v.x, acc);
+    acc = fma_bf16(w.x >> 16, v.x >> 16, acc);
+    acc = fma_bf16(w.y, v.y, acc);
+    acc = fma_bf16(w.y >> 16, v.y >> 16, acc);
+    acc = fma_bf16(w.z, v.z, acc);
+    acc = fma_bf16(w.z >> 16, v.z >> 16, acc);
+    acc = fma_bf16(w.w, v.w, acc);
+    acc = fma_bf16(w.w >> 16, v.w >> 16, acc);
     return acc;
 }
 
