@@ -252,6 +252,36 @@ int wc_gemv_batch(const wc_gemv_item *h_items, uint32_t count, uint32_t n_vec,
                   int32_t *d_status, void *stream);
 
 /*
+ * Fused decompression and matrix products on the tensor cores: for t < tokens,
+ *   y[t][r] = sum_c W[r][c] * x[t][c]
+ * with W (rows x cols, row-major BF16) given only as its WCB1 stream, as for
+ * wc_gemv; the decoded weights go from shared memory straight into tcgen05
+ * tensor-core MMAs (BF16 x BF16 -> FP32) and never reach device memory
+ * ("ZipServ: Fast and Memory-Efficient LLM Inference with Hardware-Aware
+ * Lossless Compression", Abstract: decompression fused into the GEMM). x is
+ * tokens x cols BF16 (device, 16-byte aligned, row-major), y is tokens x rows
+ * FP32 (device, 4-byte aligned, row-major); 1 <= tokens <= WC_GEMM_MAX_TOKENS;
+ * cols must be a multiple of 128 (any valid block size). The summation order
+ * is fixed, so y is the same on every run. The tensor cores' FP32 accumulation
+ * is not specified to round to nearest; every output is within
+ * cols * 2^-22 * sum_c |W[r][c] * x[t][c]| of the exact sum. The stream is
+ * checked as by wc_decompress (errors to *d_status); a stream shorter than its
+ * planes (stream_bytes below the exponent-plane offset) returns
+ * WC_ERR_CORRUPT_STREAM without launching. Suited to 16..128 tokens; for 1, 2
+ * or 4 vectors wc_gemv is faster.
+ */
+#define WC_GEMM_MAX_TOKENS 128u
+int wc_gemm(const void *d_stream, uint64_t stream_bytes, uint32_t rows, uint32_t cols,
+            uint32_t block, const void *d_x, uint32_t tokens, float *d_y,
+            int32_t *d_status, void *stream);
+
+/* wc_gemm over `count` independent matrices sharing one token count (one
+ * launch per 64 matrices); h_items is a HOST array passed as launch
+ * parameters, its x and y hold `tokens` rows each. */
+int wc_gemm_batch(const wc_gemv_item *h_items, uint32_t count, uint32_t tokens,
+                  int32_t *d_status, void *stream);
+
+/*
  * Parse a host copy of a stream's first `header_bytes` (>= 128) bytes. Fills
  * n, block and total_bytes (any may be NULL). Returns WC_ERR_CORRUPT_STREAM
  * if the header is not a WCB1 version-1 header consistent with itself.

@@ -274,6 +274,53 @@ int wc_gemv_batch(const wc_gemv_item* h_items, uint32_t count, uint32_t n_vec, i
     return WC_OK;
 }
 
+static int check_gemm_item(const wc_gemv_item& it, uint32_t tokens) {
+    if (tokens < 1 || tokens > WC_GEMM_MAX_TOKENS) return WC_ERR_INVALID_ARG;
+    if (!wc::block_ok(it.block) || it.reserved != 0 || it.stream == nullptr ||
+        (it.rows > 0 && (it.x == nullptr || it.y == nullptr)) || it.cols == 0 ||
+        it.cols % 128u != 0 || uint64_t(it.rows) * it.cols > wc::kMaxElems)
+        return WC_ERR_INVALID_ARG;
+    if (!aligned16(it.stream) || !aligned16(it.x) || (reinterpret_cast<uintptr_t>(it.y) & 3u) != 0)
+        return WC_ERR_INVALID_ARG;
+    if (it.stream_bytes < wc::make_layout(uint64_t(it.rows) * it.cols, it.block).off_exp)
+        return WC_ERR_CORRUPT_STREAM;
+    return WC_OK;
+}
+
+int wc_gemm(const void* d_stream, uint64_t stream_bytes, uint32_t rows, uint32_t cols,
+            uint32_t block, const void* d_x, uint32_t tokens, float* d_y, int32_t* d_status,
+            void* stream) {
+    wc_gemv_item it;
+    it.stream = d_stream;
+    it.stream_bytes = stream_bytes;
+    it.x = d_x;
+    it.y = d_y;
+    it.rows = rows;
+    it.cols = cols;
+    it.block = block;
+    it.reserved = 0;
+    return wc_gemm_batch(&it, 1, tokens, d_status, stream);
+}
+
+int wc_gemm_batch(const wc_gemv_item* h_items, uint32_t count, uint32_t tokens, int32_t* d_status,
+                  void* stream) {
+    if (h_items == nullptr && count > 0) return WC_ERR_INVALID_ARG;
+    for (uint32_t i = 0; i < count; ++i) {  // check everything before launching anything
+        const int rc = check_gemm_item(h_items[i], tokens);
+        if (rc != WC_OK) return rc;
+    }
+    constexpr uint32_t kChunk = wc::kGemmBatchMax;
+    wc::GemvItem chunk[kChunk];
+    for (uint32_t base = 0; base < count; base += kChunk) {
+        const uint32_t c = (count - base < kChunk) ? count - base : kChunk;
+        for (uint32_t i = 0; i < c; ++i) chunk[i] = to_gemv_item(h_items[base + i]);
+        const cudaError_t err =
+            wc::launch_gemm(chunk, c, tokens, d_status, static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return WC_ERR_CUDA;
+    }
+    return WC_OK;
+}
+
 int wc_stream_info(const void* h_header, uint64_t header_bytes, uint64_t* n, uint32_t* block,
                    uint64_t* total_bytes) {
     if (h_header == nullptr || header_bytes < WC_HEADER_BYTES) return WC_ERR_INVALID_ARG;

@@ -257,6 +257,13 @@ struct GemvItem {
 cudaError_t launch_gemv(const GemvItem* items, uint32_t count, uint32_t n_vec, int32_t* status,
                         cudaStream_t stream);
 
+// Fused decode + matrix products on the tensor cores for 1..kMaxGemmTokens
+// activation rows (wc_gemm.cu); one launch per kGemmBatchMax matrices.
+constexpr uint32_t kMaxGemmTokens = 128;
+constexpr uint32_t kGemmBatchMax = 64;
+cudaError_t launch_gemm(const GemvItem* items, uint32_t count, uint32_t tokens, int32_t* status,
+                        cudaStream_t stream);
+
 // The allocation-free encoder's fixed scratch array (wc_encode.cu).
 uint64_t noalloc_max_elems();
 cudaError_t noalloc_scratch(void** ptr, uint64_t* bytes);

@@ -107,6 +107,10 @@ def lib() -> ctypes.CDLL:
     L.wc_gemv.restype = i
     L.wc_gemv_batch.argtypes = [ctypes.POINTER(wc_gemv_item), u32, u32, vp, vp]
     L.wc_gemv_batch.restype = i
+    L.wc_gemm.argtypes = [vp, u64, u32, u32, u32, vp, u32, vp, vp, vp]
+    L.wc_gemm.restype = i
+    L.wc_gemm_batch.argtypes = [ctypes.POINTER(wc_gemv_item), u32, u32, vp, vp]
+    L.wc_gemm_batch.restype = i
     L.wc_compress_noalloc.argtypes = [vp, u64, u32, vp, u64, vp, vp, vp]
     L.wc_compress_noalloc.restype = i
     L.wc_debug_compress_stalled.argtypes = [vp, u64, u32, vp, u64, vp, vp, u64, vp, u64, vp]
@@ -163,6 +167,15 @@ def wc_gemv(d_stream, stream_bytes, rows, cols, block, d_x, n_vec, d_y, d_status
 
 def wc_gemv_batch(items, count, n_vec, d_status, stream) -> int:
     return lib().wc_gemv_batch(items, count, n_vec, d_status, stream)
+
+
+def wc_gemm(d_stream, stream_bytes, rows, cols, block, d_x, tokens, d_y, d_status, stream) -> int:
+    return lib().wc_gemm(d_stream, stream_bytes, rows, cols, block, d_x, tokens, d_y, d_status,
+                         stream)
+
+
+def wc_gemm_batch(items, count, tokens, d_status, stream) -> int:
+    return lib().wc_gemm_batch(items, count, tokens, d_status, stream)
 
 
 def wc_stream_info(h_header: bytes):
@@ -382,3 +395,31 @@ def gemv_batch(batch, n_vec: int, status: torch.Tensor, stream=None):
     arr, count = batch
     rc = wc_gemv_batch(arr, count, n_vec, status.data_ptr(), _stream_handle(stream))
     _check(rc, "wc_gemv_batch")
+
+
+GEMM_MAX_TOKENS = 128
+
+
+def gemm(stream_bytes: torch.Tensor, rows: int, cols: int, block: int, x: torch.Tensor, *,
+         nbytes: int | None = None, y: torch.Tensor | None = None,
+         status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y = x @ W.T on the tensor cores with W (rows x cols BF16) given as its stream;
+    x is (tokens, cols) BF16 with 1 <= tokens <= 128; returns FP32 (tokens, rows)."""
+    xw = as_words(x).view(-1, cols)
+    tokens = xw.shape[0]
+    if y is None:
+        y = torch.empty((tokens, rows), dtype=torch.float32, device=stream_bytes.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=stream_bytes.device)
+    rc = wc_gemm(stream_bytes.data_ptr(), stream_bytes.numel() if nbytes is None else nbytes,
+                 rows, cols, block, xw.data_ptr(), tokens, y.data_ptr(), status.data_ptr(),
+                 _stream_handle(stream))
+    _check(rc, "wc_gemm")
+    return y
+
+
+def gemm_batch(batch, tokens: int, status: torch.Tensor, stream=None):
+    """batch from make_gemv_batch (x (tokens, cols), y (tokens, rows) per item)."""
+    arr, count = batch
+    rc = wc_gemm_batch(arr, count, tokens, status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_gemm_batch")

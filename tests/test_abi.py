@@ -28,7 +28,7 @@ def test_header_declares_the_boundary():
     for f in ("wc_bound", "wc_workspace_size", "wc_compress", "wc_decompress",
               "wc_compress_batch", "wc_compress_batch_workspace_size",
               "wc_decompress_batch", "wc_stream_info", "wc_status_string", "wc_gemv",
-              "wc_gemv_batch",
+              "wc_gemv_batch", "wc_gemm", "wc_gemm_batch",
               "wc_debug_compress_stalled"):
         assert f in names
 
@@ -127,6 +127,22 @@ def test_argument_checks_before_any_launch(wclib):
     assert c.wc_gemv(16, 10**6, 4, 1024, 128, 16, 3, 16, None, None) == c.WC_ERR_INVALID_ARG  # n_vec
     assert c.wc_gemv(16, 10**6, 4, 1024, 128, 17, 1, 16, None, None) == c.WC_ERR_INVALID_ARG  # x align
     assert c.wc_gemv(16, 100, 4, 1024, 128, 16, 1, 16, None, None) == c.WC_ERR_CORRUPT_STREAM
+    # fused decode-GEMM on the tensor cores: token count, cols % 128, alignment, truncation
+    assert c.wc_gemm(16, 10**6, 4, 1024, 128, 16, 0, 16, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_gemm(16, 10**6, 4, 1024, 128, 16, 129, 16, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_gemm(16, 10**6, 4, 1000, 128, 16, 16, 16, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_gemm(16, 10**6, 4, 1024, 100, 16, 16, 16, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_gemm(16, 10**6, 4, 1024, 128, 24, 16, 16, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_gemm(24, 10**6, 4, 1024, 128, 16, 16, 16, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_gemm(16, 10**6, 4, 1024, 128, 16, 16, 18, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_gemm(16, 100, 4, 1024, 128, 16, 16, 16, None, None) == c.WC_ERR_CORRUPT_STREAM
+    gitems = (c.wc_gemv_item * 2)()
+    for it in gitems:
+        it.stream, it.stream_bytes, it.x, it.y = 16, 10**6, 16, 16
+        it.rows, it.cols, it.block, it.reserved = 4, 1024, 128, 0
+    gitems[1].reserved = 1
+    assert c.wc_gemm_batch(gitems, 2, 16, None, None) == c.WC_ERR_INVALID_ARG
+    assert c.wc_gemm_batch(None, 1, 16, None, None) == c.WC_ERR_INVALID_ARG
     # the stall test hook needs two tiles and a bounded timeout
     assert c.wc_debug_compress_stalled(16, 100, 128, 16, 10**6, 16, 16, 10**6, None, 10**6,
                                        None) == c.WC_ERR_INVALID_ARG
