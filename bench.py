@@ -518,10 +518,12 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
 # next row: fused decode + matrix-vector products over the stack's linear weights
 # ---------------------------------------------------------------------------
 def run_gemv(args):
-    """One fused wc_gemv_batch launch over the 225 linear weight matrices of the
+    """Fused decode + products over the 225 linear weight matrices of the
     8B-shaped stack (32 layers x 7 + LM head; the embedding is a lookup, not a
-    product), n_vec activation vectors, against torch's BF16 matmul (cuBLAS) on
-    the same matrices, replayed from a CUDA graph."""
+    product): one wc_gemv_batch launch with n_vec activation vectors (gemv
+    workload), or wc_gemm_batch on the tensor cores with `tokens` activation
+    rows (gemm workload, one launch per 64 matrices); against torch's BF16
+    matmul (cuBLAS) on the same matrices, replayed from a CUDA graph."""
     import torch
 
     from lossless_weight_compression_b200 import build_lib, synth, wcodec
@@ -533,7 +535,8 @@ def run_gemv(args):
     build_lib.build()
     wc = wcodec.lib()
     stream = torch.cuda.current_stream(dev)
-    nv = args.n_vec
+    gemm = args.workload == "gemm"
+    nv = args.tokens if gemm else args.n_vec
     if args.gemv_layers is None:
         mats = [(name, t) for name, t in synth.stack_tensors(dev, rank_seed_base(rank))
                 if name != "embed_tokens"]
@@ -553,10 +556,13 @@ def run_gemv(args):
                                      BLOCK) for k, (_, t) in enumerate(mats)])
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
+    entry = wc.wc_gemm_batch if gemm else wc.wc_gemv_batch
+
     def fused():
-        rc = wc.wc_gemv_batch(batch[0], batch[1], nv, status.data_ptr(), stream.cuda_stream)
+        rc = entry(batch[0], batch[1], nv, status.data_ptr(), stream.cuda_stream)
         if rc != 0:
-            raise RuntimeError("wc_gemv_batch: %s" % wc.wc_status_string(rc))
+            raise RuntimeError("%s: %s" % ("wc_gemm_batch" if gemm else "wc_gemv_batch",
+                                           wc.wc_status_string(rc)))
 
     # torch / cuBLAS on the uncompressed BF16 weights, all matrices in one graph
     ts = [t for _, t in mats]
@@ -593,7 +599,9 @@ def run_gemv(args):
     ok = status.item() == 0
     for k, t in enumerate(ts):
         ref = xs[k].double() @ t.double().T
-        bound = (t.shape[1] - 1) * 2.0 ** -24 * (xs[k].double().abs() @ t.double().abs().T)
+        # FP32 sum bound; the tensor cores' accumulation is held to 4x that
+        scale = t.shape[1] * 2.0 ** -22 if gemm else (t.shape[1] - 1) * 2.0 ** -24
+        bound = scale * (xs[k].double().abs() @ t.double().abs().T)
         ok &= bool(((ys[k].double() - ref).abs() <= bound).all())
     stream_bytes = sum(sizes)
     x_bytes = sum(x.numel() * 2 for x in xs)
@@ -601,24 +609,31 @@ def run_gemv(args):
     moved = stream_bytes + x_bytes + y_bytes  # algorithmic bytes of the launch
     peak, peak_kind = hbm_peak()
     clk = clocks.summary()
+    launches = -(-len(mats) // 64) if gemm else 1
+    what = "gemm" if gemm else "gemv"
+    kernel = ("gemm_kernel<64> (tcgen05, %d launches per step)" % launches if gemm
+              else "gemv_kernel<256,%d> (one launch per step)" % nv)
     line = {
-        "metric": "fused decode+GEMV weights/s (effective BF16 GB/s)",
+        "metric": "fused decode+%s weights/s (effective BF16 GB/s)" % what.upper(),
         "value": world * 2 * weights / t_fused / 1e9, "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * t_fused, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u16 weights, f32 accumulate", "data": "synthetic",
-        "config": {"workload": "gemv over %d linear weight matrices of the 8B-shaped stack "
-                               "(%d weights), n_vec=%d, block %d" % (len(mats), weights, nv, BLOCK),
+        "config": {"workload": "%s over %d linear weight matrices of the 8B-shaped stack "
+                               "(%d weights), %s=%d, block %d"
+                               % (what, len(mats), weights, "tokens" if gemm else "n_vec", nv,
+                                  BLOCK),
                    "l2": "weights larger than L2; no flush"},
         "roofline": {"bound": "hbm", "achieved": moved / t_fused / 1e9, "peak": peak, "unit": "GB/s",
                      "frac": moved / t_fused / 1e9 / peak, "peak_kind": peak_kind,
-                     "kernel": "gemv_kernel<256,%d> (one launch per step)" % nv,
+                     "kernel": kernel,
                      "algorithmic_bytes_per_launch": moved, "traffic": None},
         "cublas_bf16": {"ms_per_step": 1e3 * t_blas,
                         "achieved_gbs": (2 * weights + x_bytes + 2 * sum(o.numel() for o in outs))
                         / t_blas / 1e9,
                         "speedup_of_fused": t_blas / t_fused},
-        "gpu_launches": args.steps,
+        "tflops": 2.0 * weights * nv / t_fused / 1e12,
+        "gpu_launches": args.steps * launches,
         "clocks": clk,
         "verified_within_fp32_bound": ok,
     }
@@ -637,14 +652,17 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("wcodec", "reference"), default="wcodec")
-    ap.add_argument("--workload", choices=("stack", "layer", "gemv"), default="stack",
+    ap.add_argument("--workload", choices=("stack", "layer", "gemv", "gemm"), default="stack",
                     help="stack: the 8B-shaped stack (the benchmark); layer: one decoder layer "
                          "(a smaller case for profiling); gemv: fused decode + matrix-vector "
-                         "products over the stack's linear weights")
+                         "products over the stack's linear weights; gemm: the same on the "
+                         "tensor cores with --tokens activation rows")
+    ap.add_argument("--tokens", type=int, default=64,
+                    help="activation rows per product, 1..128 (gemm workload)")
     ap.add_argument("--n-vec", type=int, default=1, choices=(1, 2, 4),
                     help="activation vectors per product (gemv workload)")
     ap.add_argument("--gemv-layers", type=int, default=None,
-                    help="gemv workload on the first K decoder layers only (a smaller case)")
+                    help="gemv/gemm workload on the first K decoder layers only (a smaller case)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip timing the CPU oracle (for profiling runs)")
     ap.add_argument("--no-e2e", action="store_true",
@@ -654,7 +672,7 @@ def main(argv=None):
         log("note: fewer than 3 warm-up steps")
     if args.impl == "reference":
         return run_reference(args)
-    if args.workload == "gemv":
+    if args.workload in ("gemv", "gemm"):
         return run_gemv(args)
     return run_wcodec(args)
 

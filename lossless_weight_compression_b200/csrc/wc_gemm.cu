@@ -11,14 +11,13 @@
 // One thread block per SM, persistent. A unit is 128 consecutive rows of one
 // matrix (the MMA's M) times all tokens (its N, padded to a multiple of 16),
 // swept over cols in slices of 128:
-//   - a producer warp reads each slice's per-row block headers and offsets,
-//     checks them, and starts the copies: the slice's mantissa bytes (one 2-D
-//     TMA load, 128-byte swizzled), each row's exponent bytes (one bulk copy per
-//     row; a 128-column slice of a row is 16 whole octets of one block, 16*w
-//     bytes), and the activations (two 2-D TMA loads, 128-byte swizzled, which
-//     is the K-major layout the MMA reads);
-//   - eight decoding warps turn the staged bytes into BF16 weights and store
-//     them in the same K-major 128-byte-swizzled layout;
+//   - one thread starts each slice's mantissa bytes (one 2-D TMA load,
+//     128-byte swizzled) and another its activations (two 2-D TMA loads);
+//   - eight decoding warps own 16 rows each: a few slices ahead they check
+//     their rows' block headers and offsets and fetch each row's exponent
+//     bytes (a 128-column slice of a row is 16 whole octets of one block, 16*w
+//     contiguous bytes; 16-byte cp.async pieces), then turn the staged bytes
+//     into BF16 weights in the K-major 128-byte-swizzled layout the MMA reads;
 //   - one thread issues tcgen05.mma (BF16 x BF16 -> FP32, M = 128, K = 16) into
 //     one of two accumulators in tensor memory;
 //   - four epilogue warps move a finished accumulator out with tcgen05.ld and
@@ -43,7 +42,7 @@ constexpr uint32_t kSliceCols = 128;   // columns per pipeline slice (8 MMAs of 
 constexpr uint32_t kExpPitch = 144;    // staged exponent bytes per row (16*w <= 128, +16 spreads banks)
 constexpr uint32_t kManStage = kTileRows * kSliceCols;      // 16 KB
 constexpr uint32_t kExpStage = kTileRows * kExpPitch;       // 18 KB
-constexpr uint32_t kMetaStage = kTileRows * 2 * 16;         // t0 and t1 per row
+constexpr uint32_t kMetaStage = kTileRows * 2 * 16;         // t0, t1 per row
 constexpr uint32_t kAStage = kTileRows * kSliceCols * 2;    // 32 KB: two 64-column panels
 constexpr uint32_t kAPanel = kTileRows * 128;               // 128 rows x 128 bytes
 constexpr uint32_t kMaxRawStages = 3;
@@ -55,8 +54,8 @@ constexpr int kEpiWarp0 = 2;   // warps 2..5: warp % 4 covers the four TMEM lane
 constexpr int kEpiWarps = 4;
 constexpr int kDecWarp0 = 6;
 constexpr int kDecWarps = 8;
-constexpr int kGemmThreads = 32 * (kDecWarp0 + kDecWarps);  // 448
-constexpr int kChunksPerDecThread = int(kSliceCols / 16) * 4 / kDecWarps;  // 4
+constexpr int kXWarp = kDecWarp0 + kDecWarps;    // 14: activation loader
+constexpr int kGemmThreads = 32 * (kXWarp + 1);  // 480
 
 template <int MAXI>
 struct GemmParams {
@@ -167,6 +166,11 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared through L2 (not L1).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
 __device__ __forceinline__ void sts128(uint32_t saddr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(saddr), "r"(v.x), "r"(v.y),
                  "r"(v.z), "r"(v.w)
@@ -197,186 +201,276 @@ __device__ __forceinline__ bool gemm_wait_warp(unsigned long long* bar, uint32_t
 }
 
 // ---------------------------------------------------------------------------
-// producer warp
+// the sequence of slices a block works on: units blockIdx.x, blockIdx.x +
+// gridDim.x, ..., each swept over cols in slices of 128 (every role walks it)
 // ---------------------------------------------------------------------------
+struct Cursor {
+    uint64_t u;
+    uint32_t it, s, slices, row0;
+    bool valid;
+};
+
 template <int MAXI>
-__device__ void gemm_produce(const GemmParams<MAXI>& P, const GemmSmem& S, int lane) {
-    GemmCtl& c = *S.ctl;
-    const uint32_t R = P.raw_stages;
-    uint32_t g = 0, it = 0;
-    // phases this warp started on each barrier, to drain them if the block stops early
-    int raw_issued[kMaxRawStages] = {-1, -1, -1};
-    int x_issued[2] = {-1, -1};
-    bool ok = true;
-    for (uint64_t u = blockIdx.x; ok && u < P.total_units; u += gridDim.x) {
-        it = find_item(P, u, it);
-        const GemvItem& I = P.item[it];
-        const uint64_t n = uint64_t(I.rows) * I.cols;
-        const Layout L = make_layout(n, I.block);
-        const uint8_t* St = I.stream;
-        const uint32_t row0 = uint32_t(u - P.unit_begin[it]) * kTileRows;
-        if (row0 == 0 && lane == 0) {
-            DecodeItem d;
-            d.stream = St;
-            d.stream_bytes = I.stream_bytes;
-            check_container(d, L, P.status);
-        }
-        const uint16_t* hdr = reinterpret_cast<const uint16_t*>(St + L.off_hdr);
-        const uint32_t* offs = reinterpret_cast<const uint32_t*>(St + L.off_offs);
-        const uint32_t bmask = L.block - 1u;
-        const uint32_t slices = I.cols / kSliceCols;
-        for (uint32_t s = 0; s < slices; ++s, ++g) {
-            const uint32_t k0 = s * kSliceCols;
-            // 1. this lane's rows' block headers and offsets (loaded before the wait)
-            uint32_t h[4];
-            uint64_t sb[4], nx[4], el[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t r = uint32_t(lane) + 32u * j;
-                h[j] = 0;
-                sb[j] = nx[j] = 0;
-                el[j] = 0;
-                if (row0 + r < I.rows) {
-                    el[j] = uint64_t(row0 + r) * I.cols + k0;
-                    const uint64_t b = el[j] >> L.log2_block;
-                    h[j] = hdr[b];
-                    sb[j] = 16ull * offs[b];
-                    if ((el[j] & bmask) == 0)  // first slice of the block: check the offset chain
-                        nx[j] = b + 1 < L.nb ? 16ull * offs[b + 1] : ld_u64(St + 64);
-                }
-            }
-            // 2. a free raw stage
-            const uint32_t rs = g % R;
-            if (g >= R && !gemm_wait_warp(&c.raw_empty[rs], ((g / R) - 1) & 1u, c, P.status, 256)) {
-                ok = false;
-                break;
-            }
-            uint8_t* man = S.man + rs * kManStage;
-            uint8_t* exs = S.exp + rs * kExpStage;
-            uint4* t0 = S.meta + rs * 2 * kTileRows;
-            uint4* t1 = t0 + kTileRows;
-            // 3. check, write the decode constants, size the copies
-            uint32_t bytes[4];
-            uint64_t src[4];
-            uint32_t total = 0;
-            bool bad = false;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t r = uint32_t(lane) + 32u * j;
-                uint32_t w = h[j] >> 8, base = h[j] & 0xFFu;
-                bytes[j] = 0;
-                src[j] = 0;
-                if (row0 + r < I.rows) {
-                    bool b_bad = w > 8u || (w == 8u && base != 0u);
-                    if ((el[j] & bmask) == 0) {
-                        const uint64_t blk = el[j] >> L.log2_block;
-                        const uint64_t len = min(uint64_t(L.block), n - (blk << L.log2_block));
-                        b_bad |= sb[j] + ((len + 7) >> 3) * min(w, 8u) != nx[j];
-                    }
-                    const uint64_t seg = (el[j] & bmask) >> 3;  // first octet of the slice
-                    src[j] = L.off_exp + sb[j] + seg * min(w, 8u);
-                    b_bad |= src[j] + 16ull * min(w, 8u) > I.stream_bytes;
-                    if (b_bad) {
-                        bad = true;
-                        w = 0;
-                        base = 0;
-                    }
-                    bytes[j] = 16u * w;
-                } else {
-                    w = 0;
-                    base = 0;
-                }
-                const uint32_t m1 = (1u << w) - 1u;
-                t0[r] = make_uint4(r * kExpPitch, w, 2 * w, 4 * w);
-                t1[r] = make_uint4(m1 | (m1 << 16), (1u << (2 * w)) - 1u,
-                                   w == 8u ? 0xFFFFFFFFu : (1u << (4 * w)) - 1u,
-                                   base * 0x00800080u);
-                total += bytes[j];
-            }
-            if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) report(P.status, kStatusCorrupt);
-            total = __reduce_add_sync(0xFFFFFFFFu, total) + kManStage;
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&c.raw_full[rs], total);
-                tma_load_2d(man, &P.man_map[it], int32_t(k0), int32_t(row0), &c.raw_full[rs]);
-                raw_issued[rs] = int(g / R);
-            }
-            __syncwarp();
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                if (bytes[j])
-                    bulk_load(exs + (uint32_t(lane) + 32u * j) * kExpPitch, St + src[j], bytes[j],
-                              &c.raw_full[rs]);
-            // 4. a free activation stage (the MMAs of slice g - 2 are done)
-            const uint32_t xs = g & 1u;
-            if (g >= 2 && !gemm_wait_warp(&c.ax_empty[xs], ((g >> 1) - 1) & 1u, c, P.status, 256)) {
-                ok = false;
-                break;
-            }
-            if (lane == 0) {
-                uint8_t* xd = S.x + xs * P.nt * 256;
-                mbar_arrive_expect_tx(&c.x_full[xs], P.nt * 256);
-                tma_load_2d(xd, &P.x_map[it], int32_t(k0), 0, &c.x_full[xs]);
-                tma_load_2d(xd + P.nt * 128, &P.x_map[it], int32_t(k0 + 64), 0, &c.x_full[xs]);
-                x_issued[xs] = int(g >> 1);
-            }
-        }
+__device__ __forceinline__ Cursor cursor_at(const GemmParams<MAXI>& P, uint64_t u, uint32_t from) {
+    Cursor c = {};
+    c.u = u;
+    c.valid = u < P.total_units;
+    if (c.valid) {
+        c.it = find_item(P, u, from);
+        c.slices = P.item[c.it].cols / kSliceCols;
+        c.row0 = uint32_t(u - P.unit_begin[c.it]) * kTileRows;
     }
-    // Stopped early: let the copies already started land before the block exits.
-    if (!ok && lane == 0) {
-        for (uint32_t k = 0; k < R; ++k)
-            if (raw_issued[k] >= 0) mbar_wait(&c.raw_full[k], uint32_t(raw_issued[k]) & 1u, nullptr);
-        for (int k = 0; k < 2; ++k)
-            if (x_issued[k] >= 0) mbar_wait(&c.x_full[k], uint32_t(x_issued[k]) & 1u, nullptr);
+    return c;
+}
+
+template <int MAXI>
+__device__ __forceinline__ Cursor cursor_next(const GemmParams<MAXI>& P, const Cursor& c) {
+    if (c.s + 1 < c.slices) {
+        Cursor n = c;
+        ++n.s;
+        return n;
     }
+    return cursor_at(P, c.u + gridDim.x, c.it);
 }
 
 // ---------------------------------------------------------------------------
-// decoding warps: warp d decodes rows 32*(d%4) .. +31, chunks 4*(d/4) .. +3 of
-// every slice (a chunk is 16 columns). A lane owns one row, so each of its
-// chunks is one 16-byte swizzled mantissa load, 2w exponent bytes, and two
-// 16-byte swizzled stores; the 32 lanes of a warp hit 32 different rows, which
-// the swizzle spreads over all banks.
+// producer (one thread): the mantissa bytes of every slice, one 2-D TMA load
+// into a free raw stage; and the container header of each matrix, once.
 // ---------------------------------------------------------------------------
+template <int MAXI>
+__device__ void gemm_produce(const GemmParams<MAXI>& P, const GemmSmem& S) {
+    GemmCtl& c = *S.ctl;
+    const uint32_t R = P.raw_stages;
+    int raw_issued[kMaxRawStages] = {-1, -1, -1};  // to drain if the block stops early
+    bool ok = true;
+    uint32_t g = 0;
+    for (Cursor cur = cursor_at(P, blockIdx.x, 0); cur.valid; cur = cursor_next(P, cur), ++g) {
+        const GemvItem& I = P.item[cur.it];
+        if (cur.row0 == 0 && cur.s == 0) {
+            DecodeItem d;
+            d.stream = I.stream;
+            d.stream_bytes = I.stream_bytes;
+            check_container(d, make_layout(uint64_t(I.rows) * I.cols, I.block), P.status);
+        }
+        const uint32_t rs = g % R;
+        if (g >= R && !gemm_wait(&c.raw_empty[rs], ((g / R) - 1) & 1u, c, P.status, 256)) {
+            ok = false;
+            break;
+        }
+        mbar_arrive_expect_tx(&c.raw_full[rs], kManStage);
+        tma_load_2d(S.man + rs * kManStage, &P.man_map[cur.it], int32_t(cur.s * kSliceCols),
+                    int32_t(cur.row0), &c.raw_full[rs]);
+        raw_issued[rs] = int(g / R);
+    }
+    // Stopped early: let the copies already started land before the block exits.
+    if (!ok)
+        for (uint32_t k = 0; k < R; ++k)
+            if (raw_issued[k] >= 0) mbar_wait(&c.raw_full[k], uint32_t(raw_issued[k]) & 1u, nullptr);
+}
+
+// ---------------------------------------------------------------------------
+// activation loader (one thread): X for slice g goes into stage g % 2 once the
+// MMAs of slice g - 2 have finished reading it
+// ---------------------------------------------------------------------------
+template <int MAXI>
+__device__ void gemm_load_x(const GemmParams<MAXI>& P, const GemmSmem& S) {
+    GemmCtl& c = *S.ctl;
+    int x_issued[2] = {-1, -1};
+    bool ok = true;
+    uint32_t g = 0;
+    for (Cursor cur = cursor_at(P, blockIdx.x, 0); cur.valid; cur = cursor_next(P, cur), ++g) {
+        const uint32_t xs = g & 1u;
+        if (g >= 2 && !gemm_wait(&c.ax_empty[xs], ((g >> 1) - 1) & 1u, c, P.status, 256)) {
+            ok = false;
+            break;
+        }
+        const int32_t k0 = int32_t(cur.s * kSliceCols);
+        uint8_t* xd = S.x + xs * P.nt * 256;
+        mbar_arrive_expect_tx(&c.x_full[xs], P.nt * 256);
+        tma_load_2d(xd, &P.x_map[cur.it], k0, 0, &c.x_full[xs]);
+        tma_load_2d(xd + P.nt * 128, &P.x_map[cur.it], k0 + 64, 0, &c.x_full[xs]);
+        x_issued[xs] = int(g >> 1);
+    }
+    if (!ok)
+        for (int k = 0; k < 2; ++k)
+            if (x_issued[k] >= 0) mbar_wait(&c.x_full[k], uint32_t(x_issued[k]) & 1u, nullptr);
+}
+
+// ---------------------------------------------------------------------------
+// decoding warps. A slice is 128 rows x 8 chunks of 16 columns; eight lanes
+// share a row (lane % 8 = chunk), so a warp covers 4 rows at a time and its
+// lanes mostly agree on the row's width (the w = 4 fast path stays
+// convergent). Warp d owns rows 4*(d + 8i) + lane/8, i = 0..3, of every slice.
+//
+// Each warp prepares its own rows raw_stages - 1 slices ahead: it checks the
+// row's block header and offset when the row enters a block (loaded one slice
+// earlier still), writes the decode constants to shared memory, and fetches
+// the row's 16*w exponent bytes (lane l copies 16-byte piece l % 8, so one copy
+// instruction reads four contiguous runs) as one cp.async group per slice. No
+// other warp touches these rows' staging, so a group wait and a warp barrier
+// are all the hand-off needs; only the mantissa bytes (TMA, producer) and the
+// finished A tile (MMA) are shared.
+//
+// Per chunk: one 16-byte swizzled mantissa load, 2w exponent bytes, two 16-byte
+// swizzled stores; lanes of chunks 4..7 store their two halves in the opposite
+// order, so each store instruction of 8 lanes covers 8 distinct bank groups.
+// ---------------------------------------------------------------------------
+constexpr int kDecIters = int(kTileRows) / 4 / kDecWarps;  // rows per lane and slice
+
+// Block metadata of one row: header, offset (16-byte units) and the next
+// block's payload start (offset chain check at the block's first slice).
+struct RowMeta {
+    uint32_t blk;  // block index (~0: none)
+    uint32_t h;
+    uint32_t off;
+    uint64_t nx;
+};
+
 template <int MAXI>
 __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw, int lane) {
     GemmCtl& c = *S.ctl;
-    const uint32_t R = P.raw_stages;
-    const uint32_t r = 32u * (dw & 3) + uint32_t(lane);
-    const uint32_t c0 = uint32_t(dw >> 2) * kChunksPerDecThread;
-    const uint32_t sw = r & 7u;
-    uint32_t g = 0, it = 0;
-    for (uint64_t u = blockIdx.x; u < P.total_units; u += gridDim.x) {
-        it = find_item(P, u, it);
-        const uint32_t slices = P.item[it].cols / kSliceCols;
-        for (uint32_t s = 0; s < slices; ++s, ++g) {
-            const uint32_t rs = g % R, xs = g & 1u;
-            if (!gemm_wait_warp(&c.raw_full[rs], (g / R) & 1u, c, P.status)) return;
-            if (g >= 2 && !gemm_wait_warp(&c.ax_empty[xs], ((g >> 1) - 1) & 1u, c, P.status)) return;
-            const uint8_t* man = S.man + rs * kManStage + r * 128u;
-            const uint8_t* exs = S.exp + rs * kExpStage;
-            const uint4* meta = S.meta + rs * 2 * kTileRows;
-            const uint4 t0 = meta[r], t1 = meta[kTileRows + r];
-            const uint32_t a_row = smem_addr(S.a + xs * kAStage) + r * 128u;
+    const uint32_t R = P.raw_stages, D = R - 1;
+    const uint32_t ch = uint32_t(lane) & 7u, sub = uint32_t(lane) >> 3;
+    const uint32_t panel = (ch >> 2) * kAPanel;
+    const uint32_t j0 = (ch & 3u) * 2u;
+    const bool swap = ch >= 4u;
+    auto row_of = [&](int i) { return 4u * (uint32_t(dw) + kDecWarps * uint32_t(i)) + sub; };
+
+    RowMeta cur[kDecIters], pend[kDecIters];
+    bool pend_new[kDecIters];
+    uint32_t cur_it = ~0u;
 #pragma unroll
-            for (int i = 0; i < kChunksPerDecThread; ++i) {
-                const uint32_t ch = c0 + uint32_t(i);
-                const uint4 M = *reinterpret_cast<const uint4*>(man + (((ch & 7u) ^ sw) << 4));
-                uint4 v0, v1;
-                decode_chunk(exs, t0.x + ch * t0.z, M, t0, t1, v0, v1);
-                const uint32_t panel = a_row + (ch >> 2) * kAPanel;
-                const uint32_t j0 = (ch & 3u) * 2u;
-                sts128(panel + ((j0 ^ sw) << 4), v0);
-                sts128(panel + (((j0 + 1u) ^ sw) << 4), v1);
-            }
-            fence_proxy_async_smem();  // the tensor cores read A through the async proxy
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&c.raw_empty[rs]);
-                mbar_arrive(&c.a_full[xs]);
+    for (int i = 0; i < kDecIters; ++i) {
+        cur[i].blk = pend[i].blk = ~0u;
+        pend_new[i] = false;
+    }
+    // start the header loads slice q needs that the rows do not hold yet
+    auto load_meta = [&](const Cursor& q) {
+        if (!q.valid) return;
+        const GemvItem& I = P.item[q.it];
+        const Layout L = make_layout(uint64_t(I.rows) * I.cols, I.block);
+        const uint16_t* hdr = reinterpret_cast<const uint16_t*>(I.stream + L.off_hdr);
+        const uint32_t* offs = reinterpret_cast<const uint32_t*>(I.stream + L.off_offs);
+#pragma unroll
+        for (int i = 0; i < kDecIters; ++i) {
+            const uint32_t row = q.row0 + row_of(i);
+            pend_new[i] = false;
+            if (row < I.rows) {
+                const uint64_t el = uint64_t(row) * I.cols + q.s * kSliceCols;
+                const uint32_t b = uint32_t(el >> L.log2_block);
+                if (q.it != cur_it || b != cur[i].blk) {
+                    pend_new[i] = true;
+                    pend[i].blk = b;
+                    pend[i].h = hdr[b];
+                    pend[i].off = offs[b];
+                    pend[i].nx = b + 1 < L.nb ? 16ull * offs[b + 1] : ld_u64(I.stream + 64);
+                }
             }
         }
+    };
+    // decode constants and exponent bytes of slice a (stage a % R); one cp.async group
+    auto request = [&](uint32_t a, const Cursor& q) {
+        const uint32_t rs = a % R;
+        const GemvItem& I = P.item[q.it];
+        const uint64_t n = uint64_t(I.rows) * I.cols;
+        const Layout L = make_layout(n, I.block);
+        const uint32_t bmask = L.block - 1u;
+        uint4* t0 = S.meta + rs * 2 * kTileRows;
+        const uint32_t exs_a = smem_addr(S.exp + rs * kExpStage);
+        bool bad = false;
+#pragma unroll
+        for (int i = 0; i < kDecIters; ++i) {
+            const uint32_t r = row_of(i), row = q.row0 + r;
+            const bool fresh = pend_new[i];
+            if (fresh) cur[i] = pend[i];
+            uint32_t w = 0, base = 0;
+            uint64_t src = 0;
+            if (row < I.rows) {
+                const uint64_t el = uint64_t(row) * I.cols + q.s * kSliceCols;
+                w = cur[i].h >> 8;
+                base = cur[i].h & 0xFFu;
+                const uint64_t sb = 16ull * cur[i].off;
+                bool b_bad = w > 8u || (w == 8u && base != 0u);
+                if (fresh && (el & bmask) == 0) {  // the block's first slice
+                    const uint64_t len = min(uint64_t(L.block), n - (uint64_t(cur[i].blk) << L.log2_block));
+                    b_bad |= sb + ((len + 7) >> 3) * min(w, 8u) != cur[i].nx;
+                }
+                src = L.off_exp + sb + ((el & bmask) >> 3) * min(w, 8u);
+                b_bad |= src + 16ull * min(w, 8u) > I.stream_bytes;
+                if (b_bad) {
+                    bad = true;
+                    w = 0;
+                    base = 0;
+                }
+            }
+            if (ch == 0) {
+                const uint32_t m1 = (1u << w) - 1u;
+                t0[r] = make_uint4(r * kExpPitch, w, 2 * w, 4 * w);
+                t0[kTileRows + r] =
+                    make_uint4(m1 | (m1 << 16), (1u << (2 * w)) - 1u,
+                               w == 8u ? 0xFFFFFFFFu : (1u << (4 * w)) - 1u, base * 0x00800080u);
+            }
+            if (ch < w) cp_async16(exs_a + r * kExpPitch + 16u * ch, I.stream + src + 16u * ch);
+        }
+        cur_it = q.it;
+        if (bad) report(P.status, kStatusCorrupt);
+    };
+    auto commit = [] { asm volatile("cp.async.commit_group;" ::: "memory"); };
+
+    Cursor ahead = cursor_at(P, blockIdx.x, 0);
+    load_meta(ahead);
+    uint32_t ga = 0;
+    // prologue: slices 0 .. D-1 (one group each, empty past the end)
+    for (; ga < D; ++ga) {
+        if (ahead.valid) {
+            request(ga, ahead);
+            ahead = cursor_next(P, ahead);
+            load_meta(ahead);
+        }
+        commit();
     }
+    uint32_t g = 0;
+    for (Cursor cur_s = cursor_at(P, blockIdx.x, 0); cur_s.valid; cur_s = cursor_next(P, cur_s), ++g) {
+        if (ahead.valid) {
+            request(ga, ahead);
+            ahead = cursor_next(P, ahead);
+            load_meta(ahead);
+        }
+        ++ga;
+        commit();
+        if (D == 2)
+            asm volatile("cp.async.wait_group 2;" ::: "memory");  // slice g's group has landed
+        else
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        __syncwarp();
+        const uint32_t rs = g % R, xs = g & 1u;
+        if (!gemm_wait_warp(&c.raw_full[rs], (g / R) & 1u, c, P.status) ||
+            (g >= 2 && !gemm_wait_warp(&c.ax_empty[xs], ((g >> 1) - 1) & 1u, c, P.status)))
+            break;
+        const uint8_t* man = S.man + rs * kManStage;
+        const uint8_t* exs = S.exp + rs * kExpStage;
+        const uint4* meta = S.meta + rs * 2 * kTileRows;
+        const uint32_t a_base = smem_addr(S.a + xs * kAStage) + panel;
+#pragma unroll
+        for (int i = 0; i < kDecIters; ++i) {
+            const uint32_t r = row_of(i);
+            const uint32_t sw = r & 7u;
+            const uint4 t0 = meta[r], t1 = meta[kTileRows + r];
+            const uint4 M = *reinterpret_cast<const uint4*>(man + r * 128u + ((ch ^ sw) << 4));
+            uint4 v0, v1;
+            decode_chunk(exs, t0.x + ch * t0.z, M, t0, t1, v0, v1);
+            const uint32_t row = a_base + r * 128u;
+            sts128(row + (((j0 + (swap ? 1u : 0u)) ^ sw) << 4), swap ? v1 : v0);
+            sts128(row + (((j0 + (swap ? 0u : 1u)) ^ sw) << 4), swap ? v0 : v1);
+        }
+        fence_proxy_async_smem();  // the tensor cores read A through the async proxy
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&c.raw_empty[rs]);
+            mbar_arrive(&c.a_full[xs]);
+        }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // nothing lands after the block ends
 }
 
 // ---------------------------------------------------------------------------
@@ -510,11 +604,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
 
     if (warp == kProducerWarp) {
-        gemm_produce<MAXI>(P, S, lane);
+        if (lane == 0) gemm_produce<MAXI>(P, S);
     } else if (warp == kMmaWarp) {
         if (lane == 0) gemm_mma<MAXI>(P, S);
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiWarps) {
         gemm_epilogue<MAXI>(P, S, warp, lane);
+    } else if (warp == kXWarp) {
+        if (lane == 0) gemm_load_x<MAXI>(P, S);
     } else {
         gemm_decode<MAXI>(P, S, warp - kDecWarp0, lane);
     }
