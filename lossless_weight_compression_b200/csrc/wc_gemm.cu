@@ -13,7 +13,7 @@
 // swept over cols in slices of 128:
 //   - one thread starts each slice's mantissa bytes (one 2-D TMA load,
 //     128-byte swizzled) and another its activations (two 2-D TMA loads);
-//   - eight decoding warps own 16 rows each: a few slices ahead they check
+//   - sixteen decoding warps own 8 rows each: a few slices ahead they check
 //     their rows' block headers and offsets and fetch each row's exponent
 //     bytes (a 128-column slice of a row is 16 whole octets of one block, 16*w
 //     contiguous bytes; 16-byte cp.async pieces), then turn the staged bytes
@@ -53,9 +53,9 @@ constexpr int kMmaWarp = 1;
 constexpr int kEpiWarp0 = 2;   // warps 2..5: warp % 4 covers the four TMEM lane quarters
 constexpr int kEpiWarps = 4;
 constexpr int kDecWarp0 = 6;
-constexpr int kDecWarps = 8;
-constexpr int kXWarp = kDecWarp0 + kDecWarps;    // 14: activation loader
-constexpr int kGemmThreads = 32 * (kXWarp + 1);  // 480
+constexpr int kDecWarps = 16;
+constexpr int kXWarp = kDecWarp0 + kDecWarps;    // 22: activation loader
+constexpr int kGemmThreads = 32 * (kXWarp + 1);  // 736
 
 template <int MAXI>
 struct GemmParams {
@@ -300,16 +300,17 @@ __device__ void gemm_load_x(const GemmParams<MAXI>& P, const GemmSmem& S) {
 // decoding warps. A slice is 128 rows x 8 chunks of 16 columns; eight lanes
 // share a row (lane % 8 = chunk), so a warp covers 4 rows at a time and its
 // lanes mostly agree on the row's width (the w = 4 fast path stays
-// convergent). Warp d owns rows 4*(d + 8i) + lane/8, i = 0..3, of every slice.
+// convergent). Warp d owns rows 4*(d + 16i) + lane/8, i = 0..1, of every slice.
 //
-// Each warp prepares its own rows raw_stages - 1 slices ahead: it checks the
-// row's block header and offset when the row enters a block (loaded one slice
-// earlier still), writes the decode constants to shared memory, and fetches
-// the row's 16*w exponent bytes (lane l copies 16-byte piece l % 8, so one copy
-// instruction reads four contiguous runs) as one cp.async group per slice. No
-// other warp touches these rows' staging, so a group wait and a warp barrier
-// are all the hand-off needs; only the mantissa bytes (TMA, producer) and the
-// finished A tile (MMA) are shared.
+// Each warp prepares its own rows raw_stages - 1 slices ahead: it checks a
+// row's block header and offset when the row enters the block (the header
+// was loaded when the row entered the previous block), writes the decode
+// constants to shared memory, and fetches the row's 16*w exponent bytes
+// (lane l copies 16-byte piece l % 8, so one copy instruction reads four
+// contiguous runs) as one cp.async group per slice. No other warp touches
+// these rows' staging, so a group wait and a warp barrier are all the hand-off
+// needs; only the mantissa bytes (TMA, producer) and the finished A tile (MMA)
+// are shared.
 //
 // Per chunk: one 16-byte swizzled mantissa load, 2w exponent bytes, two 16-byte
 // swizzled stores; lanes of chunks 4..7 store their two halves in the opposite
@@ -317,14 +318,79 @@ __device__ void gemm_load_x(const GemmParams<MAXI>& P, const GemmSmem& S) {
 // ---------------------------------------------------------------------------
 constexpr int kDecIters = int(kTileRows) / 4 / kDecWarps;  // rows per lane and slice
 
-// Block metadata of one row: header, offset (16-byte units) and the next
-// block's payload start (offset chain check at the block's first slice).
-struct RowMeta {
-    uint32_t blk;  // block index (~0: none)
-    uint32_t h;
-    uint32_t off;
-    uint64_t nx;
+// State of one row for the slice being prepared: its block, the block's
+// decode parameters, where the slice's exponent bytes start, and the header of
+// the row's next block (loaded when the row enters a block, so it is in
+// registers by the time the row gets there).
+struct RowState {
+    uint64_t el;    // element index of the slice's first column
+    uint64_t src;   // stream offset of the slice's exponent bytes
+    uint32_t w, base;
+    uint32_t nh, noff;  // next block: header and offset (16-byte units)
+    uint64_t nnx;       // next block: the following block's payload start
+    bool valid;
 };
+
+// Unit-level constants of the slice being prepared.
+struct UnitState {
+    const uint8_t* stream;
+    uint64_t stream_bytes, n, nb, off_exp;
+    const uint16_t* hdr;
+    const uint32_t* offs;
+    uint32_t cols, rows, block, log2B;
+};
+
+template <int MAXI>
+__device__ __forceinline__ UnitState unit_state(const GemmParams<MAXI>& P, uint32_t it) {
+    const GemvItem& I = P.item[it];
+    UnitState U;
+    U.stream = I.stream;
+    U.stream_bytes = I.stream_bytes;
+    U.cols = I.cols;
+    U.rows = I.rows;
+    U.block = I.block;
+    const Layout L = make_layout(uint64_t(I.rows) * I.cols, I.block);
+    U.n = L.n;
+    U.nb = L.nb;
+    U.off_exp = L.off_exp;
+    U.log2B = L.log2_block;
+    U.hdr = reinterpret_cast<const uint16_t*>(I.stream + L.off_hdr);
+    U.offs = reinterpret_cast<const uint32_t*>(I.stream + L.off_offs);
+    return U;
+}
+
+// Start the loads of block b's header, offset and chain end (payload start of
+// block b + 1, or E for the last block).
+__device__ __forceinline__ void load_block(const UnitState& U, uint64_t b, uint32_t& h,
+                                           uint32_t& off, uint64_t& nx) {
+    h = U.hdr[b];
+    off = U.offs[b];
+    nx = b + 1 < U.nb ? 16ull * U.offs[b + 1] : ld_u64(U.stream + 64);
+}
+
+// The row enters block b (its header in h/off/nx): set w, base and the slice's
+// exponent offset, checking the header and, at the block's first element, the
+// offset chain; then start loading the row's next block. False if corrupt
+// (the row then decodes as w = 0).
+__device__ __forceinline__ bool enter_block(const UnitState& U, RowState& R, uint64_t row,
+                                            uint32_t h, uint32_t off, uint64_t nx) {
+    const uint32_t bmask = U.block - 1u;
+    const uint64_t b = R.el >> U.log2B;
+    uint32_t w = h >> 8, base = h & 0xFFu;
+    bool bad = w > 8u || (w == 8u && base != 0u);
+    const uint64_t sb = 16ull * off;
+    if ((R.el & bmask) == 0) {
+        const uint64_t len = min(uint64_t(U.block), U.n - (b << U.log2B));
+        bad |= sb + ((len + 7) >> 3) * min(w, 8u) != nx;
+    }
+    if (bad) w = base = 0;
+    R.w = w;
+    R.base = base;
+    R.src = U.off_exp + sb + ((R.el & bmask) >> 3) * w;
+    // the row continues into block b + 1 inside this unit's columns?
+    if (((b + 1) << U.log2B) < (row + 1) * uint64_t(U.cols)) load_block(U, b + 1, R.nh, R.noff, R.nnx);
+    return !bad;
+}
 
 template <int MAXI>
 __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw, int lane) {
@@ -336,107 +402,89 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
     const bool swap = ch >= 4u;
     auto row_of = [&](int i) { return 4u * (uint32_t(dw) + kDecWarps * uint32_t(i)) + sub; };
 
-    RowMeta cur[kDecIters], pend[kDecIters];
-    bool pend_new[kDecIters];
-    uint32_t cur_it = ~0u;
-#pragma unroll
-    for (int i = 0; i < kDecIters; ++i) {
-        cur[i].blk = pend[i].blk = ~0u;
-        pend_new[i] = false;
+    // slices this block works through
+    uint32_t total = 0;
+    {
+        uint32_t it = 0;
+        for (uint64_t u = blockIdx.x; u < P.total_units; u += gridDim.x) {
+            it = find_item(P, u, it);
+            total += P.item[it].cols / kSliceCols;
+        }
     }
-    // start the header loads slice q needs that the rows do not hold yet
-    auto load_meta = [&](const Cursor& q) {
-        if (!q.valid) return;
-        const GemvItem& I = P.item[q.it];
-        const Layout L = make_layout(uint64_t(I.rows) * I.cols, I.block);
-        const uint16_t* hdr = reinterpret_cast<const uint16_t*>(I.stream + L.off_hdr);
-        const uint32_t* offs = reinterpret_cast<const uint32_t*>(I.stream + L.off_offs);
+
+    // the slice being prepared: its unit, and each of this lane's rows
+    UnitState U = {};
+    RowState RS[kDecIters];
+    uint64_t ua = blockIdx.x;
+    uint32_t it_a = 0, sa = 0, slices_a = 0, row0_a = 0;
+    // decode constants and exponent bytes of slice a (stage a % R), as one cp.async group
+    auto prepare = [&](uint32_t a) {
+        bool bad = false;
+        if (sa == 0) {  // first slice of a unit: each row's first block, loaded here
+            it_a = find_item(P, ua, it_a);
+            U = unit_state(P, it_a);
+            slices_a = U.cols / kSliceCols;
+            row0_a = uint32_t(ua - P.unit_begin[it_a]) * kTileRows;
 #pragma unroll
-        for (int i = 0; i < kDecIters; ++i) {
-            const uint32_t row = q.row0 + row_of(i);
-            pend_new[i] = false;
-            if (row < I.rows) {
-                const uint64_t el = uint64_t(row) * I.cols + q.s * kSliceCols;
-                const uint32_t b = uint32_t(el >> L.log2_block);
-                if (q.it != cur_it || b != cur[i].blk) {
-                    pend_new[i] = true;
-                    pend[i].blk = b;
-                    pend[i].h = hdr[b];
-                    pend[i].off = offs[b];
-                    pend[i].nx = b + 1 < L.nb ? 16ull * offs[b + 1] : ld_u64(I.stream + 64);
+            for (int i = 0; i < kDecIters; ++i) {
+                const uint64_t row = row0_a + row_of(i);
+                RS[i].valid = row < U.rows;
+                RS[i].w = RS[i].base = 0;
+                if (RS[i].valid) {
+                    RS[i].el = row * U.cols;
+                    uint32_t h, off;
+                    uint64_t nx;
+                    load_block(U, RS[i].el >> U.log2B, h, off, nx);
+                    bad |= !enter_block(U, RS[i], row, h, off, nx);
                 }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kDecIters; ++i) {
+                if (!RS[i].valid) continue;
+                RS[i].el += kSliceCols;
+                if ((RS[i].el & (U.block - 1u)) == 0)
+                    bad |= !enter_block(U, RS[i], row0_a + row_of(i), RS[i].nh, RS[i].noff,
+                                        RS[i].nnx);
+                else
+                    RS[i].src += 16u * RS[i].w;
             }
         }
-    };
-    // decode constants and exponent bytes of slice a (stage a % R); one cp.async group
-    auto request = [&](uint32_t a, const Cursor& q) {
         const uint32_t rs = a % R;
-        const GemvItem& I = P.item[q.it];
-        const uint64_t n = uint64_t(I.rows) * I.cols;
-        const Layout L = make_layout(n, I.block);
-        const uint32_t bmask = L.block - 1u;
         uint4* t0 = S.meta + rs * 2 * kTileRows;
         const uint32_t exs_a = smem_addr(S.exp + rs * kExpStage);
-        bool bad = false;
 #pragma unroll
         for (int i = 0; i < kDecIters; ++i) {
-            const uint32_t r = row_of(i), row = q.row0 + r;
-            const bool fresh = pend_new[i];
-            if (fresh) cur[i] = pend[i];
-            uint32_t w = 0, base = 0;
-            uint64_t src = 0;
-            if (row < I.rows) {
-                const uint64_t el = uint64_t(row) * I.cols + q.s * kSliceCols;
-                w = cur[i].h >> 8;
-                base = cur[i].h & 0xFFu;
-                const uint64_t sb = 16ull * cur[i].off;
-                bool b_bad = w > 8u || (w == 8u && base != 0u);
-                if (fresh && (el & bmask) == 0) {  // the block's first slice
-                    const uint64_t len = min(uint64_t(L.block), n - (uint64_t(cur[i].blk) << L.log2_block));
-                    b_bad |= sb + ((len + 7) >> 3) * min(w, 8u) != cur[i].nx;
-                }
-                src = L.off_exp + sb + ((el & bmask) >> 3) * min(w, 8u);
-                b_bad |= src + 16ull * min(w, 8u) > I.stream_bytes;
-                if (b_bad) {
-                    bad = true;
-                    w = 0;
-                    base = 0;
-                }
+            const uint32_t r = row_of(i);
+            if (RS[i].valid && RS[i].src + 16u * RS[i].w > U.stream_bytes) {  // payload past the end
+                bad = true;
+                RS[i].w = RS[i].base = 0;
             }
+            const uint32_t w = RS[i].w;
             if (ch == 0) {
                 const uint32_t m1 = (1u << w) - 1u;
                 t0[r] = make_uint4(r * kExpPitch, w, 2 * w, 4 * w);
                 t0[kTileRows + r] =
                     make_uint4(m1 | (m1 << 16), (1u << (2 * w)) - 1u,
-                               w == 8u ? 0xFFFFFFFFu : (1u << (4 * w)) - 1u, base * 0x00800080u);
+                               w == 8u ? 0xFFFFFFFFu : (1u << (4 * w)) - 1u, RS[i].base * 0x00800080u);
             }
-            if (ch < w) cp_async16(exs_a + r * kExpPitch + 16u * ch, I.stream + src + 16u * ch);
+            if (ch < w) cp_async16(exs_a + r * kExpPitch + 16u * ch, U.stream + RS[i].src + 16u * ch);
         }
-        cur_it = q.it;
         if (bad) report(P.status, kStatusCorrupt);
+        if (++sa == slices_a) {
+            sa = 0;
+            ua += gridDim.x;
+        }
     };
     auto commit = [] { asm volatile("cp.async.commit_group;" ::: "memory"); };
 
-    Cursor ahead = cursor_at(P, blockIdx.x, 0);
-    load_meta(ahead);
     uint32_t ga = 0;
-    // prologue: slices 0 .. D-1 (one group each, empty past the end)
-    for (; ga < D; ++ga) {
-        if (ahead.valid) {
-            request(ga, ahead);
-            ahead = cursor_next(P, ahead);
-            load_meta(ahead);
-        }
+    for (; ga < D; ++ga) {  // prologue: slices 0 .. D-1 (one group each, empty past the end)
+        if (ga < total) prepare(ga);
         commit();
     }
-    uint32_t g = 0;
-    for (Cursor cur_s = cursor_at(P, blockIdx.x, 0); cur_s.valid; cur_s = cursor_next(P, cur_s), ++g) {
-        if (ahead.valid) {
-            request(ga, ahead);
-            ahead = cursor_next(P, ahead);
-            load_meta(ahead);
-        }
-        ++ga;
+    for (uint32_t g = 0; g < total; ++g, ++ga) {
+        if (ga < total) prepare(ga);
         commit();
         if (D == 2)
             asm volatile("cp.async.wait_group 2;" ::: "memory");  // slice g's group has landed
