@@ -297,26 +297,23 @@ __device__ void gemm_load_x(const GemmParams<MAXI>& P, const GemmSmem& S) {
 }
 
 // ---------------------------------------------------------------------------
-// decoding warps. A slice is 128 rows x 8 chunks of 16 columns; eight lanes
-// share a row (lane % 8 = chunk), so a warp covers 4 rows at a time and its
-// lanes mostly agree on the row's width (the w = 4 fast path stays
-// convergent). Warp d owns rows 4*(d + 16i) + lane/8, i = 0..1, of every slice.
+// decoding warps. A slice is 128 rows x 8 chunks of 16 columns. Warp d owns
+// rows 8d .. 8d+7 of every slice, one row per lane group of 4: lane 8q + 4b + k
+// takes row 8d + q (b = 0) or 8d + (q ^ 5) (b = 1), chunks k and k + 4 (one in
+// each 64-column panel). The two rows of a quarter-warp differ in bits 0 and 2
+// of their swizzle phase (row % 8), so the quarter's 16-byte mantissa loads and
+// its A stores each hit 8 distinct bank groups.
 //
 // Each warp prepares its own rows raw_stages - 1 slices ahead: it checks a
 // row's block header and offset when the row enters the block (the header
 // was loaded when the row entered the previous block), writes the decode
-// constants to shared memory, and fetches the row's 16*w exponent bytes
-// (lane l copies 16-byte piece l % 8, so one copy instruction reads four
-// contiguous runs) as one cp.async group per slice. No other warp touches
-// these rows' staging, so a group wait and a warp barrier are all the hand-off
-// needs; only the mantissa bytes (TMA, producer) and the finished A tile (MMA)
-// are shared.
-//
-// Per chunk: one 16-byte swizzled mantissa load, 2w exponent bytes, two 16-byte
-// swizzled stores; lanes of chunks 4..7 store their two halves in the opposite
-// order, so each store instruction of 8 lanes covers 8 distinct bank groups.
+// constants to shared memory, and fetches the row's 16*w exponent bytes (four
+// lanes per row, 16-byte cp.async pieces) as one cp.async group per slice. No
+// other warp touches these rows' staging, so a group wait and a warp barrier
+// are all the hand-off needs; only the mantissa bytes (TMA, producer) and the
+// finished A tile (MMA) are shared.
 // ---------------------------------------------------------------------------
-constexpr int kDecIters = int(kTileRows) / 4 / kDecWarps;  // rows per lane and slice
+static_assert(kDecWarps * 8 == int(kTileRows), "each decoding warp owns 8 rows");
 
 // State of one row for the slice being prepared: its block, the block's
 // decode parameters, where the slice's exponent bytes start, and the header of
@@ -396,11 +393,10 @@ template <int MAXI>
 __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw, int lane) {
     GemmCtl& c = *S.ctl;
     const uint32_t R = P.raw_stages, D = R - 1;
-    const uint32_t ch = uint32_t(lane) & 7u, sub = uint32_t(lane) >> 3;
-    const uint32_t panel = (ch >> 2) * kAPanel;
-    const uint32_t j0 = (ch & 3u) * 2u;
-    const bool swap = ch >= 4u;
-    auto row_of = [&](int i) { return 4u * (uint32_t(dw) + kDecWarps * uint32_t(i)) + sub; };
+    // lane = 8q + 4b + k: row pair q of the warp's 8 rows, member b, chunk k of a panel
+    const uint32_t k = uint32_t(lane) & 3u, q = uint32_t(lane) >> 3, b = (uint32_t(lane) >> 2) & 1u;
+    const uint32_t r = 8u * uint32_t(dw) + (b ? (q ^ 5u) : q);  // this lane's row of every slice
+    const uint32_t sw = r & 7u;
 
     // slices this block works through
     uint32_t total = 0;
@@ -412,64 +408,55 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
         }
     }
 
-    // the slice being prepared: its unit, and each of this lane's rows
+    // the slice being prepared: its unit, and this lane's row
     UnitState U = {};
-    RowState RS[kDecIters];
+    RowState RS;
     uint64_t ua = blockIdx.x;
     uint32_t it_a = 0, sa = 0, slices_a = 0, row0_a = 0;
     // decode constants and exponent bytes of slice a (stage a % R), as one cp.async group
     auto prepare = [&](uint32_t a) {
         bool bad = false;
-        if (sa == 0) {  // first slice of a unit: each row's first block, loaded here
+        if (sa == 0) {  // first slice of a unit: the row's first block, loaded here
             it_a = find_item(P, ua, it_a);
             U = unit_state(P, it_a);
             slices_a = U.cols / kSliceCols;
             row0_a = uint32_t(ua - P.unit_begin[it_a]) * kTileRows;
-#pragma unroll
-            for (int i = 0; i < kDecIters; ++i) {
-                const uint64_t row = row0_a + row_of(i);
-                RS[i].valid = row < U.rows;
-                RS[i].w = RS[i].base = 0;
-                if (RS[i].valid) {
-                    RS[i].el = row * U.cols;
-                    uint32_t h, off;
-                    uint64_t nx;
-                    load_block(U, RS[i].el >> U.log2B, h, off, nx);
-                    bad |= !enter_block(U, RS[i], row, h, off, nx);
-                }
+            const uint64_t row = row0_a + r;
+            RS.valid = row < U.rows;
+            RS.w = RS.base = 0;
+            if (RS.valid) {
+                RS.el = row * U.cols;
+                uint32_t h, off;
+                uint64_t nx;
+                load_block(U, RS.el >> U.log2B, h, off, nx);
+                bad |= !enter_block(U, RS, row, h, off, nx);
             }
-        } else {
-#pragma unroll
-            for (int i = 0; i < kDecIters; ++i) {
-                if (!RS[i].valid) continue;
-                RS[i].el += kSliceCols;
-                if ((RS[i].el & (U.block - 1u)) == 0)
-                    bad |= !enter_block(U, RS[i], row0_a + row_of(i), RS[i].nh, RS[i].noff,
-                                        RS[i].nnx);
-                else
-                    RS[i].src += 16u * RS[i].w;
-            }
+        } else if (RS.valid) {
+            RS.el += kSliceCols;
+            if ((RS.el & (U.block - 1u)) == 0)
+                bad |= !enter_block(U, RS, row0_a + r, RS.nh, RS.noff, RS.nnx);
+            else
+                RS.src += 16u * RS.w;
         }
+        if (RS.valid && RS.src + 16u * RS.w > U.stream_bytes) {  // payload past the end
+            bad = true;
+            RS.w = RS.base = 0;
+        }
+        const uint32_t w = RS.w;
         const uint32_t rs = a % R;
-        uint4* t0 = S.meta + rs * 2 * kTileRows;
-        const uint32_t exs_a = smem_addr(S.exp + rs * kExpStage);
-#pragma unroll
-        for (int i = 0; i < kDecIters; ++i) {
-            const uint32_t r = row_of(i);
-            if (RS[i].valid && RS[i].src + 16u * RS[i].w > U.stream_bytes) {  // payload past the end
-                bad = true;
-                RS[i].w = RS[i].base = 0;
-            }
-            const uint32_t w = RS[i].w;
-            if (ch == 0) {
-                const uint32_t m1 = (1u << w) - 1u;
-                t0[r] = make_uint4(r * kExpPitch, w, 2 * w, 4 * w);
-                t0[kTileRows + r] =
-                    make_uint4(m1 | (m1 << 16), (1u << (2 * w)) - 1u,
-                               w == 8u ? 0xFFFFFFFFu : (1u << (4 * w)) - 1u, RS[i].base * 0x00800080u);
-            }
-            if (ch < w) cp_async16(exs_a + r * kExpPitch + 16u * ch, U.stream + RS[i].src + 16u * ch);
+        if (k == 0) {
+            uint4* t0 = S.meta + rs * 2 * kTileRows;
+            const uint32_t m1 = (1u << w) - 1u;
+            t0[r] = make_uint4(r * kExpPitch, w, 2 * w, 4 * w);
+            t0[kTileRows + r] =
+                make_uint4(m1 | (m1 << 16), (1u << (2 * w)) - 1u,
+                           w == 8u ? 0xFFFFFFFFu : (1u << (4 * w)) - 1u, RS.base * 0x00800080u);
         }
+        // the row's 16*w exponent bytes: pieces k and k + 4 (four lanes per row)
+        const uint32_t d = smem_addr(S.exp + rs * kExpStage) + r * kExpPitch + 16u * k;
+        const uint8_t* src = U.stream + RS.src + 16u * k;
+        if (k < w) cp_async16(d, src);
+        if (k + 4u < w) cp_async16(d + 64u, src + 64u);
         if (bad) report(P.status, kStatusCorrupt);
         if (++sa == slices_a) {
             sa = 0;
@@ -495,21 +482,20 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
         if (!gemm_wait_warp(&c.raw_full[rs], (g / R) & 1u, c, P.status) ||
             (g >= 2 && !gemm_wait_warp(&c.ax_empty[xs], ((g >> 1) - 1) & 1u, c, P.status)))
             break;
-        const uint8_t* man = S.man + rs * kManStage;
+        const uint8_t* man = S.man + rs * kManStage + r * 128u;
         const uint8_t* exs = S.exp + rs * kExpStage;
         const uint4* meta = S.meta + rs * 2 * kTileRows;
-        const uint32_t a_base = smem_addr(S.a + xs * kAStage) + panel;
+        const uint4 t0 = meta[r], t1 = meta[kTileRows + r];
+        const uint32_t a_row = smem_addr(S.a + xs * kAStage) + r * 128u;
 #pragma unroll
-        for (int i = 0; i < kDecIters; ++i) {
-            const uint32_t r = row_of(i);
-            const uint32_t sw = r & 7u;
-            const uint4 t0 = meta[r], t1 = meta[kTileRows + r];
-            const uint4 M = *reinterpret_cast<const uint4*>(man + r * 128u + ((ch ^ sw) << 4));
+        for (uint32_t p = 0; p < 2; ++p) {  // the two 64-column panels
+            const uint32_t ch = 4u * p + k;
+            const uint4 M = *reinterpret_cast<const uint4*>(man + ((ch ^ sw) << 4));
             uint4 v0, v1;
             decode_chunk(exs, t0.x + ch * t0.z, M, t0, t1, v0, v1);
-            const uint32_t row = a_base + r * 128u;
-            sts128(row + (((j0 + (swap ? 1u : 0u)) ^ sw) << 4), swap ? v1 : v0);
-            sts128(row + (((j0 + (swap ? 0u : 1u)) ^ sw) << 4), swap ? v0 : v1);
+            const uint32_t row = a_row + p * kAPanel;
+            sts128(row + (((2u * k) ^ sw) << 4), v0);
+            sts128(row + (((2u * k + 1u) ^ sw) << 4), v1);
         }
         fence_proxy_async_smem();  // the tensor cores read A through the async proxy
         __syncwarp();
