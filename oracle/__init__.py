@@ -61,6 +61,11 @@ def lib() -> ctypes.CDLL:
         L.oracle_compress.restype = ctypes.c_int
         L.oracle_decompress.argtypes = [vp, u64, vp, u64, ctypes.c_uint32]
         L.oracle_decompress.restype = ctypes.c_int
+        L.oracle_bound_f32.argtypes, L.oracle_bound_f32.restype = [u64, ctypes.c_uint32], u64
+        L.oracle_compress_f32.argtypes = [vp, u64, ctypes.c_uint32, vp, u64, vp]
+        L.oracle_compress_f32.restype = ctypes.c_int
+        L.oracle_decompress_f32.argtypes = [vp, u64, vp, u64, ctypes.c_uint32]
+        L.oracle_decompress_f32.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -140,6 +145,40 @@ def decompress(stream: np.ndarray, n: int, block: int) -> np.ndarray:
     rc, out = decompress_status(stream, n, block)
     if rc != OK:
         raise ValueError("oracle_decompress failed with status %d" % rc)
+    return out
+
+
+# --- FP32 streams: high halves coded as BF16 words, low halves raw ------------
+def bound_f32(n: int, block: int) -> int:
+    return lib().oracle_bound_f32(n, block)
+
+
+def compress_f32(words: np.ndarray, block: int) -> np.ndarray:
+    """Encode FP32 bit patterns (uint32, any shape) into an FP32 stream (uint8)."""
+    words = np.ascontiguousarray(words, dtype=np.uint32).reshape(-1)
+    cap = bound_f32(words.size, block)
+    if cap == 0:
+        raise ValueError("oracle: invalid block size %r or n %d" % (block, words.size))
+    out = np.empty(cap, dtype=np.uint8)
+    nbytes = ctypes.c_uint64()
+    rc = lib().oracle_compress_f32(_ptr(words), words.size, block, _ptr(out), cap,
+                                   ctypes.byref(nbytes))
+    if rc != OK:
+        raise ValueError("oracle_compress_f32 failed with status %d" % rc)
+    return out[: nbytes.value].copy()
+
+
+def decompress_f32_status(stream: np.ndarray, n: int, block: int) -> tuple[int, np.ndarray]:
+    stream = np.ascontiguousarray(stream, dtype=np.uint8).reshape(-1)
+    out = np.zeros(n, dtype=np.uint32)
+    rc = lib().oracle_decompress_f32(_ptr(stream), stream.size, _ptr(out), n, block)
+    return rc, out
+
+
+def decompress_f32(stream: np.ndarray, n: int, block: int) -> np.ndarray:
+    rc, out = decompress_f32_status(stream, n, block)
+    if rc != OK:
+        raise ValueError("oracle_decompress_f32 failed with status %d" % rc)
     return out
 
 

@@ -30,6 +30,12 @@
  *      u32 block offsets (16-byte units), mantissa plane, exponent plane;
  *      every section starts on a 128-byte boundary and all padding is zero.
  * Decoding is the exact inverse; its result is the input, bit for bit.
+ *
+ * FP32 tensors (reading: the same block scheme applied to the FP32 exponent):
+ * the high half of an FP32 word has exactly the BF16 layout (sign, 8-bit
+ * exponent, 7 mantissa bits), so the high halves are coded as above and the
+ * low halves (16 more mantissa bits) are stored raw in a plane of their own
+ * after the mantissa plane; the header's flags bit 0 marks such a stream.
  */
 #include <stdint.h>
 #include <stdlib.h>
@@ -157,17 +163,21 @@ void oracle_unpack_octet(uint64_t octet, unsigned w, uint8_t v[8])
 /* Section layout, a function of (n, B) alone.                         */
 /* ------------------------------------------------------------------ */
 typedef struct {
-    uint64_t nb, off_hdr, off_offs, off_man, off_exp;
+    uint64_t nb, off_hdr, off_offs, off_man, off_low, off_exp;
 } layout_t;
 
-static layout_t layout_of(uint64_t n, uint32_t B)
+/* fp32 != 0: the stream of FP32 elements, whose high halves are coded as BF16
+ * words and whose low halves follow the mantissa plane as a raw u16 plane
+ * (reading: an FP32 word is a BF16 word followed by 16 more mantissa bits). */
+static layout_t layout_of(uint64_t n, uint32_t B, int fp32)
 {
     layout_t s;
     s.nb = (n + B - 1) / B;
     s.off_hdr = ORC_HEADER_BYTES;
     s.off_offs = s.off_hdr + round_up_128(2 * s.nb);
     s.off_man = s.off_offs + round_up_128(4 * s.nb);
-    s.off_exp = s.off_man + round_up_128(n);
+    s.off_low = fp32 ? s.off_man + round_up_128(n) : 0;
+    s.off_exp = fp32 ? s.off_low + round_up_128(2 * n) : s.off_man + round_up_128(n);
     return s;
 }
 
@@ -178,28 +188,33 @@ static uint64_t block_len(uint64_t n, uint32_t B, uint64_t b)
 }
 
 /* Largest possible stream: every block raw (w = 8). 0 for a bad B or n. */
-uint64_t oracle_bound(uint64_t n, uint32_t B)
+static uint64_t bound_impl(uint64_t n, uint32_t B, int fp32)
 {
     if (!block_size_allowed(B) || n > ORC_MAX_ELEMS) return 0;
-    layout_t s = layout_of(n, B);
+    layout_t s = layout_of(n, B, fp32);
     uint64_t worst = 0;
     for (uint64_t b = 0; b < s.nb; b++)
         worst += (block_len(n, B, b) + 7) / 8 * 8;
     return s.off_exp + worst;
 }
 
+uint64_t oracle_bound(uint64_t n, uint32_t B) { return bound_impl(n, B, 0); }
+uint64_t oracle_bound_f32(uint64_t n, uint32_t B) { return bound_impl(n, B, 1); }
+
 /* ------------------------------------------------------------------ */
 /* Encoder.                                                            */
 /* ------------------------------------------------------------------ */
-int oracle_compress(const uint16_t *x, uint64_t n, uint32_t B, uint8_t *out,
-                    uint64_t out_capacity, uint64_t *out_bytes)
+/* x: the 16-bit words to code; lo: NULL, or the FP32 low halves (fp32 stream). */
+static int compress_impl(const uint16_t *x, const uint16_t *lo, uint64_t n, uint32_t B,
+                         uint8_t *out, uint64_t out_capacity, uint64_t *out_bytes)
 {
+    const int fp32 = lo != NULL;
     if (!block_size_allowed(B) || n > ORC_MAX_ELEMS || out == NULL ||
         out_bytes == NULL || (n > 0 && x == NULL))
         return ORC_INVALID_ARG;
-    if (out_capacity < oracle_bound(n, B)) return ORC_BUFFER_TOO_SMALL;
+    if (out_capacity < bound_impl(n, B, fp32)) return ORC_BUFFER_TOO_SMALL;
 
-    layout_t s = layout_of(n, B);
+    layout_t s = layout_of(n, B, fp32);
     uint8_t *base = (uint8_t *)malloc(s.nb ? s.nb : 1);
     uint8_t *width = (uint8_t *)malloc(s.nb ? s.nb : 1);
     uint64_t *start = (uint64_t *)malloc((s.nb ? s.nb : 1) * sizeof(uint64_t));
@@ -229,7 +244,7 @@ int oracle_compress(const uint16_t *x, uint64_t n, uint32_t B, uint8_t *out,
     put_le(out + 4, ORC_VERSION, 2);
     put_le(out + 6, ORC_HEADER_BYTES, 2);
     put_le(out + 8, B, 4);
-    put_le(out + 12, 0, 4);
+    put_le(out + 12, (uint64_t)fp32, 4); /* flags: bit 0 = FP32 stream */
     put_le(out + 16, n, 8);
     put_le(out + 24, s.nb, 8);
     put_le(out + 32, s.off_hdr, 8);
@@ -238,6 +253,7 @@ int oracle_compress(const uint16_t *x, uint64_t n, uint32_t B, uint8_t *out,
     put_le(out + 56, s.off_exp, 8);
     put_le(out + 64, E, 8);
     put_le(out + 72, total, 8);
+    if (fp32) put_le(out + 80, s.off_low, 8);
 
     for (uint64_t b = 0; b < s.nb; b++) {
         put_le(out + s.off_hdr + 2 * b, (uint64_t)base[b] | ((uint64_t)width[b] << 8), 2);
@@ -247,6 +263,9 @@ int oracle_compress(const uint16_t *x, uint64_t n, uint32_t B, uint8_t *out,
     /* Step 1 (mantissa half): the sign+mantissa bytes, in element order. */
     for (uint64_t i = 0; i < n; i++)
         out[s.off_man + i] = oracle_signman(x[i]);
+    /* FP32: the low halves, raw, in element order. */
+    if (fp32)
+        for (uint64_t i = 0; i < n; i++) put_le(out + s.off_low + 2 * i, lo[i], 2);
 
     /* Steps 3 and 4: remap, then pack each octet into w bytes. */
     for (uint64_t b = 0; b < s.nb; b++) {
@@ -269,6 +288,35 @@ int oracle_compress(const uint16_t *x, uint64_t n, uint32_t B, uint8_t *out,
     return ORC_OK;
 }
 
+int oracle_compress(const uint16_t *x, uint64_t n, uint32_t B, uint8_t *out,
+                    uint64_t out_capacity, uint64_t *out_bytes)
+{
+    return compress_impl(x, NULL, n, B, out, out_capacity, out_bytes);
+}
+
+/* FP32: split every word into its high half (a BF16 word: sign, 8-bit
+ * exponent, 7 mantissa bits) and its low half (16 more mantissa bits). */
+int oracle_compress_f32(const uint32_t *x, uint64_t n, uint32_t B, uint8_t *out,
+                        uint64_t out_capacity, uint64_t *out_bytes)
+{
+    if (n > ORC_MAX_ELEMS || (n > 0 && x == NULL)) return ORC_INVALID_ARG;
+    uint16_t *hi = (uint16_t *)malloc((n ? n : 1) * sizeof(uint16_t));
+    uint16_t *lo = (uint16_t *)malloc((n ? n : 1) * sizeof(uint16_t));
+    if (!hi || !lo) {
+        free(hi);
+        free(lo);
+        return ORC_INVALID_ARG;
+    }
+    for (uint64_t i = 0; i < n; i++) {
+        hi[i] = (uint16_t)(x[i] >> 16);
+        lo[i] = (uint16_t)(x[i] & 0xFFFFu);
+    }
+    int rc = compress_impl(hi, lo, n, B, out, out_capacity, out_bytes);
+    free(hi);
+    free(lo);
+    return rc;
+}
+
 /* ------------------------------------------------------------------ */
 /* Decoder. Checks everything the stream definition fixes.             */
 /* ------------------------------------------------------------------ */
@@ -279,20 +327,23 @@ static int all_zero(const uint8_t *p, uint64_t count)
     return 1;
 }
 
-int oracle_decompress(const uint8_t *in, uint64_t in_bytes, uint16_t *out,
-                      uint64_t n, uint32_t B)
+/* lo: NULL, or where the low halves of an FP32 stream go. */
+static int decompress_impl(const uint8_t *in, uint64_t in_bytes, uint16_t *out, uint16_t *lo,
+                           uint64_t n, uint32_t B)
 {
+    const int fp32 = lo != NULL;
     if (!block_size_allowed(B) || n > ORC_MAX_ELEMS || in == NULL || (n > 0 && out == NULL))
         return ORC_INVALID_ARG;
     if (in_bytes < ORC_HEADER_BYTES) return ORC_CORRUPT;
 
-    layout_t s = layout_of(n, B);
+    layout_t s = layout_of(n, B, fp32);
     if (get_le(in + 0, 4) != ORC_MAGIC || get_le(in + 4, 2) != ORC_VERSION ||
         get_le(in + 6, 2) != ORC_HEADER_BYTES || get_le(in + 8, 4) != B ||
-        get_le(in + 12, 4) != 0 || get_le(in + 16, 8) != n ||
+        get_le(in + 12, 4) != (uint64_t)fp32 || get_le(in + 16, 8) != n ||
         get_le(in + 24, 8) != s.nb || get_le(in + 32, 8) != s.off_hdr ||
         get_le(in + 40, 8) != s.off_offs || get_le(in + 48, 8) != s.off_man ||
-        get_le(in + 56, 8) != s.off_exp || !all_zero(in + 80, 48))
+        get_le(in + 56, 8) != s.off_exp || get_le(in + 80, 8) != s.off_low ||
+        !all_zero(in + 88, 40))
         return ORC_CORRUPT;
     uint64_t E = get_le(in + 64, 8);
     uint64_t total = get_le(in + 72, 8);
@@ -300,8 +351,11 @@ int oracle_decompress(const uint8_t *in, uint64_t in_bytes, uint16_t *out,
 
     /* Padding between sections must be zero. */
     if (!all_zero(in + s.off_hdr + 2 * s.nb, s.off_offs - s.off_hdr - 2 * s.nb) ||
-        !all_zero(in + s.off_offs + 4 * s.nb, s.off_man - s.off_offs - 4 * s.nb) ||
-        !all_zero(in + s.off_man + n, s.off_exp - s.off_man - n))
+        !all_zero(in + s.off_offs + 4 * s.nb, s.off_man - s.off_offs - 4 * s.nb))
+        return ORC_CORRUPT;
+    if (fp32 ? (!all_zero(in + s.off_man + n, s.off_low - s.off_man - n) ||
+                !all_zero(in + s.off_low + 2 * n, s.off_exp - s.off_low - 2 * n))
+             : !all_zero(in + s.off_man + n, s.off_exp - s.off_man - n))
         return ORC_CORRUPT;
 
     /* Headers and offsets must agree with the prefix sum of the block sizes. */
@@ -335,5 +389,33 @@ int oracle_decompress(const uint8_t *in, uint64_t in_bytes, uint16_t *out,
             }
         }
     }
+    if (fp32)
+        for (uint64_t i = 0; i < n; i++) lo[i] = (uint16_t)get_le(in + s.off_low + 2 * i, 2);
     return ORC_OK;
+}
+
+int oracle_decompress(const uint8_t *in, uint64_t in_bytes, uint16_t *out,
+                      uint64_t n, uint32_t B)
+{
+    return decompress_impl(in, in_bytes, out, NULL, n, B);
+}
+
+/* FP32: decode the high halves and the low plane, then join them. */
+int oracle_decompress_f32(const uint8_t *in, uint64_t in_bytes, uint32_t *out,
+                          uint64_t n, uint32_t B)
+{
+    if (n > ORC_MAX_ELEMS || (n > 0 && out == NULL)) return ORC_INVALID_ARG;
+    uint16_t *hi = (uint16_t *)malloc((n ? n : 1) * sizeof(uint16_t));
+    uint16_t *lo = (uint16_t *)malloc((n ? n : 1) * sizeof(uint16_t));
+    if (!hi || !lo) {
+        free(hi);
+        free(lo);
+        return ORC_INVALID_ARG;
+    }
+    int rc = decompress_impl(in, in_bytes, hi, lo, n, B);
+    if (rc == ORC_OK)
+        for (uint64_t i = 0; i < n; i++) out[i] = ((uint32_t)hi[i] << 16) | lo[i];
+    free(hi);
+    free(lo);
+    return rc;
 }
