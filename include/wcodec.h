@@ -219,6 +219,26 @@ int wc_decompress_batch(const wc_batch_item *h_items, uint32_t count,
                         int32_t *d_status, void *stream);
 
 /*
+ * FP32 tensors ("ENEC: A Lossless AI Model Compression Method Enabling Fast
+ * Inference on Ascend NPUs", Abstract: the method targets AI model weights in
+ * general). The high 16 bits of an FP32 word have the BF16 layout, so the
+ * high halves are coded exactly as BF16 words and the low 16 bits are kept
+ * raw in a plane of their own (flags bit 0 of the container header set, the
+ * plane's offset at header byte 80). d_in / d_out hold n u32 words (device,
+ * 16-byte aligned); everything else as wc_compress / wc_decompress, with
+ * wc_bound_fp32 for the output capacity and wc_workspace_size for the
+ * workspace. A decoder of one kind of stream reports the other kind as
+ * WC_ERR_CORRUPT_STREAM. FP16 tensors need no entry of their own: their
+ * 16-bit words go through wc_compress / wc_decompress unchanged.
+ */
+uint64_t wc_bound_fp32(uint64_t n, uint32_t block);
+int wc_compress_fp32(const void *d_in, uint64_t n, uint32_t block, void *d_out,
+                     uint64_t out_capacity, uint64_t *d_out_bytes, void *d_workspace,
+                     uint64_t workspace_bytes, int32_t *d_status, void *stream);
+int wc_decompress_fp32(const void *d_stream, uint64_t stream_bytes, void *d_out, uint64_t n,
+                       uint32_t block, int32_t *d_status, void *stream);
+
+/*
  * Fused decompression and matrix-vector products: for j < n_vec,
  *   y[j][r] = sum_c W[r][c] * x[j][c]
  * where W (rows x cols, row-major BF16) is given only as its WCB1 stream
@@ -284,7 +304,8 @@ int wc_gemm_batch(const wc_gemv_item *h_items, uint32_t count, uint32_t tokens,
 /*
  * Parse a host copy of a stream's first `header_bytes` (>= 128) bytes. Fills
  * n, block and total_bytes (any may be NULL). Returns WC_ERR_CORRUPT_STREAM
- * if the header is not a WCB1 version-1 header consistent with itself.
+ * if the header is not a WCB1 version-1 header consistent with itself (BF16
+ * or FP32 stream; header bytes 12..15 say which).
  */
 int wc_stream_info(const void *h_header, uint64_t header_bytes,
                    uint64_t *n, uint32_t *block, uint64_t *total_bytes);

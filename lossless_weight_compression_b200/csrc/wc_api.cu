@@ -17,14 +17,14 @@ bool args_ok(uint64_t n, uint32_t block) { return wc::block_ok(block) && n <= wc
 
 int check_compress_args(const void* d_in, uint64_t n, uint32_t block, void* d_out,
                         uint64_t out_capacity, uint64_t* d_out_bytes, void* d_workspace,
-                        uint64_t workspace_bytes) {
+                        uint64_t workspace_bytes, bool fp32 = false) {
     if (!args_ok(n, block) || d_out == nullptr || d_out_bytes == nullptr || d_workspace == nullptr ||
         (n > 0 && d_in == nullptr))
         return WC_ERR_INVALID_ARG;
     if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) || !aligned16(d_workspace) ||
         (reinterpret_cast<uintptr_t>(d_out_bytes) & 7u) != 0)
         return WC_ERR_INVALID_ARG;
-    if (out_capacity < wc::bound_bytes(n, block) ||
+    if (out_capacity < wc::bound_bytes(n, block, fp32) ||
         workspace_bytes < wc::encode_workspace_bytes(wc::encode_tiles(n)))
         return WC_ERR_BUFFER_TOO_SMALL;
     return WC_OK;
@@ -54,13 +54,13 @@ uint64_t batch_workspace_bytes(const wc_compress_item* items, uint32_t count) {
     return total;
 }
 
-int check_decode_item(const wc_batch_item& it) {
+int check_decode_item(const wc_batch_item& it, bool fp32 = false) {
     if (!args_ok(it.n, it.block) || it.stream == nullptr || (it.n > 0 && it.out == nullptr) ||
         it.reserved != 0)
         return WC_ERR_INVALID_ARG;
     if (!aligned16(it.stream) || (it.n > 0 && !aligned16(it.out))) return WC_ERR_INVALID_ARG;
     // the fixed sections alone need off_exp bytes
-    if (it.stream_bytes < wc::make_layout(it.n, it.block).off_exp) return WC_ERR_CORRUPT_STREAM;
+    if (it.stream_bytes < wc::make_layout(it.n, it.block, fp32).off_exp) return WC_ERR_CORRUPT_STREAM;
     return WC_OK;
 }
 
@@ -197,6 +197,39 @@ int wc_decompress(const void* d_stream, uint64_t stream_bytes, void* d_out, uint
     return err == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
+uint64_t wc_bound_fp32(uint64_t n, uint32_t block) {
+    return args_ok(n, block) ? wc::bound_bytes(n, block, true) : 0;
+}
+
+int wc_compress_fp32(const void* d_in, uint64_t n, uint32_t block, void* d_out,
+                     uint64_t out_capacity, uint64_t* d_out_bytes, void* d_workspace,
+                     uint64_t workspace_bytes, int32_t* d_status, void* stream) {
+    const int rc = check_compress_args(d_in, n, block, d_out, out_capacity, d_out_bytes,
+                                       d_workspace, workspace_bytes, true);
+    if (rc != WC_OK) return rc;
+    const wc::EncodeItem item = to_encode_item(d_in, n, block, d_out, d_out_bytes);
+    const cudaError_t err = wc::launch_encode(&item, 1, d_workspace, d_status, kDefaultTimeoutNs,
+                                              0, static_cast<cudaStream_t>(stream), true);
+    return err == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
+int wc_decompress_fp32(const void* d_stream, uint64_t stream_bytes, void* d_out, uint64_t n,
+                       uint32_t block, int32_t* d_status, void* stream) {
+    wc_batch_item it;
+    it.stream = d_stream;
+    it.stream_bytes = stream_bytes;
+    it.out = d_out;
+    it.n = n;
+    it.block = block;
+    it.reserved = 0;
+    const int rc = check_decode_item(it, true);
+    if (rc != WC_OK) return rc;
+    const wc::DecodeItem d = to_item(it);
+    const cudaError_t err =
+        wc::launch_decode(&d, 1, d_status, static_cast<cudaStream_t>(stream), true);
+    return err == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
 int wc_decompress_batch(const wc_batch_item* h_items, uint32_t count, int32_t* d_status,
                         void* stream) {
     if (h_items == nullptr && count > 0) return WC_ERR_INVALID_ARG;
@@ -327,16 +360,18 @@ int wc_stream_info(const void* h_header, uint64_t header_bytes, uint64_t* n, uin
     const uint8_t* p = static_cast<const uint8_t*>(h_header);
     const uint64_t nn = get_le(p + 16, 8);
     const uint32_t B = uint32_t(get_le(p + 8, 4));
+    const uint64_t flags = get_le(p + 12, 4);
     if (get_le(p, 4) != wc::kMagic || get_le(p + 4, 2) != wc::kVersion ||
-        get_le(p + 6, 2) != wc::kHeaderBytes || get_le(p + 12, 4) != 0 || !args_ok(nn, B))
+        get_le(p + 6, 2) != wc::kHeaderBytes || flags > 1 || !args_ok(nn, B))
         return WC_ERR_CORRUPT_STREAM;
-    const wc::Layout L = wc::make_layout(nn, B);
+    const wc::Layout L = wc::make_layout(nn, B, flags == 1);
     const uint64_t E = get_le(p + 64, 8), total = get_le(p + 72, 8);
     if (get_le(p + 24, 8) != L.nb || get_le(p + 32, 8) != L.off_hdr ||
         get_le(p + 40, 8) != L.off_offs || get_le(p + 48, 8) != L.off_man ||
         get_le(p + 56, 8) != L.off_exp || E > nn + 8 || total != L.off_exp + E)
         return WC_ERR_CORRUPT_STREAM;
-    for (int k = 80; k < 128; ++k)
+    if (get_le(p + 80, 8) != L.off_low) return WC_ERR_CORRUPT_STREAM;
+    for (int k = 88; k < 128; ++k)
         if (p[k] != 0) return WC_ERR_CORRUPT_STREAM;
     if (n) *n = nn;
     if (block) *block = B;

@@ -40,7 +40,9 @@ namespace {
 constexpr int kConsumerWarps = kThreads / 32;  // 8
 constexpr int kProducerWarp = kConsumerWarps;
 constexpr int kDecodeThreads = kThreads + 32;  // 288
-constexpr int kStages = 4;
+// FP32 stages also hold the tile's low halves (16 KB), so they are fewer.
+template <bool F32>
+constexpr int stages_of() { return F32 ? 3 : 4; }
 
 template <int MAXI>
 struct DecodeParams {
@@ -61,16 +63,20 @@ struct __align__(16) StageInfo {
 // Per-block decode constants, computed once per block by the producer.
 //   t0 = {byte offset of the block's payload in the staged bytes, w, 2w, 4w}
 //   t1 = {M1 = m1 | m1 << 16, m2, m4, base * 0x00800080}, mk = 2^k - 1 (m4 = ~0 when 4w = 32)
+template <bool F32>
 struct __align__(16) Stage {
     uint8_t man[kTile];
     uint8_t exp[kTile + 16];
+    uint16_t low[F32 ? kTile : 8];  // FP32: the tile's low halves
     uint4 t0[kMaxBlocksPerTile];
     uint4 t1[kMaxBlocksPerTile];
     StageInfo info;
 };
 
+template <bool F32>
 struct DecodeSmem {
-    Stage stage[kStages];
+    static constexpr int kStages = stages_of<F32>();
+    Stage<F32> stage[kStages];
     unsigned long long full[kStages];
     unsigned long long empty[kStages];
     int abort;
@@ -79,11 +85,12 @@ struct DecodeSmem {
 // ---------------------------------------------------------------------------
 // producer: one warp
 // ---------------------------------------------------------------------------
-template <int MAXI>
-__device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem& sm, int lane) {
+template <int MAXI, bool F32>
+__device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem<F32>& sm, int lane) {
+    constexpr int kStages = DecodeSmem<F32>::kStages;
     uint32_t it = 0;
     DecodeItem I = P.item[0];
-    Layout L = make_layout(I.n, I.block);
+    Layout L = make_layout(I.n, I.block, F32);
     int issued_round[kStages];  // last round whose bulk copies were issued, per stage
     for (int s = 0; s < kStages; ++s) issued_round[s] = -1;
     for (uint64_t i = 0;; ++i) {
@@ -105,11 +112,11 @@ __device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem& sm, int lane) {
         if (t >= P.tile_begin[it + 1]) {  // tiles only move forward: advance the item
             while (t >= P.tile_begin[it + 1]) ++it;
             I = P.item[it];
-            L = make_layout(I.n, I.block);
+            L = make_layout(I.n, I.block, F32);
         }
         const uint64_t lt = t - P.tile_begin[it];
         if (lt == 0 && lane == 0) check_container(I, L, P.status);
-        Stage& st = sm.stage[s];
+        Stage<F32>& st = sm.stage[s];
 
         uint32_t tile_n = 0, len16 = 0, man_bytes = 0;
         uint64_t start = 0;
@@ -122,8 +129,12 @@ __device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem& sm, int lane) {
                                     st.exp, start, len16, lane);
             if (!bad) {
                 man_bytes = (tile_n + 15u) & ~15u;  // inside the 128-byte padded plane
-                if (lane == 0)
-                    st.info = StageInfo{I.out + tile_start, tile_n, L.log2_block};
+                if (lane == 0) {  // FP32 outputs are 32-bit words
+                    uint16_t* out = F32 ? reinterpret_cast<uint16_t*>(
+                                              reinterpret_cast<uint32_t*>(I.out) + tile_start)
+                                        : I.out + tile_start;
+                    st.info = StageInfo{out, tile_n, L.log2_block};
+                }
             } else {
                 if (lane == 0) report(P.status, kStatusCorrupt);
             }
@@ -137,10 +148,13 @@ __device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem& sm, int lane) {
             if (tile_n == 0) {
                 mbar_arrive(&sm.full[s]);
             } else {
-                mbar_arrive_expect_tx(&sm.full[s], man_bytes + len16);
+                const uint32_t low_bytes = F32 ? (2u * tile_n + 15u) & ~15u : 0u;
+                mbar_arrive_expect_tx(&sm.full[s], man_bytes + len16 + low_bytes);
                 const uint8_t* S = I.stream;
                 bulk_load(st.man, S + L.off_man + lt * kTile, man_bytes, &sm.full[s]);
                 if (len16) bulk_load(st.exp, S + L.off_exp + start, len16, &sm.full[s]);
+                if (F32)  // inside the 128-byte padded low plane
+                    bulk_load(st.low, S + L.off_low + 2 * lt * kTile, low_bytes, &sm.full[s]);
                 issued_round[s] = int(round);
             }
         }
@@ -150,8 +164,16 @@ __device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem& sm, int lane) {
 // ---------------------------------------------------------------------------
 // consumers: eight warps
 // ---------------------------------------------------------------------------
-template <int MAXI>
-__device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem& sm, int tid, int lane) {
+// FP32 words 2k, 2k+1 from a pair of high halves and a pair of low halves.
+__device__ __forceinline__ uint4 join_fp32(uint32_t hi01, uint32_t lo01, uint32_t hi23,
+                                           uint32_t lo23) {
+    return make_uint4(prmt(lo01, hi01, 0x5410u), prmt(lo01, hi01, 0x7632u),
+                      prmt(lo23, hi23, 0x5410u), prmt(lo23, hi23, 0x7632u));
+}
+
+template <int MAXI, bool F32>
+__device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem<F32>& sm, int tid, int lane) {
+    constexpr int kStages = DecodeSmem<F32>::kStages;
     for (uint64_t i = 0;; ++i) {
         const uint64_t t = blockIdx.x + i * gridDim.x;
         if (t >= P.total_tiles) break;
@@ -164,7 +186,7 @@ __device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem& sm, int tid, in
             }
             return;
         }
-        const Stage& st = sm.stage[s];
+        const Stage<F32>& st = sm.stage[s];
         const StageInfo info = st.info;
         const uint32_t bmask = (1u << info.log2B) - 1u;
 #pragma unroll
@@ -177,15 +199,33 @@ __device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem& sm, int tid, in
             const uint32_t q = t0.x + ((el & bmask) >> 3) * t0.y;
             uint4 r0, r1;
             decode_chunk(st.exp, q, M, t0, t1, r0, r1);
-            uint16_t* dst = info.out + el;
-            if (info.tile_n - el >= kChunk) {
-                st_stream_v4(dst, r0);
-                st_stream_v4(dst + 8, r1);
+            if (F32) {  // join each high half with its low half
+                uint32_t* dst = reinterpret_cast<uint32_t*>(info.out) + el;
+                const uint4 l0 = *reinterpret_cast<const uint4*>(st.low + el);
+                const uint4 l1 = *reinterpret_cast<const uint4*>(st.low + el + 8);
+                const uint4 y[4] = {join_fp32(r0.x, l0.x, r0.y, l0.y), join_fp32(r0.z, l0.z, r0.w, l0.w),
+                                    join_fp32(r1.x, l1.x, r1.y, l1.y), join_fp32(r1.z, l1.z, r1.w, l1.w)};
+                if (info.tile_n - el >= kChunk) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) st_stream_v4(dst + 4 * j, y[j]);
+                } else {
+                    const uint32_t words[16] = {y[0].x, y[0].y, y[0].z, y[0].w, y[1].x, y[1].y,
+                                                y[1].z, y[1].w, y[2].x, y[2].y, y[2].z, y[2].w,
+                                                y[3].x, y[3].y, y[3].z, y[3].w};
+                    const uint32_t nv = info.tile_n - el;
+                    for (uint32_t e = 0; e < nv; ++e) dst[e] = words[e];
+                }
             } else {
-                const uint32_t words[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-                const uint32_t nv = info.tile_n - el;
-                for (uint32_t e = 0; e < nv; ++e)
-                    dst[e] = uint16_t(words[e >> 1] >> (16 * (e & 1)));
+                uint16_t* dst = info.out + el;
+                if (info.tile_n - el >= kChunk) {
+                    st_stream_v4(dst, r0);
+                    st_stream_v4(dst + 8, r1);
+                } else {
+                    const uint32_t words[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+                    const uint32_t nv = info.tile_n - el;
+                    for (uint32_t e = 0; e < nv; ++e)
+                        dst[e] = uint16_t(words[e >> 1] >> (16 * (e & 1)));
+                }
             }
         }
         __syncwarp();
@@ -193,11 +233,12 @@ __device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem& sm, int tid, in
     }
 }
 
-template <int MAXI>
+template <int MAXI, bool F32>
 __global__ void __launch_bounds__(kDecodeThreads)
     decode_kernel(const __grid_constant__ DecodeParams<MAXI> P) {
+    constexpr int kStages = DecodeSmem<F32>::kStages;
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(smem_raw);
+    DecodeSmem<F32>& sm = *reinterpret_cast<DecodeSmem<F32>*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -209,14 +250,14 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
     __syncthreads();
     if (warp == kProducerWarp)
-        produce<MAXI>(P, sm, lane);
+        produce<MAXI, F32>(P, sm, lane);
     else
-        consume<MAXI>(P, sm, tid, lane);
+        consume<MAXI, F32>(P, sm, tid, lane);
 }
 
 // Persistent grid: as many resident thread blocks as the SMs hold, never more
 // than there are tiles. Computed once per device and kernel instantiation.
-template <int MAXI>
+template <int MAXI, bool F32>
 cudaError_t grid_for(uint64_t tiles, unsigned* grid) {
     static std::mutex mu;
     static int per_device[64];  // 0 = not yet known
@@ -226,14 +267,15 @@ cudaError_t grid_for(uint64_t tiles, unsigned* grid) {
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
     if (per_device[dev] == 0) {
-        err = cudaFuncSetAttribute(decode_kernel<MAXI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   int(sizeof(DecodeSmem)));
+        err = cudaFuncSetAttribute(decode_kernel<MAXI, F32>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   int(sizeof(DecodeSmem<F32>)));
         if (err != cudaSuccess) return err;
         int sms = 0, per_sm = 0;
         err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (err != cudaSuccess) return err;
-        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<MAXI>,
-                                                            kDecodeThreads, sizeof(DecodeSmem));
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<MAXI, F32>,
+                                                            kDecodeThreads, sizeof(DecodeSmem<F32>));
         if (err != cudaSuccess) return err;
         per_device[dev] = (per_sm > 0 ? per_sm : 1) * sms;
     }
@@ -242,7 +284,7 @@ cudaError_t grid_for(uint64_t tiles, unsigned* grid) {
     return cudaSuccess;
 }
 
-template <int MAXI>
+template <int MAXI, bool F32>
 cudaError_t launch_batch(const DecodeItem* items, uint32_t count, int32_t* status,
                          cudaStream_t stream) {
     static_assert(sizeof(DecodeParams<MAXI>) <= 32000, "launch parameters exceed the limit");
@@ -261,9 +303,9 @@ cudaError_t launch_batch(const DecodeItem* items, uint32_t count, int32_t* statu
     p.total_tiles = tiles;
     if (tiles == 0) return cudaSuccess;
     unsigned grid = 0;
-    cudaError_t err = grid_for<MAXI>(tiles, &grid);
+    cudaError_t err = grid_for<MAXI, F32>(tiles, &grid);
     if (err != cudaSuccess) return err;
-    decode_kernel<MAXI><<<grid, kDecodeThreads, sizeof(DecodeSmem), stream>>>(p);
+    decode_kernel<MAXI, F32><<<grid, kDecodeThreads, sizeof(DecodeSmem<F32>), stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -272,11 +314,18 @@ cudaError_t launch_batch(const DecodeItem* items, uint32_t count, int32_t* statu
 constexpr uint32_t kBatchMax = 512;
 
 cudaError_t launch_decode(const DecodeItem* items, uint32_t count, int32_t* status,
-                          cudaStream_t stream) {
-    if (count == 1) return launch_batch<1>(items, 1, status, stream);
+                          cudaStream_t stream, bool fp32) {
+    if (fp32) {  // FP32 streams: one tensor per call
+        for (uint32_t i = 0; i < count; ++i) {
+            const cudaError_t err = launch_batch<1, true>(items + i, 1, status, stream);
+            if (err != cudaSuccess) return err;
+        }
+        return cudaSuccess;
+    }
+    if (count == 1) return launch_batch<1, false>(items, 1, status, stream);
     for (uint32_t i = 0; i < count; i += kBatchMax) {
         const uint32_t c = min(kBatchMax, count - i);
-        const cudaError_t err = launch_batch<kBatchMax>(items + i, c, status, stream);
+        const cudaError_t err = launch_batch<kBatchMax, false>(items + i, c, status, stream);
         if (err != cudaSuccess) return err;
     }
     return cudaSuccess;

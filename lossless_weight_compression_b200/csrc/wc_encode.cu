@@ -37,6 +37,7 @@
 // timer, and a tile whose look-back gives up marks its state word so that
 // later tiles stop waiting too (WC_ERR_TIMEOUT).
 #include <mutex>
+#include <type_traits>
 
 #include "wc_internal.cuh"
 
@@ -73,11 +74,15 @@ struct EncodeParams {
 struct __align__(16) InInfo {
     uint64_t t, lt;    // batch tile index, tile index within its tensor
     uint64_t man_off;  // byte offset of the tile's mantissa bytes in its stream
+    uint64_t low_off;  // FP32: byte offset of the tile's low halves in its stream
     uint32_t item, tile_n, end, pad;
 };
 
+// F32: the tile's input is FP32 words; their high halves go through the same
+// path as BF16 words and their low halves straight to the stream's low plane.
+template <bool F32>
 struct __align__(16) InStage {
-    uint16_t words[kTile];
+    typename std::conditional<F32, uint32_t, uint16_t>::type words[kTile];
     InInfo info;
 };
 
@@ -92,8 +97,9 @@ struct __align__(16) OutStage {
     OutInfo info;
 };
 
+template <bool F32>
 struct EncodeSmem {
-    InStage in[kInStages];
+    InStage<F32> in[kInStages];
     OutStage out[kOutStages];
     unsigned long long in_full[kInStages], in_empty[kInStages];
     unsigned long long out_full[kOutStages], out_empty[kOutStages];
@@ -237,7 +243,8 @@ __device__ __forceinline__ void workers_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
 }
 
-__device__ __forceinline__ void give_up(EncodeSmem& sm, int32_t* status, int lane) {
+template <bool F32>
+__device__ __forceinline__ void give_up(EncodeSmem<F32>& sm, int32_t* status, int lane) {
     if (lane == 0) {
         report(status, kStatusTimeout);
         sm.abort = 1;
@@ -247,8 +254,8 @@ __device__ __forceinline__ void give_up(EncodeSmem& sm, int32_t* status, int lan
 // ---------------------------------------------------------------------------
 // producer warp
 // ---------------------------------------------------------------------------
-template <int MAXI>
-__device__ void encode_produce(const EncodeParams<MAXI>& P, EncodeSmem& sm, int lane) {
+template <int MAXI, bool F32>
+__device__ void encode_produce(const EncodeParams<MAXI>& P, EncodeSmem<F32>& sm, int lane) {
     int issued_round[kInStages];  // last round whose bulk copy was issued, per stage
     for (int s = 0; s < kInStages; ++s) issued_round[s] = -1;
     // The next tile's ticket is taken while the current tile's copy is in flight,
@@ -263,7 +270,7 @@ __device__ void encode_produce(const EncodeParams<MAXI>& P, EncodeSmem& sm, int 
             give_up(sm, P.status, lane);
             break;
         }
-        InStage& st = sm.in[s];
+        InStage<F32>& st = sm.in[s];
         const uint64_t t = t_next;
         if (t >= P.total_tiles) {
             if (lane == 0) {
@@ -277,16 +284,22 @@ __device__ void encode_produce(const EncodeParams<MAXI>& P, EncodeSmem& sm, int 
         const uint64_t lt = t - P.tile_begin[it];
         const uint64_t first = lt * kTile;
         const uint32_t tile_n = I.n ? uint32_t(min(uint64_t(kTile), I.n - first)) : 0u;
-        const uint32_t b16 = (2u * tile_n) & ~15u;  // bytes the bulk copy can move
-        const uint32_t rem = tile_n - b16 / 2u;     // trailing elements (< 8) loaded plainly
-        if (uint32_t(lane) < rem) st.words[b16 / 2 + lane] = I.in[first + b16 / 2 + lane];
-        if (lane == 0)
-            st.info = InInfo{t, lt, make_layout(I.n, I.block).off_man + first, it, tile_n, 0u, 0u};
+        constexpr uint32_t kWordBytes = F32 ? 4u : 2u;
+        const uint32_t b16 = (kWordBytes * tile_n) & ~15u;  // bytes the bulk copy can move
+        const uint32_t rem = tile_n - b16 / kWordBytes;     // trailing elements loaded plainly
+        using Word = typename std::conditional<F32, uint32_t, uint16_t>::type;
+        const Word* in_words = reinterpret_cast<const Word*>(I.in);
+        if (uint32_t(lane) < rem)
+            st.words[b16 / kWordBytes + lane] = in_words[first + b16 / kWordBytes + lane];
+        if (lane == 0) {
+            const Layout L = make_layout(I.n, I.block, F32);
+            st.info = InInfo{t, lt, L.off_man + first, L.off_low + 2 * first, it, tile_n, 0u, 0u};
+        }
         __syncwarp();
         if (lane == 0) {
             if (b16) {
                 mbar_arrive_expect_tx(&sm.in_full[s], b16);
-                bulk_load(st.words, I.in + first, b16, &sm.in_full[s]);
+                bulk_load(st.words, in_words + first, b16, &sm.in_full[s]);
                 issued_round[s] = int(round);
             } else {
                 mbar_arrive(&sm.in_full[s]);
@@ -304,8 +317,8 @@ __device__ void encode_produce(const EncodeParams<MAXI>& P, EncodeSmem& sm, int 
 // ---------------------------------------------------------------------------
 // worker warps
 // ---------------------------------------------------------------------------
-template <int MAXI>
-__device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem& sm, int tid, int lane,
+template <int MAXI, bool F32>
+__device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem<F32>& sm, int tid, int lane,
                             int warp) {
     for (uint32_t i = 0;; ++i) {
         const int s = int(i % kInStages), o = int(i % kOutStages);
@@ -316,7 +329,7 @@ __device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem& sm, int tid
             give_up(sm, P.status, lane);
             if (lane == 0) sm.worker_stop = 1;
         }
-        const InStage& in = sm.in[s];
+        const InStage<F32>& in = sm.in[s];
         OutStage& out = sm.out[o];
         InInfo info = in.info;
         if (!ok) info.end = 0, info.tile_n = 0;
@@ -350,10 +363,36 @@ __device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem& sm, int tid
             const uint32_t nv = el < tile_n ? min(uint32_t(kChunk), tile_n - el) : 0u;
             nval[k] = nv;
             if (nv) {
-                const uint4 a = *reinterpret_cast<const uint4*>(in.words + el);
-                const uint4 b = *reinterpret_cast<const uint4*>(in.words + el + 8);
-                x[k][0] = a.x; x[k][1] = a.y; x[k][2] = a.z; x[k][3] = a.w;
-                x[k][4] = b.x; x[k][5] = b.y; x[k][6] = b.z; x[k][7] = b.w;
+                if (F32) {
+                    // high halves into x (as BF16 pairs); low halves straight to the
+                    // low plane (past the end: zeros, the plane's padding)
+                    uint32_t lw[8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 a = *reinterpret_cast<const uint4*>(in.words + el + 4 * q);
+                        x[k][2 * q] = prmt(a.x, a.y, 0x7632u);
+                        x[k][2 * q + 1] = prmt(a.z, a.w, 0x7632u);
+                        lw[2 * q] = prmt(a.x, a.y, 0x5410u);
+                        lw[2 * q + 1] = prmt(a.z, a.w, 0x5410u);
+                    }
+                    if (nv < kChunk) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const uint32_t keep = (2u * j + 1 < nv) ? 0xFFFFFFFFu
+                                                  : (2u * j < nv) ? 0x0000FFFFu : 0u;
+                            lw[j] &= keep;
+                        }
+                    }
+                    const EncodeItem& Iw = P.item[info.item];
+                    uint8_t* lo_dst = Iw.out + info.low_off + 2 * el;
+                    st_stream_v4(lo_dst, make_uint4(lw[0], lw[1], lw[2], lw[3]));
+                    st_stream_v4(lo_dst + 16, make_uint4(lw[4], lw[5], lw[6], lw[7]));
+                } else {
+                    const uint4 a = *reinterpret_cast<const uint4*>(in.words + el);
+                    const uint4 b = *reinterpret_cast<const uint4*>(in.words + el + 8);
+                    x[k][0] = a.x; x[k][1] = a.y; x[k][2] = a.z; x[k][3] = a.w;
+                    x[k][4] = b.x; x[k][5] = b.y; x[k][6] = b.z; x[k][7] = b.w;
+                }
                 if (nv < kChunk) {
                     // lanes past the end repeat the first element: min and max stay put
                     const uint32_t first = x[k][0] & 0xFFFFu;
@@ -582,7 +621,7 @@ __device__ void write_container(uint8_t* out, const Layout& L, uint64_t E, int l
         uint64_t v = 0;
         switch (lane) {
             case 0: v = kMagic | (uint64_t(kVersion) << 32) | (uint64_t(kHeaderBytes) << 48); break;
-            case 1: v = L.block; break;  // flags (bytes 12..15) = 0
+            case 1: v = L.block | (uint64_t(L.fp32) << 32); break;  // flags: bit 0 = FP32
             case 2: v = L.n; break;
             case 3: v = L.nb; break;
             case 4: v = L.off_hdr; break;
@@ -591,24 +630,30 @@ __device__ void write_container(uint8_t* out, const Layout& L, uint64_t E, int l
             case 7: v = L.off_exp; break;
             case 8: v = E; break;
             case 9: v = L.off_exp + E; break;
+            case 10: v = L.off_low; break;
             default: v = 0; break;
         }
         reinterpret_cast<uint64_t*>(out)[lane] = v;
     }
 }
 
-// Zero the padding after the header, offset and mantissa sections. The bytes
-// [n, round16(n)) of the mantissa plane were stored as zeros by the last tile.
+// Zero the padding after the header, offset, mantissa and low sections. The
+// bytes [n, round16(n)) of the mantissa plane and [2n, 2 round16(n)) of the
+// low plane were stored as zeros by the last tile.
 __device__ void write_padding(uint8_t* out, const Layout& L, int lane) {
+    const uint64_t n16 = (L.n + 15) & ~uint64_t(15);
     const uint64_t a0 = L.off_hdr + 2 * L.nb, a1 = L.off_offs + 4 * L.nb;
-    const uint64_t a2 = L.off_man + ((L.n + 15) & ~uint64_t(15));
+    const uint64_t a2 = L.off_man + n16;
+    const uint64_t man_end = L.fp32 ? L.off_low : L.off_exp;
     for (uint64_t i = a0 + lane; i < L.off_offs; i += 32) out[i] = 0;
     for (uint64_t i = a1 + lane; i < L.off_man; i += 32) out[i] = 0;
-    for (uint64_t i = a2 + lane; i < L.off_exp; i += 32) out[i] = 0;
+    for (uint64_t i = a2 + lane; i < man_end; i += 32) out[i] = 0;
+    if (L.fp32)
+        for (uint64_t i = L.off_low + 2 * n16 + lane; i < L.off_exp; i += 32) out[i] = 0;
 }
 
-template <int MAXI>
-__device__ void encode_store(const EncodeParams<MAXI>& P, EncodeSmem& sm, int lane, int which) {
+template <int MAXI, bool F32>
+__device__ void encode_store(const EncodeParams<MAXI>& P, EncodeSmem<F32>& sm, int lane, int which) {
     for (uint32_t i = uint32_t(which);; i += kStoreWarps) {
         const int o = int(i % kOutStages);
         const uint32_t round = i / kOutStages;
@@ -620,7 +665,7 @@ __device__ void encode_store(const EncodeParams<MAXI>& P, EncodeSmem& sm, int la
         const OutInfo info = st.info;
         if (info.end) break;
         const EncodeItem& I = P.item[info.item];
-        const Layout L = make_layout(I.n, I.block);
+        const Layout L = make_layout(I.n, I.block, F32);
         const uint64_t first = info.lt * kTile;
         const bool last_tile = info.lt + 1 == encode_tiles(I.n);
 
@@ -670,11 +715,11 @@ __device__ void encode_store(const EncodeParams<MAXI>& P, EncodeSmem& sm, int la
     if (lane == 0) bulk_wait_all();
 }
 
-template <int MAXI>
-__global__ void __launch_bounds__(kEncodeThreads, 3)
+template <int MAXI, bool F32>
+__global__ void __launch_bounds__(kEncodeThreads, F32 ? 2 : 3)
     encode_kernel(const __grid_constant__ EncodeParams<MAXI> P) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    EncodeSmem& sm = *reinterpret_cast<EncodeSmem*>(smem_raw);
+    EncodeSmem<F32>& sm = *reinterpret_cast<EncodeSmem<F32>*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0) {
         for (int s = 0; s < kInStages; ++s) {
@@ -695,14 +740,14 @@ __global__ void __launch_bounds__(kEncodeThreads, 3)
     }
     __syncthreads();
     if (warp == kProducerWarp)
-        encode_produce<MAXI>(P, sm, lane);
+        encode_produce<MAXI, F32>(P, sm, lane);
     else if (warp >= kFirstStoreWarp)
-        encode_store<MAXI>(P, sm, lane, warp - kFirstStoreWarp);
+        encode_store<MAXI, F32>(P, sm, lane, warp - kFirstStoreWarp);
     else
-        encode_work<MAXI>(P, sm, tid, lane, warp);
+        encode_work<MAXI, F32>(P, sm, tid, lane, warp);
 }
 
-template <int MAXI>
+template <int MAXI, bool F32>
 cudaError_t encode_grid(uint64_t tiles, unsigned* grid) {
     static std::mutex mu;
     static int per_device[64];
@@ -712,14 +757,15 @@ cudaError_t encode_grid(uint64_t tiles, unsigned* grid) {
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
     if (per_device[dev] == 0) {
-        err = cudaFuncSetAttribute(encode_kernel<MAXI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   int(sizeof(EncodeSmem)));
+        err = cudaFuncSetAttribute(encode_kernel<MAXI, F32>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   int(sizeof(EncodeSmem<F32>)));
         if (err != cudaSuccess) return err;
         int sms = 0, per_sm = 0;
         err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (err != cudaSuccess) return err;
-        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_kernel<MAXI>,
-                                                            kEncodeThreads, sizeof(EncodeSmem));
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_kernel<MAXI, F32>,
+                                                            kEncodeThreads, sizeof(EncodeSmem<F32>));
         if (err != cudaSuccess) return err;
         per_device[dev] = (per_sm > 0 ? per_sm : 1) * sms;
     }
@@ -728,7 +774,7 @@ cudaError_t encode_grid(uint64_t tiles, unsigned* grid) {
     return cudaSuccess;
 }
 
-template <int MAXI>
+template <int MAXI, bool F32>
 cudaError_t encode_batch(const EncodeItem* items, uint32_t count, uint8_t* workspace,
                          int32_t* status, uint64_t timeout_ns, uint32_t first_ticket,
                          cudaStream_t stream) {
@@ -753,9 +799,9 @@ cudaError_t encode_batch(const EncodeItem* items, uint32_t count, uint8_t* works
     cudaError_t err = cudaMemsetAsync(workspace, 0, encode_workspace_bytes(tiles), stream);
     if (err != cudaSuccess) return err;
     unsigned grid = 0;
-    err = encode_grid<MAXI>(tiles, &grid);
+    err = encode_grid<MAXI, F32>(tiles, &grid);
     if (err != cudaSuccess) return err;
-    encode_kernel<MAXI><<<grid, kEncodeThreads, sizeof(EncodeSmem), stream>>>(p);
+    encode_kernel<MAXI, F32><<<grid, kEncodeThreads, sizeof(EncodeSmem<F32>), stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -765,15 +811,21 @@ constexpr uint32_t kEncodeBatchMax = 512;
 
 cudaError_t launch_encode(const EncodeItem* items, uint32_t count, void* workspace,
                           int32_t* status, uint64_t timeout_ns, uint32_t first_ticket,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, bool fp32) {
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    if (count == 1) return encode_batch<1>(items, 1, ws, status, timeout_ns, first_ticket, stream);
+    if (fp32) {  // FP32 tensors: one per call
+        if (count != 1) return cudaErrorInvalidValue;
+        return encode_batch<1, true>(items, 1, ws, status, timeout_ns, first_ticket, stream);
+    }
+    if (count == 1)
+        return encode_batch<1, false>(items, 1, ws, status, timeout_ns, first_ticket, stream);
     // Larger batches go out in launches of up to 512 tensors; each launch has
     // its own part of the workspace, so they can follow each other on the stream.
     for (uint32_t i = 0; i < count; i += kEncodeBatchMax) {
         const uint32_t c = min(kEncodeBatchMax, count - i);
         const cudaError_t err =
-            encode_batch<kEncodeBatchMax>(items + i, c, ws, status, timeout_ns, first_ticket, stream);
+            encode_batch<kEncodeBatchMax, false>(items + i, c, ws, status, timeout_ns, first_ticket,
+                                                 stream);
         if (err != cudaSuccess) return err;
         uint64_t tiles = 0;
         for (uint32_t j = 0; j < c; ++j) tiles += encode_tiles(items[i + j].n);

@@ -31,9 +31,13 @@ constexpr int kMaxBlocksPerTile = kTile / 128;                  // 64
 constexpr int32_t kStatusCorrupt = 3;
 constexpr int32_t kStatusTimeout = 5;
 
+// fp32: a stream of FP32 words, whose high halves are coded exactly as BF16
+// words and whose low halves follow the mantissa plane as a raw u16 plane
+// (off_low; 0 for BF16 streams).
 struct Layout {
-    uint64_t n, nb, off_hdr, off_offs, off_man, off_exp;
+    uint64_t n, nb, off_hdr, off_offs, off_man, off_low, off_exp;
     uint32_t block, log2_block;
+    bool fp32;
 };
 
 __host__ __device__ inline uint64_t align128(uint64_t x) { return (x + 127u) & ~uint64_t(127); }
@@ -52,7 +56,7 @@ __host__ __device__ inline uint32_t log2_pow2(uint32_t B) {
 #endif
 }
 
-__host__ __device__ inline Layout make_layout(uint64_t n, uint32_t B) {
+__host__ __device__ inline Layout make_layout(uint64_t n, uint32_t B, bool fp32 = false) {
     Layout L;
     L.n = n;
     L.block = B;
@@ -61,15 +65,17 @@ __host__ __device__ inline Layout make_layout(uint64_t n, uint32_t B) {
     L.off_hdr = kHeaderBytes;
     L.off_offs = L.off_hdr + align128(2 * L.nb);
     L.off_man = L.off_offs + align128(4 * L.nb);
-    L.off_exp = L.off_man + align128(n);
+    L.off_low = fp32 ? L.off_man + align128(n) : 0;
+    L.off_exp = fp32 ? L.off_low + align128(2 * n) : L.off_man + align128(n);
+    L.fp32 = fp32;
     return L;
 }
 
 __host__ __device__ inline uint64_t num_tiles(uint64_t n) { return (n + kTile - 1) / kTile; }
 
 // Worst-case stream size: every block raw, 8 bytes per (possibly partial) octet.
-__host__ __device__ inline uint64_t bound_bytes(uint64_t n, uint32_t B) {
-    Layout L = make_layout(n, B);
+__host__ __device__ inline uint64_t bound_bytes(uint64_t n, uint32_t B, bool fp32 = false) {
+    Layout L = make_layout(n, B, fp32);
     uint64_t full = n >> L.log2_block;
     uint64_t tail = n - (full << L.log2_block);
     return L.off_exp + full * B + ((tail + 7) / 8) * 8;
@@ -238,12 +244,15 @@ inline uint64_t encode_workspace_bytes(uint64_t tiles) { return 16 + 8 * tiles; 
 
 // One launch for `count` tensors (the launcher splits larger batches); the
 // workspace must hold encode_workspace_bytes(sum of encode_tiles) bytes.
+// fp32: the inputs are FP32 words (EncodeItem::in points at n u32 words) and
+// the streams are FP32 streams.
 cudaError_t launch_encode(const EncodeItem* items, uint32_t count, void* workspace,
                           int32_t* status, uint64_t timeout_ns, uint32_t first_ticket,
-                          cudaStream_t stream);
+                          cudaStream_t stream, bool fp32 = false);
 
+// fp32: FP32 streams decoded into n u32 words (DecodeItem::out).
 cudaError_t launch_decode(const DecodeItem* items, uint32_t count, int32_t* status,
-                          cudaStream_t stream);
+                          cudaStream_t stream, bool fp32 = false);
 
 struct GemvItem {
     const uint8_t* stream;  // WCB1 stream of W (rows x cols, row-major BF16)

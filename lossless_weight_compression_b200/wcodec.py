@@ -107,6 +107,11 @@ def lib() -> ctypes.CDLL:
     L.wc_gemv.restype = i
     L.wc_gemv_batch.argtypes = [ctypes.POINTER(wc_gemv_item), u32, u32, vp, vp]
     L.wc_gemv_batch.restype = i
+    L.wc_bound_fp32.argtypes, L.wc_bound_fp32.restype = [u64, u32], u64
+    L.wc_compress_fp32.argtypes = [vp, u64, u32, vp, u64, vp, vp, u64, vp, vp]
+    L.wc_compress_fp32.restype = i
+    L.wc_decompress_fp32.argtypes = [vp, u64, vp, u64, u32, vp, vp]
+    L.wc_decompress_fp32.restype = i
     L.wc_gemm.argtypes = [vp, u64, u32, u32, u32, vp, u32, vp, vp, vp]
     L.wc_gemm.restype = i
     L.wc_gemm_batch.argtypes = [ctypes.POINTER(wc_gemv_item), u32, u32, vp, vp]
@@ -167,6 +172,20 @@ def wc_gemv(d_stream, stream_bytes, rows, cols, block, d_x, n_vec, d_y, d_status
 
 def wc_gemv_batch(items, count, n_vec, d_status, stream) -> int:
     return lib().wc_gemv_batch(items, count, n_vec, d_status, stream)
+
+
+def wc_bound_fp32(n, block) -> int:
+    return lib().wc_bound_fp32(n, block)
+
+
+def wc_compress_fp32(d_in, n, block, d_out, out_capacity, d_out_bytes, d_ws, ws_bytes, d_status,
+                     stream) -> int:
+    return lib().wc_compress_fp32(d_in, n, block, d_out, out_capacity, d_out_bytes, d_ws,
+                                  ws_bytes, d_status, stream)
+
+
+def wc_decompress_fp32(d_stream, stream_bytes, d_out, n, block, d_status, stream) -> int:
+    return lib().wc_decompress_fp32(d_stream, stream_bytes, d_out, n, block, d_status, stream)
 
 
 def wc_gemm(d_stream, stream_bytes, rows, cols, block, d_x, tokens, d_y, d_status, stream) -> int:
@@ -423,3 +442,44 @@ def gemm_batch(batch, tokens: int, status: torch.Tensor, stream=None):
     arr, count = batch
     rc = wc_gemm_batch(arr, count, tokens, status.data_ptr(), _stream_handle(stream))
     _check(rc, "wc_gemm_batch")
+
+
+def compress_fp32(x: torch.Tensor, block: int = 1024, *, workspace: torch.Tensor | None = None,
+                  stream=None) -> Compressed:
+    """Compress a CUDA tensor of 32-bit words (FP32, read as bit patterns)."""
+    if x.element_size() != 4:
+        raise TypeError("compress_fp32 takes 32-bit words; got %s" % x.dtype)
+    words = x.contiguous().view(-1).view(torch.int32)
+    n = words.numel()
+    cap = wc_bound_fp32(n, block)
+    if cap == 0:
+        raise WcodecError(WC_ERR_INVALID_ARG, "block size %r" % (block,))
+    dev = words.device
+    buf = torch.empty((cap + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+    nbytes = torch.zeros(1, dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = workspace_for(n, block, dev)
+    rc = wc_compress_fp32(words.data_ptr() if n else None, n, block, buf.data_ptr(), buf.numel(),
+                          nbytes.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                          status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_compress_fp32")
+    return Compressed(buf, nbytes, status, n, block, tuple(x.shape), x.dtype)
+
+
+def decompress_fp32(stream_bytes: torch.Tensor, n: int, block: int, *,
+                    out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                    nbytes: int | None = None, stream=None) -> torch.Tensor:
+    """Decode an FP32 stream into n FP32 values (``out`` if given)."""
+    if out is None:
+        out = torch.empty(n, dtype=torch.float32, device=stream_bytes.device)
+    words = out.view(-1)
+    if words.numel() != n or not words.is_contiguous() or out.element_size() != 4:
+        raise ValueError("out must be a contiguous 32-bit tensor of %d elements" % n)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=stream_bytes.device)
+    size = stream_bytes.numel() if nbytes is None else nbytes
+    rc = wc_decompress_fp32(stream_bytes.data_ptr(), size, words.data_ptr() if n else None, n,
+                            block, status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_decompress_fp32")
+    return out

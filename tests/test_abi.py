@@ -29,6 +29,7 @@ def test_header_declares_the_boundary():
               "wc_compress_batch", "wc_compress_batch_workspace_size",
               "wc_decompress_batch", "wc_stream_info", "wc_status_string", "wc_gemv",
               "wc_gemv_batch", "wc_gemm", "wc_gemm_batch",
+              "wc_bound_fp32", "wc_compress_fp32", "wc_decompress_fp32",
               "wc_debug_compress_stalled"):
         assert f in names
 
@@ -47,6 +48,28 @@ def test_bound_matches_oracle(wclib, orc):
     for bad in (0, 1, 64, 127, 129, 384, 8192, 2**31):
         assert wclib.wc_bound(100, bad) == 0
     assert wclib.wc_bound(2**36, 1024) > 0 and wclib.wc_bound(2**36 + 1, 1024) == 0
+
+
+def test_fp32_bound_matches_oracle(wclib, orc):
+    rng = np.random.default_rng(1)
+    for B in BLOCKS:
+        for n in [0, 1, 7, 8, 9, B - 1, B, B + 1, 8193] + list(rng.integers(0, 10**7, 3)):
+            assert wclib.wc_bound_fp32(int(n), B) == orc.bound_f32(int(n), B)
+    assert wclib.wc_bound_fp32(100, 100) == 0
+
+
+def test_stream_info_accepts_fp32_headers(wclib, orc):
+    rng = np.random.default_rng(2)
+    x = rng.integers(0, 2**32, 5000, dtype=np.uint64).astype(np.uint32)
+    s = orc.compress_f32(x, 256)
+    rc, n, block, total = wclib.wc_stream_info(s[:128].tobytes())
+    assert (rc, n, block, total) == (0, 5000, 256, s.size)
+    bad = s[:128].copy()
+    bad[80] ^= 1  # the low plane's offset
+    assert wclib.wc_stream_info(bad.tobytes())[0] == wclib.WC_ERR_CORRUPT_STREAM
+    bad = s[:128].copy()
+    bad[12] = 2  # unknown flag
+    assert wclib.wc_stream_info(bad.tobytes())[0] == wclib.WC_ERR_CORRUPT_STREAM
 
 
 def test_workspace_size(wclib):
@@ -127,6 +150,13 @@ def test_argument_checks_before_any_launch(wclib):
     assert c.wc_gemv(16, 10**6, 4, 1024, 128, 16, 3, 16, None, None) == c.WC_ERR_INVALID_ARG  # n_vec
     assert c.wc_gemv(16, 10**6, 4, 1024, 128, 17, 1, 16, None, None) == c.WC_ERR_INVALID_ARG  # x align
     assert c.wc_gemv(16, 100, 4, 1024, 128, 16, 1, 16, None, None) == c.WC_ERR_CORRUPT_STREAM
+    # FP32 streams: capacity and truncation are checked on the host
+    assert c.wc_compress_fp32(16, 1000, 128, 16, 100, 16, 16, 10**6, None, None) == \
+        c.WC_ERR_BUFFER_TOO_SMALL
+    assert c.wc_compress_fp32(16, 1000, 100, 16, 10**6, 16, 16, 10**6, None, None) == \
+        c.WC_ERR_INVALID_ARG
+    assert c.wc_decompress_fp32(16, 100, 16, 1000, 128, None, None) == c.WC_ERR_CORRUPT_STREAM
+    assert c.wc_decompress_fp32(16, 10**6, 16, 1000, 100, None, None) == c.WC_ERR_INVALID_ARG
     # fused decode-GEMM on the tensor cores: token count, cols % 128, alignment, truncation
     assert c.wc_gemm(16, 10**6, 4, 1024, 128, 16, 0, 16, None, None) == c.WC_ERR_INVALID_ARG
     assert c.wc_gemm(16, 10**6, 4, 1024, 128, 16, 129, 16, None, None) == c.WC_ERR_INVALID_ARG

@@ -119,3 +119,22 @@ def test_fp32_malformed_streams_are_rejected(orc):
         bad[pos] = val if bad[pos] != val else val ^ 1
         assert orc.decompress_f32_status(bad, n, B)[0] == orc.CORRUPT, pos
     assert orc.decompress_f32_status(s[:-1], n, B)[0] == orc.CORRUPT
+
+
+def test_fp16_words_need_at_most_three_more_bits_than_their_exponent(orc):
+    """FP16 words through the 16-bit path: a block's width is at most bits(d) + 3,
+    d the span of the 5-bit FP16 exponents (taken from float arithmetic)."""
+    rng = np.random.default_rng(17)
+    B = 256
+    for scale in (1e-3, 0.02, 1.0, 300.0):
+        h = (rng.standard_normal(B * 40) * scale).astype(np.float16)
+        h = np.where(np.abs(h) < np.float16(6.2e-5), np.float16(6.2e-5), h)  # normals only
+        words = h.view(np.uint16)
+        _, ex = np.frexp(h.astype(np.float64))
+        for b in range(40):
+            blk, eb = words[b * B:(b + 1) * B], ex[b * B:(b + 1) * B]
+            d = int(eb.max() - eb.min())
+            base, w = orc.block_params(blk)
+            assert w <= d.bit_length() + 3
+        s = orc.compress(words, B)
+        assert np.array_equal(orc.decompress(s, words.size, B), words)
