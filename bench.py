@@ -517,6 +517,119 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
 # ---------------------------------------------------------------------------
 # next row: fused decode + matrix-vector products over the stack's linear weights
 # ---------------------------------------------------------------------------
+def run_dtype(args):
+    """FP32 or FP16 weights: encode and decode of the first K decoder layers of the
+    8B-shaped stack drawn in that dtype (same seeds as the BF16 stack). FP32
+    tensors go through wc_compress_fp32 / wc_decompress_fp32, one launch each;
+    FP16 tensors through the 16-bit batch path, one launch per direction."""
+    import torch
+
+    from lossless_weight_compression_b200 import build_lib, synth, wcodec
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    build_lib.build()
+    wc = wcodec.lib()
+    stream = torch.cuda.current_stream(dev)
+    fp32 = args.workload == "fp32"
+    dtype = torch.float32 if fp32 else torch.float16
+    layers = args.gemv_layers or 4
+    mats = [t for l in range(layers) for _, t in synth.layer_tensors(l, dev, rank_seed_base(rank), dtype)]
+    n_all = sum(t.numel() for t in mats)
+    esize = 4 if fp32 else 2
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    outs = [torch.empty_like(t) for t in mats]
+    if fp32:
+        comp = [wcodec.compress_fp32(t, BLOCK) for t in mats]
+        torch.cuda.synchronize(dev)
+        sizes = [c.size() for c in comp]
+        wss = [wcodec.workspace_for(t.numel(), BLOCK, dev) for t in mats]
+
+        def encode_all():
+            for t, c, ws in zip(mats, comp, wss):
+                rc = wc.wc_compress_fp32(t.data_ptr(), t.numel(), BLOCK, c.buffer.data_ptr(),
+                                         c.buffer.numel(), c.nbytes.data_ptr(), ws.data_ptr(),
+                                         ws.numel(), status.data_ptr(), stream.cuda_stream)
+                if rc != 0:
+                    raise RuntimeError("wc_compress_fp32: %s" % wc.wc_status_string(rc))
+
+        def decode_all():
+            for c, size, o in zip(comp, sizes, outs):
+                rc = wc.wc_decompress_fp32(c.buffer.data_ptr(), size, o.data_ptr(), o.numel(),
+                                           BLOCK, status.data_ptr(), stream.cuda_stream)
+                if rc != 0:
+                    raise RuntimeError("wc_decompress_fp32: %s" % wc.wc_status_string(rc))
+        launches = 2 * len(mats)
+        enc_kernel, dec_kernel = "encode_kernel<1,true>", "decode_kernel<1,true>"
+    else:
+        enc = wcodec.CompressBatch([t.view(-1).view(torch.int16) for t in mats], block=BLOCK)
+        enc.run()
+        torch.cuda.synchronize(dev)
+        sizes = enc.sizes()
+        batch = wcodec.make_batch([(enc.buffers[k], sizes[k], outs[k].view(-1).view(torch.int16),
+                                    mats[k].numel(), BLOCK) for k in range(len(mats))])
+
+        def encode_all():
+            enc.run()
+
+        def decode_all():
+            wcodec.decompress_batch(batch, status)
+        launches = 2
+        enc_kernel, dec_kernel = "encode_kernel<512,false>", "decode_kernel<512,false>"
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        barrier(dist, dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        barrier(dist, dev)
+        return max_over_ranks(e0.elapsed_time(e1) / 1e3 / args.steps, dist, dev)
+
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        t_enc = timed(encode_all)
+        t_dec = timed(decode_all)
+    torch.cuda.synchronize(dev)
+    ok = status.item() == 0 and all(torch.equal(a.view(-1), b.view(-1)) for a, b in zip(mats, outs))
+    stream_bytes = sum(sizes)
+    raw_bytes = esize * n_all
+    peak, peak_kind = hbm_peak()
+    moved = stream_bytes + raw_bytes
+    name = "FP32" if fp32 else "FP16"
+    line = {
+        "metric": "decode GB/s (%s out) & %% HBM roofline; compression ratio" % name,
+        "value": world * raw_bytes / t_dec / 1e9, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * t_dec, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u32" if fp32 else "u16", "data": "synthetic",
+        "config": {"workload": "first %d decoder layers of the 8B-shaped stack drawn in %s "
+                               "(%d tensors, %d elements), block %d"
+                               % (layers, name, len(mats), n_all, BLOCK),
+                   "l2": "inputs larger than L2; no flush"},
+        "roofline": {"bound": "hbm", "achieved": moved / t_dec / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": moved / t_dec / 1e9 / peak, "peak_kind": peak_kind,
+                     "kernel": dec_kernel, "algorithmic_bytes_per_launch": moved / (launches // 2),
+                     "traffic": None},
+        "compression": {"ratio": raw_bytes / stream_bytes, "stream_bytes": stream_bytes},
+        "encode": {"ms_per_step": 1e3 * t_enc, "gbs_moved": moved / t_enc / 1e9,
+                   "frac_of_peak": moved / t_enc / 1e9 / peak, "kernel": enc_kernel},
+        "gpu_launches": args.steps * launches // 2,
+        "clocks": clocks.summary(),
+        "verified_bit_exact": ok,
+    }
+    if dist is not None:
+        barrier(dist, dev)
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0 if ok else 1
+
+
 def run_gemv(args):
     """Fused decode + products over the 225 linear weight matrices of the
     8B-shaped stack (32 layers x 7 + LM head; the embedding is a lookup, not a
@@ -652,17 +765,20 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("wcodec", "reference"), default="wcodec")
-    ap.add_argument("--workload", choices=("stack", "layer", "gemv", "gemm"), default="stack",
+    ap.add_argument("--workload", choices=("stack", "layer", "gemv", "gemm", "fp32", "fp16"),
+                    default="stack",
                     help="stack: the 8B-shaped stack (the benchmark); layer: one decoder layer "
                          "(a smaller case for profiling); gemv: fused decode + matrix-vector "
                          "products over the stack's linear weights; gemm: the same on the "
-                         "tensor cores with --tokens activation rows")
+                         "tensor cores with --tokens activation rows; fp32 / fp16: encode and "
+                         "decode of the first --gemv-layers (default 4) layers in that dtype")
     ap.add_argument("--tokens", type=int, default=64,
                     help="activation rows per product, 1..128 (gemm workload)")
     ap.add_argument("--n-vec", type=int, default=1, choices=(1, 2, 4),
                     help="activation vectors per product (gemv workload)")
     ap.add_argument("--gemv-layers", type=int, default=None,
-                    help="gemv/gemm workload on the first K decoder layers only (a smaller case)")
+                    help="gemv/gemm workload on the first K decoder layers only (a smaller case); "
+                         "fp32/fp16 workloads: the number of layers (default 4)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip timing the CPU oracle (for profiling runs)")
     ap.add_argument("--no-e2e", action="store_true",
@@ -674,6 +790,8 @@ def main(argv=None):
         return run_reference(args)
     if args.workload in ("gemv", "gemm"):
         return run_gemv(args)
+    if args.workload in ("fp32", "fp16"):
+        return run_dtype(args)
     return run_wcodec(args)
 
 

@@ -48,12 +48,18 @@ def _gen(seed: int, device) -> torch.Generator:
     return g
 
 
-def gaussian_bf16(shape, std: float, seed: int, device="cpu") -> torch.Tensor:
-    """N(0, std) drawn in fp32 from ``seed`` and rounded to BF16."""
+def gaussian(shape, std: float, seed: int, device="cpu", dtype=torch.bfloat16) -> torch.Tensor:
+    """N(0, std) drawn in fp32 from ``seed`` and rounded to ``dtype`` (BF16, FP16 or
+    FP32: the same draws for every dtype)."""
     g = _gen(seed, device)
     x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
     x.mul_(std)
-    return x.to(torch.bfloat16)
+    return x if dtype == torch.float32 else x.to(dtype)
+
+
+def gaussian_bf16(shape, std: float, seed: int, device="cpu") -> torch.Tensor:
+    """N(0, std) drawn in fp32 from ``seed`` and rounded to BF16."""
+    return gaussian(shape, std, seed, device, torch.bfloat16)
 
 
 def config1(device="cpu"):
@@ -84,13 +90,14 @@ def config2(device="cpu"):
     return [("w4096_outliers", x.to(torch.bfloat16))]
 
 
-def layer_tensors(layer: int, device="cpu", seed_base: int = 10) -> Iterator[tuple[str, torch.Tensor]]:
+def layer_tensors(layer: int, device="cpu", seed_base: int = 10,
+                  dtype=torch.bfloat16) -> Iterator[tuple[str, torch.Tensor]]:
     """The seven linear weights of one decoder layer. Matrix k of layer l uses
     seed ``seed_base + 16*l + k`` for its std jitter U[0.7, 1.3] and its values."""
     for k, (name, r, c) in enumerate(LLAMA3_8B_LAYER):
         seed = seed_base + 16 * layer + k
         jitter = 0.7 + 0.6 * torch.rand((), generator=_gen(seed, "cpu")).item()
-        yield f"layers.{layer}.{name}", gaussian_bf16((r, c), 0.02 * jitter, seed, device)
+        yield f"layers.{layer}.{name}", gaussian((r, c), 0.02 * jitter, seed, device, dtype)
 
 
 def config3(device="cpu"):
