@@ -66,6 +66,14 @@ def lib() -> ctypes.CDLL:
         L.oracle_compress_f32.restype = ctypes.c_int
         L.oracle_decompress_f32.argtypes = [vp, u64, vp, u64, ctypes.c_uint32]
         L.oracle_decompress_f32.restype = ctypes.c_int
+        L.oracle_esc_block_params.argtypes = [vp, u64, vp, vp, vp]
+        L.oracle_esc_block_params.restype = None
+        L.oracle_bound_escape.argtypes = [u64, ctypes.c_uint32]
+        L.oracle_bound_escape.restype = u64
+        L.oracle_compress_escape.argtypes = [vp, u64, ctypes.c_uint32, vp, u64, vp]
+        L.oracle_compress_escape.restype = ctypes.c_int
+        L.oracle_decompress_escape.argtypes = [vp, u64, vp, u64, ctypes.c_uint32]
+        L.oracle_decompress_escape.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -198,3 +206,46 @@ def gemv(stream: np.ndarray, rows: int, cols: int, block: int, x_words: np.ndarr
         y = x @ W.T
         absum = np.abs(x) @ np.abs(W).T
     return y, absum
+
+
+# --- escape-coded streams: a window of 2^w - 1 exponents + an exception list --
+def esc_block_params(words: np.ndarray) -> tuple[int, int, int]:
+    """(base, w, exceptions) of one block of an escape-coded stream."""
+    words = np.ascontiguousarray(words, dtype=np.uint16)
+    base, w, k = ctypes.c_uint8(), ctypes.c_uint8(), ctypes.c_uint64()
+    lib().oracle_esc_block_params(_ptr(words), words.size, ctypes.byref(base),
+                                  ctypes.byref(w), ctypes.byref(k))
+    return base.value, w.value, k.value
+
+
+def bound_escape(n: int, block: int) -> int:
+    return lib().oracle_bound_escape(n, block)
+
+
+def compress_escape(words: np.ndarray, block: int) -> np.ndarray:
+    """Encode BF16 bit patterns (uint16, any shape) into an escape-coded stream."""
+    words = np.ascontiguousarray(words, dtype=np.uint16).reshape(-1)
+    cap = bound_escape(words.size, block)
+    if cap == 0:
+        raise ValueError("oracle: invalid block size %r or n %d" % (block, words.size))
+    out = np.empty(cap, dtype=np.uint8)
+    nbytes = ctypes.c_uint64()
+    rc = lib().oracle_compress_escape(_ptr(words), words.size, block, _ptr(out), cap,
+                                      ctypes.byref(nbytes))
+    if rc != OK:
+        raise ValueError("oracle_compress_escape failed with status %d" % rc)
+    return out[: nbytes.value].copy()
+
+
+def decompress_escape_status(stream: np.ndarray, n: int, block: int) -> tuple[int, np.ndarray]:
+    stream = np.ascontiguousarray(stream, dtype=np.uint8).reshape(-1)
+    out = np.zeros(n, dtype=np.uint16)
+    rc = lib().oracle_decompress_escape(_ptr(stream), stream.size, _ptr(out), n, block)
+    return rc, out
+
+
+def decompress_escape(stream: np.ndarray, n: int, block: int) -> np.ndarray:
+    rc, out = decompress_escape_status(stream, n, block)
+    if rc != OK:
+        raise ValueError("oracle_decompress_escape failed with status %d" % rc)
+    return out

@@ -36,6 +36,15 @@
  * exponent, 7 mantissa bits), so the high halves are coded as above and the
  * low halves (16 more mantissa bits) are stored raw in a plane of their own
  * after the mantissa plane; the header's flags bit 0 marks such a stream.
+ *
+ * Escape-coded streams (reading; flags bit 1): a block's w-bit codes cover a
+ * window of 2^w - 1 exponents [base, base + 2^w - 2] chosen for least size;
+ * the code 2^w - 1 marks an element outside it, whose exponent byte goes to the
+ * block's exception list right after its codes. "ZipServ: Fast and
+ * Memory-Efficient LLM Inference with Hardware-Aware Lossless Compression",
+ * Abstract, gives the direction (a fixed-length format with constant-time
+ * parallel decoding that shrinks weights further); the window and escape
+ * layout are this project's.
  */
 #include <stdint.h>
 #include <stdlib.h>
@@ -47,6 +56,8 @@
 #define ORC_CORRUPT 3
 
 #define ORC_MAGIC 0x31424357u /* the bytes "WCB1" read as a little-endian u32 */
+#define ORC_FLAG_FP32 1u      /* header flags bit 0: an FP32 stream */
+#define ORC_FLAG_ESCAPE 2u    /* header flags bit 1: an escape-coded stream */
 #define ORC_VERSION 1u
 #define ORC_HEADER_BYTES 128u
 #define ORC_MAX_ELEMS (1ull << 36)
@@ -69,6 +80,7 @@ static uint64_t get_le(const uint8_t *p, int nbytes)
 }
 
 static uint64_t round_up_128(uint64_t x) { return (x + 127u) / 128u * 128u; }
+static uint64_t round_up_16(uint64_t x) { return (x + 15u) / 16u * 16u; }
 
 static int block_size_allowed(uint32_t B)
 {
@@ -201,6 +213,27 @@ static uint64_t bound_impl(uint64_t n, uint32_t B, int fp32)
 uint64_t oracle_bound(uint64_t n, uint32_t B) { return bound_impl(n, B, 0); }
 uint64_t oracle_bound_f32(uint64_t n, uint32_t B) { return bound_impl(n, B, 1); }
 
+/* The 128-byte container header (the bytes after it are left as they are). */
+static void write_container(uint8_t *out, uint32_t B, uint32_t flags, uint64_t n,
+                            const layout_t *s, uint64_t E)
+{
+    memset(out, 0, ORC_HEADER_BYTES);
+    put_le(out + 0, ORC_MAGIC, 4);
+    put_le(out + 4, ORC_VERSION, 2);
+    put_le(out + 6, ORC_HEADER_BYTES, 2);
+    put_le(out + 8, B, 4);
+    put_le(out + 12, flags, 4);
+    put_le(out + 16, n, 8);
+    put_le(out + 24, s->nb, 8);
+    put_le(out + 32, s->off_hdr, 8);
+    put_le(out + 40, s->off_offs, 8);
+    put_le(out + 48, s->off_man, 8);
+    put_le(out + 56, s->off_exp, 8);
+    put_le(out + 64, E, 8);
+    put_le(out + 72, s->off_exp + E, 8);
+    put_le(out + 80, s->off_low, 8);
+}
+
 /* ------------------------------------------------------------------ */
 /* Encoder.                                                            */
 /* ------------------------------------------------------------------ */
@@ -240,20 +273,7 @@ static int compress_impl(const uint16_t *x, const uint16_t *lo, uint64_t n, uint
 
     /* Step 6: sections; everything not written below stays zero. */
     memset(out, 0, total);
-    put_le(out + 0, ORC_MAGIC, 4);
-    put_le(out + 4, ORC_VERSION, 2);
-    put_le(out + 6, ORC_HEADER_BYTES, 2);
-    put_le(out + 8, B, 4);
-    put_le(out + 12, (uint64_t)fp32, 4); /* flags: bit 0 = FP32 stream */
-    put_le(out + 16, n, 8);
-    put_le(out + 24, s.nb, 8);
-    put_le(out + 32, s.off_hdr, 8);
-    put_le(out + 40, s.off_offs, 8);
-    put_le(out + 48, s.off_man, 8);
-    put_le(out + 56, s.off_exp, 8);
-    put_le(out + 64, E, 8);
-    put_le(out + 72, total, 8);
-    if (fp32) put_le(out + 80, s.off_low, 8);
+    write_container(out, B, fp32 ? ORC_FLAG_FP32 : 0u, n, &s, E);
 
     for (uint64_t b = 0; b < s.nb; b++) {
         put_le(out + s.off_hdr + 2 * b, (uint64_t)base[b] | ((uint64_t)width[b] << 8), 2);
@@ -418,4 +438,220 @@ int oracle_decompress_f32(const uint8_t *in, uint64_t in_bytes, uint32_t *out,
     free(hi);
     free(lo);
     return rc;
+}
+
+/* ------------------------------------------------------------------ */
+/* Escape-coded streams (header flags bit 1).                          */
+/* ------------------------------------------------------------------ */
+/* Width w in 1..7: the window holds 2^w - 1 exponents and the code 2^w - 1
+ * is the escape. base <= 255 - (2^w - 1), so base + code never exceeds 255. */
+static unsigned escape_code(unsigned w) { return (1u << w) - 1u; }
+
+static int in_window(unsigned e, unsigned base, unsigned w)
+{
+    return e >= base && e - base < escape_code(w);
+}
+
+/* (w, base) of one block of an escape-coded stream and its number of
+ * exceptions K: the candidate of least cost ceil(L/8)*w + K among
+ *   (0, e)        when every exponent of the block equals e,
+ *   (w, base)     for 1 <= w <= 7 and 0 <= base <= 255 - (2^w - 1),
+ *   (8, 0)        the raw block,
+ * ties going to the smaller w, then to the larger base. */
+void oracle_esc_block_params(const uint16_t *x, uint64_t L, uint8_t *base, uint8_t *w,
+                             uint64_t *exceptions)
+{
+    uint64_t hist[256], below[257];
+    memset(hist, 0, sizeof hist);
+    for (uint64_t i = 0; i < L; i++) hist[oracle_exponent(x[i])]++;
+    /* below[e] = number of elements with an exponent smaller than e */
+    below[0] = 0;
+    for (unsigned e = 0; e < 256; e++) below[e + 1] = below[e] + hist[e];
+
+    const uint64_t octets = (L + 7) / 8;
+    uint64_t best_cost = 8 * octets; /* the raw block, (8, 0) */
+    unsigned best_w = 8, best_base = 0;
+    uint64_t best_k = 0;
+    for (unsigned e = 0; e < 256; e++)
+        if (L > 0 && hist[e] == L) { /* one exponent only: (0, e) costs nothing */
+            best_cost = 0, best_w = 0, best_base = e, best_k = 0;
+        }
+    for (unsigned ww = 1; ww <= 7; ww++) {
+        const unsigned m = escape_code(ww);
+        for (unsigned b = 0; b + m <= 255; b++) {
+            const uint64_t inside = below[b + m] - below[b]; /* exponents b .. b + m - 1 */
+            const uint64_t k = L - inside;
+            const uint64_t cost = octets * ww + k;
+            const int better = cost < best_cost ||
+                               (cost == best_cost && ww < best_w) ||
+                               (cost == best_cost && ww == best_w && b > best_base);
+            if (better) best_cost = cost, best_w = ww, best_base = b, best_k = k;
+        }
+    }
+    *w = (uint8_t)best_w;
+    *base = (uint8_t)best_base;
+    *exceptions = best_k;
+}
+
+/* Largest escape-coded stream: every block raw, each payload padded to 16 bytes. */
+uint64_t oracle_bound_escape(uint64_t n, uint32_t B)
+{
+    if (!block_size_allowed(B) || n > ORC_MAX_ELEMS) return 0;
+    layout_t s = layout_of(n, B, 0);
+    uint64_t worst = 0;
+    for (uint64_t b = 0; b < s.nb; b++) worst += round_up_16((block_len(n, B, b) + 7) / 8 * 8);
+    return s.off_exp + worst;
+}
+
+int oracle_compress_escape(const uint16_t *x, uint64_t n, uint32_t B, uint8_t *out,
+                           uint64_t out_capacity, uint64_t *out_bytes)
+{
+    if (!block_size_allowed(B) || n > ORC_MAX_ELEMS || out == NULL || out_bytes == NULL ||
+        (n > 0 && x == NULL))
+        return ORC_INVALID_ARG;
+    if (out_capacity < oracle_bound_escape(n, B)) return ORC_BUFFER_TOO_SMALL;
+
+    layout_t s = layout_of(n, B, 0);
+    const uint64_t slots = s.nb ? s.nb : 1;
+    uint8_t *base = (uint8_t *)malloc(slots);
+    uint8_t *width = (uint8_t *)malloc(slots);
+    uint64_t *start = (uint64_t *)malloc(slots * sizeof(uint64_t));
+    uint64_t *nexc = (uint64_t *)malloc(slots * sizeof(uint64_t));
+    if (!base || !width || !start || !nexc) {
+        free(base);
+        free(width);
+        free(start);
+        free(nexc);
+        return ORC_INVALID_ARG;
+    }
+
+    /* Window, width and number of exceptions of every block. */
+    for (uint64_t b = 0; b < s.nb; b++)
+        oracle_esc_block_params(x + b * B, block_len(n, B, b), &base[b], &width[b], &nexc[b]);
+
+    /* Exclusive prefix sum of the padded payload sizes. */
+    uint64_t running = 0;
+    for (uint64_t b = 0; b < s.nb; b++) {
+        start[b] = running;
+        running += round_up_16((block_len(n, B, b) + 7) / 8 * width[b] + nexc[b]);
+    }
+    const uint64_t E = running;
+    const uint64_t total = s.off_exp + E;
+
+    memset(out, 0, total);
+    write_container(out, B, ORC_FLAG_ESCAPE, n, &s, E);
+    for (uint64_t b = 0; b < s.nb; b++) {
+        put_le(out + s.off_hdr + 2 * b, (uint64_t)base[b] | ((uint64_t)width[b] << 8), 2);
+        put_le(out + s.off_offs + 4 * b, start[b] / 16, 4);
+    }
+    for (uint64_t i = 0; i < n; i++) out[s.off_man + i] = oracle_signman(x[i]);
+
+    /* Codes, packed as in the plain stream, then the exception list. */
+    for (uint64_t b = 0; b < s.nb; b++) {
+        const uint64_t L = block_len(n, B, b);
+        const unsigned w = width[b];
+        uint8_t *payload = out + s.off_exp + start[b];
+        uint8_t *exc = payload + (L + 7) / 8 * w;
+        uint64_t k = 0;
+        for (uint64_t j = 0; j < (L + 7) / 8; j++) {
+            uint8_t c[8];
+            for (int t = 0; t < 8; t++) {
+                const uint64_t i = 8 * j + (uint64_t)t;
+                c[t] = 0; /* lanes past the end of the block */
+                if (i >= L) continue;
+                const unsigned e = oracle_exponent(x[b * B + i]);
+                if (w == 0) {
+                    c[t] = 0; /* every exponent equals base: no code */
+                } else if (w == 8) {
+                    c[t] = (uint8_t)e; /* raw */
+                } else if (in_window(e, base[b], w)) {
+                    c[t] = (uint8_t)(e - base[b]);
+                } else {
+                    c[t] = (uint8_t)escape_code(w);
+                    exc[k++] = (uint8_t)e;
+                }
+            }
+            put_le(payload + j * w, oracle_pack_octet(c, w), (int)w);
+        }
+        (void)k; /* k == nexc[b] by construction of the block parameters */
+    }
+
+    free(base);
+    free(width);
+    free(start);
+    free(nexc);
+    *out_bytes = total;
+    return ORC_OK;
+}
+
+int oracle_decompress_escape(const uint8_t *in, uint64_t in_bytes, uint16_t *out, uint64_t n,
+                             uint32_t B)
+{
+    if (!block_size_allowed(B) || n > ORC_MAX_ELEMS || in == NULL || (n > 0 && out == NULL))
+        return ORC_INVALID_ARG;
+    if (in_bytes < ORC_HEADER_BYTES) return ORC_CORRUPT;
+
+    layout_t s = layout_of(n, B, 0);
+    if (get_le(in + 0, 4) != ORC_MAGIC || get_le(in + 4, 2) != ORC_VERSION ||
+        get_le(in + 6, 2) != ORC_HEADER_BYTES || get_le(in + 8, 4) != B ||
+        get_le(in + 12, 4) != ORC_FLAG_ESCAPE || get_le(in + 16, 8) != n ||
+        get_le(in + 24, 8) != s.nb || get_le(in + 32, 8) != s.off_hdr ||
+        get_le(in + 40, 8) != s.off_offs || get_le(in + 48, 8) != s.off_man ||
+        get_le(in + 56, 8) != s.off_exp || get_le(in + 80, 8) != 0 || !all_zero(in + 88, 40))
+        return ORC_CORRUPT;
+    const uint64_t E = get_le(in + 64, 8);
+    const uint64_t total = get_le(in + 72, 8);
+    if (E > total || total != s.off_exp + E || total > in_bytes) return ORC_CORRUPT;
+    if (!all_zero(in + s.off_hdr + 2 * s.nb, s.off_offs - s.off_hdr - 2 * s.nb) ||
+        !all_zero(in + s.off_offs + 4 * s.nb, s.off_man - s.off_offs - 4 * s.nb) ||
+        !all_zero(in + s.off_man + n, s.off_exp - s.off_man - n))
+        return ORC_CORRUPT;
+
+    const uint8_t *plane = in + s.off_exp;
+    uint64_t running = 0; /* where the next block's payload must start */
+    for (uint64_t b = 0; b < s.nb; b++) {
+        const uint64_t L = block_len(n, B, b);
+        const uint64_t h = get_le(in + s.off_hdr + 2 * b, 2);
+        const unsigned base = (unsigned)(h & 0xFFu), w = (unsigned)(h >> 8);
+        if (w > 8 || (w == 8 && base != 0)) return ORC_CORRUPT;
+        if (w >= 1 && w <= 7 && base + escape_code(w) > 255) return ORC_CORRUPT;
+        if (get_le(in + s.off_offs + 4 * b, 4) * 16 != running) return ORC_CORRUPT;
+        const uint64_t code_bytes = (L + 7) / 8 * w;
+        if (running + code_bytes > E) return ORC_CORRUPT;
+
+        /* The codes; each escape takes the next exception byte. */
+        const uint8_t *payload = plane + running;
+        uint64_t k = 0;
+        for (uint64_t j = 0; j < (L + 7) / 8; j++) {
+            uint8_t c[8];
+            oracle_unpack_octet(get_le(payload + j * w, (int)w), w, c);
+            for (int t = 0; t < 8; t++) {
+                const uint64_t i = 8 * j + (uint64_t)t;
+                if (i >= L) {
+                    if (c[t] != 0) return ORC_CORRUPT; /* unused lanes are zero */
+                    continue;
+                }
+                unsigned e;
+                if (w == 0) {
+                    e = base;
+                } else if (w == 8) {
+                    e = c[t];
+                } else if (c[t] != escape_code(w)) {
+                    e = base + c[t];
+                } else {
+                    if (running + code_bytes + k >= E) return ORC_CORRUPT;
+                    e = payload[code_bytes + k];
+                    k++;
+                    if (in_window(e, base, w)) return ORC_CORRUPT; /* not canonical */
+                }
+                out[b * B + i] = oracle_merge((uint8_t)e, in[s.off_man + b * B + i]);
+            }
+        }
+        const uint64_t size = round_up_16(code_bytes + k);
+        if (running + size > E) return ORC_CORRUPT;
+        if (!all_zero(payload + code_bytes + k, size - code_bytes - k)) return ORC_CORRUPT;
+        running += size;
+    }
+    if (running != E) return ORC_CORRUPT;
+    return ORC_OK;
 }

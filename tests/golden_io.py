@@ -21,7 +21,15 @@ def _expand(tokens):
 
 def load(name: str):
     """Returns (block, words uint16, expected stream uint8)."""
+    block, words, expected, _ = load_kind(name)
+    return block, words, expected
+
+
+def load_kind(name: str):
+    """Returns (block, words uint16, expected stream uint8, kind): kind is "plain"
+    or "escape" (an escape-coded stream, the fixture's "kind escape" line)."""
     block = total = None
+    kind = "plain"
     words, runs = [], []
     with open(os.path.join(GOLDEN_DIR, name)) as f:
         for line in f:
@@ -29,7 +37,9 @@ def load(name: str):
             if not line:
                 continue
             key, _, rest = line.partition(" ")
-            if key == "block":
+            if key == "kind":
+                kind = rest.strip()
+            elif key == "block":
                 block = int(rest)
             elif key == "words":
                 words += _expand(rest.split())
@@ -43,8 +53,10 @@ def load(name: str):
     expected = np.zeros(total, dtype=np.uint8)
     for off, data in runs:
         expected[off:off + len(data)] = data
-    return block, np.array(words, dtype=np.uint16), expected
+    return block, np.array(words, dtype=np.uint16), expected, kind
 
 
-def names():
-    return sorted(f for f in os.listdir(GOLDEN_DIR) if f.endswith(".txt") and f != "README.txt")
+def names(kind: str = "plain"):
+    """Fixture files holding streams of the given kind."""
+    files = sorted(f for f in os.listdir(GOLDEN_DIR) if f.endswith(".txt") and f != "README.txt")
+    return [f for f in files if load_kind(f)[3] == kind]
