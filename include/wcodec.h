@@ -219,6 +219,50 @@ int wc_decompress_batch(const wc_batch_item *h_items, uint32_t count,
                         int32_t *d_status, void *stream);
 
 /*
+ * Escape-coded streams (header flags bit 1): the same fixed-length block code,
+ * but a block's w-bit codes cover only a window of 2^w - 1 exponents
+ * [base, base + 2^w - 2]; the code 2^w - 1 is an escape, and the escaped
+ * elements' exponent bytes follow the block's codes, in element order, as its
+ * exception list; each block's payload is padded to 16 bytes. Per block the
+ * encoder takes the (w, base) of least size ceil(L/8)*w + exceptions (ties to
+ * the smaller w, then the larger base; one exponent only: w = 0; nothing
+ * smaller than raw: w = 8), with base + 2^w - 1 <= 255. On Gaussian weights
+ * this settles on w = 3 with a few percent of exceptions, where the plain
+ * stream needs w = 4 or 5 ("ZipServ: Fast and Memory-Efficient LLM Inference
+ * with Hardware-Aware Lossless Compression", Abstract: a fixed-length format
+ * that decodes in constant time and in parallel and shrinks weights further;
+ * the layout is this library's). Decoding stays constant-time per element:
+ * an escaped element's exception is found by a prefix count of the escapes
+ * before it in its block.
+ *
+ *  wc_bound_escape           output capacity the encoder needs (every block
+ *                            raw, payloads padded to 16 bytes); 0 if invalid
+ *  wc_workspace_size_escape  device workspace bytes of wc_compress_escape
+ *                            (4 bytes per block + 16 per 4096 blocks + 16)
+ *  wc_compress_escape        arguments as wc_compress; d_workspace is
+ *                            overwritten and need not be cleared; nothing in
+ *                            it waits, so d_status is never written
+ *  wc_decompress_escape      arguments as wc_decompress; the kernels check
+ *                            the header (flags 2), w <= 8, base 0 when raw,
+ *                            base + 2^w - 1 <= 255, that every payload holds
+ *                            its codes and exceptions and has the size they
+ *                            imply, and every read against stream_bytes;
+ *                            WC_ERR_CORRUPT_STREAM in *d_status otherwise
+ *  wc_decompress_escape_batch  wc_decompress_batch for escape-coded streams
+ * A plain stream given to an escape-coded decoder, or the other way round, is
+ * reported as WC_ERR_CORRUPT_STREAM.
+ */
+uint64_t wc_bound_escape(uint64_t n, uint32_t block);
+uint64_t wc_workspace_size_escape(uint64_t n, uint32_t block);
+int wc_compress_escape(const void *d_in, uint64_t n, uint32_t block, void *d_out,
+                       uint64_t out_capacity, uint64_t *d_out_bytes, void *d_workspace,
+                       uint64_t workspace_bytes, int32_t *d_status, void *stream);
+int wc_decompress_escape(const void *d_stream, uint64_t stream_bytes, void *d_out, uint64_t n,
+                         uint32_t block, int32_t *d_status, void *stream);
+int wc_decompress_escape_batch(const wc_batch_item *h_items, uint32_t count,
+                               int32_t *d_status, void *stream);
+
+/*
  * FP32 tensors ("ENEC: A Lossless AI Model Compression Method Enabling Fast
  * Inference on Ascend NPUs", Abstract: the method targets AI model weights in
  * general). The high 16 bits of an FP32 word have the BF16 layout, so the
@@ -304,8 +348,8 @@ int wc_gemm_batch(const wc_gemv_item *h_items, uint32_t count, uint32_t tokens,
 /*
  * Parse a host copy of a stream's first `header_bytes` (>= 128) bytes. Fills
  * n, block and total_bytes (any may be NULL). Returns WC_ERR_CORRUPT_STREAM
- * if the header is not a WCB1 version-1 header consistent with itself (BF16
- * or FP32 stream; header bytes 12..15 say which).
+ * if the header is not a WCB1 version-1 header consistent with itself (BF16,
+ * FP32 or escape-coded stream; header bytes 12..15 say which).
  */
 int wc_stream_info(const void *h_header, uint64_t header_bytes,
                    uint64_t *n, uint32_t *block, uint64_t *total_bytes);

@@ -226,7 +226,7 @@ int wc_decompress_fp32(const void* d_stream, uint64_t stream_bytes, void* d_out,
     if (rc != WC_OK) return rc;
     const wc::DecodeItem d = to_item(it);
     const cudaError_t err =
-        wc::launch_decode(&d, 1, d_status, static_cast<cudaStream_t>(stream), true);
+        wc::launch_decode(&d, 1, d_status, static_cast<cudaStream_t>(stream), wc::kKindF32);
     return err == cudaSuccess ? WC_OK : WC_ERR_CUDA;
 }
 
@@ -243,6 +243,62 @@ int wc_decompress_batch(const wc_batch_item* h_items, uint32_t count, int32_t* d
         for (uint32_t i = 0; i < c; ++i) chunk[i] = to_item(h_items[base + i]);
         const cudaError_t err =
             wc::launch_decode(chunk, c, d_status, static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return WC_ERR_CUDA;
+    }
+    return WC_OK;
+}
+
+uint64_t wc_bound_escape(uint64_t n, uint32_t block) {
+    return args_ok(n, block) ? wc::bound_bytes_escape(n, block) : 0;
+}
+
+uint64_t wc_workspace_size_escape(uint64_t n, uint32_t block) {
+    return args_ok(n, block) ? wc::escape_workspace_bytes(n, block) : 0;
+}
+
+int wc_compress_escape(const void* d_in, uint64_t n, uint32_t block, void* d_out,
+                       uint64_t out_capacity, uint64_t* d_out_bytes, void* d_workspace,
+                       uint64_t workspace_bytes, int32_t* d_status, void* stream) {
+    if (!args_ok(n, block) || d_out == nullptr || d_out_bytes == nullptr ||
+        d_workspace == nullptr || (n > 0 && d_in == nullptr))
+        return WC_ERR_INVALID_ARG;
+    if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) || !aligned16(d_workspace) ||
+        (reinterpret_cast<uintptr_t>(d_out_bytes) & 7u) != 0)
+        return WC_ERR_INVALID_ARG;
+    if (out_capacity < wc::bound_bytes_escape(n, block) ||
+        workspace_bytes < wc::escape_workspace_bytes(n, block))
+        return WC_ERR_BUFFER_TOO_SMALL;
+    const wc::EncodeItem item = to_encode_item(d_in, n, block, d_out, d_out_bytes);
+    const cudaError_t err =
+        wc::launch_encode_escape(item, d_workspace, d_status, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
+int wc_decompress_escape(const void* d_stream, uint64_t stream_bytes, void* d_out, uint64_t n,
+                         uint32_t block, int32_t* d_status, void* stream) {
+    wc_batch_item it;
+    it.stream = d_stream;
+    it.stream_bytes = stream_bytes;
+    it.out = d_out;
+    it.n = n;
+    it.block = block;
+    it.reserved = 0;
+    return wc_decompress_escape_batch(&it, 1, d_status, stream);
+}
+
+int wc_decompress_escape_batch(const wc_batch_item* h_items, uint32_t count, int32_t* d_status,
+                               void* stream) {
+    if (h_items == nullptr && count > 0) return WC_ERR_INVALID_ARG;
+    for (uint32_t i = 0; i < count; ++i) {  // validate everything before launching anything
+        const int rc = check_decode_item(h_items[i]);
+        if (rc != WC_OK) return rc;
+    }
+    wc::DecodeItem chunk[WC_BATCH_MAX];
+    for (uint32_t base = 0; base < count; base += WC_BATCH_MAX) {
+        const uint32_t c = (count - base < WC_BATCH_MAX) ? count - base : WC_BATCH_MAX;
+        for (uint32_t i = 0; i < c; ++i) chunk[i] = to_item(h_items[base + i]);
+        const cudaError_t err = wc::launch_decode(chunk, c, d_status,
+                                                  static_cast<cudaStream_t>(stream), wc::kKindEscape);
         if (err != cudaSuccess) return WC_ERR_CUDA;
     }
     return WC_OK;
@@ -362,13 +418,13 @@ int wc_stream_info(const void* h_header, uint64_t header_bytes, uint64_t* n, uin
     const uint32_t B = uint32_t(get_le(p + 8, 4));
     const uint64_t flags = get_le(p + 12, 4);
     if (get_le(p, 4) != wc::kMagic || get_le(p + 4, 2) != wc::kVersion ||
-        get_le(p + 6, 2) != wc::kHeaderBytes || flags > 1 || !args_ok(nn, B))
+        get_le(p + 6, 2) != wc::kHeaderBytes || flags > 2 || !args_ok(nn, B))
         return WC_ERR_CORRUPT_STREAM;
-    const wc::Layout L = wc::make_layout(nn, B, flags == 1);
+    const wc::Layout L = wc::make_layout(nn, B, flags == 1);  // escape-coded: the BF16 layout
     const uint64_t E = get_le(p + 64, 8), total = get_le(p + 72, 8);
     if (get_le(p + 24, 8) != L.nb || get_le(p + 32, 8) != L.off_hdr ||
         get_le(p + 40, 8) != L.off_offs || get_le(p + 48, 8) != L.off_man ||
-        get_le(p + 56, 8) != L.off_exp || E > nn + 8 || total != L.off_exp + E)
+        get_le(p + 56, 8) != L.off_exp || E > nn + 16 || total != L.off_exp + E)
         return WC_ERR_CORRUPT_STREAM;
     if (get_le(p + 80, 8) != L.off_low) return WC_ERR_CORRUPT_STREAM;
     for (int k = 88; k < 128; ++k)

@@ -30,9 +30,16 @@
 //
 // A batch of tensors is one launch: the per-tensor descriptors travel as
 // launch parameters and the producer advances through them as its tiles do.
+//
+// Escape-coded streams (header flags bit 1) use the same ring; their consumer
+// warps each own a 1024-element segment of the tile, so that an escaped
+// element's place in its block's exception list is a warp prefix count of the
+// escapes before it (segmented by block for B < 1024, carried across the
+// segment's two steps for B >= 1024, and counted over the earlier segments of
+// the block for B > 1024).
 #include <mutex>
 
-#include "wc_decode_core.cuh"
+#include "wc_escape_core.cuh"
 
 namespace wc {
 namespace {
@@ -40,9 +47,10 @@ namespace {
 constexpr int kConsumerWarps = kThreads / 32;  // 8
 constexpr int kProducerWarp = kConsumerWarps;
 constexpr int kDecodeThreads = kThreads + 32;  // 288
+constexpr int kSegment = kTile / kConsumerWarps;  // 1024: an escape consumer warp's share of a tile
 // FP32 stages also hold the tile's low halves (16 KB), so they are fewer.
-template <bool F32>
-constexpr int stages_of() { return F32 ? 3 : 4; }
+template <int KIND>
+constexpr int stages_of() { return KIND == kKindF32 ? 3 : 4; }
 
 template <int MAXI>
 struct DecodeParams {
@@ -63,34 +71,42 @@ struct __align__(16) StageInfo {
 // Per-block decode constants, computed once per block by the producer.
 //   t0 = {byte offset of the block's payload in the staged bytes, w, 2w, 4w}
 //   t1 = {M1 = m1 | m1 << 16, m2, m4, base * 0x00800080}, mk = 2^k - 1 (m4 = ~0 when 4w = 32)
-template <bool F32>
+// (escape-coded streams: see commit_tile_meta_escape)
+template <int KIND>
 struct __align__(16) Stage {
     uint8_t man[kTile];
     uint8_t exp[kTile + 16];
-    uint16_t low[F32 ? kTile : 8];  // FP32: the tile's low halves
+    uint16_t low[KIND == kKindF32 ? kTile : 8];  // FP32: the tile's low halves
     uint4 t0[kMaxBlocksPerTile];
     uint4 t1[kMaxBlocksPerTile];
     StageInfo info;
 };
 
-template <bool F32>
+template <int KIND>
 struct DecodeSmem {
-    static constexpr int kStages = stages_of<F32>();
-    Stage<F32> stage[kStages];
+    static constexpr int kStages = stages_of<KIND>();
+    Stage<KIND> stage[kStages];
     unsigned long long full[kStages];
     unsigned long long empty[kStages];
+    uint4 patch[KIND == kKindEscape ? kThreads : 1];  // escape-coded: each thread's 16 exponent bytes
     int abort;
 };
 
 // ---------------------------------------------------------------------------
 // producer: one warp
 // ---------------------------------------------------------------------------
-template <int MAXI, bool F32>
-__device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem<F32>& sm, int lane) {
-    constexpr int kStages = DecodeSmem<F32>::kStages;
+template <int KIND>
+__device__ __forceinline__ Layout layout_of_kind(uint64_t n, uint32_t B) {
+    return KIND == kKindEscape ? make_layout_escape(n, B) : make_layout(n, B, KIND == kKindF32);
+}
+
+template <int MAXI, int KIND>
+__device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem<KIND>& sm, int lane) {
+    constexpr int kStages = DecodeSmem<KIND>::kStages;
+    constexpr bool F32 = KIND == kKindF32;
     uint32_t it = 0;
     DecodeItem I = P.item[0];
-    Layout L = make_layout(I.n, I.block, F32);
+    Layout L = layout_of_kind<KIND>(I.n, I.block);
     int issued_round[kStages];  // last round whose bulk copies were issued, per stage
     for (int s = 0; s < kStages; ++s) issued_round[s] = -1;
     for (uint64_t i = 0;; ++i) {
@@ -112,11 +128,11 @@ __device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem<F32>& sm, int la
         if (t >= P.tile_begin[it + 1]) {  // tiles only move forward: advance the item
             while (t >= P.tile_begin[it + 1]) ++it;
             I = P.item[it];
-            L = make_layout(I.n, I.block, F32);
+            L = layout_of_kind<KIND>(I.n, I.block);
         }
         const uint64_t lt = t - P.tile_begin[it];
         if (lt == 0 && lane == 0) check_container(I, L, P.status);
-        Stage<F32>& st = sm.stage[s];
+        Stage<KIND>& st = sm.stage[s];
 
         uint32_t tile_n = 0, len16 = 0, man_bytes = 0;
         uint64_t start = 0;
@@ -125,8 +141,12 @@ __device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem<F32>& sm, int la
             const uint64_t tile_start = lt * kTile;
             tile_n = uint32_t(min(uint64_t(kTile), L.n - tile_start));
             const TileMeta meta = load_tile_meta(I.stream, L, tile_start, tile_n, lane);
-            bad = !commit_tile_meta(meta, I.stream, L, I.stream_bytes, tile_n, st.t0, st.t1,
-                                    st.exp, start, len16, lane);
+            if (KIND == kKindEscape)
+                bad = !commit_tile_meta_escape(meta, I.stream, L, I.stream_bytes, tile_n, st.t0,
+                                               st.t1, st.exp, start, len16, lane);
+            else
+                bad = !commit_tile_meta(meta, I.stream, L, I.stream_bytes, tile_n, st.t0, st.t1,
+                                        st.exp, start, len16, lane);
             if (!bad) {
                 man_bytes = (tile_n + 15u) & ~15u;  // inside the 128-byte padded plane
                 if (lane == 0) {  // FP32 outputs are 32-bit words
@@ -171,9 +191,10 @@ __device__ __forceinline__ uint4 join_fp32(uint32_t hi01, uint32_t lo01, uint32_
                       prmt(lo23, hi23, 0x5410u), prmt(lo23, hi23, 0x7632u));
 }
 
-template <int MAXI, bool F32>
-__device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem<F32>& sm, int tid, int lane) {
-    constexpr int kStages = DecodeSmem<F32>::kStages;
+template <int MAXI, int KIND>
+__device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem<KIND>& sm, int tid, int lane) {
+    constexpr int kStages = DecodeSmem<KIND>::kStages;
+    constexpr bool F32 = KIND == kKindF32;
     for (uint64_t i = 0;; ++i) {
         const uint64_t t = blockIdx.x + i * gridDim.x;
         if (t >= P.total_tiles) break;
@@ -186,7 +207,7 @@ __device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem<F32>& sm, int ti
             }
             return;
         }
-        const Stage<F32>& st = sm.stage[s];
+        const Stage<KIND>& st = sm.stage[s];
         const StageInfo info = st.info;
         const uint32_t bmask = (1u << info.log2B) - 1u;
 #pragma unroll
@@ -233,12 +254,134 @@ __device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem<F32>& sm, int ti
     }
 }
 
-template <int MAXI, bool F32>
+// ---------------------------------------------------------------------------
+// consumers of escape-coded streams: eight warps, one 1024-element segment each
+// ---------------------------------------------------------------------------
+// Escapes among the codes of tile elements [from, to) (all in one block, to - from
+// a multiple of 512), counted by the whole warp.
+__device__ __forceinline__ uint32_t count_escapes(const Stage<kKindEscape>& st, uint32_t from,
+                                                  uint32_t to, uint32_t log2B, int lane) {
+    const uint32_t bmask = (1u << log2B) - 1u;
+    const uint4 t0 = st.t0[from >> log2B], t1 = st.t1[from >> log2B];
+    uint32_t cnt = 0;
+    for (uint32_t el = from + 16u * uint32_t(lane); el < to; el += 512u) {
+        uint32_t E[4];
+        const uint32_t q = t0.x + ((el & bmask) >> 3) * t0.y;
+        cnt += __popc(chunk_exponents_w(t0.y, st.exp, q, t1.x, t1.y, E));
+    }
+    return __reduce_add_sync(0xFFFFFFFFu, cnt);
+}
+
+template <int MAXI>
+__device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEscape>& sm, int tid,
+                               int lane, int warp) {
+    constexpr int kStages = DecodeSmem<kKindEscape>::kStages;
+    uint8_t* patch = reinterpret_cast<uint8_t*>(&sm.patch[tid]);
+    for (uint64_t i = 0;; ++i) {
+        const uint64_t t = blockIdx.x + i * gridDim.x;
+        if (t >= P.total_tiles) break;
+        const int s = int(i % kStages);
+        const uint32_t round = uint32_t(i / kStages);
+        if (!mbar_wait(&sm.full[s], round & 1u, &sm.abort)) {
+            if (lane == 0) {
+                report(P.status, kStatusTimeout);
+                sm.abort = 1;
+            }
+            return;
+        }
+        const Stage<kKindEscape>& st = sm.stage[s];
+        const StageInfo info = st.info;
+        const uint32_t log2B = info.log2B, B = 1u << log2B, bmask = B - 1u;
+        const uint32_t group = min(B >> 4, 32u);  // lanes that hold one block in a 512-element step
+        const uint32_t seg = uint32_t(warp) * kSegment;
+        bool bad = false;
+        if (seg < info.tile_n) {  // the same for the whole warp
+            // escapes of the current block before the current step
+            uint32_t carry = 0;
+            if (B > uint32_t(kSegment) && (seg & bmask) != 0u)
+                carry = count_escapes(st, seg & ~bmask, seg, log2B, lane);
+#pragma unroll
+            for (int k = 0; k < kSegment / 512; ++k) {
+                const uint32_t step = seg + 512u * k;
+                if (step >= info.tile_n) break;
+                const uint32_t el = step + 16u * uint32_t(lane);
+                const bool active = el < info.tile_n;
+                const uint32_t bl = el >> log2B;  // < kMaxBlocksPerTile, since el < kTile
+                const uint4 t0 = st.t0[bl], t1 = st.t1[bl];
+                uint32_t E[4] = {0u, 0u, 0u, 0u};
+                uint32_t m16 = 0;
+                uint4 M = make_uint4(0u, 0u, 0u, 0u);
+                if (active) {
+                    M = *reinterpret_cast<const uint4*>(st.man + el);
+                    const uint32_t q = t0.x + ((el & bmask) >> 3) * t0.y;
+                    m16 = chunk_exponents_w(t0.y, st.exp, q, t1.x, t1.y, E);
+                    // the last chunk of a stream: bits past the block's codes are not
+                    // codes (they hold its exceptions and padding)
+                    if (info.tile_n - el < uint32_t(kChunk)) m16 &= (1u << (info.tile_n - el)) - 1u;
+                }
+                // each chunk's first exception: a prefix count over the block's chunks
+                const uint32_t c = __popc(m16);
+                uint32_t incl = c;
+                for (uint32_t d = 1; d < group; d <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d, int(group));
+                    if ((uint32_t(lane) & (group - 1u)) >= d) incl += y;
+                }
+                const uint32_t before = carry + incl - c;
+                if (B >= uint32_t(kSegment)) carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
+                if (!active) continue;
+                if (m16) {
+                    // this chunk's exceptions are staged bytes [p, p + c) of its block's payload
+                    const uint32_t p = t0.x + t0.z + before;
+                    if (p + c > t0.w) {
+                        bad = true;
+                    } else {
+                        *reinterpret_cast<uint4*>(patch) = make_uint4(E[0], E[1], E[2], E[3]);
+                        uint32_t mm = m16, pp = p;
+                        do {
+                            patch[__ffs(int(mm)) - 1] = st.exp[pp++];
+                            mm &= mm - 1u;
+                        } while (mm);
+                        const uint4 v = *reinterpret_cast<const uint4*>(patch);
+                        E[0] = v.x;
+                        E[1] = v.y;
+                        E[2] = v.z;
+                        E[3] = v.w;
+                    }
+                }
+                // the lane holding the block's last element checks its payload size
+                const uint32_t blk_end = min((bl + 1u) << log2B, info.tile_n);
+                if (blk_end - el <= uint32_t(kChunk) &&
+                    ((t0.z + before + c + 15u) & ~15u) != t0.w - t0.x)
+                    bad = true;
+                uint4 r0, r1;
+                merge_quad(E[0], M.x, r0.x, r0.y);
+                merge_quad(E[1], M.y, r0.z, r0.w);
+                merge_quad(E[2], M.z, r1.x, r1.y);
+                merge_quad(E[3], M.w, r1.z, r1.w);
+                uint16_t* dst = info.out + el;
+                if (info.tile_n - el >= uint32_t(kChunk)) {
+                    st_stream_v4(dst, r0);
+                    st_stream_v4(dst + 8, r1);
+                } else {
+                    const uint32_t words[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+                    const uint32_t nv = info.tile_n - el;
+                    for (uint32_t e = 0; e < nv; ++e)
+                        dst[e] = uint16_t(words[e >> 1] >> (16 * (e & 1)));
+                }
+            }
+        }
+        if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) report(P.status, kStatusCorrupt);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[s]);
+    }
+}
+
+template <int MAXI, int KIND>
 __global__ void __launch_bounds__(kDecodeThreads)
     decode_kernel(const __grid_constant__ DecodeParams<MAXI> P) {
-    constexpr int kStages = DecodeSmem<F32>::kStages;
+    constexpr int kStages = DecodeSmem<KIND>::kStages;
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    DecodeSmem<F32>& sm = *reinterpret_cast<DecodeSmem<F32>*>(smem_raw);
+    DecodeSmem<KIND>& sm = *reinterpret_cast<DecodeSmem<KIND>*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -250,14 +393,16 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
     __syncthreads();
     if (warp == kProducerWarp)
-        produce<MAXI, F32>(P, sm, lane);
+        produce<MAXI, KIND>(P, sm, lane);
+    else if constexpr (KIND == kKindEscape)
+        consume_escape<MAXI>(P, sm, tid, lane, warp);
     else
-        consume<MAXI, F32>(P, sm, tid, lane);
+        consume<MAXI, KIND>(P, sm, tid, lane);
 }
 
 // Persistent grid: as many resident thread blocks as the SMs hold, never more
 // than there are tiles. Computed once per device and kernel instantiation.
-template <int MAXI, bool F32>
+template <int MAXI, int KIND>
 cudaError_t grid_for(uint64_t tiles, unsigned* grid) {
     static std::mutex mu;
     static int per_device[64];  // 0 = not yet known
@@ -267,15 +412,15 @@ cudaError_t grid_for(uint64_t tiles, unsigned* grid) {
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
     if (per_device[dev] == 0) {
-        err = cudaFuncSetAttribute(decode_kernel<MAXI, F32>,
+        err = cudaFuncSetAttribute(decode_kernel<MAXI, KIND>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   int(sizeof(DecodeSmem<F32>)));
+                                   int(sizeof(DecodeSmem<KIND>)));
         if (err != cudaSuccess) return err;
         int sms = 0, per_sm = 0;
         err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (err != cudaSuccess) return err;
-        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<MAXI, F32>,
-                                                            kDecodeThreads, sizeof(DecodeSmem<F32>));
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<MAXI, KIND>,
+                                                            kDecodeThreads, sizeof(DecodeSmem<KIND>));
         if (err != cudaSuccess) return err;
         per_device[dev] = (per_sm > 0 ? per_sm : 1) * sms;
     }
@@ -284,7 +429,7 @@ cudaError_t grid_for(uint64_t tiles, unsigned* grid) {
     return cudaSuccess;
 }
 
-template <int MAXI, bool F32>
+template <int MAXI, int KIND>
 cudaError_t launch_batch(const DecodeItem* items, uint32_t count, int32_t* status,
                          cudaStream_t stream) {
     static_assert(sizeof(DecodeParams<MAXI>) <= 32000, "launch parameters exceed the limit");
@@ -303,9 +448,9 @@ cudaError_t launch_batch(const DecodeItem* items, uint32_t count, int32_t* statu
     p.total_tiles = tiles;
     if (tiles == 0) return cudaSuccess;
     unsigned grid = 0;
-    cudaError_t err = grid_for<MAXI, F32>(tiles, &grid);
+    cudaError_t err = grid_for<MAXI, KIND>(tiles, &grid);
     if (err != cudaSuccess) return err;
-    decode_kernel<MAXI, F32><<<grid, kDecodeThreads, sizeof(DecodeSmem<F32>), stream>>>(p);
+    decode_kernel<MAXI, KIND><<<grid, kDecodeThreads, sizeof(DecodeSmem<KIND>), stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -313,22 +458,29 @@ cudaError_t launch_batch(const DecodeItem* items, uint32_t count, int32_t* statu
 
 constexpr uint32_t kBatchMax = 512;
 
+template <int KIND>
+cudaError_t launch_kind(const DecodeItem* items, uint32_t count, int32_t* status,
+                        cudaStream_t stream) {
+    if (count == 1) return launch_batch<1, KIND>(items, 1, status, stream);
+    for (uint32_t i = 0; i < count; i += kBatchMax) {
+        const uint32_t c = min(kBatchMax, count - i);
+        const cudaError_t err = launch_batch<kBatchMax, KIND>(items + i, c, status, stream);
+        if (err != cudaSuccess) return err;
+    }
+    return cudaSuccess;
+}
+
 cudaError_t launch_decode(const DecodeItem* items, uint32_t count, int32_t* status,
-                          cudaStream_t stream, bool fp32) {
-    if (fp32) {  // FP32 streams: one tensor per call
+                          cudaStream_t stream, int kind) {
+    if (kind == kKindF32) {  // FP32 streams: one tensor per call
         for (uint32_t i = 0; i < count; ++i) {
-            const cudaError_t err = launch_batch<1, true>(items + i, 1, status, stream);
+            const cudaError_t err = launch_batch<1, kKindF32>(items + i, 1, status, stream);
             if (err != cudaSuccess) return err;
         }
         return cudaSuccess;
     }
-    if (count == 1) return launch_batch<1, false>(items, 1, status, stream);
-    for (uint32_t i = 0; i < count; i += kBatchMax) {
-        const uint32_t c = min(kBatchMax, count - i);
-        const cudaError_t err = launch_batch<kBatchMax, false>(items + i, c, status, stream);
-        if (err != cudaSuccess) return err;
-    }
-    return cudaSuccess;
+    if (kind == kKindEscape) return launch_kind<kKindEscape>(items, count, status, stream);
+    return launch_kind<kKindPlain>(items, count, status, stream);
 }
 
 }  // namespace wc

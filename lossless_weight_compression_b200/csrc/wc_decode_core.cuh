@@ -92,7 +92,7 @@ __device__ __forceinline__ uint64_t ld_u64(const uint8_t* p) {
 __device__ inline void check_container(const DecodeItem& I, const Layout& L, int32_t* status) {
     const uint8_t* S = I.stream;
     bool bad = ld_u64(S) != (kMagic | (uint64_t(kVersion) << 32) | (uint64_t(kHeaderBytes) << 48));
-    bad |= ld_u64(S + 8) != (uint64_t(L.block) | (uint64_t(L.fp32) << 32));  // block size, flags
+    bad |= ld_u64(S + 8) != (uint64_t(L.block) | (uint64_t(L.flags) << 32));  // block size, flags
     bad |= ld_u64(S + 16) != L.n;
     bad |= ld_u64(S + 24) != L.nb;
     bad |= ld_u64(S + 32) != L.off_hdr;
@@ -100,7 +100,7 @@ __device__ inline void check_container(const DecodeItem& I, const Layout& L, int
     bad |= ld_u64(S + 48) != L.off_man;
     bad |= ld_u64(S + 56) != L.off_exp;
     const uint64_t E = ld_u64(S + 64), total = ld_u64(S + 72);
-    bad |= E > L.n + 8 || total != L.off_exp + E || total > I.stream_bytes;
+    bad |= E > L.n + 16 || total != L.off_exp + E || total > I.stream_bytes;
     bad |= ld_u64(S + 80) != L.off_low;
     for (int k = 88; k < 128; k += 8) bad |= ld_u64(S + k) != 0;
     if (bad) report(status, kStatusCorrupt);

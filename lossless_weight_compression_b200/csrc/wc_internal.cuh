@@ -31,12 +31,18 @@ constexpr int kMaxBlocksPerTile = kTile / 128;                  // 64
 constexpr int32_t kStatusCorrupt = 3;
 constexpr int32_t kStatusTimeout = 5;
 
+// Header flags: bit 0 an FP32 stream, bit 1 an escape-coded stream.
+constexpr uint32_t kFlagF32 = 1;
+constexpr uint32_t kFlagEscape = 2;
+
 // fp32: a stream of FP32 words, whose high halves are coded exactly as BF16
 // words and whose low halves follow the mantissa plane as a raw u16 plane
-// (off_low; 0 for BF16 streams).
+// (off_low; 0 for BF16 streams). Escape-coded streams have the BF16 layout and
+// flags = kFlagEscape.
 struct Layout {
     uint64_t n, nb, off_hdr, off_offs, off_man, off_low, off_exp;
     uint32_t block, log2_block;
+    uint32_t flags;
     bool fp32;
 };
 
@@ -68,6 +74,13 @@ __host__ __device__ inline Layout make_layout(uint64_t n, uint32_t B, bool fp32 
     L.off_low = fp32 ? L.off_man + align128(n) : 0;
     L.off_exp = fp32 ? L.off_low + align128(2 * n) : L.off_man + align128(n);
     L.fp32 = fp32;
+    L.flags = fp32 ? kFlagF32 : 0u;
+    return L;
+}
+
+__host__ __device__ inline Layout make_layout_escape(uint64_t n, uint32_t B) {
+    Layout L = make_layout(n, B, false);
+    L.flags = kFlagEscape;
     return L;
 }
 
@@ -79,6 +92,14 @@ __host__ __device__ inline uint64_t bound_bytes(uint64_t n, uint32_t B, bool fp3
     uint64_t full = n >> L.log2_block;
     uint64_t tail = n - (full << L.log2_block);
     return L.off_exp + full * B + ((tail + 7) / 8) * 8;
+}
+
+// Worst-case escape-coded stream: every block raw, each payload padded to 16 bytes.
+__host__ __device__ inline uint64_t bound_bytes_escape(uint64_t n, uint32_t B) {
+    Layout L = make_layout(n, B, false);
+    uint64_t full = n >> L.log2_block;
+    uint64_t tail = n - (full << L.log2_block);
+    return L.off_exp + full * B + (((tail + 7) / 8) * 8 + 15) / 16 * 16;
 }
 
 // ---------------------------------------------------------------------------
@@ -250,9 +271,18 @@ cudaError_t launch_encode(const EncodeItem* items, uint32_t count, void* workspa
                           int32_t* status, uint64_t timeout_ns, uint32_t first_ticket,
                           cudaStream_t stream, bool fp32 = false);
 
-// fp32: FP32 streams decoded into n u32 words (DecodeItem::out).
+// Stream kinds of the decoder: BF16 (16-bit words), FP32 (decoded into n u32
+// words at DecodeItem::out) and escape-coded 16-bit streams.
+enum StreamKind : int { kKindPlain = 0, kKindF32 = 1, kKindEscape = 2 };
 cudaError_t launch_decode(const DecodeItem* items, uint32_t count, int32_t* status,
-                          cudaStream_t stream, bool fp32 = false);
+                          cudaStream_t stream, int kind = kKindPlain);
+
+// The escape-coded encoder (wc_encode_escape.cu): workspace bytes for one
+// tensor, and the launches that code it (no cross-block waits: a per-block
+// pass, a three-step scan of the block sizes, and a packing pass).
+uint64_t escape_workspace_bytes(uint64_t n, uint32_t B);
+cudaError_t launch_encode_escape(const EncodeItem& item, void* workspace, int32_t* status,
+                                 cudaStream_t stream);
 
 struct GemvItem {
     const uint8_t* stream;  // WCB1 stream of W (rows x cols, row-major BF16)

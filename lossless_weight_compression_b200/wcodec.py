@@ -120,6 +120,14 @@ def lib() -> ctypes.CDLL:
     L.wc_compress_noalloc.restype = i
     L.wc_debug_compress_stalled.argtypes = [vp, u64, u32, vp, u64, vp, vp, u64, vp, u64, vp]
     L.wc_debug_compress_stalled.restype = i
+    L.wc_bound_escape.argtypes, L.wc_bound_escape.restype = [u64, u32], u64
+    L.wc_workspace_size_escape.argtypes, L.wc_workspace_size_escape.restype = [u64, u32], u64
+    L.wc_compress_escape.argtypes = [vp, u64, u32, vp, u64, vp, vp, u64, vp, vp]
+    L.wc_compress_escape.restype = i
+    L.wc_decompress_escape.argtypes = [vp, u64, vp, u64, u32, vp, vp]
+    L.wc_decompress_escape.restype = i
+    L.wc_decompress_escape_batch.argtypes = [ctypes.POINTER(wc_batch_item), u32, vp, vp]
+    L.wc_decompress_escape_batch.restype = i
     _lib = L
     return L
 
@@ -195,6 +203,28 @@ def wc_gemm(d_stream, stream_bytes, rows, cols, block, d_x, tokens, d_y, d_statu
 
 def wc_gemm_batch(items, count, tokens, d_status, stream) -> int:
     return lib().wc_gemm_batch(items, count, tokens, d_status, stream)
+
+
+def wc_bound_escape(n, block) -> int:
+    return lib().wc_bound_escape(n, block)
+
+
+def wc_workspace_size_escape(n, block) -> int:
+    return lib().wc_workspace_size_escape(n, block)
+
+
+def wc_compress_escape(d_in, n, block, d_out, out_capacity, d_out_bytes, d_ws, ws_bytes, d_status,
+                       stream) -> int:
+    return lib().wc_compress_escape(d_in, n, block, d_out, out_capacity, d_out_bytes, d_ws,
+                                    ws_bytes, d_status, stream)
+
+
+def wc_decompress_escape(d_stream, stream_bytes, d_out, n, block, d_status, stream) -> int:
+    return lib().wc_decompress_escape(d_stream, stream_bytes, d_out, n, block, d_status, stream)
+
+
+def wc_decompress_escape_batch(items, count, d_status, stream) -> int:
+    return lib().wc_decompress_escape_batch(items, count, d_status, stream)
 
 
 def wc_stream_info(h_header: bytes):
@@ -483,3 +513,53 @@ def decompress_fp32(stream_bytes: torch.Tensor, n: int, block: int, *,
                             block, status.data_ptr(), _stream_handle(stream))
     _check(rc, "wc_decompress_fp32")
     return out
+
+
+# ---------------------------------------------------------------------------
+# escape-coded streams (a window of 2^w - 1 exponents per block + exceptions)
+# ---------------------------------------------------------------------------
+def compress_escape(x: torch.Tensor, block: int = 1024, *, workspace: torch.Tensor | None = None,
+                    stream=None) -> Compressed:
+    """Compress a CUDA tensor of 16-bit words into an escape-coded stream."""
+    words = as_words(x)
+    n = words.numel()
+    cap = wc_bound_escape(n, block)
+    if cap == 0:
+        raise WcodecError(WC_ERR_INVALID_ARG, "block size %r" % (block,))
+    dev = words.device
+    buf = torch.empty((cap + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+    nbytes = torch.zeros(1, dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    if workspace is None:
+        ws = wc_workspace_size_escape(n, block)
+        workspace = torch.empty((ws + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+    rc = wc_compress_escape(words.data_ptr() if n else None, n, block, buf.data_ptr(),
+                            buf.numel(), nbytes.data_ptr(), workspace.data_ptr(),
+                            workspace.numel(), status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_compress_escape")
+    return Compressed(buf, nbytes, status, n, block, tuple(x.shape), x.dtype)
+
+
+def decompress_escape(stream_bytes: torch.Tensor, n: int, block: int, *,
+                      out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                      nbytes: int | None = None, stream=None) -> torch.Tensor:
+    """Decode an escape-coded stream into n 16-bit values (``out`` if given)."""
+    if out is None:
+        out = torch.empty(n, dtype=torch.bfloat16, device=stream_bytes.device)
+    words = out.view(-1)
+    if words.numel() != n or not words.is_contiguous() or out.element_size() != 2:
+        raise ValueError("out must be a contiguous 16-bit tensor of %d elements" % n)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=stream_bytes.device)
+    size = stream_bytes.numel() if nbytes is None else nbytes
+    rc = wc_decompress_escape(stream_bytes.data_ptr(), size, words.data_ptr() if n else None, n,
+                              block, status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_decompress_escape")
+    return out
+
+
+def decompress_escape_batch(batch, status: torch.Tensor, stream=None):
+    """Decode escape-coded streams (a batch from ``make_batch``), one launch per 512."""
+    arr, count = batch
+    rc = wc_decompress_escape_batch(arr, count, status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_decompress_escape_batch")

@@ -186,3 +186,38 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(wcodec, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="not built"):
         wcodec.lib()
+
+
+def test_escape_bound_matches_oracle(wclib, orc):
+    rng = np.random.default_rng(2)
+    for B in BLOCKS:
+        for n in [0, 1, 7, 8, 9, B - 1, B, B + 1, 8193] + list(rng.integers(0, 10**7, 3)):
+            assert wclib.wc_bound_escape(int(n), B) == orc.bound_escape(int(n), B)
+            assert wclib.wc_workspace_size_escape(int(n), B) >= 16
+    assert wclib.wc_bound_escape(100, 100) == 0 and wclib.wc_workspace_size_escape(100, 100) == 0
+
+
+def test_escape_entry_points_check_arguments_before_launching(wclib):
+    # fake, aligned device addresses: every call below must return before any launch
+    n, B = 10_000, 1024
+    cap, ws = wclib.wc_bound_escape(n, B), wclib.wc_workspace_size_escape(n, B)
+    rc = wclib.wc_compress_escape(1 << 20, n, 1000, 1 << 21, cap, 1 << 22, 1 << 23, ws, None, None)
+    assert rc == wclib.WC_ERR_INVALID_ARG                   # block size
+    rc = wclib.wc_compress_escape(1 << 20, n, B, (1 << 21) + 8, cap, 1 << 22, 1 << 23, ws, None, None)
+    assert rc == wclib.WC_ERR_INVALID_ARG                   # misaligned output
+    rc = wclib.wc_compress_escape(1 << 20, n, B, 1 << 21, cap - 1, 1 << 22, 1 << 23, ws, None, None)
+    assert rc == wclib.WC_ERR_BUFFER_TOO_SMALL              # output capacity
+    rc = wclib.wc_compress_escape(1 << 20, n, B, 1 << 21, cap, 1 << 22, 1 << 23, ws - 1, None, None)
+    assert rc == wclib.WC_ERR_BUFFER_TOO_SMALL              # workspace
+    rc = wclib.wc_decompress_escape(1 << 20, 100, 1 << 21, n, B, None, None)
+    assert rc == wclib.WC_ERR_CORRUPT_STREAM                # shorter than the fixed sections
+    rc = wclib.wc_decompress_escape_batch(None, 3, None, None)
+    assert rc == wclib.WC_ERR_INVALID_ARG
+
+
+def test_stream_info_reads_escape_headers(wclib, orc):
+    words = (np.random.default_rng(3).standard_normal(5000) * 0.02).astype(np.float32)
+    words = (words.view(np.uint32) >> 16).astype(np.uint16)
+    s = orc.compress_escape(words, 256)
+    rc, n, b, total = wclib.wc_stream_info(bytes(s[:128]))
+    assert rc == wclib.WC_OK and (n, b, total) == (5000, 256, s.size)
