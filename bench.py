@@ -438,11 +438,13 @@ def run_wcodec(args):
 
 
 def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stream, dist, dev,
-            n_total):
+            n_total, entry="wc_decompress_batch"):
     """Same metric through the public C-ABI, but each step first copies the
     compressed streams from pinned host memory and ends by reading the status
-    word back; the copies are inside the timed region."""
+    word back; the copies are inside the timed region. `entry` is the batched
+    decoder of the streams' kind."""
     import torch
+    decode_batch = getattr(wc, entry)
     total = sum(sizes)
     try:
         host = torch.empty(total, dtype=torch.uint8, pin_memory=True)
@@ -461,9 +463,9 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
     def step():
         for k, s in enumerate(sizes):
             bufs[k][:s].copy_(views[k], non_blocking=True)
-        rc = wc.wc_decompress_batch(batch[0], batch[1], dec_status.data_ptr(), sh)
+        rc = decode_batch(batch[0], batch[1], dec_status.data_ptr(), sh)
         if rc != 0:
-            raise RuntimeError("wc_decompress_batch: %s" % wc.wc_status_string(rc))
+            raise RuntimeError("%s: %s" % (entry, wc.wc_status_string(rc)))
         status_host.copy_(dec_status, non_blocking=True)
 
     steps = max(1, min(args.steps, 5))
@@ -512,6 +514,146 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
                                "unit": "GB/s", "h2d_bytes_per_step": 2 * n_total,
                                "speedup_of_compressed_path": raw_sec / sec}
     return result
+
+
+# ---------------------------------------------------------------------------
+# next row: escape-coded streams of the whole stack
+# ---------------------------------------------------------------------------
+def run_escape(args):
+    """The 8B-shaped stack as escape-coded streams (a window of 2^w - 1
+    exponents per block plus an exception list): each tensor encoded with
+    wc_compress_escape (five launches per tensor, outside the metric), then the
+    whole stack decoded by one wc_decompress_escape_batch launch per step."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from lossless_weight_compression_b200 import build_lib, synth, wcodec
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    build_lib.build()
+    wc = wcodec.lib()
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    names, inputs = [], []
+    hist = torch.zeros(256, dtype=torch.int64, device=dev)
+    tensors = (synth.stack_tensors(dev, rank_seed_base(rank)) if args.workload == "escape"
+               else synth.layer_tensors(0, dev, rank_seed_base(rank)))
+    for name, t in tensors:
+        words = t.view(-1).view(torch.int16)
+        hist += torch.bincount(((words.to(torch.int32) >> 7) & 0xFF), minlength=256)
+        names.append(name)
+        inputs.append(words)
+    n_total = sum(w.numel() for w in inputs)
+    bufs = [torch.empty((wc.wc_bound_escape(w.numel(), BLOCK) + 15) // 16 * 16, dtype=torch.uint8,
+                        device=dev) for w in inputs]
+    ws_bytes = max(wc.wc_workspace_size_escape(w.numel(), BLOCK) for w in inputs)
+    ws = torch.empty((ws_bytes + 15) // 16 * 16, dtype=torch.uint8, device=dev)
+    nbytes = torch.zeros(len(inputs), dtype=torch.int64, device=dev)
+    status = torch.zeros(2, dtype=torch.int32, device=dev)
+    outs = [torch.empty(w.numel(), dtype=torch.int16, device=dev) for w in inputs]
+
+    def encode_all():
+        for k, w in enumerate(inputs):
+            rc = wc.wc_compress_escape(w.data_ptr(), w.numel(), BLOCK, bufs[k].data_ptr(),
+                                       bufs[k].numel(), nbytes[k:].data_ptr(), ws.data_ptr(),
+                                       ws.numel(), status[0:].data_ptr(), sh)
+            if rc != 0:
+                raise RuntimeError("wc_compress_escape: %s" % wc.wc_status_string(rc))
+
+    encode_all()
+    torch.cuda.synchronize(dev)
+    sizes = nbytes.cpu().tolist()
+    batch = wcodec.make_batch([(bufs[k], sizes[k], outs[k], inputs[k].numel(), BLOCK)
+                               for k in range(len(inputs))])
+    dec_status = status[1:]
+
+    def decode_all():
+        rc = wc.wc_decompress_escape_batch(batch[0], batch[1], dec_status.data_ptr(), sh)
+        if rc != 0:
+            raise RuntimeError("wc_decompress_escape_batch: %s" % wc.wc_status_string(rc))
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        barrier(dist, dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        barrier(dist, dev)
+        return max_over_ranks(e0.elapsed_time(e1) / 1e3 / args.steps, dist, dev)
+
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        t_enc = timed(encode_all)
+        t_dec = timed(decode_all)
+    torch.cuda.synchronize(dev)
+    verified = bool((status == 0).all().item()) and all(
+        torch.equal(a, b) for a, b in zip(inputs, outs)) and nbytes.cpu().tolist() == sizes
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stream, dist,
+                      dev, n_total, entry="wc_decompress_escape_batch")
+    stream_total = sum(sizes)
+    bytes_out = 2 * n_total
+    moved = stream_total + bytes_out
+    peak, peak_kind = hbm_peak()
+    p = hist.double() / hist.sum()
+    H = float(-(p[p > 0] * torch.log2(p[p > 0])).sum())
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        torch.set_num_threads(1)
+        q = [w for nm, w in zip(names, inputs) if nm.endswith("q_proj")][0]
+        qw = q.cpu().numpy().view(np.uint16)
+        oracle.build()
+        t0 = time.perf_counter()
+        sref = oracle.compress_escape(qw, BLOCK)
+        t1 = time.perf_counter()
+        back = oracle.decompress_escape(sref, qw.size, BLOCK)
+        t2 = time.perf_counter()
+        same = bool(np.array_equal(back, qw)) and bool(np.array_equal(
+            sref, bufs[names.index([nm for nm in names if nm.endswith("q_proj")][0])]
+            [:sref.size].cpu().numpy()))
+        cpu = {"value": 2 * qw.size / (t2 - t1) / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": "the first q_proj of the workload (%d elements) copied to the host, "
+                         "encoded then decoded once by the single-threaded C oracle; decode "
+                         "timed (encode %.4f GB/s); oracle stream equals the GPU's: %s"
+                         % (qw.size, 2 * qw.size / (t1 - t0) / 1e9, same)}
+        verified &= same
+    line = {
+        "metric": "escape-coded decode GB/s (BF16 out) & % HBM roofline; compression ratio",
+        "value": world * bytes_out / t_dec / 1e9, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * t_dec, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u16", "data": "synthetic",
+        "config": {"workload": (WORKLOAD if args.workload == "escape" else LAYER_WORKLOAD)
+                   + "; escape-coded streams", "block": BLOCK, "tensors": len(inputs),
+                   "l2": "inputs larger than L2; no flush"},
+        "roofline": {"bound": "hbm", "achieved": moved / t_dec / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": moved / t_dec / 1e9 / peak, "peak_kind": peak_kind,
+                     "kernel": "decode_kernel<512,escape> (one launch per step)",
+                     "algorithmic_bytes_per_launch": moved, "traffic": None},
+        "compression": {"ratio": bytes_out / stream_total, "stream_bytes": stream_total,
+                        "exponent_entropy_bits": H, "entropy_bound_ratio": 16.0 / (8.0 + H)},
+        "encode": {"ms_per_step": 1e3 * t_enc, "gbs_moved": moved / t_enc / 1e9,
+                   "frac_of_peak": moved / t_enc / 1e9 / peak,
+                   "kernels": "esc_params, esc_reduce, esc_top, esc_down, esc_pack per tensor"},
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+        "verified_bit_exact": verified,
+        "cpu_baseline": cpu,
+    }
+    if dist is not None:
+        barrier(dist, dev)
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0 if verified else 1
 
 
 # ---------------------------------------------------------------------------
@@ -765,10 +907,12 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("wcodec", "reference"), default="wcodec")
-    ap.add_argument("--workload", choices=("stack", "layer", "gemv", "gemm", "fp32", "fp16"),
+    ap.add_argument("--workload", choices=("stack", "layer", "gemv", "gemm", "fp32", "fp16",
+                                           "escape", "escape-layer"),
                     default="stack",
                     help="stack: the 8B-shaped stack (the benchmark); layer: one decoder layer "
-                         "(a smaller case for profiling); gemv: fused decode + matrix-vector "
+                         "(a smaller case for profiling); escape / escape-layer: the same as "
+                         "escape-coded streams; gemv: fused decode + matrix-vector "
                          "products over the stack's linear weights; gemm: the same on the "
                          "tensor cores with --tokens activation rows; fp32 / fp16: encode and "
                          "decode of the first --gemv-layers (default 4) layers in that dtype")
@@ -792,6 +936,8 @@ def main(argv=None):
         return run_gemv(args)
     if args.workload in ("fp32", "fp16"):
         return run_dtype(args)
+    if args.workload in ("escape", "escape-layer"):
+        return run_escape(args)
     return run_wcodec(args)
 
 

@@ -38,6 +38,7 @@
 // segment's two steps for B >= 1024, and counted over the earlier segments of
 // the block for B > 1024).
 #include <mutex>
+#include <type_traits>
 
 #include "wc_escape_core.cuh"
 
@@ -78,7 +79,8 @@ struct __align__(16) Stage {
     uint8_t exp[kTile + 16];
     uint16_t low[KIND == kKindF32 ? kTile : 8];  // FP32: the tile's low halves
     uint4 t0[kMaxBlocksPerTile];
-    uint4 t1[kMaxBlocksPerTile];
+    // escape-coded stages keep 8 bytes here, so that three thread blocks fit an SM
+    typename std::conditional<KIND == kKindEscape, uint2, uint4>::type t1[kMaxBlocksPerTile];
     StageInfo info;
 };
 
@@ -141,7 +143,7 @@ __device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem<KIND>& sm, int l
             const uint64_t tile_start = lt * kTile;
             tile_n = uint32_t(min(uint64_t(kTile), L.n - tile_start));
             const TileMeta meta = load_tile_meta(I.stream, L, tile_start, tile_n, lane);
-            if (KIND == kKindEscape)
+            if constexpr (KIND == kKindEscape)
                 bad = !commit_tile_meta_escape(meta, I.stream, L, I.stream_bytes, tile_n, st.t0,
                                                st.t1, st.exp, start, len16, lane);
             else
@@ -258,18 +260,103 @@ __device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem<KIND>& sm, int t
 // consumers of escape-coded streams: eight warps, one 1024-element segment each
 // ---------------------------------------------------------------------------
 // Escapes among the codes of tile elements [from, to) (all in one block, to - from
-// a multiple of 512), counted by the whole warp.
-__device__ __forceinline__ uint32_t count_escapes(const Stage<kKindEscape>& st, uint32_t from,
-                                                  uint32_t to, uint32_t log2B, int lane) {
+// a multiple of 512), counted by the whole warp. Only blocks longer than a
+// consumer warp's segment (B > 1024) need it.
+__device__ __noinline__ uint32_t count_escapes(const Stage<kKindEscape>& st, uint32_t from,
+                                               uint32_t to, uint32_t log2B, int lane) {
     const uint32_t bmask = (1u << log2B) - 1u;
-    const uint4 t0 = st.t0[from >> log2B], t1 = st.t1[from >> log2B];
+    const uint4 t0 = st.t0[from >> log2B];
+    const uint2 t1 = st.t1[from >> log2B];
     uint32_t cnt = 0;
     for (uint32_t el = from + 16u * uint32_t(lane); el < to; el += 512u) {
-        uint32_t E[4];
+        uint32_t E[4], esc[4];
         const uint32_t q = t0.x + ((el & bmask) >> 3) * t0.y;
-        cnt += __popc(chunk_exponents_w(t0.y, st.exp, q, t1.x, t1.y, E));
+        chunk_exponents_w(t0.y, st.exp, q, t1.x, t1.y, E, esc);
+        cnt += escape_count(esc);
     }
     return __reduce_add_sync(0xFFFFFFFFu, cnt);
+}
+
+// One chunk of an escape-coded tile in a consumer lane's registers.
+struct EscChunk {
+    uint32_t el;      // first element (tile-relative)
+    uint32_t E[4];    // exponent bytes
+    uint32_t esc[4];  // escape flags (bit 8t+7 of word j: element 4j+t)
+    uint4 M;          // sign+mantissa bytes
+    uint4 t0;         // its block's constants
+    uint32_t count;   // escapes in the chunk
+    bool active;
+};
+
+__device__ __forceinline__ void load_esc_chunk(const Stage<kKindEscape>& st, uint32_t el,
+                                               uint32_t tile_n, uint32_t log2B, EscChunk& c) {
+    c.el = el;
+    c.active = el < tile_n;
+    c.count = 0;
+    if (!c.active) return;
+    const uint32_t bl = el >> log2B;
+    c.t0 = st.t0[bl];
+    const uint2 t1 = st.t1[bl];
+    c.M = *reinterpret_cast<const uint4*>(st.man + el);
+    const uint32_t q = c.t0.x + ((el & ((1u << log2B) - 1u)) >> 3) * c.t0.y;
+    chunk_exponents_w(c.t0.y, st.exp, q, t1.x, t1.y, c.E, c.esc);
+    const uint32_t nv = tile_n - el;
+    if (nv < uint32_t(kChunk)) {
+        // the last chunk of a stream: bits past the block's codes are not codes
+        // (they hold its exceptions and padding)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int valid = int(nv) - 4 * j;
+            if (valid < 4) c.esc[j] &= valid <= 0 ? 0u : (0xFFFFFFFFu >> (32 - 8 * valid));
+        }
+    }
+    c.count = escape_count(c.esc);
+}
+
+// Patch the chunk's escaped elements with their exceptions (staged bytes
+// [before-th exception of the block, ...)), check the block's payload size if
+// the chunk holds the block's last element, and store the 16 BF16 words.
+__device__ __forceinline__ bool finish_esc_chunk(const Stage<kKindEscape>& st, EscChunk& c,
+                                                 uint32_t before, uint32_t tile_n, uint32_t log2B,
+                                                 uint8_t* patch, uint16_t* out) {
+    bool bad = false;
+    if (c.count) {
+        const uint32_t p = c.t0.x + c.t0.z + before;
+        if (p + c.count > c.t0.w) {
+            bad = true;
+        } else {
+            *reinterpret_cast<uint4*>(patch) = make_uint4(c.E[0], c.E[1], c.E[2], c.E[3]);
+            uint32_t mm = escape_mask(c.esc), pp = p;
+            do {
+                patch[__ffs(int(mm)) - 1] = st.exp[pp++];
+                mm &= mm - 1u;
+            } while (mm);
+            const uint4 v = *reinterpret_cast<const uint4*>(patch);
+            c.E[0] = v.x;
+            c.E[1] = v.y;
+            c.E[2] = v.z;
+            c.E[3] = v.w;
+        }
+    }
+    const uint32_t blk_end = min(((c.el >> log2B) + 1u) << log2B, tile_n);
+    if (blk_end - c.el <= uint32_t(kChunk) &&
+        ((c.t0.z + before + c.count + 15u) & ~15u) != c.t0.w - c.t0.x)
+        bad = true;
+    uint4 r0, r1;
+    merge_quad(c.E[0], c.M.x, r0.x, r0.y);
+    merge_quad(c.E[1], c.M.y, r0.z, r0.w);
+    merge_quad(c.E[2], c.M.z, r1.x, r1.y);
+    merge_quad(c.E[3], c.M.w, r1.z, r1.w);
+    uint16_t* dst = out + c.el;
+    if (tile_n - c.el >= uint32_t(kChunk)) {
+        st_stream_v4(dst, r0);
+        st_stream_v4(dst + 8, r1);
+    } else {
+        const uint32_t words[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+        const uint32_t nv = tile_n - c.el;
+        for (uint32_t e = 0; e < nv; ++e) dst[e] = uint16_t(words[e >> 1] >> (16 * (e & 1)));
+    }
+    return bad;
 }
 
 template <int MAXI>
@@ -291,84 +378,35 @@ __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEsca
         }
         const Stage<kKindEscape>& st = sm.stage[s];
         const StageInfo info = st.info;
-        const uint32_t log2B = info.log2B, B = 1u << log2B, bmask = B - 1u;
+        const uint32_t log2B = info.log2B, B = 1u << log2B;
         const uint32_t group = min(B >> 4, 32u);  // lanes that hold one block in a 512-element step
         const uint32_t seg = uint32_t(warp) * kSegment;
         bool bad = false;
         if (seg < info.tile_n) {  // the same for the whole warp
-            // escapes of the current block before the current step
+            // escapes of the segment's block before the segment
             uint32_t carry = 0;
-            if (B > uint32_t(kSegment) && (seg & bmask) != 0u)
-                carry = count_escapes(st, seg & ~bmask, seg, log2B, lane);
-#pragma unroll
-            for (int k = 0; k < kSegment / 512; ++k) {
-                const uint32_t step = seg + 512u * k;
-                if (step >= info.tile_n) break;
-                const uint32_t el = step + 16u * uint32_t(lane);
-                const bool active = el < info.tile_n;
-                const uint32_t bl = el >> log2B;  // < kMaxBlocksPerTile, since el < kTile
-                const uint4 t0 = st.t0[bl], t1 = st.t1[bl];
-                uint32_t E[4] = {0u, 0u, 0u, 0u};
-                uint32_t m16 = 0;
-                uint4 M = make_uint4(0u, 0u, 0u, 0u);
-                if (active) {
-                    M = *reinterpret_cast<const uint4*>(st.man + el);
-                    const uint32_t q = t0.x + ((el & bmask) >> 3) * t0.y;
-                    m16 = chunk_exponents_w(t0.y, st.exp, q, t1.x, t1.y, E);
-                    // the last chunk of a stream: bits past the block's codes are not
-                    // codes (they hold its exceptions and padding)
-                    if (info.tile_n - el < uint32_t(kChunk)) m16 &= (1u << (info.tile_n - el)) - 1u;
-                }
-                // each chunk's first exception: a prefix count over the block's chunks
-                const uint32_t c = __popc(m16);
-                uint32_t incl = c;
-                for (uint32_t d = 1; d < group; d <<= 1) {
-                    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d, int(group));
-                    if ((uint32_t(lane) & (group - 1u)) >= d) incl += y;
-                }
-                const uint32_t before = carry + incl - c;
-                if (B >= uint32_t(kSegment)) carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
-                if (!active) continue;
-                if (m16) {
-                    // this chunk's exceptions are staged bytes [p, p + c) of its block's payload
-                    const uint32_t p = t0.x + t0.z + before;
-                    if (p + c > t0.w) {
-                        bad = true;
-                    } else {
-                        *reinterpret_cast<uint4*>(patch) = make_uint4(E[0], E[1], E[2], E[3]);
-                        uint32_t mm = m16, pp = p;
-                        do {
-                            patch[__ffs(int(mm)) - 1] = st.exp[pp++];
-                            mm &= mm - 1u;
-                        } while (mm);
-                        const uint4 v = *reinterpret_cast<const uint4*>(patch);
-                        E[0] = v.x;
-                        E[1] = v.y;
-                        E[2] = v.z;
-                        E[3] = v.w;
-                    }
-                }
-                // the lane holding the block's last element checks its payload size
-                const uint32_t blk_end = min((bl + 1u) << log2B, info.tile_n);
-                if (blk_end - el <= uint32_t(kChunk) &&
-                    ((t0.z + before + c + 15u) & ~15u) != t0.w - t0.x)
-                    bad = true;
-                uint4 r0, r1;
-                merge_quad(E[0], M.x, r0.x, r0.y);
-                merge_quad(E[1], M.y, r0.z, r0.w);
-                merge_quad(E[2], M.z, r1.x, r1.y);
-                merge_quad(E[3], M.w, r1.z, r1.w);
-                uint16_t* dst = info.out + el;
-                if (info.tile_n - el >= uint32_t(kChunk)) {
-                    st_stream_v4(dst, r0);
-                    st_stream_v4(dst + 8, r1);
-                } else {
-                    const uint32_t words[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-                    const uint32_t nv = info.tile_n - el;
-                    for (uint32_t e = 0; e < nv; ++e)
-                        dst[e] = uint16_t(words[e >> 1] >> (16 * (e & 1)));
-                }
+            if (B > uint32_t(kSegment) && (seg & (B - 1u)) != 0u)
+                carry = count_escapes(st, seg & ~(B - 1u), seg, log2B, lane);
+            // both 512-element steps of the segment at once: chunk k of this lane
+            // starts at seg + 512k + 16 lane
+            EscChunk c0, c1;
+            load_esc_chunk(st, seg + 16u * uint32_t(lane), info.tile_n, log2B, c0);
+            load_esc_chunk(st, seg + 512u + 16u * uint32_t(lane), info.tile_n, log2B, c1);
+            // one prefix count for both steps: step k's counts in bits [16k, 16k + 16)
+            const uint32_t v = c0.count | (c1.count << 16);
+            uint32_t incl = v;
+            for (uint32_t d = 1; d < group; d <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d, int(group));
+                if ((uint32_t(lane) & (group - 1u)) >= d) incl += y;
             }
+            const uint32_t excl = incl - v;
+            uint32_t before0 = excl & 0xFFFFu, before1 = excl >> 16;
+            if (B >= uint32_t(kSegment)) {  // step 1 continues step 0's block
+                before0 += carry;
+                before1 += carry + (__shfl_sync(0xFFFFFFFFu, incl, 31) & 0xFFFFu);
+            }
+            if (c0.active) bad |= finish_esc_chunk(st, c0, before0, info.tile_n, log2B, patch, info.out);
+            if (c1.active) bad |= finish_esc_chunk(st, c1, before1, info.tile_n, log2B, patch, info.out);
         }
         if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) report(P.status, kStatusCorrupt);
         __syncwarp();

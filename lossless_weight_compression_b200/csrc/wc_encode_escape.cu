@@ -253,8 +253,14 @@ __global__ void __launch_bounds__(kEscThreads) esc_down_kernel(const EscParams P
 // ---------------------------------------------------------------------------
 // pack: one warp per block
 // ---------------------------------------------------------------------------
+// Each warp builds its block's payload (at most B <= 4096 bytes, a raw block's)
+// in shared memory and writes it out with 16-byte stores.
+constexpr int kPackStageBytes = 4096;
+
 __global__ void __launch_bounds__(kEscThreads) esc_pack_kernel(const EscParams P) {
+    __shared__ __align__(16) uint8_t stage_all[kEscWarps][kPackStageBytes];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint8_t* stage = stage_all[warp];
     const Layout& L = P.L;
     for (uint64_t b = uint64_t(blockIdx.x) * kEscWarps + warp; b < L.nb;
          b += uint64_t(gridDim.x) * kEscWarps) {
@@ -265,6 +271,7 @@ __global__ void __launch_bounds__(kEscThreads) esc_pack_kernel(const EscParams P
         const uint32_t code_bytes = ((len + 7) >> 3) * w;
         uint8_t* payload =
             P.out + L.off_exp + 16ull * reinterpret_cast<const uint32_t*>(P.out + L.off_offs)[b];
+        __syncwarp();  // the previous block's payload has left the stage
         const uint16_t* x = P.in + first;
         uint32_t carry = 0;  // escapes of the block before the current step
         for (uint32_t step = 0; step < len; step += 32 * kChunk) {
@@ -314,15 +321,18 @@ __global__ void __launch_bounds__(kEscThreads) esc_pack_kernel(const EscParams P
             carry += __shfl_sync(0xFFFFFFFFu, incl, 31);
             for (uint32_t mm = m16; mm; mm &= mm - 1u) {
                 const uint32_t i = uint32_t(__ffs(int(mm))) - 1u;
-                payload[pos++] = uint8_t(ex[i >> 2] >> (8 * (i & 3u)));
+                stage[pos++] = uint8_t(ex[i >> 2] >> (8 * (i & 3u)));
             }
             if (nv == kChunk)
-                pack_chunk_w(w, V, payload + (el >> 3) * w);
+                pack_chunk_w(w, V, stage + (el >> 3) * w);
             else if (nv)
-                pack_chunk_tail(w, V, payload + (el >> 3) * w, (nv > 8 ? 2u : 1u) * w);
+                pack_chunk_tail(w, V, stage + (el >> 3) * w, (nv > 8 ? 2u : 1u) * w);
         }
         const uint32_t used = code_bytes + carry, padded = (used + 15u) & ~15u;
-        if (uint32_t(lane) < padded - used) payload[used + lane] = 0;
+        if (uint32_t(lane) < padded - used) stage[used + lane] = 0;
+        __syncwarp();
+        for (uint32_t k = 16u * uint32_t(lane); k < padded; k += 16u * 32u)
+            st_stream_v4(payload + k, *reinterpret_cast<const uint4*>(stage + k));
     }
 }
 

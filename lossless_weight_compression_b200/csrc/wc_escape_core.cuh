@@ -82,22 +82,22 @@ __device__ __forceinline__ uint32_t quad_to_bytes(uint32_t Q) {
 }
 
 // The 16 codes of a chunk as exponent bytes: E[j] holds elements 4j..4j+3
-// (base added; escaped elements hold base + 2^W - 1 until patched). Returns the
-// chunk's escape mask, bit t for element t.
+// (base added; escaped elements hold base + 2^W - 1 until patched), and
+// esc[j] has bit 8t+7 set when element 4j+t is escaped.
 template <int W>
-__device__ __forceinline__ uint32_t chunk_exponents(const uint8_t* exp, uint32_t q, uint32_t base4,
-                                                    uint32_t esc_add, uint32_t E[4]) {
+__device__ __forceinline__ void chunk_exponents(const uint8_t* exp, uint32_t q, uint32_t base4,
+                                                uint32_t esc_add, uint32_t E[4], uint32_t esc[4]) {
     if constexpr (W == 0) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) E[j] = base4;
-        return 0u;
+        for (int j = 0; j < 4; ++j) E[j] = base4, esc[j] = 0u;
     } else if constexpr (W == 8) {  // raw block: the codes are the exponents
         const uint4 v = *reinterpret_cast<const uint4*>(exp + q);
         E[0] = v.x;
         E[1] = v.y;
         E[2] = v.z;
         E[3] = v.w;
-        return 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) esc[j] = 0u;
     } else {
         uint32_t X[4] = {0u, 0u, 0u, 0u};
         fetch_chunk_bits<W>(exp, q, X);
@@ -106,34 +106,45 @@ __device__ __forceinline__ uint32_t chunk_exponents(const uint8_t* exp, uint32_t
         V[1] = quad_to_bytes<W>(chunk_quad<W, 1>(X));
         V[2] = quad_to_bytes<W>(chunk_quad<W, 2>(X));
         V[3] = quad_to_bytes<W>(chunk_quad<W, 3>(X));
-        uint32_t m16 = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             // a byte equals 2^W - 1 (the largest value it can hold) exactly when
             // adding 0x80 - (2^W - 1) sets its top bit; no carries leave a byte
-            const uint32_t esc = (V[j] + esc_add) & 0x80808080u;
-            // bits 7, 15, 23, 31 -> bits 28..31 (the products' other bits do not
-            // overlap, so nothing carries into them), then into place
-            m16 |= ((esc * 0x00204081u) >> 28) << (4 * j);
+            esc[j] = (V[j] + esc_add) & 0x80808080u;
             E[j] = V[j] + base4;
         }
-        return m16;
     }
 }
 
-__device__ __forceinline__ uint32_t chunk_exponents_w(uint32_t w, const uint8_t* exp, uint32_t q,
-                                                      uint32_t base4, uint32_t esc_add,
-                                                      uint32_t E[4]) {
+// The escapes of a chunk: their number, from the four escape words at once
+// (their flag bits are moved to distinct positions and counted together).
+__device__ __forceinline__ uint32_t escape_count(const uint32_t esc[4]) {
+    return __popc(esc[0] | (esc[1] >> 1) | (esc[2] >> 2) | (esc[3] >> 3));
+}
+
+// ... and their mask, bit t for element t: bits 7, 15, 23, 31 of a word go to
+// bits 28..31 of one product (its other bits do not overlap, so nothing
+// carries into them), then into place.
+__device__ __forceinline__ uint32_t escape_mask(const uint32_t esc[4]) {
+    uint32_t m16 = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m16 |= ((esc[j] * 0x00204081u) >> 28) << (4 * j);
+    return m16;
+}
+
+__device__ __forceinline__ void chunk_exponents_w(uint32_t w, const uint8_t* exp, uint32_t q,
+                                                  uint32_t base4, uint32_t esc_add, uint32_t E[4],
+                                                  uint32_t esc[4]) {
     switch (w) {
-        case 0: return chunk_exponents<0>(exp, q, base4, esc_add, E);
-        case 1: return chunk_exponents<1>(exp, q, base4, esc_add, E);
-        case 2: return chunk_exponents<2>(exp, q, base4, esc_add, E);
-        case 3: return chunk_exponents<3>(exp, q, base4, esc_add, E);
-        case 4: return chunk_exponents<4>(exp, q, base4, esc_add, E);
-        case 5: return chunk_exponents<5>(exp, q, base4, esc_add, E);
-        case 6: return chunk_exponents<6>(exp, q, base4, esc_add, E);
-        case 7: return chunk_exponents<7>(exp, q, base4, esc_add, E);
-        default: return chunk_exponents<8>(exp, q, base4, esc_add, E);
+        case 0: chunk_exponents<0>(exp, q, base4, esc_add, E, esc); break;
+        case 1: chunk_exponents<1>(exp, q, base4, esc_add, E, esc); break;
+        case 2: chunk_exponents<2>(exp, q, base4, esc_add, E, esc); break;
+        case 3: chunk_exponents<3>(exp, q, base4, esc_add, E, esc); break;
+        case 4: chunk_exponents<4>(exp, q, base4, esc_add, E, esc); break;
+        case 5: chunk_exponents<5>(exp, q, base4, esc_add, E, esc); break;
+        case 6: chunk_exponents<6>(exp, q, base4, esc_add, E, esc); break;
+        case 7: chunk_exponents<7>(exp, q, base4, esc_add, E, esc); break;
+        default: chunk_exponents<8>(exp, q, base4, esc_add, E, esc); break;
     }
 }
 
@@ -148,7 +159,7 @@ __device__ __forceinline__ void merge_quad(uint32_t E, uint32_t S, uint32_t& lo,
 // block's decode constants:
 //   t0 = {payload start within the staged bytes, w, code bytes ceil(L/8)*w,
 //         payload end within the staged bytes}
-//   t1 = {base * 0x01010101, (0x80 - (2^w - 1)) * 0x01010101 for 1 <= w <= 7, 0, 0}
+//   t1 = {base * 0x01010101, (0x80 - (2^w - 1)) * 0x01010101 for 1 <= w <= 7}
 // Checks: w <= 8; base 0 when w == 8; base + 2^w - 1 <= 255 when 1 <= w <= 7;
 // every payload holds its codes and is no longer than a raw block's (16-byte
 // padded); the tile's payload inside stream_bytes. The exact payload size
@@ -157,7 +168,7 @@ __device__ __forceinline__ void merge_quad(uint32_t E, uint32_t S, uint32_t& lo,
 // Called by all 32 lanes of a warp.
 __device__ inline bool commit_tile_meta_escape(const TileMeta& m, const uint8_t* S,
                                                const Layout& L, uint64_t stream_bytes,
-                                               uint32_t tile_n, uint4* t0, uint4* t1,
+                                               uint32_t tile_n, uint4* t0, uint2* t1,
                                                uint8_t* exp_stage, uint64_t& start,
                                                uint32_t& len16, int lane) {
     const uint32_t log2B = L.log2_block, B = L.block;
@@ -193,8 +204,8 @@ __device__ inline bool commit_tile_meta_escape(const TileMeta& m, const uint8_t*
             const uint32_t m1 = (1u << w) - 1u;
             t0[b] = make_uint4(uint32_t(m.sb[j] - start), w, ((len + 7) >> 3) * w,
                                uint32_t(m.nx[j] - start));
-            t1[b] = make_uint4(base * 0x01010101u,
-                               (w >= 1u && w <= 7u) ? (0x80u - m1) * 0x01010101u : 0u, 0u, 0u);
+            t1[b] = make_uint2(base * 0x01010101u,
+                               (w >= 1u && w <= 7u) ? (0x80u - m1) * 0x01010101u : 0u);
         }
     }
     const uint32_t len = uint32_t(end - start);
