@@ -90,7 +90,6 @@ struct DecodeSmem {
     Stage<KIND> stage[kStages];
     unsigned long long full[kStages];
     unsigned long long empty[kStages];
-    uint4 patch[KIND == kKindEscape ? kThreads : 1];  // escape-coded: each thread's 16 exponent bytes
     int abort;
 };
 
@@ -271,7 +270,7 @@ __device__ __noinline__ uint32_t count_escapes(const Stage<kKindEscape>& st, uin
     for (uint32_t el = from + 16u * uint32_t(lane); el < to; el += 512u) {
         uint32_t E[4], esc[4];
         const uint32_t q = t0.x + ((el & bmask) >> 3) * t0.y;
-        chunk_exponents_w(t0.y, st.exp, q, t1.x, t1.y, E, esc);
+        chunk_exponents_rt(st.exp, q, t0.y, t1.x, t1.y, E, esc);
         cnt += escape_count(esc);
     }
     return __reduce_add_sync(0xFFFFFFFFu, cnt);
@@ -280,30 +279,36 @@ __device__ __noinline__ uint32_t count_escapes(const Stage<kKindEscape>& st, uin
 // One chunk of an escape-coded tile in a consumer lane's registers.
 struct EscChunk {
     uint32_t el;      // first element (tile-relative)
+    uint32_t q;       // staged byte of its first code
     uint32_t E[4];    // exponent bytes
     uint32_t esc[4];  // escape flags (bit 8t+7 of word j: element 4j+t)
     uint4 M;          // sign+mantissa bytes
     uint4 t0;         // its block's constants
+    uint2 t1;
     uint32_t count;   // escapes in the chunk
     bool active;
 };
 
-__device__ __forceinline__ void load_esc_chunk(const Stage<kKindEscape>& st, uint32_t el,
-                                               uint32_t tile_n, uint32_t log2B, EscChunk& c) {
+__device__ __forceinline__ void load_esc_meta(const Stage<kKindEscape>& st, uint32_t el,
+                                              uint32_t tile_n, uint32_t log2B, EscChunk& c) {
     c.el = el;
     c.active = el < tile_n;
     c.count = 0;
-    if (!c.active) return;
-    const uint32_t bl = el >> log2B;
-    c.t0 = st.t0[bl];
-    const uint2 t1 = st.t1[bl];
-    c.M = *reinterpret_cast<const uint4*>(st.man + el);
-    const uint32_t q = c.t0.x + ((el & ((1u << log2B) - 1u)) >> 3) * c.t0.y;
-    chunk_exponents_w(c.t0.y, st.exp, q, t1.x, t1.y, c.E, c.esc);
-    const uint32_t nv = tile_n - el;
+    // an inactive chunk (past the end of the tile) decodes staged byte 0 as
+    // width 3 and is never stored
+    const uint32_t bl = c.active ? el >> log2B : 0u;
+    c.t0 = c.active ? st.t0[bl] : make_uint4(0u, 3u, 0u, 0u);
+    c.t1 = st.t1[bl];
+    c.M = *reinterpret_cast<const uint4*>(st.man + (c.active ? el : 0u));
+    c.q = c.t0.x + ((el & ((1u << log2B) - 1u)) >> 3) * c.t0.y;
+    if (!c.active) c.q = 0;
+}
+
+// The last chunk of a stream: bits past the block's codes are not codes (they
+// hold its exceptions and padding).
+__device__ __forceinline__ void finish_esc_codes(uint32_t tile_n, EscChunk& c) {
+    const uint32_t nv = tile_n - c.el;
     if (nv < uint32_t(kChunk)) {
-        // the last chunk of a stream: bits past the block's codes are not codes
-        // (they hold its exceptions and padding)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int valid = int(nv) - 4 * j;
@@ -313,33 +318,71 @@ __device__ __forceinline__ void load_esc_chunk(const Stage<kKindEscape>& st, uin
     c.count = escape_count(c.esc);
 }
 
-// Patch the chunk's escaped elements with their exceptions (staged bytes
-// [before-th exception of the block, ...)), check the block's payload size if
-// the chunk holds the block's last element, and store the 16 BF16 words.
+// Decode the codes of a lane's chunks: 3-bit codes (the width escape-coded
+// Gaussian weights take) through code specialised on the width, any other
+// width through the run-time path.
+// Both chunks are first decoded as 3-bit codes without a branch (so that their
+// shared-memory loads can be scheduled together); a chunk of another width is
+// then decoded again through the run-time path.
+__device__ __forceinline__ void decode_esc_pair(const Stage<kKindEscape>& st, uint32_t tile_n,
+                                                EscChunk& c0, EscChunk& c1) {
+    chunk_exponents<3>(st.exp, c0.q, c0.t1.x, c0.t1.y, c0.E, c0.esc);
+    chunk_exponents<3>(st.exp, c1.q, c1.t1.x, c1.t1.y, c1.E, c1.esc);
+    if (c0.t0.y != 3u) chunk_exponents_rt(st.exp, c0.q, c0.t0.y, c0.t1.x, c0.t1.y, c0.E, c0.esc);
+    if (c1.t0.y != 3u) chunk_exponents_rt(st.exp, c1.q, c1.t0.y, c1.t1.x, c1.t1.y, c1.E, c1.esc);
+    if (c0.active) finish_esc_codes(tile_n, c0);
+    if (c1.active) finish_esc_codes(tile_n, c1);
+}
+
+// Put the chunk's exceptions -- staged bytes [p, p + count), in element order --
+// into its escaped bytes. A word with one escape (all but a few in a thousand
+// for Gaussian weights) takes its exception with a byte mask; a word with more
+// goes byte by byte.
+__device__ __forceinline__ void patch_esc_chunk(const uint8_t* exp, uint32_t p, EscChunk& c) {
+    uint32_t k[4], multi = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {  // without branches: a word without escapes keeps its bytes
+        const uint32_t esc = c.esc[j];
+        k[j] = __popc(esc);
+        multi |= k[j] >> 1;
+        const uint32_t mask = (esc >> 7) * 0xFFu;
+        c.E[j] ^= (c.E[j] ^ (uint32_t(exp[p]) * 0x01010101u)) & mask;
+        p += k[j];
+    }
+    if (multi) {  // some word holds two or more escapes: place its bytes one by one
+#pragma unroll
+        for (int j = 3; j >= 0; --j) {
+            p -= k[j];
+            if (k[j] > 1u) {
+                uint32_t m = c.esc[j], r = p, E = c.E[j];
+                do {
+                    const uint32_t byte = (uint32_t(__ffs(int(m))) - 1u) >> 3;  // bit 8b + 7 -> b
+                    const uint32_t sel = (0x3210u & ~(0xFu << (4 * byte))) | (4u << (4 * byte));
+                    E = prmt(E, exp[r++], sel);
+                    m &= m - 1u;
+                } while (m);
+                c.E[j] = E;
+            }
+        }
+    }
+}
+
+// Patch the chunk's escaped elements with their exceptions (the `before`-th
+// exception of its block onwards), check the block's payload size if the
+// chunk holds the block's last element, and store the 16 BF16 words.
 __device__ __forceinline__ bool finish_esc_chunk(const Stage<kKindEscape>& st, EscChunk& c,
                                                  uint32_t before, uint32_t tile_n, uint32_t log2B,
-                                                 uint8_t* patch, uint16_t* out) {
+                                                 uint16_t* out) {
     bool bad = false;
     if (c.count) {
         const uint32_t p = c.t0.x + c.t0.z + before;
-        if (p + c.count > c.t0.w) {
+        if (p + c.count > c.t0.w)
             bad = true;
-        } else {
-            *reinterpret_cast<uint4*>(patch) = make_uint4(c.E[0], c.E[1], c.E[2], c.E[3]);
-            uint32_t mm = escape_mask(c.esc), pp = p;
-            do {
-                patch[__ffs(int(mm)) - 1] = st.exp[pp++];
-                mm &= mm - 1u;
-            } while (mm);
-            const uint4 v = *reinterpret_cast<const uint4*>(patch);
-            c.E[0] = v.x;
-            c.E[1] = v.y;
-            c.E[2] = v.z;
-            c.E[3] = v.w;
-        }
+        else
+            patch_esc_chunk(st.exp, p, c);
     }
-    const uint32_t blk_end = min(((c.el >> log2B) + 1u) << log2B, tile_n);
-    if (blk_end - c.el <= uint32_t(kChunk) &&
+    const uint32_t next = c.el + uint32_t(kChunk);
+    if (((next & ((1u << log2B) - 1u)) == 0u || next >= tile_n) &&
         ((c.t0.z + before + c.count + 15u) & ~15u) != c.t0.w - c.t0.x)
         bad = true;
     uint4 r0, r1;
@@ -363,7 +406,7 @@ template <int MAXI>
 __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEscape>& sm, int tid,
                                int lane, int warp) {
     constexpr int kStages = DecodeSmem<kKindEscape>::kStages;
-    uint8_t* patch = reinterpret_cast<uint8_t*>(&sm.patch[tid]);
+    (void)tid;
     for (uint64_t i = 0;; ++i) {
         const uint64_t t = blockIdx.x + i * gridDim.x;
         if (t >= P.total_tiles) break;
@@ -379,7 +422,6 @@ __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEsca
         const Stage<kKindEscape>& st = sm.stage[s];
         const StageInfo info = st.info;
         const uint32_t log2B = info.log2B, B = 1u << log2B;
-        const uint32_t group = min(B >> 4, 32u);  // lanes that hold one block in a 512-element step
         const uint32_t seg = uint32_t(warp) * kSegment;
         bool bad = false;
         if (seg < info.tile_n) {  // the same for the whole warp
@@ -390,14 +432,25 @@ __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEsca
             // both 512-element steps of the segment at once: chunk k of this lane
             // starts at seg + 512k + 16 lane
             EscChunk c0, c1;
-            load_esc_chunk(st, seg + 16u * uint32_t(lane), info.tile_n, log2B, c0);
-            load_esc_chunk(st, seg + 512u + 16u * uint32_t(lane), info.tile_n, log2B, c1);
-            // one prefix count for both steps: step k's counts in bits [16k, 16k + 16)
+            load_esc_meta(st, seg + 16u * uint32_t(lane), info.tile_n, log2B, c0);
+            load_esc_meta(st, seg + 512u + 16u * uint32_t(lane), info.tile_n, log2B, c1);
+            decode_esc_pair(st, info.tile_n, c0, c1);
+            // one prefix count for both steps (step k's counts in bits [16k, 16k + 16)),
+            // segmented by block: B/16 lanes hold one block of a step when B < 512
             const uint32_t v = c0.count | (c1.count << 16);
             uint32_t incl = v;
-            for (uint32_t d = 1; d < group; d <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d, int(group));
-                if ((uint32_t(lane) & (group - 1u)) >= d) incl += y;
+            if (B >= 512u) {
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+                    if (lane >= d) incl += y;
+                }
+            } else {
+                const uint32_t group = B >> 4;
+                for (uint32_t d = 1; d < group; d <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d, int(group));
+                    if ((uint32_t(lane) & (group - 1u)) >= d) incl += y;
+                }
             }
             const uint32_t excl = incl - v;
             uint32_t before0 = excl & 0xFFFFu, before1 = excl >> 16;
@@ -405,8 +458,8 @@ __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEsca
                 before0 += carry;
                 before1 += carry + (__shfl_sync(0xFFFFFFFFu, incl, 31) & 0xFFFFu);
             }
-            if (c0.active) bad |= finish_esc_chunk(st, c0, before0, info.tile_n, log2B, patch, info.out);
-            if (c1.active) bad |= finish_esc_chunk(st, c1, before1, info.tile_n, log2B, patch, info.out);
+            if (c0.active) bad |= finish_esc_chunk(st, c0, before0, info.tile_n, log2B, info.out);
+            if (c1.active) bad |= finish_esc_chunk(st, c1, before1, info.tile_n, log2B, info.out);
         }
         if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) report(P.status, kStatusCorrupt);
         __syncwarp();

@@ -116,6 +116,40 @@ __device__ __forceinline__ void chunk_exponents(const uint8_t* exp, uint32_t q, 
     }
 }
 
+// chunk_exponents for a width known only at run time (0..8), the same result:
+// the chunk's two octets are fetched as 64-bit strings, each split into two
+// quads, each quad spread into bytes with run-time shifts.
+__device__ __forceinline__ void chunk_exponents_rt(const uint8_t* exp, uint32_t q, uint32_t w,
+                                                   uint32_t base4, uint32_t esc_add, uint32_t E[4],
+                                                   uint32_t esc[4]) {
+    if (w == 0u) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) E[j] = base4, esc[j] = 0u;
+        return;
+    }
+    const uint32_t* s32 = reinterpret_cast<const uint32_t*>(exp);
+    uint32_t lo[2], hi[2];
+    fetch_octet(s32, q, lo[0], hi[0]);
+    fetch_octet(s32, q + w, lo[1], hi[1]);
+    const uint32_t w4 = 4u * w;
+    const uint32_t m4 = w == 8u ? 0xFFFFFFFFu : (1u << w4) - 1u;
+    const uint32_t M2 = (1u << (2u * w)) - 1u, m1x2 = ((1u << w) - 1u) * 0x00010001u;
+    const uint32_t sh2 = 16u - 2u * w, sh1 = 8u - w;
+    // raw blocks (w = 8) hold any byte: they have no escape code
+    const uint32_t detect = w == 8u ? 0u : 0x80808080u;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const uint32_t Q[2] = {lo[k] & m4, __funnelshift_rc(lo[k], hi[k], w4) & m4};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t t = (Q[h] & M2) | ((Q[h] << sh2) & (M2 << 16));
+            const uint32_t V = (t & m1x2) | ((t << sh1) & (m1x2 << 8));
+            esc[2 * k + h] = (V + esc_add) & detect;
+            E[2 * k + h] = V + base4;
+        }
+    }
+}
+
 // The escapes of a chunk: their number, from the four escape words at once
 // (their flag bits are moved to distinct positions and counted together).
 __device__ __forceinline__ uint32_t escape_count(const uint32_t esc[4]) {
