@@ -438,11 +438,14 @@ def run_wcodec(args):
 
 
 def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stream, dist, dev,
-            n_total, entry="wc_decompress_batch"):
-    """Same metric through the public C-ABI, but each step first copies the
-    compressed streams from pinned host memory and ends by reading the status
-    word back; the copies are inside the timed region. `entry` is the batched
-    decoder of the streams' kind."""
+            n_total, entry="wc_decompress_batch", host_flags=0):
+    """Same metric through the public C-ABI with the compressed streams in pinned
+    host memory and a read of the status word back every step, both inside the
+    timed region, by two paths: (a) copy the streams to the device
+    (cudaMemcpyAsync per tensor), then one batched decode (`entry`); (b) one
+    wc_decompress_host_batch launch that reads the streams over the host link
+    itself (`host_flags`: the streams' kind). The faster path is the line's
+    value; both are reported."""
     import torch
     decode_batch = getattr(wc, entry)
     total = sum(sizes)
@@ -481,10 +484,41 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
     sec = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, dev)
     ok = status_host.item() == 0 and all(torch.equal(a, b) for a, b in zip(inputs, outs))
     world = dist.get_world_size() if dist is not None else 1
-    result = {"value": whole_job_gbs(world, 2 * n_total, steps, sec), "unit": "GB/s",
-              "h2d_bytes_per_step": total, "d2h_bytes_per_step": 4, "steps": steps,
-              "verified_bit_exact": bool(ok)}
-    del host, views
+    copy_path = {"value": whole_job_gbs(world, 2 * n_total, steps, sec), "unit": "GB/s",
+                 "h2d_bytes_per_step": total, "d2h_bytes_per_step": 4, "steps": steps,
+                 "path": "cudaMemcpyAsync of each stream, then %s" % entry,
+                 "verified_bit_exact": bool(ok)}
+
+    # (b) the decoder reads the pinned streams itself
+    for o in outs:
+        o.fill_(-1)
+    hbatch = wcodec.make_batch([(views[k], sizes[k], outs[k], inputs[k].numel(), BLOCK)
+                                for k in range(len(sizes))])
+
+    def fused_step():
+        rc = wc.wc_decompress_host_batch(hbatch[0], hbatch[1], host_flags, dec_status.data_ptr(), sh)
+        if rc != 0:
+            raise RuntimeError("wc_decompress_host_batch: %s" % wc.wc_status_string(rc))
+        status_host.copy_(dec_status, non_blocking=True)
+
+    fused_step()
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    e0.record(stream)
+    for _ in range(steps):
+        fused_step()
+    e1.record(stream)
+    barrier(dist, dev)
+    fsec = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, dev)
+    fok = status_host.item() == 0 and all(torch.equal(a, b) for a, b in zip(inputs, outs))
+    fused_path = {"value": whole_job_gbs(world, 2 * n_total, steps, fsec), "unit": "GB/s",
+                  "h2d_bytes_per_step": total, "d2h_bytes_per_step": 4, "steps": steps,
+                  "path": "wc_decompress_host_batch (the decoder reads the pinned streams)",
+                  "verified_bit_exact": bool(fok)}
+    best, other = (fused_path, copy_path) if fsec < sec else (copy_path, fused_path)
+    result = dict(best)
+    result["other_path"] = other
+    del host, views, hbatch
     # context: the same weights moved uncompressed (BF16, pinned host -> device), no decode
     try:
         raw = torch.empty(2 * n_total, dtype=torch.uint8, pin_memory=True)
@@ -512,7 +546,7 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
     raw_sec = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, dev)
     result["bf16_h2d_only"] = {"value": whole_job_gbs(world, 2 * n_total, steps, raw_sec),
                                "unit": "GB/s", "h2d_bytes_per_step": 2 * n_total,
-                               "speedup_of_compressed_path": raw_sec / sec}
+                               "speedup_of_compressed_path": raw_sec / min(sec, fsec)}
     return result
 
 
@@ -597,7 +631,7 @@ def run_escape(args):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stream, dist,
-                      dev, n_total, entry="wc_decompress_escape_batch")
+                      dev, n_total, entry="wc_decompress_escape_batch", host_flags=2)
     stream_total = sum(sizes)
     bytes_out = 2 * n_total
     moved = stream_total + bytes_out

@@ -263,6 +263,27 @@ int wc_decompress_escape_batch(const wc_batch_item *h_items, uint32_t count,
                                int32_t *d_status, void *stream);
 
 /*
+ * Decompression fused with the host-to-device transfer ("ENEC: A Lossless AI
+ * Model Compression Method Enabling Fast Inference on Ascend NPUs", Abstract:
+ * compressed weights cut the transfer in weight-transfer-bound inference).
+ * The streams stay in page-locked host memory (cudaHostAlloc, cudaMallocHost
+ * or cudaHostRegister; anything else returns WC_ERR_INVALID_ARG) and the
+ * decoder reads each tile's bytes over the host link itself, decoding earlier
+ * tiles meanwhile, into BF16 in device memory: no device buffer holds the
+ * compressed streams, and only the compressed bytes cross the link.
+ *   h_items / h_stream  as wc_decompress_batch / wc_decompress, except that each
+ *                       stream pointer is a HOST pointer (16-byte aligned); the
+ *                       host memory must not change until the work is done
+ *   flags               0 for plain streams, WC_FLAG_ESCAPE for escape-coded ones
+ * Checks and errors as wc_decompress (d_status); FP32 streams are not taken.
+ */
+#define WC_FLAG_ESCAPE 2u
+int wc_decompress_host(const void *h_stream, uint64_t stream_bytes, void *d_out, uint64_t n,
+                       uint32_t block, uint32_t flags, int32_t *d_status, void *stream);
+int wc_decompress_host_batch(const wc_batch_item *h_items, uint32_t count, uint32_t flags,
+                             int32_t *d_status, void *stream);
+
+/*
  * FP32 tensors ("ENEC: A Lossless AI Model Compression Method Enabling Fast
  * Inference on Ascend NPUs", Abstract: the method targets AI model weights in
  * general). The high 16 bits of an FP32 word have the BF16 layout, so the

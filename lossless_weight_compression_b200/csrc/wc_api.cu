@@ -304,6 +304,55 @@ int wc_decompress_escape_batch(const wc_batch_item* h_items, uint32_t count, int
     return WC_OK;
 }
 
+// The device's address of page-locked host memory (cudaHostAlloc, cudaMallocHost
+// or cudaHostRegister); nullptr for any other pointer. A host-side query: it
+// neither allocates nor synchronizes.
+static const void* mapped_host_address(const void* h) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, h) != cudaSuccess) {
+        (void)cudaGetLastError();  // a failed query leaves a (non-sticky) error: clear it
+        return nullptr;
+    }
+    return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
+int wc_decompress_host_batch(const wc_batch_item* h_items, uint32_t count, uint32_t flags,
+                             int32_t* d_status, void* stream) {
+    if ((h_items == nullptr && count > 0) || (flags != 0u && flags != WC_FLAG_ESCAPE))
+        return WC_ERR_INVALID_ARG;
+    for (uint32_t i = 0; i < count; ++i) {  // validate everything before launching anything
+        const int rc = check_decode_item(h_items[i]);
+        if (rc != WC_OK) return rc;
+        const void* dev = mapped_host_address(h_items[i].stream);
+        if (dev == nullptr || !aligned16(dev)) return WC_ERR_INVALID_ARG;
+    }
+    const int kind = flags == WC_FLAG_ESCAPE ? wc::kKindEscape : wc::kKindPlain;
+    wc::DecodeItem chunk[WC_BATCH_MAX];
+    for (uint32_t base = 0; base < count; base += WC_BATCH_MAX) {
+        const uint32_t c = (count - base < WC_BATCH_MAX) ? count - base : WC_BATCH_MAX;
+        for (uint32_t i = 0; i < c; ++i) {
+            chunk[i] = to_item(h_items[base + i]);
+            chunk[i].stream = static_cast<const uint8_t*>(mapped_host_address(h_items[base + i].stream));
+        }
+        const cudaError_t err = wc::launch_decode(chunk, c, d_status,
+                                                  static_cast<cudaStream_t>(stream), kind, true);
+        if (err != cudaSuccess) return WC_ERR_CUDA;
+    }
+    return WC_OK;
+}
+
+int wc_decompress_host(const void* h_stream, uint64_t stream_bytes, void* d_out, uint64_t n,
+                       uint32_t block, uint32_t flags, int32_t* d_status, void* stream) {
+    wc_batch_item it;
+    it.stream = h_stream;
+    it.stream_bytes = stream_bytes;
+    it.out = d_out;
+    it.n = n;
+    it.block = block;
+    it.reserved = 0;
+    return wc_decompress_host_batch(&it, 1, flags, d_status, stream);
+}
+
 static int check_gemv_item(const wc_gemv_item& it, uint32_t n_vec) {
     if (n_vec != 1 && n_vec != 2 && n_vec != 4) return WC_ERR_INVALID_ARG;
     if (!wc::block_ok(it.block) || it.reserved != 0 || it.stream == nullptr ||

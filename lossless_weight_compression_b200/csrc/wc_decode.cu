@@ -101,7 +101,31 @@ __device__ __forceinline__ Layout layout_of_kind(uint64_t n, uint32_t B) {
     return KIND == kKindEscape ? make_layout_escape(n, B) : make_layout(n, B, KIND == kKindF32);
 }
 
-template <int MAXI, int KIND>
+// Copy `bytes` (a multiple of 16) from page-locked host memory, read through the
+// device's mapping of it, into shared memory: 16-byte loads by the whole warp,
+// four in flight per lane (2 KB per warp round trip; the grid's hundreds of
+// producers keep the host link busy).
+__device__ __forceinline__ void warp_copy_from_host(uint8_t* dst, const uint8_t* src,
+                                                    uint32_t bytes, int lane) {
+    for (uint32_t base = 0; base < bytes; base += 32u * 16u * 4u) {
+        uint4 v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t off = base + (uint32_t(k) * 32u + uint32_t(lane)) * 16u;
+            if (off < bytes) v[k] = *reinterpret_cast<const uint4*>(src + off);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const uint32_t off = base + (uint32_t(k) * 32u + uint32_t(lane)) * 16u;
+            if (off < bytes) *reinterpret_cast<uint4*>(dst + off) = v[k];
+        }
+    }
+}
+
+// HOST: the streams are in page-locked host memory; the producer reads each
+// tile's bytes over the host link itself instead of issuing bulk copies, so
+// the transfer and the decode of earlier tiles overlap in one launch.
+template <int MAXI, int KIND, bool HOST>
 __device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem<KIND>& sm, int lane) {
     constexpr int kStages = DecodeSmem<KIND>::kStages;
     constexpr bool F32 = KIND == kKindF32;
@@ -165,8 +189,14 @@ __device__ void produce(const DecodeParams<MAXI>& P, DecodeSmem<KIND>& sm, int l
             tile_n = 0;
         }
         __syncwarp();
+        if (HOST && tile_n != 0) {
+            const uint8_t* S = I.stream;
+            warp_copy_from_host(st.man, S + L.off_man + lt * kTile, man_bytes, lane);
+            if (len16) warp_copy_from_host(st.exp, S + L.off_exp + start, len16, lane);
+            __syncwarp();  // every lane's stores precede lane 0's arrive
+        }
         if (lane == 0) {
-            if (tile_n == 0) {
+            if (tile_n == 0 || HOST) {
                 mbar_arrive(&sm.full[s]);
             } else {
                 const uint32_t low_bytes = F32 ? (2u * tile_n + 15u) & ~15u : 0u;
@@ -467,7 +497,7 @@ __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEsca
     }
 }
 
-template <int MAXI, int KIND>
+template <int MAXI, int KIND, bool HOST>
 __global__ void __launch_bounds__(kDecodeThreads)
     decode_kernel(const __grid_constant__ DecodeParams<MAXI> P) {
     constexpr int kStages = DecodeSmem<KIND>::kStages;
@@ -484,7 +514,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
     __syncthreads();
     if (warp == kProducerWarp)
-        produce<MAXI, KIND>(P, sm, lane);
+        produce<MAXI, KIND, HOST>(P, sm, lane);
     else if constexpr (KIND == kKindEscape)
         consume_escape<MAXI>(P, sm, tid, lane, warp);
     else
@@ -493,7 +523,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
 
 // Persistent grid: as many resident thread blocks as the SMs hold, never more
 // than there are tiles. Computed once per device and kernel instantiation.
-template <int MAXI, int KIND>
+template <int MAXI, int KIND, bool HOST>
 cudaError_t grid_for(uint64_t tiles, unsigned* grid) {
     static std::mutex mu;
     static int per_device[64];  // 0 = not yet known
@@ -503,14 +533,14 @@ cudaError_t grid_for(uint64_t tiles, unsigned* grid) {
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
     if (per_device[dev] == 0) {
-        err = cudaFuncSetAttribute(decode_kernel<MAXI, KIND>,
+        err = cudaFuncSetAttribute(decode_kernel<MAXI, KIND, HOST>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    int(sizeof(DecodeSmem<KIND>)));
         if (err != cudaSuccess) return err;
         int sms = 0, per_sm = 0;
         err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (err != cudaSuccess) return err;
-        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<MAXI, KIND>,
+        err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<MAXI, KIND, HOST>,
                                                             kDecodeThreads, sizeof(DecodeSmem<KIND>));
         if (err != cudaSuccess) return err;
         per_device[dev] = (per_sm > 0 ? per_sm : 1) * sms;
@@ -520,7 +550,7 @@ cudaError_t grid_for(uint64_t tiles, unsigned* grid) {
     return cudaSuccess;
 }
 
-template <int MAXI, int KIND>
+template <int MAXI, int KIND, bool HOST>
 cudaError_t launch_batch(const DecodeItem* items, uint32_t count, int32_t* status,
                          cudaStream_t stream) {
     static_assert(sizeof(DecodeParams<MAXI>) <= 32000, "launch parameters exceed the limit");
@@ -539,9 +569,9 @@ cudaError_t launch_batch(const DecodeItem* items, uint32_t count, int32_t* statu
     p.total_tiles = tiles;
     if (tiles == 0) return cudaSuccess;
     unsigned grid = 0;
-    cudaError_t err = grid_for<MAXI, KIND>(tiles, &grid);
+    cudaError_t err = grid_for<MAXI, KIND, HOST>(tiles, &grid);
     if (err != cudaSuccess) return err;
-    decode_kernel<MAXI, KIND><<<grid, kDecodeThreads, sizeof(DecodeSmem<KIND>), stream>>>(p);
+    decode_kernel<MAXI, KIND, HOST><<<grid, kDecodeThreads, sizeof(DecodeSmem<KIND>), stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -549,29 +579,33 @@ cudaError_t launch_batch(const DecodeItem* items, uint32_t count, int32_t* statu
 
 constexpr uint32_t kBatchMax = 512;
 
-template <int KIND>
+template <int KIND, bool HOST>
 cudaError_t launch_kind(const DecodeItem* items, uint32_t count, int32_t* status,
                         cudaStream_t stream) {
-    if (count == 1) return launch_batch<1, KIND>(items, 1, status, stream);
+    if (count == 1) return launch_batch<1, KIND, HOST>(items, 1, status, stream);
     for (uint32_t i = 0; i < count; i += kBatchMax) {
         const uint32_t c = min(kBatchMax, count - i);
-        const cudaError_t err = launch_batch<kBatchMax, KIND>(items + i, c, status, stream);
+        const cudaError_t err = launch_batch<kBatchMax, KIND, HOST>(items + i, c, status, stream);
         if (err != cudaSuccess) return err;
     }
     return cudaSuccess;
 }
 
 cudaError_t launch_decode(const DecodeItem* items, uint32_t count, int32_t* status,
-                          cudaStream_t stream, int kind) {
-    if (kind == kKindF32) {  // FP32 streams: one tensor per call
+                          cudaStream_t stream, int kind, bool host_streams) {
+    if (kind == kKindF32) {  // FP32 streams: one tensor per call, device streams only
+        if (host_streams) return cudaErrorInvalidValue;
         for (uint32_t i = 0; i < count; ++i) {
-            const cudaError_t err = launch_batch<1, kKindF32>(items + i, 1, status, stream);
+            const cudaError_t err = launch_batch<1, kKindF32, false>(items + i, 1, status, stream);
             if (err != cudaSuccess) return err;
         }
         return cudaSuccess;
     }
-    if (kind == kKindEscape) return launch_kind<kKindEscape>(items, count, status, stream);
-    return launch_kind<kKindPlain>(items, count, status, stream);
+    if (kind == kKindEscape)
+        return host_streams ? launch_kind<kKindEscape, true>(items, count, status, stream)
+                            : launch_kind<kKindEscape, false>(items, count, status, stream);
+    return host_streams ? launch_kind<kKindPlain, true>(items, count, status, stream)
+                        : launch_kind<kKindPlain, false>(items, count, status, stream);
 }
 
 }  // namespace wc

@@ -274,8 +274,10 @@ cudaError_t launch_encode(const EncodeItem* items, uint32_t count, void* workspa
 // Stream kinds of the decoder: BF16 (16-bit words), FP32 (decoded into n u32
 // words at DecodeItem::out) and escape-coded 16-bit streams.
 enum StreamKind : int { kKindPlain = 0, kKindF32 = 1, kKindEscape = 2 };
+// host_streams: every DecodeItem::stream is the device's address of page-locked
+// host memory, read by the kernel over the host link (plain and escape-coded kinds).
 cudaError_t launch_decode(const DecodeItem* items, uint32_t count, int32_t* status,
-                          cudaStream_t stream, int kind = kKindPlain);
+                          cudaStream_t stream, int kind = kKindPlain, bool host_streams = false);
 
 // The escape-coded encoder (wc_encode_escape.cu): workspace bytes for one
 // tensor, and the launches that code it (no cross-block waits: a per-block

@@ -128,6 +128,10 @@ def lib() -> ctypes.CDLL:
     L.wc_decompress_escape.restype = i
     L.wc_decompress_escape_batch.argtypes = [ctypes.POINTER(wc_batch_item), u32, vp, vp]
     L.wc_decompress_escape_batch.restype = i
+    L.wc_decompress_host.argtypes = [vp, u64, vp, u64, u32, u32, vp, vp]
+    L.wc_decompress_host.restype = i
+    L.wc_decompress_host_batch.argtypes = [ctypes.POINTER(wc_batch_item), u32, u32, vp, vp]
+    L.wc_decompress_host_batch.restype = i
     _lib = L
     return L
 
@@ -225,6 +229,18 @@ def wc_decompress_escape(d_stream, stream_bytes, d_out, n, block, d_status, stre
 
 def wc_decompress_escape_batch(items, count, d_status, stream) -> int:
     return lib().wc_decompress_escape_batch(items, count, d_status, stream)
+
+
+WC_FLAG_ESCAPE = 2
+
+
+def wc_decompress_host(h_stream, stream_bytes, d_out, n, block, flags, d_status, stream) -> int:
+    return lib().wc_decompress_host(h_stream, stream_bytes, d_out, n, block, flags, d_status,
+                                    stream)
+
+
+def wc_decompress_host_batch(items, count, flags, d_status, stream) -> int:
+    return lib().wc_decompress_host_batch(items, count, flags, d_status, stream)
 
 
 def wc_stream_info(h_header: bytes):
@@ -563,3 +579,12 @@ def decompress_escape_batch(batch, status: torch.Tensor, stream=None):
     arr, count = batch
     rc = wc_decompress_escape_batch(arr, count, status.data_ptr(), _stream_handle(stream))
     _check(rc, "wc_decompress_escape_batch")
+
+
+def decompress_host_batch(batch, status: torch.Tensor, escape: bool = False, stream=None):
+    """Decode streams held in page-locked host memory (a batch from ``make_batch``
+    whose stream tensors are pinned CPU tensors) straight into device outputs."""
+    arr, count = batch
+    rc = wc_decompress_host_batch(arr, count, WC_FLAG_ESCAPE if escape else 0,
+                                  status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_decompress_host_batch")

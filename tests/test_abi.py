@@ -221,3 +221,10 @@ def test_stream_info_reads_escape_headers(wclib, orc):
     s = orc.compress_escape(words, 256)
     rc, n, b, total = wclib.wc_stream_info(bytes(s[:128]))
     assert rc == wclib.WC_OK and (n, b, total) == (5000, 256, s.size)
+
+
+def test_host_stream_decode_checks_flags_before_anything(wclib):
+    item = (wclib.wc_batch_item * 1)()
+    for bad_flags in (1, 3, 4):
+        assert wclib.wc_decompress_host_batch(item, 1, bad_flags, None, None) == wclib.WC_ERR_INVALID_ARG
+    assert wclib.wc_decompress_host_batch(None, 2, 0, None, None) == wclib.WC_ERR_INVALID_ARG
