@@ -555,9 +555,9 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
 # ---------------------------------------------------------------------------
 def run_escape(args):
     """The 8B-shaped stack as escape-coded streams (a window of 2^w - 1
-    exponents per block plus an exception list): each tensor encoded with
-    wc_compress_escape (five launches per tensor, outside the metric), then the
-    whole stack decoded by one wc_decompress_escape_batch launch per step."""
+    exponents per block plus an exception list): all tensors encoded by one
+    wc_compress_escape_batch call (five launches), then the whole stack decoded
+    by one wc_decompress_escape_batch launch per step (the metric)."""
     import numpy as np
     import torch
 
@@ -582,25 +582,20 @@ def run_escape(args):
         names.append(name)
         inputs.append(words)
     n_total = sum(w.numel() for w in inputs)
-    bufs = [torch.empty((wc.wc_bound_escape(w.numel(), BLOCK) + 15) // 16 * 16, dtype=torch.uint8,
-                        device=dev) for w in inputs]
-    ws_bytes = max(wc.wc_workspace_size_escape(w.numel(), BLOCK) for w in inputs)
-    ws = torch.empty((ws_bytes + 15) // 16 * 16, dtype=torch.uint8, device=dev)
-    nbytes = torch.zeros(len(inputs), dtype=torch.int64, device=dev)
+    enc = wcodec.CompressBatch(inputs, block=BLOCK, escape=True)
+    bufs, nbytes = enc.buffers, enc.nbytes
     status = torch.zeros(2, dtype=torch.int32, device=dev)
     outs = [torch.empty(w.numel(), dtype=torch.int16, device=dev) for w in inputs]
 
-    def encode_all():
-        for k, w in enumerate(inputs):
-            rc = wc.wc_compress_escape(w.data_ptr(), w.numel(), BLOCK, bufs[k].data_ptr(),
-                                       bufs[k].numel(), nbytes[k:].data_ptr(), ws.data_ptr(),
-                                       ws.numel(), status[0:].data_ptr(), sh)
-            if rc != 0:
-                raise RuntimeError("wc_compress_escape: %s" % wc.wc_status_string(rc))
+    def encode_all():  # five launches for the whole batch
+        rc = wc.wc_compress_escape_batch(enc.items, enc.count, enc.workspace.data_ptr(),
+                                         enc.workspace.numel(), status[0:].data_ptr(), sh)
+        if rc != 0:
+            raise RuntimeError("wc_compress_escape_batch: %s" % wc.wc_status_string(rc))
 
     encode_all()
     torch.cuda.synchronize(dev)
-    sizes = nbytes.cpu().tolist()
+    sizes = enc.sizes()
     batch = wcodec.make_batch([(bufs[k], sizes[k], outs[k], inputs[k].numel(), BLOCK)
                                for k in range(len(inputs))])
     dec_status = status[1:]
@@ -627,7 +622,7 @@ def run_escape(args):
         t_dec = timed(decode_all)
     torch.cuda.synchronize(dev)
     verified = bool((status == 0).all().item()) and all(
-        torch.equal(a, b) for a, b in zip(inputs, outs)) and nbytes.cpu().tolist() == sizes
+        torch.equal(a, b) for a, b in zip(inputs, outs)) and enc.sizes() == sizes
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stream, dist,
@@ -675,7 +670,8 @@ def run_escape(args):
                         "exponent_entropy_bits": H, "entropy_bound_ratio": 16.0 / (8.0 + H)},
         "encode": {"ms_per_step": 1e3 * t_enc, "gbs_moved": moved / t_enc / 1e9,
                    "frac_of_peak": moved / t_enc / 1e9 / peak,
-                   "kernels": "esc_params, esc_reduce, esc_top, esc_down, esc_pack per tensor"},
+                   "kernels": "esc_params, esc_reduce, esc_top, esc_down, esc_pack (one launch "
+                              "each for the batch)"},
         "e2e": e2e,
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),

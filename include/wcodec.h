@@ -263,6 +263,18 @@ int wc_decompress_escape_batch(const wc_batch_item *h_items, uint32_t count,
                                int32_t *d_status, void *stream);
 
 /*
+ * wc_compress_escape over `count` tensors (h_items as for wc_compress_batch,
+ * out_capacity >= wc_bound_escape(n, block) each), in five launches per 512
+ * tensors; every stream equals the one wc_compress_escape writes. d_workspace
+ * (device, 16-byte aligned, need not be cleared) holds at least
+ * wc_compress_escape_batch_workspace_size bytes (0 if an item's n or block is
+ * invalid). Every item is checked before anything is launched.
+ */
+uint64_t wc_compress_escape_batch_workspace_size(const wc_compress_item *h_items, uint32_t count);
+int wc_compress_escape_batch(const wc_compress_item *h_items, uint32_t count, void *d_workspace,
+                             uint64_t workspace_bytes, int32_t *d_status, void *stream);
+
+/*
  * Decompression fused with the host-to-device transfer ("ENEC: A Lossless AI
  * Model Compression Method Enabling Fast Inference on Ascend NPUs", Abstract:
  * compressed weights cut the transfer in weight-transfer-bound inference).

@@ -253,25 +253,87 @@ uint64_t wc_bound_escape(uint64_t n, uint32_t block) {
 }
 
 uint64_t wc_workspace_size_escape(uint64_t n, uint32_t block) {
-    return args_ok(n, block) ? wc::escape_workspace_bytes(n, block) : 0;
+    if (!args_ok(n, block)) return 0;
+    const wc::EncodeItem item = to_encode_item(nullptr, n, block, nullptr, nullptr);
+    return wc::escape_workspace_bytes(&item, 1);
+}
+
+static int check_escape_item(const void* d_in, uint64_t n, uint32_t block, const void* d_out,
+                             uint64_t out_capacity, const uint64_t* d_out_bytes) {
+    if (!args_ok(n, block) || d_out == nullptr || d_out_bytes == nullptr ||
+        (n > 0 && d_in == nullptr))
+        return WC_ERR_INVALID_ARG;
+    if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) ||
+        (reinterpret_cast<uintptr_t>(d_out_bytes) & 7u) != 0)
+        return WC_ERR_INVALID_ARG;
+    if (out_capacity < wc::bound_bytes_escape(n, block)) return WC_ERR_BUFFER_TOO_SMALL;
+    return WC_OK;
 }
 
 int wc_compress_escape(const void* d_in, uint64_t n, uint32_t block, void* d_out,
                        uint64_t out_capacity, uint64_t* d_out_bytes, void* d_workspace,
                        uint64_t workspace_bytes, int32_t* d_status, void* stream) {
-    if (!args_ok(n, block) || d_out == nullptr || d_out_bytes == nullptr ||
-        d_workspace == nullptr || (n > 0 && d_in == nullptr))
-        return WC_ERR_INVALID_ARG;
-    if ((n > 0 && !aligned16(d_in)) || !aligned16(d_out) || !aligned16(d_workspace) ||
-        (reinterpret_cast<uintptr_t>(d_out_bytes) & 7u) != 0)
-        return WC_ERR_INVALID_ARG;
-    if (out_capacity < wc::bound_bytes_escape(n, block) ||
-        workspace_bytes < wc::escape_workspace_bytes(n, block))
-        return WC_ERR_BUFFER_TOO_SMALL;
+    (void)d_status;  // nothing in these kernels waits, so nothing can time out
+    const int rc = check_escape_item(d_in, n, block, d_out, out_capacity, d_out_bytes);
+    if (rc != WC_OK) return rc;
+    if (d_workspace == nullptr || !aligned16(d_workspace)) return WC_ERR_INVALID_ARG;
     const wc::EncodeItem item = to_encode_item(d_in, n, block, d_out, d_out_bytes);
+    if (workspace_bytes < wc::escape_workspace_bytes(&item, 1)) return WC_ERR_BUFFER_TOO_SMALL;
     const cudaError_t err =
-        wc::launch_encode_escape(item, d_workspace, d_status, static_cast<cudaStream_t>(stream));
+        wc::launch_encode_escape(&item, 1, d_workspace, static_cast<cudaStream_t>(stream));
     return err == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}
+
+// Host-side copies of a batch's items (at most this many per call of the helpers below).
+static uint64_t escape_batch_workspace(const wc_compress_item* h_items, uint32_t count) {
+    uint64_t total = 0;
+    wc::EncodeItem chunk[WC_BATCH_MAX];
+    for (uint32_t base = 0; base < count; base += WC_BATCH_MAX) {
+        const uint32_t c = (count - base < WC_BATCH_MAX) ? count - base : WC_BATCH_MAX;
+        for (uint32_t i = 0; i < c; ++i) {
+            const wc_compress_item& it = h_items[base + i];
+            chunk[i] = to_encode_item(it.in, it.n, it.block, it.out, it.out_bytes);
+        }
+        total += wc::escape_workspace_bytes(chunk, c);
+    }
+    return total;
+}
+
+uint64_t wc_compress_escape_batch_workspace_size(const wc_compress_item* h_items, uint32_t count) {
+    if (h_items == nullptr && count > 0) return 0;
+    for (uint32_t i = 0; i < count; ++i)
+        if (!args_ok(h_items[i].n, h_items[i].block)) return 0;
+    return escape_batch_workspace(h_items, count);
+}
+
+int wc_compress_escape_batch(const wc_compress_item* h_items, uint32_t count, void* d_workspace,
+                             uint64_t workspace_bytes, int32_t* d_status, void* stream) {
+    (void)d_status;
+    if (h_items == nullptr && count > 0) return WC_ERR_INVALID_ARG;
+    if (count == 0) return WC_OK;
+    for (uint32_t i = 0; i < count; ++i) {  // check everything before launching anything
+        const wc_compress_item& it = h_items[i];
+        if (it.reserved != 0) return WC_ERR_INVALID_ARG;
+        const int rc = check_escape_item(it.in, it.n, it.block, it.out, it.out_capacity,
+                                         it.out_bytes);
+        if (rc != WC_OK) return rc;
+    }
+    if (d_workspace == nullptr || !aligned16(d_workspace)) return WC_ERR_INVALID_ARG;
+    if (workspace_bytes < escape_batch_workspace(h_items, count)) return WC_ERR_BUFFER_TOO_SMALL;
+    wc::EncodeItem chunk[WC_BATCH_MAX];
+    uint8_t* ws = static_cast<uint8_t*>(d_workspace);
+    for (uint32_t base = 0; base < count; base += WC_BATCH_MAX) {
+        const uint32_t c = (count - base < WC_BATCH_MAX) ? count - base : WC_BATCH_MAX;
+        for (uint32_t i = 0; i < c; ++i) {
+            const wc_compress_item& it = h_items[base + i];
+            chunk[i] = to_encode_item(it.in, it.n, it.block, it.out, it.out_bytes);
+        }
+        const cudaError_t err =
+            wc::launch_encode_escape(chunk, c, ws, static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return WC_ERR_CUDA;
+        ws += wc::escape_workspace_bytes(chunk, c);
+    }
+    return WC_OK;
 }
 
 int wc_decompress_escape(const void* d_stream, uint64_t stream_bytes, void* d_out, uint64_t n,

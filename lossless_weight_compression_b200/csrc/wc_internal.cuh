@@ -279,11 +279,12 @@ enum StreamKind : int { kKindPlain = 0, kKindF32 = 1, kKindEscape = 2 };
 cudaError_t launch_decode(const DecodeItem* items, uint32_t count, int32_t* status,
                           cudaStream_t stream, int kind = kKindPlain, bool host_streams = false);
 
-// The escape-coded encoder (wc_encode_escape.cu): workspace bytes for one
-// tensor, and the launches that code it (no cross-block waits: a per-block
-// pass, a three-step scan of the block sizes, and a packing pass).
-uint64_t escape_workspace_bytes(uint64_t n, uint32_t B);
-cudaError_t launch_encode_escape(const EncodeItem& item, void* workspace, int32_t* status,
+// The escape-coded encoder (wc_encode_escape.cu): workspace bytes for a batch
+// of tensors, and the launches that code them (five per batch of up to 512
+// tensors, no cross-block waits: a per-block pass, a three-step scan of the
+// block sizes, and a packing pass).
+uint64_t escape_workspace_bytes(const EncodeItem* items, uint32_t count);
+cudaError_t launch_encode_escape(const EncodeItem* items, uint32_t count, void* workspace,
                                  cudaStream_t stream);
 
 struct GemvItem {

@@ -128,6 +128,10 @@ def lib() -> ctypes.CDLL:
     L.wc_decompress_escape.restype = i
     L.wc_decompress_escape_batch.argtypes = [ctypes.POINTER(wc_batch_item), u32, vp, vp]
     L.wc_decompress_escape_batch.restype = i
+    L.wc_compress_escape_batch_workspace_size.argtypes = [ctypes.POINTER(wc_compress_item), u32]
+    L.wc_compress_escape_batch_workspace_size.restype = u64
+    L.wc_compress_escape_batch.argtypes = [ctypes.POINTER(wc_compress_item), u32, vp, u64, vp, vp]
+    L.wc_compress_escape_batch.restype = i
     L.wc_decompress_host.argtypes = [vp, u64, vp, u64, u32, u32, vp, vp]
     L.wc_decompress_host.restype = i
     L.wc_decompress_host_batch.argtypes = [ctypes.POINTER(wc_batch_item), u32, u32, vp, vp]
@@ -232,6 +236,15 @@ def wc_decompress_escape_batch(items, count, d_status, stream) -> int:
 
 
 WC_FLAG_ESCAPE = 2
+
+
+def wc_compress_escape_batch_workspace_size(items, count) -> int:
+    return lib().wc_compress_escape_batch_workspace_size(items, count)
+
+
+def wc_compress_escape_batch(items, count, d_workspace, workspace_bytes, d_status, stream) -> int:
+    return lib().wc_compress_escape_batch(items, count, d_workspace, workspace_bytes, d_status,
+                                          stream)
 
 
 def wc_decompress_host(h_stream, stream_bytes, d_out, n, block, flags, d_status, stream) -> int:
@@ -360,14 +373,17 @@ def decompress_compressed(c: Compressed, out: torch.Tensor | None = None, status
 
 class CompressBatch:
     """Reusable buffers and descriptors for compressing a fixed list of tensors
-    in one call: ``run()`` enqueues one encoder launch per 512 tensors."""
+    in one call: ``run()`` enqueues one encoder launch per 512 tensors (five for
+    escape-coded streams, ``escape=True``)."""
 
-    def __init__(self, tensors, block=1024):
+    def __init__(self, tensors, block=1024, escape=False):
+        self.escape = escape
+        bound = wc_bound_escape if escape else wc_bound
         self.words = [as_words(t) for t in tensors]
         dev = self.words[0].device if self.words else torch.device("cuda")
         k = len(self.words)
         self.blocks = list(block) if isinstance(block, (list, tuple)) else [block] * k
-        self.buffers = [torch.empty((wc_bound(w.numel(), b) + 15) // 16 * 16,
+        self.buffers = [torch.empty((bound(w.numel(), b) + 15) // 16 * 16,
                                     dtype=torch.uint8, device=dev)
                         for w, b in zip(self.words, self.blocks)]
         self.nbytes = torch.zeros(max(1, k), dtype=torch.int64, device=dev)
@@ -382,17 +398,18 @@ class CompressBatch:
             it.out = self.buffers[j].data_ptr()
             it.out_capacity = self.buffers[j].numel()
             it.out_bytes = self.nbytes[j:].data_ptr()
-        ws = wc_compress_batch_workspace_size(self.items, k)
+        ws = (wc_compress_escape_batch_workspace_size if escape
+              else wc_compress_batch_workspace_size)(self.items, k)
         if k and ws == 0:
-            raise WcodecError(WC_ERR_INVALID_ARG, "wc_compress_batch_workspace_size")
+            raise WcodecError(WC_ERR_INVALID_ARG, "workspace size")
         self.workspace = torch.empty(max(16, (ws + 15) // 16 * 16), dtype=torch.uint8, device=dev)
         self.count = k
 
     def run(self, stream=None):
-        rc = wc_compress_batch(self.items, self.count, self.workspace.data_ptr(),
-                               self.workspace.numel(), self.status.data_ptr(),
-                               _stream_handle(stream))
-        _check(rc, "wc_compress_batch")
+        entry = wc_compress_escape_batch if self.escape else wc_compress_batch
+        rc = entry(self.items, self.count, self.workspace.data_ptr(), self.workspace.numel(),
+                   self.status.data_ptr(), _stream_handle(stream))
+        _check(rc, entry.__name__)
 
     def sizes(self) -> list[int]:
         return self.nbytes[: self.count].cpu().tolist()

@@ -224,3 +224,34 @@ def test_random_metadata_corruption_leaves_device_healthy(orc, wclib, cuda):
         assert st in (0, wclib.WC_ERR_CORRUPT_STREAM)
     dec, st = gpu_decompress_escape(wclib, good, words.size, B, cuda)
     assert st == 0 and np.array_equal(dec, words)
+
+
+def test_batch_compress_matches_oracle(orc, wclib, cuda):
+    """One wc_compress_escape_batch call over tensors of mixed sizes and block sizes
+    (an empty one included): every stream equals the oracle's."""
+    rng = np.random.default_rng(24)
+    shapes = [(0, 256), (1, 128), (8191, 512), (8193, 4096), (100_003, 128), (1 << 20, 1024),
+              (3 * 8192 + 5, 2048), (65536, 256)]
+    words = [random_words(rng, n, KINDS[k % len(KINDS)]) for k, (n, _) in enumerate(shapes)]
+    batch = wclib.CompressBatch([to_gpu_words(w, cuda) for w in words],
+                                block=[B for _, B in shapes], escape=True)
+    batch.run()
+    torch.cuda.synchronize()
+    sizes = batch.sizes()
+    for j, ((n, B), w) in enumerate(zip(shapes, words)):
+        got = batch.buffers[j][: sizes[j]].cpu().numpy()
+        assert np.array_equal(got, orc.compress_escape(w, B)), (n, B)
+
+
+def test_batch_compress_spans_launches(orc, wclib, cuda):
+    """More tensors than one launch takes (700 > 512): each launch has its own
+    part of the workspace."""
+    rng = np.random.default_rng(25)
+    words = [random_words(rng, int(rng.integers(0, 20000)), "mixed") for _ in range(700)]
+    batch = wclib.CompressBatch([to_gpu_words(w, cuda) for w in words], block=256, escape=True)
+    batch.run()
+    torch.cuda.synchronize()
+    sizes = batch.sizes()
+    for j in range(0, 700, 7):
+        got = batch.buffers[j][: sizes[j]].cpu().numpy()
+        assert np.array_equal(got, orc.compress_escape(words[j], 256))
