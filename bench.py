@@ -687,6 +687,105 @@ def run_escape(args):
 
 
 # ---------------------------------------------------------------------------
+# every workload at every block size it names, both stream kinds
+# ---------------------------------------------------------------------------
+def run_sweep(args):
+    """Encode and decode timings of workloads 1, 2, 3 and 5 at each of their block
+    sizes, as plain and as escape-coded streams (one batched launch per
+    direction; workload 4 is the default benchmark). A case whose input, stream
+    and output together fit in the 126 MB L2 is flagged L2-resident: its GB/s
+    are cache, not HBM, figures. Every decode is checked against its input."""
+    import torch
+
+    from lossless_weight_compression_b200 import build_lib, synth, wcodec
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    build_lib.build()
+    wc = wcodec.lib()
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = hbm_peak()
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    rows, ok_all = [], True
+
+    def timed(fn, reps):
+        for _ in range(args.warmup):
+            fn()
+        barrier(dist, dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        barrier(dist, dev)
+        return max_over_ranks(e0.elapsed_time(e1) / 1e3 / reps, dist, dev)
+
+    with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+        for cfg in (1, 2, 3, 5):
+            wl = synth.WORKLOADS[cfg]
+            tensors = [t.view(-1).view(torch.int16) for _, t in wl.make(dev)]
+            n = sum(t.numel() for t in tensors)
+            counts = torch.zeros(256, dtype=torch.int64, device=dev)
+            for t in tensors:
+                counts += torch.bincount(((t.to(torch.int32) >> 7) & 0xFF), minlength=256)
+            p = counts.double() / counts.sum()
+            H = float(-(p[p > 0] * torch.log2(p[p > 0])).sum())
+            for B in wl.blocks:
+                for escape in (False, True):
+                    enc = wcodec.CompressBatch(tensors, block=B, escape=escape)
+                    enc.run()
+                    torch.cuda.synchronize(dev)
+                    sizes = enc.sizes()
+                    outs = [torch.empty_like(t) for t in tensors]
+                    status = torch.zeros(1, dtype=torch.int32, device=dev)
+                    batch = wcodec.make_batch([(enc.buffers[k], sizes[k], outs[k], t.numel(), B)
+                                               for k, t in enumerate(tensors)])
+                    dec = wcodec.decompress_escape_batch if escape else wcodec.decompress_batch
+                    reps = max(args.steps, int(2e9 // (2 * n)))  # a few hundred ms per case at most
+                    t_enc = timed(enc.run, reps)
+                    t_dec = timed(lambda: dec(batch, status), reps)
+                    torch.cuda.synchronize(dev)
+                    ok = (status.item() == 0 and enc.status.item() == 0
+                          and all(torch.equal(a, b) for a, b in zip(tensors, outs)))
+                    ok_all &= ok
+                    C = sum(sizes)
+                    moved = 2 * n + C
+                    rows.append({
+                        "workload": cfg, "name": wl.name, "block": B,
+                        "stream": "escape-coded" if escape else "plain", "elements": n,
+                        "ratio": 2 * n / C, "exponent_entropy_bits": H,
+                        "entropy_bound_ratio": 16.0 / (8.0 + H),
+                        "encode_ms": 1e3 * t_enc, "decode_ms": 1e3 * t_dec,
+                        "encode_gbs_bf16_in": world * 2 * n / t_enc / 1e9,
+                        "decode_gbs_bf16_out": world * 2 * n / t_dec / 1e9,
+                        "decode_frac_of_peak": moved / t_dec / 1e9 / peak,
+                        "encode_frac_of_peak": moved / t_enc / 1e9 / peak,
+                        "l2_resident": moved + 2 * n <= l2_bytes,
+                        "verified_bit_exact": ok})
+                    del enc, outs, batch
+            del tensors
+    line = {
+        "metric": "encode / decode GB/s and compression ratio per workload and block size",
+        "value": None, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u16", "data": "synthetic",
+        "config": {"workload": "sweep: workloads 1, 2, 3, 5 at each of their block sizes, plain "
+                               "and escape-coded streams", "peak_gbs": peak, "peak_kind": peak_kind,
+                   "l2_bytes": l2_bytes},
+        "sweep": rows, "clocks": clocks.summary(), "verified_bit_exact": ok_all,
+        "gpu_launches": None,
+    }
+    if dist is not None:
+        barrier(dist, dev)
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0 if ok_all else 1
+
+
+# ---------------------------------------------------------------------------
 # next row: fused decode + matrix-vector products over the stack's linear weights
 # ---------------------------------------------------------------------------
 def run_dtype(args):
@@ -938,11 +1037,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("wcodec", "reference"), default="wcodec")
     ap.add_argument("--workload", choices=("stack", "layer", "gemv", "gemm", "fp32", "fp16",
-                                           "escape", "escape-layer"),
+                                           "escape", "escape-layer", "sweep"),
                     default="stack",
                     help="stack: the 8B-shaped stack (the benchmark); layer: one decoder layer "
                          "(a smaller case for profiling); escape / escape-layer: the same as "
-                         "escape-coded streams; gemv: fused decode + matrix-vector "
+                         "escape-coded streams; sweep: workloads 1, 2, 3, 5 at each of their "
+                         "block sizes, both stream kinds; gemv: fused decode + matrix-vector "
                          "products over the stack's linear weights; gemm: the same on the "
                          "tensor cores with --tokens activation rows; fp32 / fp16: encode and "
                          "decode of the first --gemv-layers (default 4) layers in that dtype")
@@ -968,6 +1068,8 @@ def main(argv=None):
         return run_dtype(args)
     if args.workload in ("escape", "escape-layer"):
         return run_escape(args)
+    if args.workload == "sweep":
+        return run_sweep(args)
     return run_wcodec(args)
 
 
