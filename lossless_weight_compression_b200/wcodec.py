@@ -307,6 +307,7 @@ class Compressed:
     block: int
     shape: tuple
     dtype: torch.dtype
+    escape: bool = False  # an escape-coded stream (header flags bit 1)
 
     def size(self) -> int:
         return int(self.nbytes.item())
@@ -365,10 +366,11 @@ def decompress(stream_bytes: torch.Tensor, n: int, block: int, *, out: torch.Ten
 
 def decompress_compressed(c: Compressed, out: torch.Tensor | None = None, status=None,
                           stream=None) -> torch.Tensor:
-    """Decode a ``Compressed`` back into its original shape and dtype."""
+    """Decode a ``Compressed`` (plain or escape-coded) back into its original shape and dtype."""
     if out is None:
         out = torch.empty(c.shape, dtype=c.dtype, device=c.buffer.device)
-    return decompress(c.buffer, c.n, c.block, out=out, status=status, stream=stream)
+    fn = decompress_escape if c.escape else decompress
+    return fn(c.buffer, c.n, c.block, out=out, status=status, stream=stream)
 
 
 class CompressBatch:
@@ -570,7 +572,7 @@ def compress_escape(x: torch.Tensor, block: int = 1024, *, workspace: torch.Tens
                             buf.numel(), nbytes.data_ptr(), workspace.data_ptr(),
                             workspace.numel(), status.data_ptr(), _stream_handle(stream))
     _check(rc, "wc_compress_escape")
-    return Compressed(buf, nbytes, status, n, block, tuple(x.shape), x.dtype)
+    return Compressed(buf, nbytes, status, n, block, tuple(x.shape), x.dtype, escape=True)
 
 
 def decompress_escape(stream_bytes: torch.Tensor, n: int, block: int, *,

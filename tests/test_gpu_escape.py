@@ -255,3 +255,12 @@ def test_batch_compress_spans_launches(orc, wclib, cuda):
     for j in range(0, 700, 7):
         got = batch.buffers[j][: sizes[j]].cpu().numpy()
         assert np.array_equal(got, orc.compress_escape(words[j], 256))
+
+
+def test_torch_helpers_round_trip_either_kind(wclib, cuda):
+    w = torch.randn(1000, 777, device=cuda).mul_(0.02).to(torch.bfloat16)
+    for c in (wclib.compress(w, 512), wclib.compress_escape(w, 512)):
+        y = wclib.decompress_compressed(c)
+        torch.cuda.synchronize()
+        assert y.shape == w.shape and y.dtype == w.dtype
+        assert torch.equal(y.view(torch.int16), w.view(torch.int16))
