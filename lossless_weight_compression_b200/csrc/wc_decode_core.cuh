@@ -66,22 +66,27 @@ __device__ __forceinline__ void decode_chunk_w4(const uint8_t* exp_stage, uint32
     r1.w = (prmt(M.w, 0u, 0x3322u) & 0x807F807Fu) | (prmt(e1, o1, 0xF7B3u) * 128u + base7);
 }
 
+// One chunk of 16 elements at any width (0..8), as two octets through decode_octet.
+__device__ __forceinline__ void decode_chunk_any(const uint8_t* exp_stage, uint32_t q, uint4 M,
+                                                 uint4 t0, uint4 t1, uint4& r0, uint4& r1) {
+    const uint32_t w = t0.y;
+    const uint32_t* s32 = reinterpret_cast<const uint32_t*>(exp_stage);
+    const uint32_t sh = 16u - w;
+    uint32_t lo0, hi0, lo1, hi1;
+    fetch_octet(s32, q, lo0, hi0);
+    fetch_octet(s32, q + w, lo1, hi1);
+    r0 = decode_octet(lo0, hi0, M.x, M.y, t0.z, t0.w, sh, t1);
+    r1 = decode_octet(lo1, hi1, M.z, M.w, t0.z, t0.w, sh, t1);
+}
+
 // One chunk of 16 elements at any width: the w = 4 path above, else two octets
 // through decode_octet.
 __device__ __forceinline__ void decode_chunk(const uint8_t* exp_stage, uint32_t q, uint4 M,
                                             uint4 t0, uint4 t1, uint4& r0, uint4& r1) {
-    const uint32_t w = t0.y;
-    if (w == 4u) {
+    if (t0.y == 4u)
         decode_chunk_w4(exp_stage, q, M, t1.w, r0, r1);
-    } else {
-        const uint32_t* s32 = reinterpret_cast<const uint32_t*>(exp_stage);
-        const uint32_t sh = 16u - w;
-        uint32_t lo0, hi0, lo1, hi1;
-        fetch_octet(s32, q, lo0, hi0);
-        fetch_octet(s32, q + w, lo1, hi1);
-        r0 = decode_octet(lo0, hi0, M.x, M.y, t0.z, t0.w, sh, t1);
-        r1 = decode_octet(lo1, hi1, M.z, M.w, t0.z, t0.w, sh, t1);
-    }
+    else
+        decode_chunk_any(exp_stage, q, M, t0, t1, r0, r1);
 }
 
 __device__ __forceinline__ uint64_t ld_u64(const uint8_t* p) {

@@ -487,12 +487,19 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
         const uint4* meta = S.meta + rs * 2 * kTileRows;
         const uint4 t0 = meta[r], t1 = meta[kTileRows + r];
         const uint32_t a_row = smem_addr(S.a + xs * kAStage) + r * 128u;
+        // The warp's eight rows lie in different blocks: if any of them is not of
+        // width 4, every lane takes the general path (one path for the warp instead
+        // of both, one after the other).
+        const bool all_w4 = __all_sync(0xFFFFFFFFu, t0.y == 4u);
 #pragma unroll
         for (uint32_t p = 0; p < 2; ++p) {  // the two 64-column panels
             const uint32_t ch = 4u * p + k;
             const uint4 M = *reinterpret_cast<const uint4*>(man + ((ch ^ sw) << 4));
             uint4 v0, v1;
-            decode_chunk(exs, t0.x + ch * t0.z, M, t0, t1, v0, v1);
+            if (all_w4)
+                decode_chunk_w4(exs, t0.x + ch * t0.z, M, t1.w, v0, v1);
+            else
+                decode_chunk_any(exs, t0.x + ch * t0.z, M, t0, t1, v0, v1);
             const uint32_t row = a_row + p * kAPanel;
             sts128(row + (((2u * k) ^ sw) << 4), v0);
             sts128(row + (((2u * k + 1u) ^ sw) << 4), v1);
