@@ -243,8 +243,9 @@ __device__ void gemm_produce(const GemmParams<MAXI>& P, const GemmSmem& S) {
     const uint32_t R = P.raw_stages;
     int raw_issued[kMaxRawStages] = {-1, -1, -1};  // to drain if the block stops early
     bool ok = true;
-    uint32_t g = 0;
-    for (Cursor cur = cursor_at(P, blockIdx.x, 0); cur.valid; cur = cursor_next(P, cur), ++g) {
+    uint32_t g = 0, rs = 0, round = 0;  // slice g goes to raw stage rs = g % R in round g / R
+    for (Cursor cur = cursor_at(P, blockIdx.x, 0); cur.valid;
+         cur = cursor_next(P, cur), ++g, rs = rs + 1 == R ? (++round, 0u) : rs + 1) {
         const GemvItem& I = P.item[cur.it];
         if (cur.row0 == 0 && cur.s == 0) {
             DecodeItem d;
@@ -252,15 +253,14 @@ __device__ void gemm_produce(const GemmParams<MAXI>& P, const GemmSmem& S) {
             d.stream_bytes = I.stream_bytes;
             check_container(d, make_layout(uint64_t(I.rows) * I.cols, I.block), P.status);
         }
-        const uint32_t rs = g % R;
-        if (g >= R && !gemm_wait(&c.raw_empty[rs], ((g / R) - 1) & 1u, c, P.status, 256)) {
+        if (round > 0 && !gemm_wait(&c.raw_empty[rs], (round - 1) & 1u, c, P.status, 256)) {
             ok = false;
             break;
         }
         mbar_arrive_expect_tx(&c.raw_full[rs], kManStage);
         tma_load_2d(S.man + rs * kManStage, &P.man_map[cur.it], int32_t(cur.s * kSliceCols),
                     int32_t(cur.row0), &c.raw_full[rs]);
-        raw_issued[rs] = int(g / R);
+        raw_issued[rs] = int(round);
     }
     // Stopped early: let the copies already started land before the block exits.
     if (!ok)
@@ -413,6 +413,7 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
     RowState RS;
     uint64_t ua = blockIdx.x;
     uint32_t it_a = 0, sa = 0, slices_a = 0, row0_a = 0;
+    uint32_t rs_a = 0;  // raw stage of the slice being prepared: (its index) % R, kept incrementally
     // decode constants and exponent bytes of slice a (stage a % R), as one cp.async group
     auto prepare = [&](uint32_t a) {
         bool bad = false;
@@ -443,7 +444,9 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
             RS.w = RS.base = 0;
         }
         const uint32_t w = RS.w;
-        const uint32_t rs = a % R;
+        (void)a;
+        const uint32_t rs = rs_a;
+        rs_a = rs_a + 1 == R ? 0u : rs_a + 1;
         if (k == 0) {
             uint4* t0 = S.meta + rs * 2 * kTileRows;
             const uint32_t m1 = (1u << w) - 1u;
@@ -465,7 +468,7 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
     };
     auto commit = [] { asm volatile("cp.async.commit_group;" ::: "memory"); };
 
-    uint32_t ga = 0;
+    uint32_t ga = 0, rs_g = 0, round_g = 0;  // slice g: raw stage g % R, round g / R
     for (; ga < D; ++ga) {  // prologue: slices 0 .. D-1 (one group each, empty past the end)
         if (ga < total) prepare(ga);
         commit();
@@ -478,8 +481,10 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
         else
             asm volatile("cp.async.wait_group 1;" ::: "memory");
         __syncwarp();
-        const uint32_t rs = g % R, xs = g & 1u;
-        if (!gemm_wait_warp(&c.raw_full[rs], (g / R) & 1u, c, P.status) ||
+        const uint32_t rs = rs_g, xs = g & 1u;
+        const uint32_t raw_parity = round_g & 1u;
+        if (rs_g + 1 == R) rs_g = 0, ++round_g; else ++rs_g;
+        if (!gemm_wait_warp(&c.raw_full[rs], raw_parity, c, P.status) ||
             (g >= 2 && !gemm_wait_warp(&c.ax_empty[xs], ((g >> 1) - 1) & 1u, c, P.status)))
             break;
         const uint8_t* man = S.man + rs * kManStage + r * 128u;
