@@ -414,8 +414,8 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
     uint64_t ua = blockIdx.x;
     uint32_t it_a = 0, sa = 0, slices_a = 0, row0_a = 0;
     uint32_t rs_a = 0;  // raw stage of the slice being prepared: (its index) % R, kept incrementally
-    // decode constants and exponent bytes of slice a (stage a % R), as one cp.async group
-    auto prepare = [&](uint32_t a) {
+    // decode constants and exponent bytes of the next slice (into stage rs_a), as one cp.async group
+    auto prepare = [&]() {
         bool bad = false;
         if (sa == 0) {  // first slice of a unit: the row's first block, loaded here
             it_a = find_item(P, ua, it_a);
@@ -444,7 +444,6 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
             RS.w = RS.base = 0;
         }
         const uint32_t w = RS.w;
-        (void)a;
         const uint32_t rs = rs_a;
         rs_a = rs_a + 1 == R ? 0u : rs_a + 1;
         if (k == 0) {
@@ -470,11 +469,11 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
 
     uint32_t ga = 0, rs_g = 0, round_g = 0;  // slice g: raw stage g % R, round g / R
     for (; ga < D; ++ga) {  // prologue: slices 0 .. D-1 (one group each, empty past the end)
-        if (ga < total) prepare(ga);
+        if (ga < total) prepare();
         commit();
     }
     for (uint32_t g = 0; g < total; ++g, ++ga) {
-        if (ga < total) prepare(ga);
+        if (ga < total) prepare();
         commit();
         if (D == 2)
             asm volatile("cp.async.wait_group 2;" ::: "memory");  // slice g's group has landed
