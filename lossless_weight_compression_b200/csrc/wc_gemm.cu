@@ -30,6 +30,7 @@
 
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "wc_decode_core.cuh"
@@ -201,26 +202,52 @@ __device__ __forceinline__ bool gemm_wait_warp(unsigned long long* bar, uint32_t
 }
 
 // ---------------------------------------------------------------------------
-// the sequence of slices a block works on: units blockIdx.x, blockIdx.x +
-// gridDim.x, ..., each swept over cols in slices of 128 (every role walks it)
+// The units a block works on, in rounds of gridDim.x: round k takes unit
+// k*G + b when k is even and k*G + G-1-b when k is odd (b = blockIdx.x,
+// G = gridDim.x), a snake over the blocks. The host numbers a batch's units
+// longest first, so a block that took one of the long units of a round takes
+// one of the short units of the next. Every role walks the same sequence; only
+// the last round can be partial, so the first unit past the end ends the walk.
 // ---------------------------------------------------------------------------
-struct Cursor {
+struct UnitWalk {
     uint64_t u;
+    uint32_t odd;  // round parity
+    __device__ __forceinline__ void start() {
+        u = blockIdx.x;
+        odd = 0;
+    }
+    __device__ __forceinline__ void next() {
+        u += odd ? 1u + 2u * blockIdx.x : 2u * gridDim.x - 1u - 2u * blockIdx.x;
+        odd ^= 1u;
+    }
+};
+
+// the sequence of slices a block works on: its units, each swept over cols in
+// slices of 128 (the producer and the activation loader walk it)
+struct Cursor {
+    UnitWalk w;
     uint32_t it, s, slices, row0;
     bool valid;
 };
 
 template <int MAXI>
-__device__ __forceinline__ Cursor cursor_at(const GemmParams<MAXI>& P, uint64_t u, uint32_t from) {
+__device__ __forceinline__ Cursor cursor_at(const GemmParams<MAXI>& P, UnitWalk w, uint32_t from) {
     Cursor c = {};
-    c.u = u;
-    c.valid = u < P.total_units;
+    c.w = w;
+    c.valid = w.u < P.total_units;
     if (c.valid) {
-        c.it = find_item(P, u, from);
+        c.it = find_item(P, w.u, from);
         c.slices = P.item[c.it].cols / kSliceCols;
-        c.row0 = uint32_t(u - P.unit_begin[c.it]) * kTileRows;
+        c.row0 = uint32_t(w.u - P.unit_begin[c.it]) * kTileRows;
     }
     return c;
+}
+
+template <int MAXI>
+__device__ __forceinline__ Cursor cursor_first(const GemmParams<MAXI>& P) {
+    UnitWalk w;
+    w.start();
+    return cursor_at(P, w, 0);
 }
 
 template <int MAXI>
@@ -230,7 +257,9 @@ __device__ __forceinline__ Cursor cursor_next(const GemmParams<MAXI>& P, const C
         ++n.s;
         return n;
     }
-    return cursor_at(P, c.u + gridDim.x, c.it);
+    UnitWalk w = c.w;
+    w.next();
+    return cursor_at(P, w, c.it);
 }
 
 // ---------------------------------------------------------------------------
@@ -244,7 +273,7 @@ __device__ void gemm_produce(const GemmParams<MAXI>& P, const GemmSmem& S) {
     int raw_issued[kMaxRawStages] = {-1, -1, -1};  // to drain if the block stops early
     bool ok = true;
     uint32_t g = 0, rs = 0, round = 0;  // slice g goes to raw stage rs = g % R in round g / R
-    for (Cursor cur = cursor_at(P, blockIdx.x, 0); cur.valid;
+    for (Cursor cur = cursor_first(P); cur.valid;
          cur = cursor_next(P, cur), ++g, rs = rs + 1 == R ? (++round, 0u) : rs + 1) {
         const GemvItem& I = P.item[cur.it];
         if (cur.row0 == 0 && cur.s == 0) {
@@ -278,7 +307,7 @@ __device__ void gemm_load_x(const GemmParams<MAXI>& P, const GemmSmem& S) {
     int x_issued[2] = {-1, -1};
     bool ok = true;
     uint32_t g = 0;
-    for (Cursor cur = cursor_at(P, blockIdx.x, 0); cur.valid; cur = cursor_next(P, cur), ++g) {
+    for (Cursor cur = cursor_first(P); cur.valid; cur = cursor_next(P, cur), ++g) {
         const uint32_t xs = g & 1u;
         if (g >= 2 && !gemm_wait(&c.ax_empty[xs], ((g >> 1) - 1) & 1u, c, P.status, 256)) {
             ok = false;
@@ -402,8 +431,9 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
     uint32_t total = 0;
     {
         uint32_t it = 0;
-        for (uint64_t u = blockIdx.x; u < P.total_units; u += gridDim.x) {
-            it = find_item(P, u, it);
+        UnitWalk w;
+        for (w.start(); w.u < P.total_units; w.next()) {
+            it = find_item(P, w.u, it);
             total += P.item[it].cols / kSliceCols;
         }
     }
@@ -411,17 +441,18 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
     // the slice being prepared: its unit, and this lane's row
     UnitState U = {};
     RowState RS;
-    uint64_t ua = blockIdx.x;
+    UnitWalk wa;
+    wa.start();
     uint32_t it_a = 0, sa = 0, slices_a = 0, row0_a = 0;
     uint32_t rs_a = 0;  // raw stage of the slice being prepared: (its index) % R, kept incrementally
     // decode constants and exponent bytes of the next slice (into stage rs_a), as one cp.async group
     auto prepare = [&]() {
         bool bad = false;
         if (sa == 0) {  // first slice of a unit: the row's first block, loaded here
-            it_a = find_item(P, ua, it_a);
+            it_a = find_item(P, wa.u, it_a);
             U = unit_state(P, it_a);
             slices_a = U.cols / kSliceCols;
-            row0_a = uint32_t(ua - P.unit_begin[it_a]) * kTileRows;
+            row0_a = uint32_t(wa.u - P.unit_begin[it_a]) * kTileRows;
             const uint64_t row = row0_a + r;
             RS.valid = row < U.rows;
             RS.w = RS.base = 0;
@@ -462,7 +493,7 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
         if (bad) report(P.status, kStatusCorrupt);
         if (++sa == slices_a) {
             sa = 0;
-            ua += gridDim.x;
+            wa.next();
         }
     };
     auto commit = [] { asm volatile("cp.async.commit_group;" ::: "memory"); };
@@ -529,8 +560,9 @@ __device__ void gemm_mma(const GemmParams<MAXI>& P, const GemmSmem& S) {
     const uint32_t xstage = P.nt * 256, xpanel = P.nt * 128;
     uint32_t g = 0, j = 0, it = 0;
     bool issued = false;
-    for (uint64_t u = blockIdx.x; u < P.total_units; u += gridDim.x, ++j) {
-        it = find_item(P, u, it);
+    UnitWalk w;
+    for (w.start(); w.u < P.total_units; w.next(), ++j) {
+        it = find_item(P, w.u, it);
         const uint32_t slices = P.item[it].cols / kSliceCols;
         const uint32_t buf = j & 1u;
         if (j >= 2 && !gemm_wait(&c.acc_empty[buf], ((j >> 1) - 1) & 1u, c, P.status)) break;
@@ -576,10 +608,11 @@ __device__ void gemm_epilogue(const GemmParams<MAXI>& P, const GemmSmem& S, int 
     GemmCtl& c = *S.ctl;
     const uint32_t q = uint32_t(warp) & 3u;
     uint32_t j = 0, it = 0;
-    for (uint64_t u = blockIdx.x; u < P.total_units; u += gridDim.x, ++j) {
-        it = find_item(P, u, it);
+    UnitWalk w;
+    for (w.start(); w.u < P.total_units; w.next(), ++j) {
+        it = find_item(P, w.u, it);
         const GemvItem& I = P.item[it];
-        const uint32_t row = uint32_t(u - P.unit_begin[it]) * kTileRows + 32u * q + uint32_t(lane);
+        const uint32_t row = uint32_t(w.u - P.unit_begin[it]) * kTileRows + 32u * q + uint32_t(lane);
         const uint32_t buf = j & 1u;
         if (!gemm_wait_warp(&c.acc_full[buf], (j >> 1) & 1u, c, P.status, 512)) return;
         tc_fence_after();
@@ -702,9 +735,15 @@ cudaError_t gemm_launch(const GemvItem* items, uint32_t count, uint32_t tokens, 
     p.raw_stages = gemm_smem_bytes(p.nt, 3) <= kSmemLimit ? 3 : 2;
     p.tmem_cols = 32;
     while (p.tmem_cols < 2 * p.nt) p.tmem_cols *= 2;
+    // Units are numbered longest first (matrices by decreasing column count,
+    // ties in the caller's order) for the blocks' snake walk.
+    uint32_t order[MAXI];
+    for (uint32_t i = 0; i < count; ++i) order[i] = i;
+    std::stable_sort(order, order + count,
+                     [&](uint32_t a, uint32_t b) { return items[a].cols > items[b].cols; });
     uint64_t units = 0;
     for (uint32_t i = 0; i < count; ++i) {
-        const GemvItem& I = items[i];
+        const GemvItem& I = items[order[i]];
         p.item[i] = I;
         p.unit_begin[i] = units;
         units += (uint64_t(I.rows) + kTileRows - 1) / kTileRows;
