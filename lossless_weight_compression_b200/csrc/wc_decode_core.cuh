@@ -45,17 +45,16 @@ __device__ __forceinline__ uint4 decode_octet(uint32_t lo, uint32_t hi, uint32_t
     return r;
 }
 
-// The common case w = 4, as one chunk of 16 elements: its two octets are the 8
-// bytes at q (8-byte aligned: q = payload offset + 4 * (element offset in the
-// block / 8)), element t in nibble t. Low nibbles give the even elements, high
-// nibbles the odd ones; a byte permute then places elements 2k and 2k+1 in
-// the two 16-bit lanes of a word, using the permute's sign-replicating
-// selectors on bytes below 0x80 as zero bytes. Same result as decode_octet.
-__device__ __forceinline__ void decode_chunk_w4(const uint8_t* exp_stage, uint32_t q, uint4 M,
-                                                uint32_t base7, uint4& r0, uint4& r1) {
-    const uint2 F = *reinterpret_cast<const uint2*>(exp_stage + q);
-    const uint32_t e0 = F.x & 0x0F0F0F0Fu, o0 = (F.x >> 4) & 0x0F0F0F0Fu;  // elements 0..7
-    const uint32_t e1 = F.y & 0x0F0F0F0Fu, o1 = (F.y >> 4) & 0x0F0F0F0Fu;  // elements 8..15
+// The common case w = 4: an octet is 4 bytes, element t in nibble t. Low
+// nibbles give the even elements, high nibbles the odd ones; a byte permute
+// then places elements 2k and 2k+1 in the two 16-bit lanes of a word, using
+// the permute's sign-replicating selectors on bytes below 0x80 as zero bytes.
+// Same result as decode_octet. Two octets f0, f1 with their sign+mantissa
+// bytes in M.xy and M.zw:
+__device__ __forceinline__ void decode_octets_w4(uint32_t f0, uint32_t f1, uint4 M, uint32_t base7,
+                                                 uint4& r0, uint4& r1) {
+    const uint32_t e0 = f0 & 0x0F0F0F0Fu, o0 = (f0 >> 4) & 0x0F0F0F0Fu;  // octet 0
+    const uint32_t e1 = f1 & 0x0F0F0F0Fu, o1 = (f1 >> 4) & 0x0F0F0F0Fu;  // octet 1
     r0.x = (prmt(M.x, 0u, 0x1100u) & 0x807F807Fu) | (prmt(e0, o0, 0xC480u) * 128u + base7);
     r0.y = (prmt(M.x, 0u, 0x3322u) & 0x807F807Fu) | (prmt(e0, o0, 0xD591u) * 128u + base7);
     r0.z = (prmt(M.y, 0u, 0x1100u) & 0x807F807Fu) | (prmt(e0, o0, 0xE6A2u) * 128u + base7);
@@ -66,17 +65,31 @@ __device__ __forceinline__ void decode_chunk_w4(const uint8_t* exp_stage, uint32
     r1.w = (prmt(M.w, 0u, 0x3322u) & 0x807F807Fu) | (prmt(e1, o1, 0xF7B3u) * 128u + base7);
 }
 
+// One chunk of 16 elements at w = 4: its two octets are the 8 bytes at q
+// (8-byte aligned: q = payload offset + 4 * (element offset in the block / 8)).
+__device__ __forceinline__ void decode_chunk_w4(const uint8_t* exp_stage, uint32_t q, uint4 M,
+                                                uint32_t base7, uint4& r0, uint4& r1) {
+    const uint2 F = *reinterpret_cast<const uint2*>(exp_stage + q);
+    decode_octets_w4(F.x, F.y, M, base7, r0, r1);
+}
+
+// Two octets of any width (0..8) starting at bytes q0 and q1 of the staged
+// exponent bytes, with their sign+mantissa bytes in M.xy and M.zw.
+__device__ __forceinline__ void decode_octets_any(const uint8_t* exp_stage, uint32_t q0, uint32_t q1,
+                                                  uint4 M, uint4 t0, uint4 t1, uint4& r0, uint4& r1) {
+    const uint32_t* s32 = reinterpret_cast<const uint32_t*>(exp_stage);
+    const uint32_t sh = 16u - t0.y;
+    uint32_t lo0, hi0, lo1, hi1;
+    fetch_octet(s32, q0, lo0, hi0);
+    fetch_octet(s32, q1, lo1, hi1);
+    r0 = decode_octet(lo0, hi0, M.x, M.y, t0.z, t0.w, sh, t1);
+    r1 = decode_octet(lo1, hi1, M.z, M.w, t0.z, t0.w, sh, t1);
+}
+
 // One chunk of 16 elements at any width (0..8), as two octets through decode_octet.
 __device__ __forceinline__ void decode_chunk_any(const uint8_t* exp_stage, uint32_t q, uint4 M,
                                                  uint4 t0, uint4 t1, uint4& r0, uint4& r1) {
-    const uint32_t w = t0.y;
-    const uint32_t* s32 = reinterpret_cast<const uint32_t*>(exp_stage);
-    const uint32_t sh = 16u - w;
-    uint32_t lo0, hi0, lo1, hi1;
-    fetch_octet(s32, q, lo0, hi0);
-    fetch_octet(s32, q + w, lo1, hi1);
-    r0 = decode_octet(lo0, hi0, M.x, M.y, t0.z, t0.w, sh, t1);
-    r1 = decode_octet(lo1, hi1, M.z, M.w, t0.z, t0.w, sh, t1);
+    decode_octets_any(exp_stage, q, q + t0.y, M, t0, t1, r0, r1);
 }
 
 // One chunk of 16 elements at any width: the w = 4 path above, else two octets

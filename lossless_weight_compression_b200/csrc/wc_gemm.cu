@@ -43,7 +43,7 @@ constexpr uint32_t kSliceCols = 128;   // columns per pipeline slice (8 MMAs of 
 constexpr uint32_t kExpPitch = 144;    // staged exponent bytes per row (16*w <= 128, +16 spreads banks)
 constexpr uint32_t kManStage = kTileRows * kSliceCols;      // 16 KB
 constexpr uint32_t kExpStage = kTileRows * kExpPitch;       // 18 KB
-constexpr uint32_t kMetaStage = kTileRows * 2 * 16;         // t0, t1 per row
+constexpr uint32_t kMetaStage = kTileRows * 4;              // w | base << 8 per row
 constexpr uint32_t kAStage = kTileRows * kSliceCols * 2;    // 32 KB: two 64-column panels
 constexpr uint32_t kAPanel = kTileRows * 128;               // 128 rows x 128 bytes
 constexpr uint32_t kMaxRawStages = 3;
@@ -92,7 +92,7 @@ struct GemmSmem {
     uint8_t* x;     // 2 stages of nt * 256 bytes
     uint8_t* man;   // raw_stages stages
     uint8_t* exp;
-    uint4* meta;    // per stage: t0[128], t1[128]
+    uint32_t* meta;  // per stage: w | base << 8 of each row
 };
 
 __host__ __device__ inline uint32_t gemm_smem_bytes(uint32_t nt, uint32_t raw_stages) {
@@ -344,18 +344,37 @@ __device__ void gemm_load_x(const GemmParams<MAXI>& P, const GemmSmem& S) {
 // ---------------------------------------------------------------------------
 static_assert(kDecWarps * 8 == int(kTileRows), "each decoding warp owns 8 rows");
 
-// State of one row for the slice being prepared: its block, the block's
-// decode parameters, where the slice's exponent bytes start, and the header of
-// the row's next block (loaded when the row enters a block, so it is in
-// registers by the time the row gets there).
+// State of one row for the slice being prepared: where its exponent bytes
+// start, how many of its block's elements are left from there, the block's
+// width and base, and the header of the row's next block (loaded
+// when the row enters a block, so it is in registers by the time the row gets
+// there). Everything but the byte pointer and the count changes only when the
+// row enters a block: once every block / 128 slices.
 struct RowState {
-    uint64_t el;    // element index of the slice's first column
-    uint64_t src;   // stream offset of the slice's exponent bytes
+    uint64_t b;          // the row's current block
+    const uint8_t* src;  // the slice's exponent bytes
+    uint32_t left;       // elements from the slice's first column to the block's end
     uint32_t w, base;
-    uint32_t nh, noff;  // next block: header and offset (16-byte units)
-    uint64_t nnx;       // next block: the following block's payload start
+    uint32_t nh, noff;   // next block: header and offset (16-byte units)
+    uint64_t nnx;        // next block: the following block's payload start
     bool valid;
 };
+
+__device__ __forceinline__ void set_width(RowState& R, uint32_t w, uint32_t base) {
+    R.w = w;
+    R.base = base;
+}
+
+// Decode constants of a row from its width and base, in the form decode_octet
+// takes: t0 = {row offset, w, 2w, 4w}, t1 = {pair masks, 2w-bit mask, 4w-bit
+// mask, base << 7 in both 16-bit lanes}.
+__device__ __forceinline__ void row_constants(uint32_t row_off, uint32_t w, uint32_t base,
+                                              uint4& t0, uint4& t1) {
+    const uint32_t m1 = (1u << w) - 1u;
+    t0 = make_uint4(row_off, w, 2 * w, 4 * w);
+    t1 = make_uint4(m1 | (m1 << 16), (1u << (2 * w)) - 1u,
+                    w == 8u ? 0xFFFFFFFFu : (1u << (4 * w)) - 1u, base * 0x00800080u);
+}
 
 // Unit-level constants of the slice being prepared.
 struct UnitState {
@@ -394,25 +413,27 @@ __device__ __forceinline__ void load_block(const UnitState& U, uint64_t b, uint3
     nx = b + 1 < U.nb ? 16ull * U.offs[b + 1] : ld_u64(U.stream + 64);
 }
 
-// The row enters block b (its header in h/off/nx): set w, base and the slice's
-// exponent offset, checking the header and, at the block's first element, the
-// offset chain; then start loading the row's next block. False if corrupt
-// (the row then decodes as w = 0).
+// The row enters the block holding element el (its header in h/off/nx; el is
+// a slice's first column): set the width, the decode constants, the slice's
+// exponent bytes and the block's remaining elements, checking the header, that
+// the block's payload lies inside the stream (so no slice of it reads past the
+// end) and, at the block's first element, the offset chain; then start loading
+// the row's next block. False if corrupt (the row then decodes as w = 0).
 __device__ __forceinline__ bool enter_block(const UnitState& U, RowState& R, uint64_t row,
-                                            uint32_t h, uint32_t off, uint64_t nx) {
-    const uint32_t bmask = U.block - 1u;
-    const uint64_t b = R.el >> U.log2B;
+                                            uint64_t el, uint32_t h, uint32_t off, uint64_t nx) {
+    const uint64_t b = el >> U.log2B;
+    const uint32_t ob = uint32_t(el) & (U.block - 1u);  // the slice's offset in the block
+    const uint64_t len = min(uint64_t(U.block), U.n - (b << U.log2B));
     uint32_t w = h >> 8, base = h & 0xFFu;
     bool bad = w > 8u || (w == 8u && base != 0u);
-    const uint64_t sb = 16ull * off;
-    if ((R.el & bmask) == 0) {
-        const uint64_t len = min(uint64_t(U.block), U.n - (b << U.log2B));
-        bad |= sb + ((len + 7) >> 3) * min(w, 8u) != nx;
-    }
+    const uint64_t sb = 16ull * off, end = sb + ((len + 7) >> 3) * min(w, 8u);
+    if (ob == 0) bad |= end != nx;
+    bad |= U.off_exp + end > U.stream_bytes;
     if (bad) w = base = 0;
-    R.w = w;
-    R.base = base;
-    R.src = U.off_exp + sb + ((R.el & bmask) >> 3) * w;
+    R.b = b;
+    R.left = uint32_t(len) - ob;
+    R.src = U.stream + U.off_exp + sb + (ob >> 3) * w;
+    set_width(R, w, base);
     // the row continues into block b + 1 inside this unit's columns?
     if (((b + 1) << U.log2B) < (row + 1) * uint64_t(U.cols)) load_block(U, b + 1, R.nh, R.noff, R.nnx);
     return !bad;
@@ -423,9 +444,19 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
     GemmCtl& c = *S.ctl;
     const uint32_t R = P.raw_stages, D = R - 1;
     // lane = 8q + 4b + k: row pair q of the warp's 8 rows, member b, chunk k of a panel
+    // preparing: lane = 8q + 4b + k prepares row r (four lanes per row)
     const uint32_t k = uint32_t(lane) & 3u, q = uint32_t(lane) >> 3, b = (uint32_t(lane) >> 2) & 1u;
-    const uint32_t r = 8u * uint32_t(dw) + (b ? (q ^ 5u) : q);  // this lane's row of every slice
-    const uint32_t sw = r & 7u;
+    const uint32_t r = 8u * uint32_t(dw) + (b ? (q ^ 5u) : q);
+    // decoding: eight lanes per row, four rows per step, two steps per slice.
+    // Lane c = lane % 8 of a row takes 16 of its 128 columns, octets o0 and o1
+    // (2c, 2c+1 in the first panel; 2c+1, 2c in the second, so that the 8 lanes
+    // of a row store to 8 distinct bank groups each time). Step 0 takes the
+    // warp's rows 0,4,1,5 (slots 0..3), step 1 rows 2,6,3,7: the two rows of a
+    // half-warp are four apart, so their exponent and mantissa loads fall in
+    // complementary bank halves.
+    const uint32_t c8 = uint32_t(lane) & 7u, slot = uint32_t(lane) >> 3, pp = c8 >> 2;
+    const uint32_t o0 = 2u * c8 + pp, o1 = 2u * c8 + 1u - pp;
+    const uint32_t row_s0 = 8u * uint32_t(dw) + (slot >> 1) + 4u * (slot & 1u), row_s1 = row_s0 + 2u;
 
     // slices this block works through
     uint32_t total = 0;
@@ -440,12 +471,14 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
 
     // the slice being prepared: its unit, and this lane's row
     UnitState U = {};
-    RowState RS;
+    RowState RS = {};
     UnitWalk wa;
     wa.start();
     uint32_t it_a = 0, sa = 0, slices_a = 0, row0_a = 0;
     uint32_t rs_a = 0;  // raw stage of the slice being prepared: (its index) % R, kept incrementally
-    // decode constants and exponent bytes of the next slice (into stage rs_a), as one cp.async group
+    const uint32_t row_off = r * kExpPitch;                          // the row in an exponent stage
+    const uint32_t exp_lane = smem_addr(S.exp) + row_off + 16u * k;  // this lane's pieces in stage 0
+    // width, base and exponent bytes of the next slice (into stage rs_a), as one cp.async group
     auto prepare = [&]() {
         bool bad = false;
         if (sa == 0) {  // first slice of a unit: the row's first block, loaded here
@@ -455,39 +488,29 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
             row0_a = uint32_t(wa.u - P.unit_begin[it_a]) * kTileRows;
             const uint64_t row = row0_a + r;
             RS.valid = row < U.rows;
-            RS.w = RS.base = 0;
+            set_width(RS, 0, 0);
+            RS.left = 0;
             if (RS.valid) {
-                RS.el = row * U.cols;
+                const uint64_t el = row * U.cols;
                 uint32_t h, off;
                 uint64_t nx;
-                load_block(U, RS.el >> U.log2B, h, off, nx);
-                bad |= !enter_block(U, RS, row, h, off, nx);
+                load_block(U, el >> U.log2B, h, off, nx);
+                bad |= !enter_block(U, RS, row, el, h, off, nx);
             }
         } else if (RS.valid) {
-            RS.el += kSliceCols;
-            if ((RS.el & (U.block - 1u)) == 0)
-                bad |= !enter_block(U, RS, row0_a + r, RS.nh, RS.noff, RS.nnx);
+            RS.left -= kSliceCols;
+            if (RS.left == 0)  // the slice starts the row's next block
+                bad |= !enter_block(U, RS, row0_a + r, (RS.b + 1) << U.log2B, RS.nh, RS.noff, RS.nnx);
             else
                 RS.src += 16u * RS.w;
-        }
-        if (RS.valid && RS.src + 16u * RS.w > U.stream_bytes) {  // payload past the end
-            bad = true;
-            RS.w = RS.base = 0;
         }
         const uint32_t w = RS.w;
         const uint32_t rs = rs_a;
         rs_a = rs_a + 1 == R ? 0u : rs_a + 1;
-        if (k == 0) {
-            uint4* t0 = S.meta + rs * 2 * kTileRows;
-            const uint32_t m1 = (1u << w) - 1u;
-            t0[r] = make_uint4(r * kExpPitch, w, 2 * w, 4 * w);
-            t0[kTileRows + r] =
-                make_uint4(m1 | (m1 << 16), (1u << (2 * w)) - 1u,
-                           w == 8u ? 0xFFFFFFFFu : (1u << (4 * w)) - 1u, RS.base * 0x00800080u);
-        }
+        if (k == 0) S.meta[rs * kTileRows + r] = w | (RS.base << 8);
         // the row's 16*w exponent bytes: pieces k and k + 4 (four lanes per row)
-        const uint32_t d = smem_addr(S.exp + rs * kExpStage) + r * kExpPitch + 16u * k;
-        const uint8_t* src = U.stream + RS.src + 16u * k;
+        const uint32_t d = exp_lane + rs * kExpStage;
+        const uint8_t* src = RS.src + 16u * k;
         if (k < w) cp_async16(d, src);
         if (k + 4u < w) cp_async16(d + 64u, src + 64u);
         if (bad) report(P.status, kStatusCorrupt);
@@ -517,27 +540,43 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
         if (!gemm_wait_warp(&c.raw_full[rs], raw_parity, c, P.status) ||
             (g >= 2 && !gemm_wait_warp(&c.ax_empty[xs], ((g >> 1) - 1) & 1u, c, P.status)))
             break;
-        const uint8_t* man = S.man + rs * kManStage + r * 128u;
+        const uint8_t* man = S.man + rs * kManStage;
         const uint8_t* exs = S.exp + rs * kExpStage;
-        const uint4* meta = S.meta + rs * 2 * kTileRows;
-        const uint4 t0 = meta[r], t1 = meta[kTileRows + r];
-        const uint32_t a_row = smem_addr(S.a + xs * kAStage) + r * 128u;
-        // The warp's eight rows lie in different blocks: if any of them is not of
-        // width 4, every lane takes the general path (one path for the warp instead
-        // of both, one after the other).
-        const bool all_w4 = __all_sync(0xFFFFFFFFu, t0.y == 4u);
+        const uint32_t* meta = S.meta + rs * kTileRows;
+        const uint32_t a_tile = smem_addr(S.a + xs * kAStage) + pp * kAPanel;
+        // Every load of both steps first, the exponent words at their width-4
+        // places: a step whose four rows are all of width 4 (the common case)
+        // decodes from them; otherwise the step takes the general path, which
+        // fetches its octets again at the rows' widths.
+        uint32_t mw[2], f[2][2];
+        uint4 M[2];
 #pragma unroll
-        for (uint32_t p = 0; p < 2; ++p) {  // the two 64-column panels
-            const uint32_t ch = 4u * p + k;
-            const uint4 M = *reinterpret_cast<const uint4*>(man + ((ch ^ sw) << 4));
+        for (uint32_t st = 0; st < 2; ++st) {
+            const uint32_t rr = st ? row_s1 : row_s0;
+            mw[st] = meta[rr];
+            const uint8_t* mp = man + rr * 128u + ((c8 ^ (rr & 7u)) << 4);
+            const uint2 h0 = *reinterpret_cast<const uint2*>(mp + 8u * pp);
+            const uint2 h1 = *reinterpret_cast<const uint2*>(mp + 8u - 8u * pp);
+            M[st] = make_uint4(h0.x, h0.y, h1.x, h1.y);
+            const uint8_t* ep = exs + rr * kExpPitch;
+            f[st][0] = *reinterpret_cast<const uint32_t*>(ep + 4u * o0);
+            f[st][1] = *reinterpret_cast<const uint32_t*>(ep + 4u * o1);
+        }
+#pragma unroll
+        for (uint32_t st = 0; st < 2; ++st) {
+            const uint32_t rr = st ? row_s1 : row_s0;
+            const uint32_t sw = rr & 7u, w = mw[st] & 0xFFu, base = mw[st] >> 8;
             uint4 v0, v1;
-            if (all_w4)
-                decode_chunk_w4(exs, t0.x + ch * t0.z, M, t1.w, v0, v1);
-            else
-                decode_chunk_any(exs, t0.x + ch * t0.z, M, t0, t1, v0, v1);
-            const uint32_t row = a_row + p * kAPanel;
-            sts128(row + (((2u * k) ^ sw) << 4), v0);
-            sts128(row + (((2u * k + 1u) ^ sw) << 4), v1);
+            if (__all_sync(0xFFFFFFFFu, w == 4u)) {
+                decode_octets_w4(f[st][0], f[st][1], M[st], base * 0x00800080u, v0, v1);
+            } else {
+                uint4 t0, t1;
+                row_constants(rr * kExpPitch, w, base, t0, t1);
+                decode_octets_any(exs, t0.x + o0 * w, t0.x + o1 * w, M[st], t0, t1, v0, v1);
+            }
+            const uint32_t row = a_tile + rr * 128u;
+            sts128(row + (((o0 & 7u) ^ sw) << 4), v0);
+            sts128(row + (((o1 & 7u) ^ sw) << 4), v1);
         }
         fence_proxy_async_smem();  // the tensor cores read A through the async proxy
         __syncwarp();
@@ -651,7 +690,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     p += P.raw_stages * kManStage;
     S.exp = p;
     p += P.raw_stages * kExpStage;
-    S.meta = reinterpret_cast<uint4*>(p);
+    S.meta = reinterpret_cast<uint32_t*>(p);
     GemmCtl& c = *S.ctl;
     if (tid == 0) {
         for (uint32_t s = 0; s < kMaxRawStages; ++s) {
