@@ -23,9 +23,9 @@
 //                     with coalesced 16-byte stores: their position needs no
 //                     prefix), reduce per-block min/max, compute widths and
 //                     the tile-local scan, publish the tile's byte count at
-//                     once, and pack the exponent payload into one of six
+//                     once, and pack the exponent payload into one of four
 //                     output stages -- none of this waits on other tiles;
-//   4 store warps     take alternate tiles; each runs the look-back over a
+//   2 store warps     take alternate tiles; each runs the look-back over a
 //                     256-tile window per round trip (wide enough to keep up
 //                     with the rate at which tiles start), publishes the
 //                     inclusive prefix, writes the block headers and offsets,

@@ -13,11 +13,12 @@
 // swept over cols in slices of 128:
 //   - one thread starts each slice's mantissa bytes (one 2-D TMA load,
 //     128-byte swizzled) and another its activations (two 2-D TMA loads);
-//   - sixteen decoding warps own 8 rows each: a few slices ahead they check
-//     their rows' block headers and offsets and fetch each row's exponent
-//     bytes (a 128-column slice of a row is 16 whole octets of one block, 16*w
-//     contiguous bytes; 16-byte cp.async pieces), then turn the staged bytes
-//     into BF16 weights in the K-major 128-byte-swizzled layout the MMA reads;
+//   - four preparing warps, a few slices ahead, check each row's block
+//     header and offset and fetch the row's exponent bytes (a 128-column slice
+//     of a row is 16 whole octets of one block, 16*w contiguous bytes; 16-byte
+//     cp.async pieces);
+//   - sixteen decoding warps own 8 rows each and turn the staged bytes into
+//     BF16 weights in the K-major 128-byte-swizzled layout the MMA reads;
 //   - one thread issues tcgen05.mma (BF16 x BF16 -> FP32, M = 128, K = 16) into
 //     one of two accumulators in tensor memory;
 //   - four epilogue warps move a finished accumulator out with tcgen05.ld and
@@ -56,7 +57,9 @@ constexpr int kEpiWarps = 4;
 constexpr int kDecWarp0 = 6;
 constexpr int kDecWarps = 16;
 constexpr int kXWarp = kDecWarp0 + kDecWarps;    // 22: activation loader
-constexpr int kGemmThreads = 32 * (kXWarp + 1);  // 736
+constexpr int kPrepWarp0 = kXWarp + 1;           // 23..26: one lane per row of the tile
+constexpr int kPrepWarps = 4;
+constexpr int kGemmThreads = 32 * (kPrepWarp0 + kPrepWarps);  // 864
 
 template <int MAXI>
 struct GemmParams {
@@ -79,6 +82,7 @@ struct GemmParams {
 // every 8 rows of 128 bytes and is a function of the address.
 struct GemmCtl {
     unsigned long long raw_full[kMaxRawStages], raw_empty[kMaxRawStages];
+    unsigned long long exp_full[kMaxRawStages];  // a stage's exponent bytes and row words are in
     unsigned long long a_full[2], x_full[2], ax_empty[2];
     unsigned long long acc_full[2], acc_empty[2];
     unsigned long long drain;
@@ -165,6 +169,12 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         "[%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
         : "memory");
+}
+
+// The mbarrier's current phase also waits for every cp.async this thread has
+// started so far (no net arrival: the thread still arrives itself).
+__device__ __forceinline__ void cp_async_mbar_arrive(unsigned long long* bar) {
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 // 16-byte asynchronous copy global -> shared through L2 (not L1).
@@ -326,21 +336,18 @@ __device__ void gemm_load_x(const GemmParams<MAXI>& P, const GemmSmem& S) {
 }
 
 // ---------------------------------------------------------------------------
-// decoding warps. A slice is 128 rows x 8 chunks of 16 columns. Warp d owns
-// rows 8d .. 8d+7 of every slice, one row per lane group of 4: lane 8q + 4b + k
-// takes row 8d + q (b = 0) or 8d + (q ^ 5) (b = 1), chunks k and k + 4 (one in
-// each 64-column panel). The two rows of a quarter-warp differ in bits 0 and 2
-// of their swizzle phase (row % 8), so the quarter's 16-byte mantissa loads and
-// its A stores each hit 8 distinct bank groups.
+// preparing and decoding warps. A slice is 128 rows x 128 columns.
 //
-// Each warp prepares its own rows raw_stages - 1 slices ahead: it checks a
-// row's block header and offset when the row enters the block (the header
-// was loaded when the row entered the previous block), writes the decode
-// constants to shared memory, and fetches the row's 16*w exponent bytes (four
-// lanes per row, 16-byte cp.async pieces) as one cp.async group per slice. No
-// other warp touches these rows' staging, so a group wait and a warp barrier
-// are all the hand-off needs; only the mantissa bytes (TMA, producer) and the
-// finished A tile (MMA) are shared.
+// Four preparing warps run a few slices ahead, one lane per row: a lane checks
+// its row's block header and offset when the row enters a block (the header
+// was loaded when the row entered the previous block), writes the row's width
+// and base to the slice's stage, and fetches the row's 16*w exponent bytes
+// (16-byte cp.async pieces). An mbarrier per stage hands the staged bytes
+// over; it completes once every row's lane has arrived and all their copies
+// have landed.
+//
+// Sixteen decoding warps own 8 rows each and turn the staged bytes into BF16
+// weights in the K-major 128-byte-swizzled layout the MMA reads.
 // ---------------------------------------------------------------------------
 static_assert(kDecWarps * 8 == int(kTileRows), "each decoding warp owns 8 rows");
 
@@ -439,16 +446,74 @@ __device__ __forceinline__ bool enter_block(const UnitState& U, RowState& R, uin
     return !bad;
 }
 
+// Preparing warps: lane l of preparing warp p owns row 32p + l of every slice.
+// For each slice, once the decoding warps have freed its stage, the lane writes
+// its row's width and base word and starts the row's 16*w exponent bytes
+// (16-byte cp.async pieces); the stage's exp_full barrier then completes when
+// all 128 rows have done so and all their copies have landed.
+template <int MAXI>
+__device__ void gemm_prepare(const GemmParams<MAXI>& P, const GemmSmem& S, int pw, int lane) {
+    GemmCtl& c = *S.ctl;
+    const uint32_t R = P.raw_stages;
+    const uint32_t r = 32u * uint32_t(pw) + uint32_t(lane);
+    const uint32_t exp_row = smem_addr(S.exp) + r * kExpPitch;
+    UnitState U = {};
+    RowState RS = {};
+    UnitWalk wk;
+    wk.start();
+    uint32_t it = 0, sa = 0, slices = 0, row0 = 0;
+    uint32_t rs = 0, round = 0;  // slice a: raw stage a % R, round a / R
+    while (wk.u < P.total_units) {
+        bool bad = false;
+        if (sa == 0) {  // first slice of a unit: the row's first block, loaded here
+            it = find_item(P, wk.u, it);
+            U = unit_state(P, it);
+            slices = U.cols / kSliceCols;
+            row0 = uint32_t(wk.u - P.unit_begin[it]) * kTileRows;
+            const uint64_t row = row0 + r;
+            RS.valid = row < U.rows;
+            set_width(RS, 0, 0);
+            RS.left = 0;
+            if (RS.valid) {
+                const uint64_t el = row * U.cols;
+                uint32_t h, off;
+                uint64_t nx;
+                load_block(U, el >> U.log2B, h, off, nx);
+                bad |= !enter_block(U, RS, row, el, h, off, nx);
+            }
+        } else if (RS.valid) {
+            RS.left -= kSliceCols;
+            if (RS.left == 0)  // the slice starts the row's next block
+                bad |= !enter_block(U, RS, row0 + r, (RS.b + 1) << U.log2B, RS.nh, RS.noff, RS.nnx);
+            else
+                RS.src += 16u * RS.w;
+        }
+        if (bad) report(P.status, kStatusCorrupt);
+        // the stage is free once the decoding warps are done with slice a - R
+        if (round > 0 && !gemm_wait_warp(&c.raw_empty[rs], (round - 1) & 1u, c, P.status)) break;
+        const uint32_t w = RS.w;
+        S.meta[rs * kTileRows + r] = w | (RS.base << 8);
+        const uint32_t d = exp_row + rs * kExpStage;
+#pragma unroll
+        for (uint32_t j = 0; j < 8; ++j)
+            if (j < w) cp_async16(d + 16u * j, RS.src + 16u * j);
+        cp_async_mbar_arrive(&c.exp_full[rs]);
+        mbar_arrive(&c.exp_full[rs]);
+        if (++sa == slices) {
+            sa = 0;
+            wk.next();
+        }
+        if (rs + 1 == R) rs = 0, ++round; else ++rs;
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // nothing lands after the block ends
+}
+
 template <int MAXI>
 __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw, int lane) {
     GemmCtl& c = *S.ctl;
-    const uint32_t R = P.raw_stages, D = R - 1;
-    // lane = 8q + 4b + k: row pair q of the warp's 8 rows, member b, chunk k of a panel
-    // preparing: lane = 8q + 4b + k prepares row r (four lanes per row)
-    const uint32_t k = uint32_t(lane) & 3u, q = uint32_t(lane) >> 3, b = (uint32_t(lane) >> 2) & 1u;
-    const uint32_t r = 8u * uint32_t(dw) + (b ? (q ^ 5u) : q);
-    // decoding: eight lanes per row, four rows per step, two steps per slice.
-    // Lane c = lane % 8 of a row takes 16 of its 128 columns, octets o0 and o1
+    const uint32_t R = P.raw_stages;
+    // Eight lanes per row, four rows per step, two steps per slice. Lane
+    // c = lane % 8 of a row takes 16 of its 128 columns, octets o0 and o1
     // (2c, 2c+1 in the first panel; 2c+1, 2c in the second, so that the 8 lanes
     // of a row store to 8 distinct bank groups each time). Step 0 takes the
     // warp's rows 0,4,1,5 (slots 0..3), step 1 rows 2,6,3,7: the two rows of a
@@ -469,75 +534,13 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
         }
     }
 
-    // the slice being prepared: its unit, and this lane's row
-    UnitState U = {};
-    RowState RS = {};
-    UnitWalk wa;
-    wa.start();
-    uint32_t it_a = 0, sa = 0, slices_a = 0, row0_a = 0;
-    uint32_t rs_a = 0;  // raw stage of the slice being prepared: (its index) % R, kept incrementally
-    const uint32_t row_off = r * kExpPitch;                          // the row in an exponent stage
-    const uint32_t exp_lane = smem_addr(S.exp) + row_off + 16u * k;  // this lane's pieces in stage 0
-    // width, base and exponent bytes of the next slice (into stage rs_a), as one cp.async group
-    auto prepare = [&]() {
-        bool bad = false;
-        if (sa == 0) {  // first slice of a unit: the row's first block, loaded here
-            it_a = find_item(P, wa.u, it_a);
-            U = unit_state(P, it_a);
-            slices_a = U.cols / kSliceCols;
-            row0_a = uint32_t(wa.u - P.unit_begin[it_a]) * kTileRows;
-            const uint64_t row = row0_a + r;
-            RS.valid = row < U.rows;
-            set_width(RS, 0, 0);
-            RS.left = 0;
-            if (RS.valid) {
-                const uint64_t el = row * U.cols;
-                uint32_t h, off;
-                uint64_t nx;
-                load_block(U, el >> U.log2B, h, off, nx);
-                bad |= !enter_block(U, RS, row, el, h, off, nx);
-            }
-        } else if (RS.valid) {
-            RS.left -= kSliceCols;
-            if (RS.left == 0)  // the slice starts the row's next block
-                bad |= !enter_block(U, RS, row0_a + r, (RS.b + 1) << U.log2B, RS.nh, RS.noff, RS.nnx);
-            else
-                RS.src += 16u * RS.w;
-        }
-        const uint32_t w = RS.w;
-        const uint32_t rs = rs_a;
-        rs_a = rs_a + 1 == R ? 0u : rs_a + 1;
-        if (k == 0) S.meta[rs * kTileRows + r] = w | (RS.base << 8);
-        // the row's 16*w exponent bytes: pieces k and k + 4 (four lanes per row)
-        const uint32_t d = exp_lane + rs * kExpStage;
-        const uint8_t* src = RS.src + 16u * k;
-        if (k < w) cp_async16(d, src);
-        if (k + 4u < w) cp_async16(d + 64u, src + 64u);
-        if (bad) report(P.status, kStatusCorrupt);
-        if (++sa == slices_a) {
-            sa = 0;
-            wa.next();
-        }
-    };
-    auto commit = [] { asm volatile("cp.async.commit_group;" ::: "memory"); };
-
-    uint32_t ga = 0, rs_g = 0, round_g = 0;  // slice g: raw stage g % R, round g / R
-    for (; ga < D; ++ga) {  // prologue: slices 0 .. D-1 (one group each, empty past the end)
-        if (ga < total) prepare();
-        commit();
-    }
-    for (uint32_t g = 0; g < total; ++g, ++ga) {
-        if (ga < total) prepare();
-        commit();
-        if (D == 2)
-            asm volatile("cp.async.wait_group 2;" ::: "memory");  // slice g's group has landed
-        else
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-        __syncwarp();
+    uint32_t rs_g = 0, round_g = 0;  // slice g: raw stage g % R, round g / R
+    for (uint32_t g = 0; g < total; ++g) {
         const uint32_t rs = rs_g, xs = g & 1u;
         const uint32_t raw_parity = round_g & 1u;
         if (rs_g + 1 == R) rs_g = 0, ++round_g; else ++rs_g;
         if (!gemm_wait_warp(&c.raw_full[rs], raw_parity, c, P.status) ||
+            !gemm_wait_warp(&c.exp_full[rs], raw_parity, c, P.status) ||
             (g >= 2 && !gemm_wait_warp(&c.ax_empty[xs], ((g >> 1) - 1) & 1u, c, P.status)))
             break;
         const uint8_t* man = S.man + rs * kManStage;
@@ -585,7 +588,6 @@ __device__ void gemm_decode(const GemmParams<MAXI>& P, const GemmSmem& S, int dw
             mbar_arrive(&c.a_full[xs]);
         }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");  // nothing lands after the block ends
 }
 
 // ---------------------------------------------------------------------------
@@ -696,6 +698,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (uint32_t s = 0; s < kMaxRawStages; ++s) {
             mbar_init(&c.raw_full[s], 1);
             mbar_init(&c.raw_empty[s], kDecWarps);
+            mbar_init(&c.exp_full[s], 32 * kPrepWarps);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&c.a_full[s], kDecWarps);
@@ -728,6 +731,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         gemm_epilogue<MAXI>(P, S, warp, lane);
     } else if (warp == kXWarp) {
         if (lane == 0) gemm_load_x<MAXI>(P, S);
+    } else if (warp >= kPrepWarp0) {
+        gemm_prepare<MAXI>(P, S, warp - kPrepWarp0, lane);
     } else {
         gemm_decode<MAXI>(P, S, warp - kDecWarp0, lane);
     }
