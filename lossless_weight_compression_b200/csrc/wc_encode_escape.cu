@@ -110,13 +110,20 @@ __device__ __forceinline__ void exponent_range(uint4 v, uint32_t& lo, uint32_t& 
 
 template <int MAXI>
 __global__ void __launch_bounds__(kEscThreads) esc_params_kernel(const __grid_constant__ EscBatch<MAXI> P) {
-    // Each lane counts its own elements in byte counters laid out [exponent][lane]
-    // (no atomics; lanes that share a 32-bit word sit in one bank, so at most a
-    // 4-way conflict); a block gives a lane at most B / 32 <= 128 elements. Only
-    // the rows of exponents lo..hi of the block are cleared, counted and summed.
+    // Each lane counts its own elements in byte counters laid out [exponent][lane];
+    // a block gives a lane at most B / 32 <= 128 elements, so a byte never carries
+    // into its neighbour. An increment is a shared-memory reduction on the
+    // 32-bit word holding the lane's byte (no value returned): unlike a byte
+    // read-modify-write, increments of one lane that may hit the same counter do
+    // not wait for one another. Only the rows of exponents lo..hi of the block
+    // are cleared, counted and summed.
     extern __shared__ __align__(16) uint8_t params_smem[];  // kParamsSmem bytes
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint8_t* cnt = params_smem + warp * (256 * 32);
+    // the word of row e holding this lane's counter, and the lane's byte in it
+    uint32_t* cnt_lane = reinterpret_cast<uint32_t*>(cnt + (lane & ~3));
+    const uint32_t one = 1u << (8 * (lane & 3));
+    auto count = [&](uint32_t e) { atomicAdd(cnt_lane + 8 * e, one); };
     uint32_t* h = reinterpret_cast<uint32_t*>(params_smem + kEscWarps * (256 * 32)) + warp * kHistWords;
     for (uint64_t gb = uint64_t(blockIdx.x) * kEscWarps + warp; gb < P.total_blocks;
          gb += uint64_t(gridDim.x) * kEscWarps) {
@@ -184,8 +191,7 @@ __global__ void __launch_bounds__(kEscThreads) esc_params_kernel(const __grid_co
                 split_quad(keep[k].x, keep[k].y, s0, e0);
                 split_quad(keep[k].z, keep[k].w, s1, e1);
 #pragma unroll
-                for (int t = 0; t < 8; ++t)
-                    cnt[(((t < 4 ? e0 : e1) >> (8 * (t & 3))) & 0xFFu) * 32 + lane] += 1;
+                for (int t = 0; t < 8; ++t) count(((t < 4 ? e0 : e1) >> (8 * (t & 3))) & 0xFFu);
             }
         }
         for (uint32_t g = uint32_t(lane) + 32u * kKeep; g < groups; g += 32) {
@@ -194,11 +200,9 @@ __global__ void __launch_bounds__(kEscThreads) esc_params_kernel(const __grid_co
             split_quad(v.x, v.y, s0, e0);
             split_quad(v.z, v.w, s1, e1);
 #pragma unroll
-            for (int t = 0; t < 8; ++t)
-                cnt[(((t < 4 ? e0 : e1) >> (8 * (t & 3))) & 0xFFu) * 32 + lane] += 1;
+            for (int t = 0; t < 8; ++t) count(((t < 4 ? e0 : e1) >> (8 * (t & 3))) & 0xFFu);
         }
-        for (uint32_t i = 8 * groups + lane; i < len; i += 32)
-            cnt[((uint32_t(x[i]) >> 7) & 0xFFu) * 32 + lane] += 1;
+        for (uint32_t i = 8 * groups + lane; i < len; i += 32) count((uint32_t(x[i]) >> 7) & 0xFFu);
         __syncwarp();
 
         // h[j] <- elements with an exponent below lo + j, for j = 0..span (lane l
