@@ -139,23 +139,24 @@ __global__ void __launch_bounds__(kEscThreads) esc_params_kernel(const __grid_co
 
         // pass 1: sign+mantissa bytes out, exponent range. A lane's share of a
         // block of up to 1024 elements (four 16-byte groups) is loaded at once and
-        // kept for pass 2; longer blocks are read again.
+        // its exponent bytes kept for pass 2; longer blocks are read again.
         constexpr uint32_t kKeep = 4;
-        uint4 keep[kKeep];
+        uint4 in[kKeep];
 #pragma unroll
         for (uint32_t k = 0; k < kKeep; ++k) {
             const uint32_t g = uint32_t(lane) + 32u * k;
-            keep[k] = g < groups ? ld_stream_v4(x + 8 * g) : make_uint4(0u, 0u, 0u, 0u);
+            in[k] = g < groups ? ld_stream_v4(x + 8 * g) : make_uint4(0u, 0u, 0u, 0u);
         }
         uint32_t lo = 255u, hi = 0u;
+        uint2 keep[kKeep];  // exponent bytes of the kept groups
 #pragma unroll
         for (uint32_t k = 0; k < kKeep; ++k) {
             const uint32_t g = uint32_t(lane) + 32u * k;
             if (g < groups) {
-                const uint4 v = keep[k];
-                uint32_t s0, s1, e0, e1;
-                split_quad(v.x, v.y, s0, e0);
-                split_quad(v.z, v.w, s1, e1);
+                const uint4 v = in[k];
+                uint32_t s0, s1;
+                split_quad(v.x, v.y, s0, keep[k].x);
+                split_quad(v.z, v.w, s1, keep[k].y);
                 *reinterpret_cast<uint2*>(man + 8 * g) = make_uint2(s0, s1);
                 exponent_range(v, lo, hi);
             }
@@ -187,11 +188,9 @@ __global__ void __launch_bounds__(kEscThreads) esc_params_kernel(const __grid_co
 #pragma unroll
         for (uint32_t k = 0; k < kKeep; ++k) {
             if (uint32_t(lane) + 32u * k < groups) {
-                uint32_t s0, s1, e0, e1;
-                split_quad(keep[k].x, keep[k].y, s0, e0);
-                split_quad(keep[k].z, keep[k].w, s1, e1);
 #pragma unroll
-                for (int t = 0; t < 8; ++t) count(((t < 4 ? e0 : e1) >> (8 * (t & 3))) & 0xFFu);
+                for (int t = 0; t < 8; ++t)
+                    count(((t < 4 ? keep[k].x : keep[k].y) >> (8 * (t & 3))) & 0xFFu);
             }
         }
         for (uint32_t g = uint32_t(lane) + 32u * kKeep; g < groups; g += 32) {
