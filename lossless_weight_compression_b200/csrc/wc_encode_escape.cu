@@ -83,6 +83,20 @@ __device__ __forceinline__ uint32_t owner(const uint64_t* begin, uint32_t count,
     return uint32_t(lo);
 }
 
+// The same, for a walk over increasing units: a scan forward from the tensor
+// of the previous unit (usually one cached comparison) instead of a binary
+// search of dependent loads from the launch parameters.
+template <int MAXI>
+__device__ __forceinline__ uint32_t owner_from(const uint64_t* begin, uint32_t count, uint64_t u,
+                                               uint32_t from) {
+    if constexpr (MAXI == 1) {
+        return 0;
+    } else {
+        while (from + 1 < count && begin[from + 1] <= u) ++from;
+        return from;
+    }
+}
+
 __device__ __forceinline__ uint32_t block_len(const Layout& L, uint64_t b) {
     const uint64_t first = b << L.log2_block;
     return uint32_t(min(uint64_t(L.block), L.n - first));
@@ -125,9 +139,10 @@ __global__ void __launch_bounds__(kEscThreads) esc_params_kernel(const __grid_co
     const uint32_t one = 1u << (8 * (lane & 3));
     auto count = [&](uint32_t e) { atomicAdd(cnt_lane + 8 * e, one); };
     uint32_t* h = reinterpret_cast<uint32_t*>(params_smem + kEscWarps * (256 * 32)) + warp * kHistWords;
+    uint32_t it = 0;
     for (uint64_t gb = uint64_t(blockIdx.x) * kEscWarps + warp; gb < P.total_blocks;
          gb += uint64_t(gridDim.x) * kEscWarps) {
-        const uint32_t it = owner<MAXI>(P.block_begin, P.count, gb);
+        it = owner_from<MAXI>(P.block_begin, P.count, gb, it);
         const EscItem& I = P.item[it];
         const Layout L = make_layout_escape(I.n, I.block);
         const uint64_t b = gb - P.block_begin[it];
@@ -517,9 +532,10 @@ __global__ void __launch_bounds__(kEscThreads) esc_pack_kernel(const __grid_cons
     __shared__ __align__(16) uint8_t stage_all[kEscWarps][kPackStageBytes];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint8_t* stage = stage_all[warp];
+    uint32_t it = 0;
     for (uint64_t gb = uint64_t(blockIdx.x) * kEscWarps + warp; gb < P.total_blocks;
          gb += uint64_t(gridDim.x) * kEscWarps) {
-        const uint32_t it = owner<MAXI>(P.block_begin, P.count, gb);
+        it = owner_from<MAXI>(P.block_begin, P.count, gb, it);
         const EscItem& I = P.item[it];
         const Layout L = make_layout_escape(I.n, I.block);
         const uint64_t b = gb - P.block_begin[it];
