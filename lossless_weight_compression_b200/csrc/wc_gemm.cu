@@ -421,8 +421,8 @@ __device__ __forceinline__ void load_block(const UnitState& U, uint64_t b, uint3
 }
 
 // The row enters the block holding element el (its header in h/off/nx; el is
-// a slice's first column): set the width, the decode constants, the slice's
-// exponent bytes and the block's remaining elements, checking the header, that
+// a slice's first column): set the width and base, the slice's exponent
+// bytes and the block's remaining elements, checking the header, that
 // the block's payload lies inside the stream (so no slice of it reads past the
 // end) and, at the block's first element, the offset chain; then start loading
 // the row's next block. False if corrupt (the row then decodes as w = 0).
