@@ -250,31 +250,37 @@ __global__ void __launch_bounds__(kEscThreads) esc_params_kernel(const __grid_co
         if (lane == 0) h[0] = 0;
         __syncwarp();
 
-        // the least-cost candidate: ties to the smaller w (strict comparisons in
-        // increasing w), then the larger base (the maximum of count << 8 | base).
-        // For a width the best base lies in [min(lo, hmax), min(hi, hmax)],
-        // hmax = 255 - (2^w - 1): a window starting below lo holds no more than
-        // one starting there (ties go to the larger base), one above hi holds
-        // nothing.
+        // The least-cost candidate: ties to the smaller w, then the larger base,
+        // i.e. the minimum of cost << 11 | w << 8 | (255 - base) (cost <= 8 * 512 +
+        // 4096 < 2^13). For a width the best base lies in [min(lo, hmax),
+        // min(hi, hmax)], hmax = 255 - (2^w - 1): a window starting below lo holds
+        // no more than one starting there (ties go to the larger base), one above
+        // hi holds nothing. All widths are searched at once: lanes 4(w-1) ..
+        // 4(w-1)+3 take width w = 1..7, every fourth base each, and one warp
+        // minimum picks the winner.
         const uint32_t octets = (len + 7) >> 3;
         uint32_t best_cost = 0xFFFFFFFFu, best_w = 8, best_base = 0, best_k = 0;
-        if (lo == hi) best_cost = 0, best_w = 0, best_base = lo, best_k = 0;
-#pragma unroll
-        for (uint32_t w = 1; w <= 7; ++w) {
-            const uint32_t m = (1u << w) - 1u, hmax = 255u - m;
-            const uint32_t b0 = min(lo, hmax), b1 = min(hi, hmax);
-            uint32_t key = 0;
-            for (uint32_t base = b0 + uint32_t(lane); base <= b1; base += 32) {
-                // elements below e: 0 up to lo, h[e - lo] inside, len above hi
-                const uint32_t top = base + m;
-                const uint32_t below_top = top > hi ? len : h[top - lo];
-                const uint32_t below_base = base <= lo ? 0u : h[base - lo];
-                key = max(key, ((below_top - below_base) << 8) | base);
+        if (lo == hi) {
+            best_cost = 0, best_w = 0, best_base = lo, best_k = 0;
+        } else {
+            uint32_t key = 0xFFFFFFFFu;
+            if (lane < 28) {
+                const uint32_t w = uint32_t(lane >> 2) + 1u, m = (1u << w) - 1u, hmax = 255u - m;
+                const uint32_t b1 = min(hi, hmax);
+                for (uint32_t base = min(lo, hmax) + uint32_t(lane & 3); base <= b1; base += 4) {
+                    // elements below e: 0 up to lo, h[e - lo] inside, len above hi
+                    const uint32_t top = base + m;
+                    const uint32_t below_top = top > hi ? len : h[top - lo];
+                    const uint32_t below_base = base <= lo ? 0u : h[base - lo];
+                    const uint32_t cost = octets * w + len - (below_top - below_base);
+                    key = min(key, (cost << 11) | (w << 8) | (255u - base));
+                }
             }
-            key = __reduce_max_sync(0xFFFFFFFFu, key);
-            const uint32_t k = len - (key >> 8);
-            const uint32_t cost = octets * w + k;
-            if (cost < best_cost) best_cost = cost, best_w = w, best_base = key & 0xFFu, best_k = k;
+            key = __reduce_min_sync(0xFFFFFFFFu, key);
+            best_cost = key >> 11;
+            best_w = (key >> 8) & 7u;
+            best_base = 255u - (key & 0xFFu);
+            best_k = best_cost - octets * best_w;
         }
         if (8 * octets < best_cost) best_cost = 8 * octets, best_w = 8, best_base = 0, best_k = 0;
         if (lane == 0) {
