@@ -185,3 +185,21 @@ def test_gemm_reports_corrupt_stream(orc, wclib, cuda):
     y, status = run_gpu(wclib, stream, rows, cols, B, x, cuda)
     assert status == 0
     check_bound(y, y_ref, absum, cols)
+
+
+def test_gemm_refuses_escape_coded_stream(orc, wclib, cuda):
+    """The fused product decodes plain streams only: an escape-coded stream of the
+    same matrix is reported as corrupt (its container header carries the escape
+    flag), every read staying inside the stream, and the device stays usable."""
+    rng = np.random.default_rng(55)
+    rows, cols, B = 256, 1024, 512
+    W = rand_bf16(rng, (rows, cols), 0.02)
+    x = rand_bf16(rng, (16, cols), 1.0)
+    esc = orc.compress_escape(W.reshape(-1), B)
+    _, status = run_gpu(wclib, esc, rows, cols, B, x, cuda)
+    assert status == 3
+    stream = orc.compress(W, B)
+    y_ref, absum = orc.gemv(stream, rows, cols, B, x)
+    y, status = run_gpu(wclib, stream, rows, cols, B, x, cuda)
+    assert status == 0
+    check_bound(y, y_ref, absum, cols)

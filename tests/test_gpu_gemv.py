@@ -118,3 +118,19 @@ def test_gemv_reports_corrupt_stream(orc, wclib, cuda):
     bad[128 + 2 * 5 + 1] = 9  # block 5: w = 9
     _, status = run_gpu(wclib, bad, rows, cols, B, rand_bf16(rng, (1, cols), 1.0), cuda)
     assert status == 3
+
+
+def test_gemv_refuses_escape_coded_stream(orc, wclib, cuda):
+    """Plain streams only: an escape-coded stream of the same matrix is reported as
+    corrupt, and the device stays usable."""
+    rng = np.random.default_rng(44)
+    rows, cols, B = 64, 2048, 1024
+    W = rand_bf16(rng, (rows, cols), 0.02)
+    x = rand_bf16(rng, (1, cols), 1.0)
+    _, status = run_gpu(wclib, orc.compress_escape(W.reshape(-1), B), rows, cols, B, x, cuda)
+    assert status == 3
+    stream = orc.compress(W, B)
+    y_ref, absum = orc.gemv(stream, rows, cols, B, x)
+    y, status = run_gpu(wclib, stream, rows, cols, B, x, cuda)
+    assert status == 0
+    check_bound(y, y_ref, absum, cols)
