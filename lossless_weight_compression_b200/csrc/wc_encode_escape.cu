@@ -459,20 +459,20 @@ __device__ __forceinline__ void load_chunk_words(const uint16_t* x, uint32_t el,
 // block's exception list (a warp prefix count on top of `carry`), the
 // exceptions and the packed codes into `stage`.
 template <uint32_t W>
-__device__ __forceinline__ void pack_step(const uint16_t* x, const uint32_t xw[8], uint32_t el,
+__device__ __forceinline__ void pack_step(const uint32_t xw[8], uint32_t el,
                                           uint32_t nv, uint32_t base4, uint32_t code_bytes,
                                           uint32_t& carry, uint8_t* stage, int lane) {
-    uint32_t V[4], esc[4];
+    uint32_t V[4], esc[4], E[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        uint32_t s4, e4;
-        split_quad(xw[2 * j], xw[2 * j + 1], s4, e4);
+        uint32_t s4;
+        split_quad(xw[2 * j], xw[2 * j + 1], s4, E[j]);
         if constexpr (W == 0) {
             V[j] = 0u, esc[j] = 0u;
         } else if constexpr (W == 8) {
-            V[j] = e4, esc[j] = 0u;
+            V[j] = E[j], esc[j] = 0u;
         } else {
-            esc[j] = codes4<W>(e4, base4, V[j]);
+            esc[j] = codes4<W>(E[j], base4, V[j]);
         }
     }
     if (nv < kChunk) {  // lanes past the end take code 0 and no escape
@@ -499,9 +499,11 @@ __device__ __forceinline__ void pack_step(const uint16_t* x, const uint32_t xw[8
         uint32_t m16 = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) m16 |= ((esc[j] * 0x00204081u) >> 28) << (4 * j);
+        // the chunk's 16 exponent bytes, already in registers
+        const uint64_t e_lo = E[0] | (uint64_t(E[1]) << 32), e_hi = E[2] | (uint64_t(E[3]) << 32);
         for (; m16; m16 &= m16 - 1u) {  // exceptions in element order
             const uint32_t i = uint32_t(__ffs(int(m16))) - 1u;
-            stage[pos++] = uint8_t(x[el + i] >> 7);
+            stage[pos++] = uint8_t((i < 8 ? e_lo : e_hi) >> (8 * (i & 7u)));
         }
     }
     if (nv == kChunk)
@@ -524,9 +526,9 @@ __device__ __forceinline__ uint32_t pack_block(const uint16_t* x, uint32_t len, 
         uint32_t xa[8], xb[8], na, nb;
         load_chunk_words(x, el0, len, xa, na);
         load_chunk_words(x, el1, len, xb, nb);
-        pack_step<W>(x, xa, el0, na, base4, code_bytes, carry, stage, lane);
+        pack_step<W>(xa, el0, na, base4, code_bytes, carry, stage, lane);
         if (step + 32 * kChunk < len)  // the same for the whole warp
-            pack_step<W>(x, xb, el1, nb, base4, code_bytes, carry, stage, lane);
+            pack_step<W>(xb, el1, nb, base4, code_bytes, carry, stage, lane);
     }
     const uint32_t used = code_bytes + carry, padded = (used + 15u) & ~15u;
     if (uint32_t(lane) < padded - used) stage[used + lane] = 0;
