@@ -362,10 +362,12 @@ int wc_gemv_batch(const wc_gemv_item *h_items, uint32_t count, uint32_t n_vec,
  * is fixed, so y is the same on every run. The tensor cores' FP32 accumulation
  * is not specified to round to nearest; every output is within
  * cols * 2^-22 * sum_c |W[r][c] * x[t][c]| of the exact sum. The stream is
- * checked as by wc_decompress (errors to *d_status); a stream shorter than its
- * planes (stream_bytes below the exponent-plane offset) returns
- * WC_ERR_CORRUPT_STREAM without launching. Suited to 16..128 tokens; for 1, 2
- * or 4 vectors wc_gemv is faster.
+ * checked as by wc_decompress (errors to *d_status; an escape-coded or FP32
+ * stream is reported as corrupt); a stream shorter than its planes
+ * (stream_bytes below the exponent-plane offset) returns WC_ERR_CORRUPT_STREAM
+ * without launching. Faster than wc_gemv at every token count, one included
+ * (the token count is padded to a multiple of 16 inside); wc_gemv keeps the
+ * tighter round-to-nearest bound of a plain FP32 sum.
  */
 #define WC_GEMM_MAX_TOKENS 128u
 int wc_gemm(const void *d_stream, uint64_t stream_bytes, uint32_t rows, uint32_t cols,
