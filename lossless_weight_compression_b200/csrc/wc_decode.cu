@@ -84,12 +84,23 @@ struct __align__(16) Stage {
     StageInfo info;
 };
 
+// Escape-coded tiles with blocks longer than a consumer warp's segment: each
+// warp's escape total for the stage's tile, and a barrier per stage on which
+// all eight consumer warps arrive for every such tile (each warp keeps the
+// barriers' phases: the warps see the same tiles in the same order).
+struct EscSegments {
+    uint32_t count[stages_of<kKindEscape>()][kConsumerWarps];
+    unsigned long long done[stages_of<kKindEscape>()];
+};
+struct NoEscSegments {};
+
 template <int KIND>
 struct DecodeSmem {
     static constexpr int kStages = stages_of<KIND>();
     Stage<KIND> stage[kStages];
     unsigned long long full[kStages];
     unsigned long long empty[kStages];
+    typename std::conditional<KIND == kKindEscape, EscSegments, NoEscSegments>::type seg;
     int abort;
 };
 
@@ -288,24 +299,6 @@ __device__ void consume(const DecodeParams<MAXI>& P, DecodeSmem<KIND>& sm, int t
 // ---------------------------------------------------------------------------
 // consumers of escape-coded streams: eight warps, one 1024-element segment each
 // ---------------------------------------------------------------------------
-// Escapes among the codes of tile elements [from, to) (all in one block, to - from
-// a multiple of 512), counted by the whole warp. Only blocks longer than a
-// consumer warp's segment (B > 1024) need it.
-__device__ __noinline__ uint32_t count_escapes(const Stage<kKindEscape>& st, uint32_t from,
-                                               uint32_t to, uint32_t log2B, int lane) {
-    const uint32_t bmask = (1u << log2B) - 1u;
-    const uint4 t0 = st.t0[from >> log2B];
-    const uint2 t1 = st.t1[from >> log2B];
-    uint32_t cnt = 0;
-    for (uint32_t el = from + 16u * uint32_t(lane); el < to; el += 512u) {
-        uint32_t E[4], esc[4];
-        const uint32_t q = t0.x + ((el & bmask) >> 3) * t0.y;
-        chunk_exponents_rt(st.exp, q, t0.y, t1.x, t1.y, E, esc);
-        cnt += escape_count(esc);
-    }
-    return __reduce_add_sync(0xFFFFFFFFu, cnt);
-}
-
 // One chunk of an escape-coded tile in a consumer lane's registers.
 struct EscChunk {
     uint32_t el;      // first element (tile-relative)
@@ -437,6 +430,7 @@ __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEsca
                                int lane, int warp) {
     constexpr int kStages = DecodeSmem<kKindEscape>::kStages;
     (void)tid;
+    uint32_t seg_phase = 0;  // bit s: parity of stage s's next segment-total phase
     for (uint64_t i = 0;; ++i) {
         const uint64_t t = blockIdx.x + i * gridDim.x;
         if (t >= P.total_tiles) break;
@@ -454,21 +448,19 @@ __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEsca
         const uint32_t log2B = info.log2B, B = 1u << log2B;
         const uint32_t seg = uint32_t(warp) * kSegment;
         bool bad = false;
-        if (seg < info.tile_n) {  // the same for the whole warp
-            // escapes of the segment's block before the segment
-            uint32_t carry = 0;
-            if (B > uint32_t(kSegment) && (seg & (B - 1u)) != 0u)
-                carry = count_escapes(st, seg & ~(B - 1u), seg, log2B, lane);
-            // both 512-element steps of the segment at once: chunk k of this lane
-            // starts at seg + 512k + 16 lane
-            EscChunk c0, c1;
+        const bool active = seg < info.tile_n;  // the same for the whole warp
+        // both 512-element steps of the segment at once: chunk k of this lane
+        // starts at seg + 512k + 16 lane
+        EscChunk c0, c1;
+        uint32_t incl = 0, v = 0;
+        if (active) {
             load_esc_meta(st, seg + 16u * uint32_t(lane), info.tile_n, log2B, c0);
             load_esc_meta(st, seg + 512u + 16u * uint32_t(lane), info.tile_n, log2B, c1);
             decode_esc_pair(st, info.tile_n, c0, c1);
             // one prefix count for both steps (step k's counts in bits [16k, 16k + 16)),
             // segmented by block: B/16 lanes hold one block of a step when B < 512
-            const uint32_t v = c0.count | (c1.count << 16);
-            uint32_t incl = v;
+            v = c0.count | (c1.count << 16);
+            incl = v;
             if (B >= 512u) {
 #pragma unroll
                 for (int d = 1; d < 32; d <<= 1) {
@@ -482,11 +474,34 @@ __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEsca
                     if ((uint32_t(lane) & (group - 1u)) >= d) incl += y;
                 }
             }
+        }
+        // Blocks longer than a segment: the escapes of the block's earlier
+        // segments, from the other warps' totals.
+        const uint32_t last = B >= uint32_t(kSegment) ? __shfl_sync(0xFFFFFFFFu, incl, 31) : 0u;
+        uint32_t carry = 0;
+        if (B > uint32_t(kSegment)) {
+            if (lane == 0) {
+                sm.seg.count[s][warp] = (last & 0xFFFFu) + (last >> 16);
+                mbar_arrive(&sm.seg.done[s]);
+            }
+            const uint32_t parity = (seg_phase >> s) & 1u;
+            seg_phase ^= 1u << s;
+            if (!mbar_wait(&sm.seg.done[s], parity, &sm.abort)) {
+                if (lane == 0) {
+                    report(P.status, kStatusTimeout);
+                    sm.abort = 1;
+                }
+                return;
+            }
+            for (uint32_t w = (seg & ~(B - 1u)) / uint32_t(kSegment); w < uint32_t(warp); ++w)
+                carry += sm.seg.count[s][w];
+        }
+        if (active) {
             const uint32_t excl = incl - v;
             uint32_t before0 = excl & 0xFFFFu, before1 = excl >> 16;
             if (B >= uint32_t(kSegment)) {  // step 1 continues step 0's block
                 before0 += carry;
-                before1 += carry + (__shfl_sync(0xFFFFFFFFu, incl, 31) & 0xFFFFu);
+                before1 += carry + (last & 0xFFFFu);
             }
             if (c0.active) bad |= finish_esc_chunk(st, c0, before0, info.tile_n, log2B, info.out);
             if (c1.active) bad |= finish_esc_chunk(st, c1, before1, info.tile_n, log2B, info.out);
@@ -509,6 +524,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
             mbar_init(&sm.full[s], 1);                // the producer's arrive (+ copied bytes)
             mbar_init(&sm.empty[s], kConsumerWarps);  // one arrive per consumer warp
         }
+        if constexpr (KIND == kKindEscape)
+            for (int s = 0; s < kStages; ++s) mbar_init(&sm.seg.done[s], kConsumerWarps);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
