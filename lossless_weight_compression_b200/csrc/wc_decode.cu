@@ -35,8 +35,9 @@
 // warps each own a 1024-element segment of the tile, so that an escaped
 // element's place in its block's exception list is a warp prefix count of the
 // escapes before it (segmented by block for B < 1024, carried across the
-// segment's two steps for B >= 1024, and counted over the earlier segments of
-// the block for B > 1024).
+// segment's two steps for B >= 1024, and, for B > 1024, offset by the escape
+// totals of the block's earlier segments, which their warps post to shared
+// memory).
 #include <mutex>
 #include <type_traits>
 
