@@ -16,14 +16,16 @@
 //
 // Five launches per batch of up to kEscBatchMax tensors, none of which waits
 // on another thread block; the tensors' blocks (and scan chunks) are numbered
-// across the batch and each unit finds its tensor by binary search over the
-// launch parameters:
+// across the batch, a scan chunk finds its tensor by binary search over the
+// launch parameters and a warp walking blocks by scanning forward from its
+// previous block's tensor:
 //   params     one warp per block: split (the sign+mantissa bytes go straight
-//              to the mantissa plane), a 256-bin exponent histogram from
-//              lane-private byte counters in shared memory (no atomics) summed
-//              with dp4a, its prefix counts, and for each w the window of most
-//              elements (one warp maximum over all bases); writes the block
-//              header and the padded size in 16-byte units
+//              to the mantissa plane), a 256-bin exponent histogram in
+//              lane-private byte counters in shared memory (incremented by
+//              shared-memory reductions on the lane's word, summed with dp4a),
+//              its prefix counts, and the least-cost (w, base) with all widths
+//              searched at once (four lanes per width, one warp minimum);
+//              writes the block header and the padded size in 16-byte units
 //   reduce     one thread block per 4096 blocks of a tensor: their sizes' sum
 //   top        one warp per tensor: the exclusive prefix of its chunk sums, the
 //              exponent-plane size E, the container header and section padding,
