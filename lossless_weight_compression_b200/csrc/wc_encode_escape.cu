@@ -110,16 +110,26 @@ __device__ __forceinline__ uint32_t block_len(const Layout& L, uint64_t b) {
 // Smallest and largest exponent of the 16-bit words in v (the exponent is the
 // top byte of a word's 15-bit magnitude, so 16-bit lane minima and maxima of
 // the sign-cleared words give them).
-__device__ __forceinline__ void exponent_range(uint4 v, uint32_t& lo, uint32_t& hi) {
+// Running per-lane minimum and maximum of the sign-cleared words, two 16-bit
+// lanes at a time (mn starts at 0xFFFFFFFF, mx at 0); exponent_bounds turns
+// them into exponent bytes once per block.
+__device__ __forceinline__ void magnitude_range(uint4 v, uint32_t& mn, uint32_t& mx) {
     const uint32_t a = v.x & 0x7FFF7FFFu, b = v.y & 0x7FFF7FFFu, c = v.z & 0x7FFF7FFFu,
                    d = v.w & 0x7FFF7FFFu;
-    uint32_t mn, mx;
-    asm("min.u16x2 %0, %1, %2;" : "=r"(mn) : "r"(a), "r"(b));
+    asm("min.u16x2 %0, %0, %1;" : "+r"(mn) : "r"(a));
+    asm("min.u16x2 %0, %0, %1;" : "+r"(mn) : "r"(b));
     asm("min.u16x2 %0, %0, %1;" : "+r"(mn) : "r"(c));
     asm("min.u16x2 %0, %0, %1;" : "+r"(mn) : "r"(d));
-    asm("max.u16x2 %0, %1, %2;" : "=r"(mx) : "r"(a), "r"(b));
+    asm("max.u16x2 %0, %0, %1;" : "+r"(mx) : "r"(a));
+    asm("max.u16x2 %0, %0, %1;" : "+r"(mx) : "r"(b));
     asm("max.u16x2 %0, %0, %1;" : "+r"(mx) : "r"(c));
     asm("max.u16x2 %0, %0, %1;" : "+r"(mx) : "r"(d));
+}
+
+// Folds a magnitude range into an exponent range [lo, hi] (a lane that saw no
+// word keeps lo = 511, above every exponent, and hi = 0).
+__device__ __forceinline__ void exponent_bounds(uint32_t mn, uint32_t mx, uint32_t& lo,
+                                                uint32_t& hi) {
     lo = min(lo, min(mn & 0xFFFFu, mn >> 16) >> 7);
     hi = max(hi, max(mx & 0xFFFFu, mx >> 16) >> 7);
 }
@@ -164,7 +174,7 @@ __global__ void __launch_bounds__(kEscThreads) esc_params_kernel(const __grid_co
             const uint32_t g = uint32_t(lane) + 32u * k;
             in[k] = g < groups ? ld_stream_v4(x + 8 * g) : make_uint4(0u, 0u, 0u, 0u);
         }
-        uint32_t lo = 255u, hi = 0u;
+        uint32_t mn = 0xFFFFFFFFu, mx = 0u;  // magnitude range, two lanes at a time
         uint2 keep[kKeep];  // exponent bytes of the kept groups
 #pragma unroll
         for (uint32_t k = 0; k < kKeep; ++k) {
@@ -175,7 +185,7 @@ __global__ void __launch_bounds__(kEscThreads) esc_params_kernel(const __grid_co
                 split_quad(v.x, v.y, s0, keep[k].x);
                 split_quad(v.z, v.w, s1, keep[k].y);
                 *reinterpret_cast<uint2*>(man + 8 * g) = make_uint2(s0, s1);
-                exponent_range(v, lo, hi);
+                magnitude_range(v, mn, mx);
             }
         }
         for (uint32_t g = uint32_t(lane) + 32u * kKeep; g < groups; g += 32) {
@@ -184,8 +194,10 @@ __global__ void __launch_bounds__(kEscThreads) esc_params_kernel(const __grid_co
             split_quad(v.x, v.y, s0, e0);
             split_quad(v.z, v.w, s1, e1);
             *reinterpret_cast<uint2*>(man + 8 * g) = make_uint2(s0, s1);
-            exponent_range(v, lo, hi);
+            magnitude_range(v, mn, mx);
         }
+        uint32_t lo = 511u, hi = 0u;
+        exponent_bounds(mn, mx, lo, hi);
         for (uint32_t i = 8 * groups + lane; i < len; i += 32) {  // the ragged end of a tensor
             const uint32_t w16 = x[i];
             const uint32_t e = (w16 >> 7) & 0xFFu;
