@@ -199,9 +199,33 @@ def ncu_traffic_per_elem():
 # ---------------------------------------------------------------------------
 # the CPU oracle, timed (cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
+def host_info():
+    """The host the oracle runs on: its usable core count and CPU model."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": cores, "cpu_model": model}
+
+
+ORACLE_SAMPLE = ("layer 0 of the stack (7 tensors, 218,103,808 elements) copied to the host; "
+                 "the single-threaded C oracle encodes each tensor once (timed apart), then "
+                 "decodes all seven per step (the metric)")
+
+
 def oracle_sample_words(device_tensors=None):
-    """The bounded sample the oracle is timed on: layer 0 of the stack
-    (7 tensors, 218,103,808 elements), as host uint16 arrays."""
+    """The bounded sample the oracle is timed on, in both the cpu_baseline and the
+    reference arm: layer 0 of the stack (7 tensors, 218,103,808 elements), as
+    host uint16 arrays."""
     import numpy as np
     import torch
 
@@ -217,57 +241,57 @@ def oracle_sample_words(device_tensors=None):
     return out
 
 
-def time_oracle(sample, block=BLOCK):
-    """Encode then decode each tensor with the oracle; returns
-    (decode GB/s BF16-out, encode GB/s BF16-in, elements)."""
-    import numpy as np
+class OracleTimer:
+    """The oracle on a host sample: encode() once, then decode_step() per step."""
 
-    import oracle
-    oracle.build()
-    n_total = sum(w.size for _, w in sample)
-    t_enc = t_dec = 0.0
-    for _, w in sample:
+    def __init__(self, sample, block=BLOCK):
+        import oracle
+        oracle.build()
+        self.oracle, self.sample, self.block = oracle, sample, block
+        self.n = sum(w.size for _, w in sample)
+        self.streams = None
+
+    def encode(self):
+        """Encode every tensor once; returns BF16-in GB/s."""
         t0 = time.perf_counter()
-        s = oracle.compress(w, block)
-        t1 = time.perf_counter()
-        d = oracle.decompress(s, w.size, block)
-        t2 = time.perf_counter()
-        if not np.array_equal(d, w):
-            raise RuntimeError("oracle round trip failed")
-        t_enc += t1 - t0
-        t_dec += t2 - t1
-    return 2 * n_total / t_dec / 1e9, 2 * n_total / t_enc / 1e9, n_total
+        self.streams = [self.oracle.compress(w, self.block) for _, w in self.sample]
+        return 2 * self.n / (time.perf_counter() - t0) / 1e9
+
+    def decode_step(self):
+        """Decode every tensor once and check it; returns the seconds spent decoding."""
+        import numpy as np
+        sec = 0.0
+        for (_, w), s in zip(self.sample, self.streams):
+            t0 = time.perf_counter()
+            d = self.oracle.decompress(s, w.size, self.block)
+            sec += time.perf_counter() - t0
+            if not np.array_equal(d, w):
+                raise RuntimeError("oracle round trip failed")
+        return sec
 
 
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
-    import numpy as np  # noqa: F401
     import torch
-
-    from lossless_weight_compression_b200 import synth
     torch.set_num_threads(1)
-    # each step: the oracle encodes and decodes layer 0's q_proj (16,777,216 elements)
-    sample = [(n, w) for n, w in oracle_sample_words() if n.endswith("q_proj")]
+    timer = OracleTimer(oracle_sample_words())
+    enc_gbs = timer.encode()
     for _ in range(args.warmup):
-        time_oracle(sample)
-    dec_times, n_step = [], sample[0][1].size
-    for _ in range(args.steps):
-        dec_gbs, _, _ = time_oracle(sample)
-        dec_times.append(2 * n_step / dec_gbs / 1e9)
-    total = sum(dec_times)
-    value = 2 * n_step * args.steps / total / 1e9
+        timer.decode_step()
+    total = sum(timer.decode_step() for _ in range(args.steps))
+    value = 2 * timer.n * args.steps / total / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "block": BLOCK,
-                   "sample": "per step: layers.0.q_proj (16,777,216 elements) of the stack"},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": "layers.0.q_proj of the stack, encoded then decoded by the "
-                                   "single-threaded C oracle each step; decode timed"},
+                   "sample": "per step: " + ORACLE_SAMPLE},
+        "cpu_baseline": dict({"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                              "sample": ORACLE_SAMPLE, "encode_gbs_bf16_in": enc_gbs},
+                             **host_info()),
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -277,6 +301,171 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
+def timed_steps(fn, steps, warmup, stream, dist, dev):
+    """Seconds per call of fn: `warmup` untimed calls, then `steps` calls between
+    two CUDA events on `stream`, barriers on both sides, max over ranks."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    barrier(dist, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    barrier(dist, dev)
+    return max_over_ranks(e0.elapsed_time(e1) / 1e3 / steps, dist, dev)
+
+
+def escape_phase(args, wc, wcodec, inputs, outs, stream, dist, dev, world):
+    """The same tensors as escape-coded streams: one wc_compress_escape_batch call
+    (five launches) and one wc_decompress_escape_batch launch, each timed over
+    the step count; every decoded tensor checked against its input."""
+    import torch
+    sh = stream.cuda_stream
+    n_total = sum(w.numel() for w in inputs)
+    enc = wcodec.CompressBatch(inputs, block=BLOCK, escape=True)
+    status = torch.zeros(2, dtype=torch.int32, device=dev)
+
+    def encode_all():
+        rc = wc.wc_compress_escape_batch(enc.items, enc.count, enc.workspace.data_ptr(),
+                                         enc.workspace.numel(), status[0:].data_ptr(), sh)
+        if rc != 0:
+            raise RuntimeError("wc_compress_escape_batch: %s" % wc.wc_status_string(rc))
+
+    encode_all()
+    torch.cuda.synchronize(dev)
+    sizes = enc.sizes()
+    batch = wcodec.make_batch([(enc.buffers[k], sizes[k], outs[k], inputs[k].numel(), BLOCK)
+                               for k in range(len(inputs))])
+
+    def decode_all():
+        rc = wc.wc_decompress_escape_batch(batch[0], batch[1], status[1:].data_ptr(), sh)
+        if rc != 0:
+            raise RuntimeError("wc_decompress_escape_batch: %s" % wc.wc_status_string(rc))
+
+    for o in outs:
+        o.fill_(-1)
+    torch.cuda.nvtx.range_push("escape-coded encode")
+    t_enc = timed_steps(encode_all, args.steps, args.warmup, stream, dist, dev)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.nvtx.range_push("escape-coded decode")
+    t_dec = timed_steps(decode_all, args.steps, args.warmup, stream, dist, dev)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize(dev)
+    ok = (bool((status == 0).all().item()) and enc.sizes() == sizes
+          and all(torch.equal(a, b) for a, b in zip(inputs, outs)))
+    C = sum(sizes)
+    moved = C + 2 * n_total
+    peak, peak_kind = hbm_peak()
+    out = {"value": world * 2 * n_total / t_dec / 1e9, "unit": "GB/s (BF16 out)",
+           "ms_per_step": 1e3 * t_dec,
+           "roofline": {"bound": "hbm", "achieved": moved / t_dec / 1e9, "peak": peak,
+                        "unit": "GB/s", "frac": moved / t_dec / 1e9 / peak,
+                        "peak_kind": peak_kind,
+                        "kernel": "decode_kernel<512,escape> (one launch per step)",
+                        "algorithmic_bytes_per_launch": moved},
+           "compression": {"ratio": 2 * n_total / C, "stream_bytes": C},
+           "encode": {"ms_per_step": 1e3 * t_enc, "achieved_hbm_gbs": moved / t_enc / 1e9,
+                      "frac_of_peak": moved / t_enc / 1e9 / peak,
+                      "kernels": "esc_params, esc_reduce, esc_top, esc_down, esc_pack (one "
+                                 "launch each per step)"},
+           "gpu_launches": args.steps * 6,
+           "verified_bit_exact": ok}
+    del enc, batch
+    torch.cuda.empty_cache()
+    return out, ok
+
+
+def fused_phase(args, wc, wcodec, mats, streams, sizes, nv, gemm, stream, dist, dev, world,
+                escape=False):
+    """Fused decode + products over weight matrices given as streams: one
+    wc_gemm_batch call (tensor cores, `nv` activation rows, one launch per 64
+    matrices) or one wc_gemv_batch launch (`nv` vectors), against torch's BF16
+    matmul (cuBLAS) on the uncompressed matrices replayed from a CUDA graph.
+    mats: (rows, cols) BF16 tensors; streams/sizes: their streams. Every output
+    is checked against the float64 product of the uncompressed weights."""
+    import torch
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    xs = [torch.randn((nv, t.shape[1]), generator=g, device=dev).to(torch.bfloat16) for t in mats]
+    ys = [torch.empty((nv, t.shape[0]), dtype=torch.float32, device=dev) for t in mats]
+    batch = wcodec.make_gemv_batch([(streams[k], sizes[k], xs[k], ys[k], t.shape[0], t.shape[1],
+                                     BLOCK) for k, t in enumerate(mats)])
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    if gemm:
+        entry, ename = (wc.wc_gemm_batch, "wc_gemm_batch")
+    else:
+        entry, ename = (wc.wc_gemv_batch, "wc_gemv_batch")
+    flags = 2 if escape else 0
+
+    def fused():
+        if flags:
+            rc = wc.wc_gemm_batch_flags(batch[0], batch[1], nv, flags, status.data_ptr(),
+                                        stream.cuda_stream)
+        else:
+            rc = entry(batch[0], batch[1], nv, status.data_ptr(), stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError("%s: %s" % (ename, wc.wc_status_string(rc)))
+
+    outs = [torch.empty((nv, t.shape[0]), dtype=torch.bfloat16, device=dev) for t in mats]
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for _ in range(2):
+            for k, t in enumerate(mats):
+                torch.matmul(xs[k], t.T, out=outs[k])
+    stream.wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for k, t in enumerate(mats):
+            torch.matmul(xs[k], t.T, out=outs[k])
+    what = "gemm" if gemm else "gemv"
+    torch.cuda.nvtx.range_push("fused decode+%s, %d rows" % (what, nv))
+    t_fused = timed_steps(fused, args.steps, args.warmup, stream, dist, dev)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.nvtx.range_push("cuBLAS BF16, %d rows" % nv)
+    t_blas = timed_steps(graph.replay, args.steps, args.warmup, stream, dist, dev)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize(dev)
+    ok = status.item() == 0
+    for k, t in enumerate(mats):
+        ref = xs[k].double() @ t.double().T
+        # FP32 sum bound; the tensor cores' accumulation is held to 4x that
+        scale = t.shape[1] * 2.0 ** -22 if gemm else (t.shape[1] - 1) * 2.0 ** -24
+        bound = scale * (xs[k].double().abs() @ t.double().abs().T)
+        ok &= bool(((ys[k].double() - ref).abs() <= bound).all())
+        del ref, bound
+    weights = sum(t.numel() for t in mats)
+    stream_bytes = sum(sizes)
+    x_bytes = sum(x.numel() * 2 for x in xs)
+    y_bytes = sum(y.numel() * 4 for y in ys)
+    moved = stream_bytes + x_bytes + y_bytes
+    peak, peak_kind = hbm_peak()
+    launches = -(-len(mats) // 64) if gemm else -(-len(mats) // 256)
+    kernel = ("gemm_kernel<64%s> (tcgen05, %d launches per step)"
+              % (",escape" if escape else "", launches) if gemm
+              else "gemv_kernel<256,%d> (%d launches per step)" % (nv, launches))
+    out = {"tokens" if gemm else "n_vec": nv,
+           "value": world * 2 * weights / t_fused / 1e9, "unit": "GB/s (effective BF16 weights)",
+           "ms_per_step": 1e3 * t_fused,
+           "roofline": {"bound": "hbm", "achieved": moved / t_fused / 1e9, "peak": peak,
+                        "unit": "GB/s", "frac": moved / t_fused / 1e9 / peak,
+                        "peak_kind": peak_kind, "kernel": kernel,
+                        "algorithmic_bytes_per_launch": moved / launches},
+           "cublas_bf16": {"ms_per_step": 1e3 * t_blas,
+                           "achieved_gbs": (2 * weights + x_bytes + 2 * sum(o.numel() for o in outs))
+                           / t_blas / 1e9,
+                           "speedup_of_fused": t_blas / t_fused},
+           "tflops": 2.0 * weights * nv / t_fused / 1e12,
+           "stream": "escape-coded" if escape else "plain",
+           "gpu_launches": args.steps * launches,
+           "verified_within_fp32_bound": bool(ok)}
+    del graph, xs, ys, outs
+    torch.cuda.empty_cache()
+    return out, bool(ok)
+
+
 def run_wcodec(args):
     import torch
 
@@ -295,7 +484,7 @@ def run_wcodec(args):
 
     # ---- workload, resident in HBM ------------------------------------------------
     t0 = time.time()
-    names, inputs = [], []
+    names, inputs, shapes = [], [], []
     hist = torch.zeros(256, dtype=torch.int64, device=dev)
     if args.workload == "stack":
         tensors = synth.stack_tensors(dev, rank_seed_base(rank))
@@ -306,6 +495,7 @@ def run_wcodec(args):
         hist += torch.bincount(((words.to(torch.int32) >> 7) & 0xFF), minlength=256)
         names.append(name)
         inputs.append(words)
+        shapes.append(tuple(t.shape))
     n_total = sum(w.numel() for w in inputs)
     log("rank %d: generated %d tensors, %d elements in %.1f s" % (rank, len(inputs), n_total,
                                                                    time.time() - t0))
@@ -348,12 +538,16 @@ def run_wcodec(args):
     barrier(dist, dev)
     with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
         for k in range(args.steps):
+            torch.cuda.nvtx.range_push("encode (A1-A4), step %d" % k)
             ev[k][0].record(stream)
             encode_all()
             ev[k][1].record(stream)
+            torch.cuda.nvtx.range_pop()
+            torch.cuda.nvtx.range_push("decode (A5), step %d" % k)
             ev[k][2].record(stream)
             decode_all()
             ev[k][3].record(stream)
+            torch.cuda.nvtx.range_pop()
         barrier(dist, dev)
     enc_ms = [e[0].elapsed_time(e[1]) for e in ev]
     dec_ms = [e[2].elapsed_time(e[3]) for e in ev]
@@ -371,6 +565,24 @@ def run_wcodec(args):
     if not args.no_e2e:
         e2e = run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stream, dist,
                       dev, n_total)
+
+    # ---- the next rows on the same weights: escape-coded streams, fused products --------
+    extra_ok = True
+    escape = None
+    if not args.no_escape:
+        escape, ok = escape_phase(args, wc, wcodec, inputs, outs, stream, dist, dev, world)
+        extra_ok &= ok
+    fused = []
+    if args.fused_tokens:
+        # the linear weights (the embedding is a lookup, not a product), as the plain
+        # streams the main encoder wrote
+        idx = [k for k, nm in enumerate(names) if nm != "embed_tokens"]
+        mats = [inputs[k].view(torch.bfloat16).view(shapes[k]) for k in idx]
+        for nv in args.fused_tokens:
+            res, ok = fused_phase(args, wc, wcodec, mats, [bufs[k] for k in idx],
+                                  [sizes[k] for k in idx], nv, True, stream, dist, dev, world)
+            fused.append(res)
+            extra_ok &= ok
 
     # ---- figures ---------------------------------------------------------------------
     bytes_out = 2 * n_total
@@ -390,12 +602,13 @@ def run_wcodec(args):
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            sample = oracle_sample_words(list(zip(names, inputs)))
-            cdec, cenc, cn = time_oracle(sample)
-            cpu = {"value": cdec, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                   "sample": "layer 0 of the stack (7 tensors, %d elements) copied to the host, "
-                             "encoded then decoded once by the single-threaded C oracle; decode "
-                             "timed (encode %.4f GB/s)" % (cn, cenc)}
+            timer = OracleTimer(oracle_sample_words(list(zip(names, inputs))))
+            cenc = timer.encode()
+            reps = 3
+            csec = sum(timer.decode_step() for _ in range(reps))
+            cpu = dict({"value": 2 * timer.n * reps / csec / 1e9, "unit": "GB/s", "cores": 1,
+                        "kind": "oracle", "sample": ORACLE_SAMPLE + "; %d steps" % reps,
+                        "encode_gbs_bf16_in": cenc}, **host_info())
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
@@ -428,13 +641,15 @@ def run_wcodec(args):
             "clocks": clk,
             "verified_bit_exact": verified,
             "cpu_baseline": cpu,
+            "escape_coded": escape,
+            "fused_gemm": fused or None,
         }
     if dist is not None:
         barrier(dist, dev)
         dist.destroy_process_group()
     if line is not None:
         print(json.dumps(line), flush=True)
-    return 0 if verified else 1
+    return 0 if (verified and extra_ok) else 1
 
 
 def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stream, dist, dev,
@@ -444,8 +659,8 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
     timed region, by two paths: (a) copy the streams to the device
     (cudaMemcpyAsync per tensor), then one batched decode (`entry`); (b) one
     wc_decompress_host_batch launch that reads the streams over the host link
-    itself (`host_flags`: the streams' kind). The faster path is the line's
-    value; both are reported."""
+    itself (`host_flags`: the streams' kind). Path (b), the library call alone,
+    is the line's value; (a) is reported beside it."""
     import torch
     decode_batch = getattr(wc, entry)
     total = sum(sizes)
@@ -515,9 +730,10 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
                   "h2d_bytes_per_step": total, "d2h_bytes_per_step": 4, "steps": steps,
                   "path": "wc_decompress_host_batch (the decoder reads the pinned streams)",
                   "verified_bit_exact": bool(fok)}
-    best, other = (fused_path, copy_path) if fsec < sec else (copy_path, fused_path)
-    result = dict(best)
-    result["other_path"] = other
+    # the value: the library's own host-stream entry point, C-ABI end to end; the
+    # copy engines' path (torch copies, then the library's device decode) beside it
+    result = dict(fused_path)
+    result["copy_then_decode"] = copy_path
     del host, views, hbatch
     # context: the same weights moved uncompressed (BF16, pinned host -> device), no decode
     try:
@@ -546,7 +762,8 @@ def run_e2e(args, wc, wcodec, bufs, sizes, batch, dec_status, inputs, outs, stre
     raw_sec = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, dev)
     result["bf16_h2d_only"] = {"value": whole_job_gbs(world, 2 * n_total, steps, raw_sec),
                                "unit": "GB/s", "h2d_bytes_per_step": 2 * n_total,
-                               "speedup_of_compressed_path": raw_sec / min(sec, fsec)}
+                               "speedup_of_host_stream_decode": raw_sec / fsec,
+                               "speedup_of_copy_then_decode": raw_sec / sec}
     return result
 
 
@@ -904,10 +1121,10 @@ def run_dtype(args):
 def run_gemv(args):
     """Fused decode + products over the 225 linear weight matrices of the
     8B-shaped stack (32 layers x 7 + LM head; the embedding is a lookup, not a
-    product): one wc_gemv_batch launch with n_vec activation vectors (gemv
-    workload), or wc_gemm_batch on the tensor cores with `tokens` activation
-    rows (gemm workload, one launch per 64 matrices); against torch's BF16
-    matmul (cuBLAS) on the same matrices, replayed from a CUDA graph."""
+    product): wc_gemv_batch with n_vec activation vectors (gemv workload), or
+    wc_gemm_batch on the tensor cores with `tokens` activation rows (gemm
+    workload, one launch per 64 matrices); against torch's BF16 matmul (cuBLAS)
+    on the same matrices, replayed from a CUDA graph."""
     import torch
 
     from lossless_weight_compression_b200 import build_lib, synth, wcodec
@@ -928,100 +1145,32 @@ def run_gemv(args):
         mats = [m for l in range(args.gemv_layers)
                 for m in synth.layer_tensors(l, dev, rank_seed_base(rank))]
     weights = sum(t.numel() for _, t in mats)
-    enc = wcodec.CompressBatch([t for _, t in mats], block=BLOCK)
+    enc = wcodec.CompressBatch([t for _, t in mats], block=BLOCK, escape=args.escape_streams)
     enc.run()
     torch.cuda.synchronize(dev)
     sizes = enc.sizes()
-    g = torch.Generator(device=dev)
-    g.manual_seed(7)
-    xs = [torch.randn((nv, t.shape[1]), generator=g, device=dev).to(torch.bfloat16) for _, t in mats]
-    ys = [torch.empty((nv, t.shape[0]), dtype=torch.float32, device=dev) for _, t in mats]
-    batch = wcodec.make_gemv_batch([(enc.buffers[k], sizes[k], xs[k], ys[k], t.shape[0], t.shape[1],
-                                     BLOCK) for k, (_, t) in enumerate(mats)])
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-
-    entry = wc.wc_gemm_batch if gemm else wc.wc_gemv_batch
-
-    def fused():
-        rc = entry(batch[0], batch[1], nv, status.data_ptr(), stream.cuda_stream)
-        if rc != 0:
-            raise RuntimeError("%s: %s" % ("wc_gemm_batch" if gemm else "wc_gemv_batch",
-                                           wc.wc_status_string(rc)))
-
-    # torch / cuBLAS on the uncompressed BF16 weights, all matrices in one graph
-    ts = [t for _, t in mats]
-    outs = [torch.empty((nv, t.shape[0]), dtype=torch.bfloat16, device=dev) for t in ts]
-    side = torch.cuda.Stream(dev)
-    side.wait_stream(stream)
-    with torch.cuda.stream(side):
-        for _ in range(2):
-            for k, t in enumerate(ts):
-                torch.matmul(xs[k], t.T, out=outs[k])
-    stream.wait_stream(side)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for k, t in enumerate(ts):
-            torch.matmul(xs[k], t.T, out=outs[k])
-
-    def timed(fn, steps):
-        for _ in range(args.warmup):
-            fn()
-        barrier(dist, dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(steps):
-            fn()
-        e1.record(stream)
-        barrier(dist, dev)
-        return max_over_ranks(e0.elapsed_time(e1) / 1e3 / steps, dist, dev)
-
     with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
-        t_fused = timed(fused, args.steps)
-        t_blas = timed(graph.replay, args.steps)
-    torch.cuda.synchronize(dev)
-    # verification against the decoded weights in FP64 (outside the timed region)
-    ok = status.item() == 0
-    for k, t in enumerate(ts):
-        ref = xs[k].double() @ t.double().T
-        # FP32 sum bound; the tensor cores' accumulation is held to 4x that
-        scale = t.shape[1] * 2.0 ** -22 if gemm else (t.shape[1] - 1) * 2.0 ** -24
-        bound = scale * (xs[k].double().abs() @ t.double().abs().T)
-        ok &= bool(((ys[k].double() - ref).abs() <= bound).all())
-    stream_bytes = sum(sizes)
-    x_bytes = sum(x.numel() * 2 for x in xs)
-    y_bytes = sum(y.numel() * 4 for y in ys)
-    moved = stream_bytes + x_bytes + y_bytes  # algorithmic bytes of the launch
-    peak, peak_kind = hbm_peak()
-    clk = clocks.summary()
-    launches = -(-len(mats) // 64) if gemm else 1
+        res, ok = fused_phase(args, wc, wcodec, [t for _, t in mats], enc.buffers, sizes, nv, gemm,
+                              stream, dist, dev, world, escape=args.escape_streams)
     what = "gemm" if gemm else "gemv"
-    kernel = ("gemm_kernel<64> (tcgen05, %d launches per step)" % launches if gemm
-              else "gemv_kernel<256,%d> (one launch per step)" % nv)
     line = {
         "metric": "fused decode+%s weights/s (effective BF16 GB/s)" % what.upper(),
-        "value": world * 2 * weights / t_fused / 1e9, "unit": "GB/s",
+        "value": res["value"], "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * t_fused, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u16 weights, f32 accumulate", "data": "synthetic",
         "config": {"workload": "%s over %d linear weight matrices of the 8B-shaped stack "
-                               "(%d weights), %s=%d, block %d"
+                               "(%d weights), %s=%d, block %d, %s streams"
                                % (what, len(mats), weights, "tokens" if gemm else "n_vec", nv,
-                                  BLOCK),
+                                  BLOCK, res["stream"]),
                    "l2": "weights larger than L2; no flush"},
-        "roofline": {"bound": "hbm", "achieved": moved / t_fused / 1e9, "peak": peak, "unit": "GB/s",
-                     "frac": moved / t_fused / 1e9 / peak, "peak_kind": peak_kind,
-                     "kernel": kernel,
-                     "algorithmic_bytes_per_launch": moved, "traffic": None},
-        "cublas_bf16": {"ms_per_step": 1e3 * t_blas,
-                        "achieved_gbs": (2 * weights + x_bytes + 2 * sum(o.numel() for o in outs))
-                        / t_blas / 1e9,
-                        "speedup_of_fused": t_blas / t_fused},
-        "tflops": 2.0 * weights * nv / t_fused / 1e12,
-        "gpu_launches": args.steps * launches,
-        "clocks": clk,
+        "roofline": res["roofline"],
+        "cublas_bf16": res["cublas_bf16"],
+        "tflops": res["tflops"],
+        "gpu_launches": res["gpu_launches"],
+        "clocks": clocks.summary(),
         "verified_within_fp32_bound": ok,
     }
-    del graph
     if dist is not None:
         barrier(dist, dev)
         dist.destroy_process_group()
@@ -1057,6 +1206,14 @@ def main(argv=None):
                     help="skip timing the CPU oracle (for profiling runs)")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end (pinned host memory) measurement")
+    ap.add_argument("--no-escape", action="store_true",
+                    help="stack/layer workloads: skip the escape-coded streams' measurement")
+    ap.add_argument("--fused-tokens", type=lambda v: [int(t) for t in v.split(",") if t],
+                    default=[1, 16, 128],
+                    help="stack/layer workloads: token counts of the fused decode+GEMM "
+                         "measurement on the same streams (comma list; empty to skip)")
+    ap.add_argument("--escape-streams", action="store_true",
+                    help="gemm workload: multiply from escape-coded streams")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         log("note: fewer than 3 warm-up steps")

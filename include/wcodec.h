@@ -160,7 +160,10 @@ int wc_compress_batch(const wc_compress_item *h_items, uint32_t count,
  *    WC_ERR_BUFFER_TOO_SMALL before anything is looked up or enqueued.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    before any stream capture. The address is kept for the life of the
+ *    process: after cudaDeviceReset on a device it belongs to a context that
+ *    no longer exists, so do not call this entry point on that device again
+ *    in the same process.
  *  - All calls share the one array and it keeps what the last call left;
  *    every call clears the part it uses on `stream` before its kernel runs.
  *    Calls that can overlap on the GPU (unordered streams, several host

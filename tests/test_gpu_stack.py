@@ -2,13 +2,16 @@
 16.06 GB BF16) compressed in one wc_compress_batch call and decoded in one
 wc_decompress_batch call -- the launch configuration the benchmark times.
 
-The oracle cannot encode 8 billion elements in test time, so the checks are
-(a) decode(encode(x)) == x for every tensor, bit for bit, on the device;
-(b) every stream's size, E and block headers against the closed form, computed
+Checks:
+(a) every one of the 226 streams byte for byte against the oracle's stream of
+    the same tensor (the oracle runs tensor by tensor on a thread per host
+    core, with bounded host memory);
+(b) decode(encode(x)) == x for every tensor, bit for bit, on the device;
+(c) every stream's size, E and block headers against the closed form, computed
     from per-block exponent min/max with plain PyTorch reductions;
-(c) sampled blocks of every tensor byte for byte against the oracle: a block's
-    header and exponent payload do not depend on the rest of the tensor, so the
-    oracle's encoding of the block alone must reproduce them.
+(d) sampled blocks of every tensor byte for byte against the oracle's encoding
+    of the block alone: a block's header and exponent payload do not depend on
+    the rest of the tensor.
 """
 import numpy as np
 import pytest
@@ -59,6 +62,16 @@ def stack(wclib, cuda):
     yield names, tensors, enc
     del enc, tensors
     torch.cuda.empty_cache()
+
+
+def test_stack_every_stream_matches_oracle(orc, wclib, cuda, stack):
+    from stack_oracle import compare_all
+    names, tensors, enc = stack
+    sizes = enc.sizes()
+    items = ((names[k], tensors[k], enc.buffers[k][:sizes[k]]) for k in range(len(tensors)))
+    bad, count = compare_all(items, lambda w: orc.compress(w, B))
+    assert count == 226
+    assert not bad, bad
 
 
 def test_stack_round_trip_in_one_launch_each_way(wclib, cuda, stack):

@@ -3,16 +3,18 @@ tensors, 8,029,995,008 elements, 16.06 GB BF16) compressed by one
 wc_compress_escape_batch call and decoded by one wc_decompress_escape_batch
 call -- the launch configuration `bench.py --workload escape` times.
 
-The oracle cannot encode 8 billion elements in test time, so the checks are
-(a) decode(encode(x)) == x for every tensor, bit for bit, on the device;
-(b) every block's width and base, every offset, E and every stream's size
+Checks:
+(a) every one of the 226 streams byte for byte against the oracle's
+    escape-coded stream of the same tensor (the oracle runs tensor by tensor on
+    a thread per host core, with bounded host memory);
+(b) decode(encode(x)) == x for every tensor, bit for bit, on the device;
+(c) every block's width and base, every offset, E and every stream's size
     against the choice rule recomputed here with plain PyTorch reductions (a
     256-bin exponent histogram per block, every window of every width, ties to
     the smaller width and then the larger base);
-(c) sampled blocks of every tensor byte for byte against the oracle: a block's
-    header and payload (codes, exception list, padding) do not depend on the
-    rest of the tensor, so the oracle's encoding of the block alone must
-    reproduce them.
+(d) sampled blocks of every tensor byte for byte against the oracle's encoding
+    of the block alone: a block's header and payload (codes, exception list,
+    padding) do not depend on the rest of the tensor.
 """
 import numpy as np
 import pytest
@@ -83,6 +85,16 @@ def stack(wclib, cuda):
     yield names, tensors, enc
     del enc, tensors
     torch.cuda.empty_cache()
+
+
+def test_escape_stack_every_stream_matches_oracle(orc, wclib, cuda, stack):
+    from stack_oracle import compare_all
+    names, tensors, enc = stack
+    sizes = enc.sizes()
+    items = ((names[k], tensors[k], enc.buffers[k][:sizes[k]]) for k in range(len(tensors)))
+    bad, count = compare_all(items, lambda w: orc.compress_escape(w, B))
+    assert count == 226
+    assert not bad, bad
 
 
 def test_escape_stack_round_trip_in_one_batch_each_way(wclib, cuda, stack):

@@ -1,13 +1,15 @@
-"""wc_compress_noalloc, the allocation-free encoder entry point, against wc_compress.
+"""wc_compress_noalloc, the allocation-free encoder entry point, against wc_compress
+and the oracle.
 
 Callers that cannot allocate device memory -- an engine that has reserved the
 GPU's memory for its own pools, or a path that must not stall on the device
 synchronisation cudaMalloc/cudaFree may imply -- use wc_compress_noalloc,
 which keeps the encoder's look-back state in a fixed array inside the library
 instead of a caller workspace. Its stream must be byte-for-byte the stream
-wc_compress writes for the same input (the codec is integer work, so the
-tolerance is zero), on two calls in a row: the second call reuses the array
-the first one left behind. Everything goes through the C-ABI.
+wc_compress writes for the same input and the oracle's stream of it (the codec
+is integer work, so the tolerance is zero), on two calls in a row: the second
+call reuses the array the first one left behind. Everything goes through the
+C-ABI.
 
 This file is named to be collected last.
 """
@@ -50,12 +52,14 @@ def _noalloc(wc, x, block):
     return out[: int(nbytes.item())].cpu().numpy()
 
 
-def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(wclib, cuda):
+def test_noalloc_matches_workspace_entry_on_two_calls_in_a_row(orc, wclib, cuda):
     for x, block in _inputs(cuda):
         expected = _with_workspace(wclib, x, block)
         got = _noalloc(wclib, x, block)
         assert got.size == expected.size
         assert np.array_equal(got, expected)
+        ref = orc.compress(x.cpu().numpy().view(np.uint16), block)
+        assert np.array_equal(got, ref)
 
 
 def test_noalloc_rejects_sizes_beyond_its_array(wclib, cuda):
