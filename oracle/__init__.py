@@ -74,6 +74,16 @@ def lib() -> ctypes.CDLL:
         L.oracle_compress_escape.restype = ctypes.c_int
         L.oracle_decompress_escape.argtypes = [vp, u64, vp, u64, ctypes.c_uint32]
         L.oracle_decompress_escape.restype = ctypes.c_int
+        L.oracle_tans_normalize.argtypes = [vp, ctypes.c_uint32, vp]
+        L.oracle_tans_normalize.restype = None
+        L.oracle_tans_table.argtypes = [vp, ctypes.c_uint32, vp, vp, vp]
+        L.oracle_tans_table.restype = None
+        L.oracle_bound_tans.argtypes = [u64, ctypes.c_uint32, ctypes.c_uint32]
+        L.oracle_bound_tans.restype = u64
+        L.oracle_compress_tans.argtypes = [vp, u64, ctypes.c_uint32, ctypes.c_uint32, vp, u64, vp]
+        L.oracle_compress_tans.restype = ctypes.c_int
+        L.oracle_decompress_tans.argtypes = [vp, u64, vp, u64, ctypes.c_uint32]
+        L.oracle_decompress_tans.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -248,4 +258,59 @@ def decompress_escape(stream: np.ndarray, n: int, block: int) -> np.ndarray:
     rc, out = decompress_escape_status(stream, n, block)
     if rc != OK:
         raise ValueError("oracle_decompress_escape failed with status %d" % rc)
+    return out
+
+
+# --- tANS-coded streams: the exponents entropy-coded, 32 interleaved lanes ---
+def tans_normalize(counts, R: int) -> np.ndarray:
+    """Normalized counts (sum 2^R) of a 256-bin exponent histogram."""
+    c = np.ascontiguousarray(counts, dtype=np.uint64)
+    assert c.size == 256
+    f = np.zeros(256, dtype=np.uint16)
+    lib().oracle_tans_normalize(_ptr(c), R, _ptr(f))
+    return f
+
+
+def tans_table(freq, R: int):
+    """(sym, nb, next) of every one of the 2^R decoder states."""
+    f = np.ascontiguousarray(freq, dtype=np.uint16)
+    L = 1 << R
+    sym = np.zeros(L, np.uint8)
+    nb = np.zeros(L, np.uint8)
+    nxt = np.zeros(L, np.uint16)
+    lib().oracle_tans_table(_ptr(f), R, _ptr(sym), _ptr(nb), _ptr(nxt))
+    return sym, nb, nxt
+
+
+def bound_tans(n: int, chunk: int, R: int) -> int:
+    return lib().oracle_bound_tans(n, chunk, R)
+
+
+def compress_tans(words: np.ndarray, chunk: int, R: int = 11) -> np.ndarray:
+    """Encode BF16 bit patterns into a tANS-coded stream (chunk elements per
+    chunk, 2^R table states)."""
+    words = np.ascontiguousarray(words, dtype=np.uint16).reshape(-1)
+    cap = bound_tans(words.size, chunk, R)
+    if cap == 0:
+        raise ValueError("oracle: invalid chunk %r, R %r or n %d" % (chunk, R, words.size))
+    out = np.empty(cap, dtype=np.uint8)
+    nbytes = ctypes.c_uint64()
+    rc = lib().oracle_compress_tans(_ptr(words), words.size, chunk, R, _ptr(out), cap,
+                                    ctypes.byref(nbytes))
+    if rc != OK:
+        raise ValueError("oracle_compress_tans failed with status %d" % rc)
+    return out[: nbytes.value].copy()
+
+
+def decompress_tans_status(stream: np.ndarray, n: int, chunk: int) -> tuple[int, np.ndarray]:
+    stream = np.ascontiguousarray(stream, dtype=np.uint8).reshape(-1)
+    out = np.zeros(n, dtype=np.uint16)
+    rc = lib().oracle_decompress_tans(_ptr(stream), stream.size, _ptr(out), n, chunk)
+    return rc, out
+
+
+def decompress_tans(stream: np.ndarray, n: int, chunk: int) -> np.ndarray:
+    rc, out = decompress_tans_status(stream, n, chunk)
+    if rc != OK:
+        raise ValueError("oracle_decompress_tans failed with status %d" % rc)
     return out

@@ -655,3 +655,380 @@ int oracle_decompress_escape(const uint8_t *in, uint64_t in_bytes, uint16_t *out
     if (running != E) return ORC_CORRUPT;
     return ORC_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* tANS-coded streams (reading; flags bit 2).                          */
+/* ------------------------------------------------------------------ */
+/*
+ * "MINE: Entropy-coded Memory-efficient Inference for Large Language Models",
+ * Abstract: a GPU entropy coder of the tANS family (dtANS-LLM) that exploits
+ * the non-uniform distribution of weight values and exposes hyper-parameters
+ * trading compression ratio against decoding cost. The abstract gives no
+ * format. Reading: the exponent bytes are coded by tabled asymmetric numeral
+ * systems (Duda's tANS) over one normalized histogram per tensor, with L = 2^R
+ * states; the sign+mantissa bytes stay raw as in every other stream kind.
+ * The tensor is cut into chunks of C elements; a chunk is 32 interleaved lane
+ * streams (lane l codes the chunk's elements l, l + 32, ...), each with its
+ * own state, sharing one stream of 32-bit words that the lanes take in turn
+ * (decode order: step by step, lanes in order). R and C are the
+ * hyper-parameters.
+ *
+ * Layout: the WCB1 container header with flags = 4, the chunk size C in the
+ * block-size field, nb = number of chunks and R in bytes 88..91;
+ *   off_hdr  256 u16 normalized counts f[e] (sum L; all 0 when n = 0)
+ *   off_offs nb u32 chunk offsets, 16-byte units, from off_exp
+ *   off_man  n sign+mantissa bytes
+ *   off_exp  per chunk: 32 u16 initial decoder states, then the u32 words,
+ *            then zeros up to a multiple of 16 bytes
+ * Decoding a lane: state X in [0, L); per element: refill when fewer than R
+ * bits are buffered (the next word goes above the buffered bits), then
+ * e = sym[X], X = next[X] + (the low nb[X] buffered bits), which are dropped.
+ * A valid chunk ends with every state 0 and has fewer than 4 unused words.
+ */
+#define ORC_FLAG_TANS 4u
+#define ORC_TANS_LANES 32u
+
+static int tans_chunk_allowed(uint32_t C)
+{
+    return C == 1024 || C == 2048 || C == 4096 || C == 8192; /* reading */
+}
+
+static int tans_log_allowed(uint32_t R) { return R >= 8 && R <= 12; } /* reading */
+
+static unsigned floor_log2(uint32_t v)
+{
+    unsigned k = 0;
+    while ((v >> (k + 1)) != 0) k++;
+    return k;
+}
+
+/* Normalize exponent counts to a sum of L = 2^R (reading of the
+ * normalization, which the page leaves open): every present exponent gets
+ * max(1, floor(count * L / total)); the shortfall goes to, and any excess
+ * comes off, the entry with the largest normalized count (the smaller
+ * exponent on ties), one at a time. */
+void oracle_tans_normalize(const uint64_t counts[256], uint32_t R, uint16_t freq[256])
+{
+    const uint32_t L = 1u << R;
+    uint64_t total = 0;
+    for (int e = 0; e < 256; e++) total += counts[e];
+    uint64_t sum = 0;
+    for (int e = 0; e < 256; e++) {
+        uint64_t f = 0;
+        if (counts[e] > 0) {
+            f = counts[e] * L / total;
+            if (f == 0) f = 1;
+        }
+        freq[e] = (uint16_t)f;
+        sum += f;
+    }
+    if (total == 0) return;
+    while (sum != L) {
+        int big = 0;
+        for (int e = 1; e < 256; e++)
+            if (freq[e] > freq[big]) big = e;
+        if (sum < L) {
+            freq[big]++;
+            sum++;
+        } else {
+            freq[big]--;
+            sum--;
+        }
+    }
+}
+
+/* Decoding table of the normalized counts (sum L): the exponents are spread
+ * over the L states with the odd step L/2 + L/8 + 3 (which visits every
+ * state once), then state X holding the v-th occurrence of e (v counted from
+ * f[e]) decodes to e with nb = R - floor(log2 v) bits and next = v * 2^nb - L.
+ * pos[e][v - f[e]] = X is the encoder's inverse map (pos_base[e] indexes it). */
+static void tans_tables(const uint16_t freq[256], uint32_t R, uint8_t *sym, uint8_t *nbits,
+                        uint16_t *next, uint16_t *pos, uint32_t pos_base[256])
+{
+    const uint32_t L = 1u << R, step = (L >> 1) + (L >> 3) + 3;
+    uint32_t p = 0, acc = 0;
+    for (int e = 0; e < 256; e++) {
+        pos_base[e] = acc;
+        acc += freq[e];
+        for (uint32_t i = 0; i < freq[e]; i++) {
+            sym[p] = (uint8_t)e;
+            p = (p + step) & (L - 1);
+        }
+    }
+    uint32_t seen[256];
+    for (int e = 0; e < 256; e++) seen[e] = freq[e];
+    for (uint32_t X = 0; X < L; X++) {
+        const unsigned e = sym[X];
+        const uint32_t v = seen[e]++;
+        const unsigned nb = R - floor_log2(v);
+        nbits[X] = (uint8_t)nb;
+        next[X] = (uint16_t)((v << nb) - L);
+        pos[pos_base[e] + (v - freq[e])] = (uint16_t)X;
+    }
+}
+
+/* The decoding table alone (for the tests): sym, nb and next of every state. */
+void oracle_tans_table(const uint16_t freq[256], uint32_t R, uint8_t *sym, uint8_t *nbits,
+                       uint16_t *next)
+{
+    uint16_t *pos = malloc(2 * ((size_t)1 << R));
+    uint32_t pos_base[256];
+    if (pos == NULL) return;
+    tans_tables(freq, R, sym, nbits, next, pos, pos_base);
+    free(pos);
+}
+
+static uint64_t tans_chunk_len(uint64_t n, uint32_t C, uint64_t c)
+{
+    const uint64_t start = c * (uint64_t)C;
+    return (n - start < C) ? n - start : C;
+}
+
+typedef struct {
+    uint64_t nb, off_hdr, off_offs, off_man, off_exp;
+} tans_layout_t;
+
+static tans_layout_t tans_layout(uint64_t n, uint32_t C)
+{
+    tans_layout_t s;
+    s.nb = (n + C - 1) / C;
+    s.off_hdr = ORC_HEADER_BYTES;
+    s.off_offs = s.off_hdr + 512;
+    s.off_man = s.off_offs + round_up_128(4 * s.nb);
+    s.off_exp = s.off_man + round_up_128(n);
+    return s;
+}
+
+/* Words of one lane: the refill rule can buffer at most R - 1 bits before a
+ * refill and consumes at most R bits per element, so a lane of k elements
+ * takes at most 1 + floor(k * R / (33 - R)) words (each refill is followed by
+ * at least 33 - R consumed bits before the next). */
+uint64_t oracle_bound_tans(uint64_t n, uint32_t C, uint32_t R)
+{
+    if (!tans_chunk_allowed(C) || !tans_log_allowed(R) || n > ORC_MAX_ELEMS) return 0;
+    tans_layout_t s = tans_layout(n, C);
+    uint64_t worst = 0;
+    for (uint64_t c = 0; c < s.nb; c++) {
+        const uint64_t len = tans_chunk_len(n, C, c);
+        const uint64_t k = (len + ORC_TANS_LANES - 1) / ORC_TANS_LANES;
+        const uint64_t words = ORC_TANS_LANES * (1 + k * R / (33 - R));
+        worst += round_up_16(2 * ORC_TANS_LANES + 4 * words);
+    }
+    return s.off_exp + worst;
+}
+
+int oracle_compress_tans(const uint16_t *x, uint64_t n, uint32_t C, uint32_t R, uint8_t *out,
+                         uint64_t out_capacity, uint64_t *out_bytes)
+{
+    if (!tans_chunk_allowed(C) || !tans_log_allowed(R) || n > ORC_MAX_ELEMS || out == NULL ||
+        out_bytes == NULL || (n > 0 && x == NULL))
+        return ORC_INVALID_ARG;
+    if (out_capacity < oracle_bound_tans(n, C, R)) return ORC_BUFFER_TOO_SMALL;
+    const uint32_t L = 1u << R;
+    tans_layout_t s = tans_layout(n, C);
+    memset(out, 0, s.off_exp);
+
+    /* the histogram of the exponents and its normalization */
+    uint64_t counts[256] = {0};
+    for (uint64_t i = 0; i < n; i++) counts[oracle_exponent(x[i])]++;
+    uint16_t freq[256];
+    oracle_tans_normalize(counts, R, freq);
+    for (int e = 0; e < 256; e++) put_le(out + s.off_hdr + 2 * e, freq[e], 2);
+    for (uint64_t i = 0; i < n; i++) out[s.off_man + i] = oracle_signman(x[i]);
+
+    uint8_t *sym = malloc(L), *nbits = malloc(L);
+    uint16_t *next = malloc(2 * (size_t)L), *pos = malloc(2 * (size_t)L);
+    uint16_t *val = malloc(2 * (size_t)C);
+    uint8_t *len_bits = malloc(C);
+    /* a lane's words: at most 1 + floor(k * R / (33 - R)) for k elements */
+    const uint64_t lane_cap = 2 + (uint64_t)(C / ORC_TANS_LANES) * R / (33 - R);
+    uint32_t *lane_words = malloc(4 * (size_t)lane_cap * ORC_TANS_LANES);
+    uint32_t pos_base[256];
+    if (!sym || !nbits || !next || !pos || !val || !len_bits || !lane_words) {
+        free(sym); free(nbits); free(next); free(pos); free(val); free(len_bits);
+        free(lane_words);
+        return ORC_INVALID_ARG;
+    }
+    tans_tables(freq, R, sym, nbits, next, pos, pos_base);
+
+    uint64_t running = 0;
+    for (uint64_t c = 0; c < s.nb; c++) {
+        const uint64_t first = c * (uint64_t)C, len = tans_chunk_len(n, C, c);
+        uint8_t *payload = out + s.off_exp + running;
+        put_le(out + s.off_offs + 4 * c, running / 16, 4);
+        /* 1. every lane coded backwards from its last element: each element
+         *    gives the bits its decoding will read (value, count), element by
+         *    element in chunk order */
+        for (uint32_t l = 0; l < ORC_TANS_LANES; l++) {
+            uint32_t state = L; /* the encoder's state lives in [L, 2L) */
+            const uint64_t steps = len > l ? (len - l + ORC_TANS_LANES - 1) / ORC_TANS_LANES : 0;
+            for (uint64_t k = steps; k-- > 0;) {
+                const uint64_t i = l + k * ORC_TANS_LANES;
+                const unsigned e = oracle_exponent(x[first + i]);
+                const uint32_t f = freq[e];
+                unsigned nb = 0;
+                while ((state >> nb) >= 2 * f) nb++;
+                val[i] = (uint16_t)(state & ((1u << nb) - 1u));
+                len_bits[i] = (uint8_t)nb;
+                state = L + pos[pos_base[e] + ((state >> nb) - f)];
+            }
+            put_le(payload + 2 * l, state - L, 2); /* the decoder's first state */
+        }
+        /* 2. each lane's bits in element order, bit by bit, 32 to a word */
+        uint64_t lane_bits[ORC_TANS_LANES] = {0};
+        for (uint32_t l = 0; l < ORC_TANS_LANES; l++) {
+            uint32_t *lw = lane_words + (uint64_t)l * lane_cap;
+            memset(lw, 0, 4 * (size_t)lane_cap);
+            for (uint64_t j = l; j < len; j += ORC_TANS_LANES)
+                for (unsigned b = 0; b < len_bits[j]; b++, lane_bits[l]++)
+                    if ((val[j] >> b) & 1u) lw[lane_bits[l] / 32] |= 1u << (lane_bits[l] % 32);
+        }
+        /* 3. the words, in the order the decoder takes them: step by step,
+         *    lanes in order, a lane refilling when it holds fewer than R bits */
+        uint64_t words = 0;
+        uint32_t cnt[ORC_TANS_LANES] = {0};   /* bits buffered by the decoder */
+        uint64_t taken[ORC_TANS_LANES] = {0}; /* words of the lane already taken */
+        const uint64_t max_steps = (len + ORC_TANS_LANES - 1) / ORC_TANS_LANES;
+        for (uint64_t k = 0; k < max_steps; k++) {
+            for (uint32_t l = 0; l < ORC_TANS_LANES; l++) {
+                const uint64_t i = l + k * ORC_TANS_LANES;
+                if (i >= len || cnt[l] >= R) continue;
+                if (2 * ORC_TANS_LANES + 4 * (words + 1) > out_capacity - s.off_exp - running ||
+                    taken[l] >= lane_cap) {
+                    free(sym); free(nbits); free(next); free(pos); free(val); free(len_bits);
+                    free(lane_words);
+                    return ORC_BUFFER_TOO_SMALL;
+                }
+                put_le(payload + 2 * ORC_TANS_LANES + 4 * words,
+                       lane_words[(uint64_t)l * lane_cap + taken[l]], 4);
+                words++;
+                taken[l]++;
+                cnt[l] += 32;
+            }
+            for (uint32_t l = 0; l < ORC_TANS_LANES; l++) {
+                const uint64_t i = l + k * ORC_TANS_LANES;
+                if (i < len) cnt[l] -= len_bits[i];
+            }
+        }
+        const uint64_t size = round_up_16(2 * ORC_TANS_LANES + 4 * words);
+        memset(payload + 2 * ORC_TANS_LANES + 4 * words, 0,
+               size - 2 * ORC_TANS_LANES - 4 * words);
+        running += size;
+    }
+    free(sym); free(nbits); free(next); free(pos); free(val); free(len_bits);
+    free(lane_words);
+
+    layout_t hdr;
+    hdr.nb = s.nb;
+    hdr.off_hdr = s.off_hdr;
+    hdr.off_offs = s.off_offs;
+    hdr.off_man = s.off_man;
+    hdr.off_low = 0;
+    hdr.off_exp = s.off_exp;
+    write_container(out, C, ORC_FLAG_TANS, n, &hdr, running);
+    put_le(out + 88, R, 4);
+    *out_bytes = s.off_exp + running;
+    return ORC_OK;
+}
+
+int oracle_decompress_tans(const uint8_t *in, uint64_t in_bytes, uint16_t *out, uint64_t n,
+                           uint32_t C)
+{
+    if (!tans_chunk_allowed(C) || n > ORC_MAX_ELEMS || in == NULL || (n > 0 && out == NULL))
+        return ORC_INVALID_ARG;
+    if (in_bytes < ORC_HEADER_BYTES) return ORC_CORRUPT;
+    tans_layout_t s = tans_layout(n, C);
+    const uint32_t R = (uint32_t)get_le(in + 88, 4);
+    if (get_le(in + 0, 4) != ORC_MAGIC || get_le(in + 4, 2) != ORC_VERSION ||
+        get_le(in + 6, 2) != ORC_HEADER_BYTES || get_le(in + 8, 4) != C ||
+        get_le(in + 12, 4) != ORC_FLAG_TANS || get_le(in + 16, 8) != n ||
+        get_le(in + 24, 8) != s.nb || get_le(in + 32, 8) != s.off_hdr ||
+        get_le(in + 40, 8) != s.off_offs || get_le(in + 48, 8) != s.off_man ||
+        get_le(in + 56, 8) != s.off_exp || get_le(in + 80, 8) != 0 ||
+        !tans_log_allowed(R) || !all_zero(in + 92, 36))
+        return ORC_CORRUPT;
+    const uint64_t E = get_le(in + 64, 8);
+    const uint64_t total = get_le(in + 72, 8);
+    if (E > total || total != s.off_exp + E || total > in_bytes) return ORC_CORRUPT;
+    if (!all_zero(in + s.off_offs + 4 * s.nb, s.off_man - s.off_offs - 4 * s.nb) ||
+        !all_zero(in + s.off_man + n, s.off_exp - s.off_man - n))
+        return ORC_CORRUPT;
+    const uint32_t L = 1u << R;
+    uint16_t freq[256];
+    uint64_t sum = 0;
+    for (int e = 0; e < 256; e++) {
+        freq[e] = (uint16_t)get_le(in + s.off_hdr + 2 * e, 2);
+        sum += freq[e];
+    }
+    if (sum != (n > 0 ? L : 0)) return ORC_CORRUPT;
+    if (n == 0) return E == 0 ? ORC_OK : ORC_CORRUPT;
+
+    uint8_t *sym = malloc(L), *nbits = malloc(L);
+    uint16_t *next = malloc(2 * (size_t)L), *pos = malloc(2 * (size_t)L);
+    uint32_t pos_base[256];
+    if (!sym || !nbits || !next || !pos) {
+        free(sym); free(nbits); free(next); free(pos);
+        return ORC_INVALID_ARG;
+    }
+    tans_tables(freq, R, sym, nbits, next, pos, pos_base);
+    int rc = ORC_OK;
+    uint64_t running = 0;
+    for (uint64_t c = 0; c < s.nb && rc == ORC_OK; c++) {
+        const uint64_t first = c * (uint64_t)C, len = tans_chunk_len(n, C, c);
+        const uint64_t start = 16 * get_le(in + s.off_offs + 4 * c, 4);
+        const uint64_t end = c + 1 < s.nb ? 16 * get_le(in + s.off_offs + 4 * (c + 1), 4) : E;
+        if (start != running || end < start + 2 * ORC_TANS_LANES || end > E) {
+            rc = ORC_CORRUPT;
+            break;
+        }
+        const uint8_t *payload = in + s.off_exp + start;
+        const uint64_t avail = (end - start - 2 * ORC_TANS_LANES) / 4;
+        uint32_t X[ORC_TANS_LANES], cnt[ORC_TANS_LANES];
+        uint64_t buf[ORC_TANS_LANES];
+        for (uint32_t l = 0; l < ORC_TANS_LANES; l++) {
+            X[l] = (uint32_t)get_le(payload + 2 * l, 2);
+            cnt[l] = 0;
+            buf[l] = 0;
+            if (X[l] >= L || (l >= len && X[l] != 0)) rc = ORC_CORRUPT;
+        }
+        uint64_t words = 0;
+        const uint64_t max_steps = (len + ORC_TANS_LANES - 1) / ORC_TANS_LANES;
+        for (uint64_t k = 0; k < max_steps && rc == ORC_OK; k++) {
+            for (uint32_t l = 0; l < ORC_TANS_LANES; l++) {
+                const uint64_t i = l + k * ORC_TANS_LANES;
+                if (i >= len) continue;
+                if (cnt[l] < R) {
+                    if (words >= avail) {
+                        rc = ORC_CORRUPT;
+                        break;
+                    }
+                    buf[l] |= get_le(payload + 2 * ORC_TANS_LANES + 4 * words, 4) << cnt[l];
+                    cnt[l] += 32;
+                    words++;
+                }
+            }
+            for (uint32_t l = 0; l < ORC_TANS_LANES && rc == ORC_OK; l++) {
+                const uint64_t i = l + k * ORC_TANS_LANES;
+                if (i >= len) continue;
+                const unsigned nb = nbits[X[l]];
+                const unsigned e = sym[X[l]];
+                X[l] = next[X[l]] + (uint32_t)(buf[l] & ((1u << nb) - 1u));
+                buf[l] >>= nb;
+                cnt[l] -= nb;
+                out[first + i] = oracle_merge((uint8_t)e, in[s.off_man + first + i]);
+            }
+        }
+        if (rc != ORC_OK) break;
+        /* every lane back at state 0, no bits left over, padding zero */
+        for (uint32_t l = 0; l < ORC_TANS_LANES; l++)
+            if (X[l] != 0 || buf[l] != 0) rc = ORC_CORRUPT;
+        if (avail - words > 3 ||
+            !all_zero(payload + 2 * ORC_TANS_LANES + 4 * words,
+                      end - start - 2 * ORC_TANS_LANES - 4 * words))
+            rc = ORC_CORRUPT;
+        running = end;
+    }
+    if (rc == ORC_OK && running != E) rc = ORC_CORRUPT;
+    free(sym); free(nbits); free(next); free(pos);
+    return rc;
+}

@@ -26,9 +26,21 @@ def load(name: str):
 
 
 def load_kind(name: str):
-    """Returns (block, words uint16, expected stream uint8, kind): kind is "plain"
-    or "escape" (an escape-coded stream, the fixture's "kind escape" line)."""
-    block = total = None
+    """Returns (block, words uint16, expected stream uint8, kind): kind is "plain",
+    "escape" (an escape-coded stream, the fixture's "kind escape" line) or "tans"
+    (a tANS-coded stream; its table log is read by load_tans)."""
+    return _load(name)[:4]
+
+
+def load_tans(name: str):
+    """Returns (chunk size, table log R, words uint16, expected stream uint8)."""
+    block, words, expected, kind, R = _load(name)
+    assert kind == "tans"
+    return block, R, words, expected
+
+
+def _load(name: str):
+    block = total = R = None
     kind = "plain"
     words, runs = [], []
     with open(os.path.join(GOLDEN_DIR, name)) as f:
@@ -41,6 +53,8 @@ def load_kind(name: str):
                 kind = rest.strip()
             elif key == "block":
                 block = int(rest)
+            elif key == "tablelog":
+                R = int(rest)
             elif key == "words":
                 words += _expand(rest.split())
             elif key == "total":
@@ -53,7 +67,7 @@ def load_kind(name: str):
     expected = np.zeros(total, dtype=np.uint8)
     for off, data in runs:
         expected[off:off + len(data)] = data
-    return block, np.array(words, dtype=np.uint16), expected, kind
+    return block, np.array(words, dtype=np.uint16), expected, kind, R
 
 
 def names(kind: str = "plain"):
