@@ -317,10 +317,12 @@ def timed_steps(fn, steps, warmup, stream, dist, dev):
     return max_over_ranks(e0.elapsed_time(e1) / 1e3 / steps, dist, dev)
 
 
-def escape_phase(args, wc, wcodec, inputs, outs, stream, dist, dev, world):
+def escape_phase(args, wc, wcodec, inputs, outs, stream, dist, dev, world, mats=None):
     """The same tensors as escape-coded streams: one wc_compress_escape_batch call
     (five launches) and one wc_decompress_escape_batch launch, each timed over
-    the step count; every decoded tensor checked against its input."""
+    the step count; every decoded tensor checked against its input. mats:
+    (index, (rows, cols) BF16 view) of the linear weights, multiplied from
+    their escape-coded streams on the tensor cores at args.fused_tokens."""
     import torch
     sh = stream.cuda_stream
     n_total = sum(w.numel() for w in inputs)
@@ -372,9 +374,74 @@ def escape_phase(args, wc, wcodec, inputs, outs, stream, dist, dev, world):
                                  "launch each per step)"},
            "gpu_launches": args.steps * 6,
            "verified_bit_exact": ok}
+    fused = []
+    for nv in (args.fused_tokens if mats else []):
+        res, fok = fused_phase(args, wc, wcodec, [m for _, m in mats],
+                               [enc.buffers[k] for k, _ in mats], [sizes[k] for k, _ in mats],
+                               nv, True, stream, dist, dev, world, escape=True)
+        fused.append(res)
+        ok &= fok
+    out["fused_gemm"] = fused or None
+    out["verified_bit_exact"] = ok
     del enc, batch
     torch.cuda.empty_cache()
     return out, ok
+
+
+TANS_CHUNK = 4096
+TANS_LOG = 11
+
+
+def tans_phase(args, wc, wcodec, inputs, outs, stream, dist, dev, world):
+    """The same tensors as tANS-coded streams (exponents entropy-coded, chunks
+    of 4096 elements as 32 interleaved lane streams, 2^11 states): one
+    wc_compress_tans_batch call (five launches) and one wc_decompress_tans_batch
+    launch, each timed over the step count; every decoded tensor checked
+    against its input."""
+    import torch
+    n_total = sum(w.numel() for w in inputs)
+    enc = wcodec.CompressBatch(inputs, block=TANS_CHUNK, tans_log=TANS_LOG)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    enc.run(stream)
+    torch.cuda.synchronize(dev)
+    sizes = enc.sizes()
+    batch = wcodec.make_batch([(enc.buffers[k], sizes[k], outs[k], inputs[k].numel(), TANS_CHUNK)
+                               for k in range(len(inputs))])
+
+    def decode_all():
+        wcodec.decompress_tans_batch(batch, status, stream)
+
+    for o in outs:
+        o.fill_(-1)
+    torch.cuda.nvtx.range_push("tANS encode")
+    t_enc = timed_steps(lambda: enc.run(stream), args.steps, args.warmup, stream, dist, dev)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.nvtx.range_push("tANS decode")
+    t_dec = timed_steps(decode_all, args.steps, args.warmup, stream, dist, dev)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize(dev)
+    ok = (status.item() == 0 and enc.sizes() == sizes
+          and all(torch.equal(a, b) for a, b in zip(inputs, outs)))
+    C = sum(sizes)
+    moved = C + 2 * n_total
+    peak, peak_kind = hbm_peak()
+    out = {"value": world * 2 * n_total / t_dec / 1e9, "unit": "GB/s (BF16 out)",
+           "ms_per_step": 1e3 * t_dec, "chunk": TANS_CHUNK, "table_log": TANS_LOG,
+           "roofline": {"bound": "hbm", "achieved": moved / t_dec / 1e9, "peak": peak,
+                        "unit": "GB/s", "frac": moved / t_dec / 1e9 / peak,
+                        "peak_kind": peak_kind,
+                        "kernel": "tans_decode_kernel<256> (one launch per step)",
+                        "algorithmic_bytes_per_launch": moved},
+           "compression": {"ratio": 2 * n_total / C, "stream_bytes": C},
+           "encode": {"ms_per_step": 1e3 * t_enc, "achieved_hbm_gbs": moved / t_enc / 1e9,
+                      "frac_of_peak": moved / t_enc / 1e9 / peak,
+                      "kernels": "tans_hist, tans_plan, tans_encode (twice), tans_scan (five "
+                                 "launches per step)"},
+           "gpu_launches": args.steps * 6,
+           "verified_bit_exact": bool(ok)}
+    del enc, batch
+    torch.cuda.empty_cache()
+    return out, bool(ok)
 
 
 def fused_phase(args, wc, wcodec, mats, streams, sizes, nv, gemm, stream, dist, dev, world,
@@ -568,16 +635,21 @@ def run_wcodec(args):
 
     # ---- the next rows on the same weights: escape-coded streams, fused products --------
     extra_ok = True
+    # the linear weights (the embedding is a lookup, not a product)
+    idx = [k for k, nm in enumerate(names) if nm != "embed_tokens"]
+    mats = [inputs[k].view(torch.bfloat16).view(shapes[k]) for k in idx]
     escape = None
     if not args.no_escape:
-        escape, ok = escape_phase(args, wc, wcodec, inputs, outs, stream, dist, dev, world)
+        escape, ok = escape_phase(args, wc, wcodec, inputs, outs, stream, dist, dev, world,
+                                  list(zip(idx, mats)))
+        extra_ok &= ok
+    tans = None
+    if not args.no_tans:
+        tans, ok = tans_phase(args, wc, wcodec, inputs, outs, stream, dist, dev, world)
         extra_ok &= ok
     fused = []
     if args.fused_tokens:
-        # the linear weights (the embedding is a lookup, not a product), as the plain
-        # streams the main encoder wrote
-        idx = [k for k, nm in enumerate(names) if nm != "embed_tokens"]
-        mats = [inputs[k].view(torch.bfloat16).view(shapes[k]) for k in idx]
+        # from the plain streams the main encoder wrote
         for nv in args.fused_tokens:
             res, ok = fused_phase(args, wc, wcodec, mats, [bufs[k] for k in idx],
                                   [sizes[k] for k in idx], nv, True, stream, dist, dev, world)
@@ -642,6 +714,7 @@ def run_wcodec(args):
             "verified_bit_exact": verified,
             "cpu_baseline": cpu,
             "escape_coded": escape,
+            "tans_coded": tans,
             "fused_gemm": fused or None,
         }
     if dist is not None:
@@ -1208,6 +1281,8 @@ def main(argv=None):
                     help="skip the end-to-end (pinned host memory) measurement")
     ap.add_argument("--no-escape", action="store_true",
                     help="stack/layer workloads: skip the escape-coded streams' measurement")
+    ap.add_argument("--no-tans", action="store_true",
+                    help="stack/layer workloads: skip the tANS-coded streams' measurement")
     ap.add_argument("--fused-tokens", type=lambda v: [int(t) for t in v.split(",") if t],
                     default=[1, 16, 128],
                     help="stack/layer workloads: token counts of the fused decode+GEMM "

@@ -355,8 +355,9 @@ int wc_gemv_batch(const wc_gemv_item *h_items, uint32_t count, uint32_t n_vec,
  * Fused decompression and matrix products on the tensor cores: for t < tokens,
  *   y[t][r] = sum_c W[r][c] * x[t][c]
  * with W (rows x cols, row-major BF16) given only as its WCB1 stream, as for
- * wc_gemv; the decoded weights go from shared memory straight into tcgen05
- * tensor-core MMAs (BF16 x BF16 -> FP32) and never reach device memory
+ * wc_gemv; the decoded weights go from the SM's own memories (shared memory,
+ * then tensor memory) straight into tcgen05 tensor-core MMAs (BF16 x BF16 ->
+ * FP32) and never reach device memory
  * ("ZipServ: Fast and Memory-Efficient LLM Inference with Hardware-Aware
  * Lossless Compression", Abstract: decompression fused into the GEMM). x is
  * tokens x cols BF16 (device, 16-byte aligned, row-major), y is tokens x rows
@@ -384,10 +385,84 @@ int wc_gemm_batch(const wc_gemv_item *h_items, uint32_t count, uint32_t tokens,
                   int32_t *d_status, void *stream);
 
 /*
+ * wc_gemm_batch for either stream kind: flags 0 (plain WCB1 streams, exactly
+ * wc_gemm_batch) or WC_FLAG_ESCAPE (escape-coded streams, as written by
+ * wc_compress_escape). The escape-coded product is the combination the
+ * ZipServ abstract describes ("ZipServ: Fast and Memory-Efficient LLM
+ * Inference with Hardware-Aware Lossless Compression", Abstract: a compact
+ * fixed-length format decoded in constant time, in parallel, directly into the
+ * tensor-core operands): an element's code sits at a closed-form position and
+ * an escaped element takes the next byte of its block's exception list. For
+ * escape-coded streams every row must be whole blocks (cols a multiple of
+ * block; else WC_ERR_INVALID_ARG). Results, bound and determinism as
+ * wc_gemm. The stream is checked for what the kernel reads (each block's width
+ * and window, the offset chain against the codes, the exception list against
+ * the escape count and outside the window, every read inside stream_bytes);
+ * a stream of the other kind is reported as corrupt. Any other flags value:
+ * WC_ERR_INVALID_ARG.
+ */
+int wc_gemm_batch_flags(const wc_gemv_item *h_items, uint32_t count, uint32_t tokens,
+                        uint32_t flags, int32_t *d_status, void *stream);
+
+/*
+ * tANS-coded streams (header flags 4): the exponent bytes entropy-coded by
+ * tabled asymmetric numeral systems ("MINE: Entropy-coded Memory-efficient
+ * Inference for Large Language Models", Abstract: a GPU entropy coder of the
+ * tANS family, dtANS-LLM, exploiting the non-uniform distribution of weights,
+ * with hyper-parameters that trade compression ratio against decoding cost;
+ * the format is this library's reading). One normalized histogram per tensor
+ * with 2^table_log states (table_log 8..12); the tensor is cut into chunks of
+ * `chunk` elements (1024, 2048, 4096 or 8192), each coded as 32 interleaved
+ * lane streams (lane l: the chunk's elements l, l + 32, ...) that share one
+ * stream of 32-bit words, taken in turn by the lanes holding fewer than
+ * table_log bits; the sign+mantissa bytes stay raw. Unlike the fixed-length
+ * streams, a lane's position in the word stream is only known after its
+ * previous element ("ZipServ ...", Abstract: variable-length codes break SIMT
+ * parallelism), so one warp decodes one chunk step by step.
+ * Layout: the WCB1 header (flags 4, the chunk size in the block field, the
+ * table log at byte 88), 256 u16 normalized counts at byte 128, u32 chunk
+ * offsets (16-byte units) at byte 640, the mantissa plane, then per chunk 32
+ * u16 first states, the words and zero padding to 16 bytes.
+ *
+ *  wc_bound_tans        output capacity the encoder needs; 0 if invalid
+ *  wc_compress_tans_batch_workspace_size
+ *                       device workspace of wc_compress_tans[_batch]: 2 KB per
+ *                       tensor and 4 bytes per chunk (per WC_BATCH_MAX tensors)
+ *  wc_compress_tans[_batch]
+ *                       encode (items' block = the chunk size): five launches
+ *                       per WC_BATCH_MAX tensors, none waiting on another
+ *                       thread block; the workspace is overwritten (cleared by
+ *                       the call on `stream`); *out_bytes receives each size
+ *  wc_decompress_tans[_batch]
+ *                       decode (block = the chunk size): one launch per 256
+ *                       tensors. The kernels check the header, that the counts
+ *                       sum to 2^table_log, every chunk's offsets and first
+ *                       states, every word read against its chunk's payload,
+ *                       and that every lane ends in state 0 with fewer than 4
+ *                       unused words; WC_ERR_CORRUPT_STREAM in *d_status
+ *                       otherwise, with every read inside stream_bytes. A
+ *                       stream shorter than its fixed sections returns
+ *                       WC_ERR_CORRUPT_STREAM without launching.
+ * Device pointers 16-byte aligned; the library allocates nothing.
+ */
+uint64_t wc_bound_tans(uint64_t n, uint32_t chunk, uint32_t table_log);
+uint64_t wc_compress_tans_batch_workspace_size(const wc_compress_item *h_items, uint32_t count);
+int wc_compress_tans(const void *d_in, uint64_t n, uint32_t chunk, uint32_t table_log,
+                     void *d_out, uint64_t out_capacity, uint64_t *d_out_bytes,
+                     void *d_workspace, uint64_t workspace_bytes, void *stream);
+int wc_compress_tans_batch(const wc_compress_item *h_items, uint32_t count, uint32_t table_log,
+                           void *d_workspace, uint64_t workspace_bytes, void *stream);
+int wc_decompress_tans(const void *d_stream, uint64_t stream_bytes, void *d_out, uint64_t n,
+                       uint32_t chunk, int32_t *d_status, void *stream);
+int wc_decompress_tans_batch(const wc_batch_item *h_items, uint32_t count, int32_t *d_status,
+                             void *stream);
+
+/*
  * Parse a host copy of a stream's first `header_bytes` (>= 128) bytes. Fills
  * n, block and total_bytes (any may be NULL). Returns WC_ERR_CORRUPT_STREAM
  * if the header is not a WCB1 version-1 header consistent with itself (BF16,
- * FP32 or escape-coded stream; header bytes 12..15 say which).
+ * FP32, escape-coded or tANS-coded stream; header bytes 12..15 say which; for
+ * a tANS-coded stream `block` is its chunk size).
  */
 int wc_stream_info(const void *h_header, uint64_t header_bytes,
                    uint64_t *n, uint32_t *block, uint64_t *total_bytes);

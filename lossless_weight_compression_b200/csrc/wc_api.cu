@@ -366,6 +366,120 @@ int wc_decompress_escape_batch(const wc_batch_item* h_items, uint32_t count, int
     return WC_OK;
 }
 
+static int check_tans_item(const wc_batch_item& it) {
+    if (!wc::tans_chunk_ok(it.block) || it.n > wc::kMaxElems || it.stream == nullptr ||
+        (it.n > 0 && it.out == nullptr) || it.reserved != 0)
+        return WC_ERR_INVALID_ARG;
+    if (!aligned16(it.stream) || (it.n > 0 && !aligned16(it.out))) return WC_ERR_INVALID_ARG;
+    if (it.stream_bytes < wc::tans_fixed_bytes(it.n, it.block)) return WC_ERR_CORRUPT_STREAM;
+    return WC_OK;
+}
+
+uint64_t wc_bound_tans(uint64_t n, uint32_t chunk, uint32_t table_log) {
+    if (!wc::tans_chunk_ok(chunk) || table_log < 8 || table_log > 12 || n > wc::kMaxElems) return 0;
+    return wc::tans_bound_bytes(n, chunk, table_log);
+}
+
+static int tans_encode_items(const wc_compress_item* h_items, uint32_t count, uint32_t table_log,
+                             wc::EncodeItem* items) {
+    if (table_log < 8 || table_log > 12) return WC_ERR_INVALID_ARG;
+    for (uint32_t i = 0; i < count; ++i) {
+        const wc_compress_item& it = h_items[i];
+        if (!wc::tans_chunk_ok(it.block) || it.n > wc::kMaxElems || it.out == nullptr ||
+            it.out_bytes == nullptr || (it.n > 0 && it.in == nullptr) || it.reserved != 0)
+            return WC_ERR_INVALID_ARG;
+        if ((it.n > 0 && !aligned16(it.in)) || !aligned16(it.out) ||
+            (reinterpret_cast<uintptr_t>(it.out_bytes) & 7u) != 0)
+            return WC_ERR_INVALID_ARG;
+        if (it.out_capacity < wc::tans_bound_bytes(it.n, it.block, table_log))
+            return WC_ERR_BUFFER_TOO_SMALL;
+        items[i] = to_encode_item(it.in, it.n, it.block, it.out, it.out_bytes);
+    }
+    return WC_OK;
+}
+
+uint64_t wc_compress_tans_batch_workspace_size(const wc_compress_item* h_items, uint32_t count) {
+    if (h_items == nullptr && count > 0) return 0;
+    uint64_t total = 0;
+    for (uint32_t base = 0; base < count; base += WC_BATCH_MAX) {
+        const uint32_t c = (count - base < WC_BATCH_MAX) ? count - base : WC_BATCH_MAX;
+        wc::EncodeItem items[WC_BATCH_MAX];
+        for (uint32_t i = 0; i < c; ++i) {
+            items[i].n = h_items[base + i].n;
+            items[i].block = wc::tans_chunk_ok(h_items[base + i].block) ? h_items[base + i].block : 1024u;
+        }
+        total += wc::tans_workspace_bytes(items, c);
+    }
+    return total;
+}
+
+int wc_compress_tans_batch(const wc_compress_item* h_items, uint32_t count, uint32_t table_log,
+                           void* d_workspace, uint64_t workspace_bytes, void* stream) {
+    if ((h_items == nullptr && count > 0) || (count > 0 && d_workspace == nullptr) ||
+        (count > 0 && !aligned16(d_workspace)))
+        return WC_ERR_INVALID_ARG;
+    if (workspace_bytes < wc_compress_tans_batch_workspace_size(h_items, count))
+        return WC_ERR_BUFFER_TOO_SMALL;
+    uint8_t* ws = static_cast<uint8_t*>(d_workspace);
+    for (uint32_t base = 0; base < count; base += WC_BATCH_MAX) {
+        const uint32_t c = (count - base < WC_BATCH_MAX) ? count - base : WC_BATCH_MAX;
+        wc::EncodeItem items[WC_BATCH_MAX];
+        uint32_t logs[WC_BATCH_MAX];
+        const int rc = tans_encode_items(h_items + base, c, table_log, items);
+        if (rc != WC_OK) return rc;
+        for (uint32_t i = 0; i < c; ++i) logs[i] = table_log;
+        const cudaError_t err =
+            wc::launch_encode_tans(items, logs, c, ws, static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return WC_ERR_CUDA;
+        ws += wc::tans_workspace_bytes(items, c);
+    }
+    return WC_OK;
+}
+
+int wc_compress_tans(const void* d_in, uint64_t n, uint32_t chunk, uint32_t table_log, void* d_out,
+                     uint64_t out_capacity, uint64_t* d_out_bytes, void* d_workspace,
+                     uint64_t workspace_bytes, void* stream) {
+    wc_compress_item it;
+    it.in = d_in;
+    it.n = n;
+    it.block = chunk;
+    it.reserved = 0;
+    it.out = d_out;
+    it.out_capacity = out_capacity;
+    it.out_bytes = d_out_bytes;
+    return wc_compress_tans_batch(&it, 1, table_log, d_workspace, workspace_bytes, stream);
+}
+
+int wc_decompress_tans_batch(const wc_batch_item* h_items, uint32_t count, int32_t* d_status,
+                             void* stream) {
+    if (h_items == nullptr && count > 0) return WC_ERR_INVALID_ARG;
+    for (uint32_t i = 0; i < count; ++i) {  // validate everything before launching anything
+        const int rc = check_tans_item(h_items[i]);
+        if (rc != WC_OK) return rc;
+    }
+    wc::DecodeItem chunk[WC_BATCH_MAX];
+    for (uint32_t base = 0; base < count; base += WC_BATCH_MAX) {
+        const uint32_t c = (count - base < WC_BATCH_MAX) ? count - base : WC_BATCH_MAX;
+        for (uint32_t i = 0; i < c; ++i) chunk[i] = to_item(h_items[base + i]);
+        const cudaError_t err =
+            wc::launch_decode_tans(chunk, c, d_status, static_cast<cudaStream_t>(stream));
+        if (err != cudaSuccess) return WC_ERR_CUDA;
+    }
+    return WC_OK;
+}
+
+int wc_decompress_tans(const void* d_stream, uint64_t stream_bytes, void* d_out, uint64_t n,
+                       uint32_t chunk, int32_t* d_status, void* stream) {
+    wc_batch_item it;
+    it.stream = d_stream;
+    it.stream_bytes = stream_bytes;
+    it.out = d_out;
+    it.n = n;
+    it.block = chunk;
+    it.reserved = 0;
+    return wc_decompress_tans_batch(&it, 1, d_status, stream);
+}
+
 // The device's address of page-locked host memory (cudaHostAlloc, cudaMallocHost
 // or cudaHostRegister); nullptr for any other pointer. A host-side query: it
 // neither allocates nor synchronizes.
@@ -474,12 +588,13 @@ int wc_gemv_batch(const wc_gemv_item* h_items, uint32_t count, uint32_t n_vec, i
     return WC_OK;
 }
 
-static int check_gemm_item(const wc_gemv_item& it, uint32_t tokens) {
+static int check_gemm_item(const wc_gemv_item& it, uint32_t tokens, bool escape) {
     if (tokens < 1 || tokens > WC_GEMM_MAX_TOKENS) return WC_ERR_INVALID_ARG;
     if (!wc::block_ok(it.block) || it.reserved != 0 || it.stream == nullptr ||
         (it.rows > 0 && (it.x == nullptr || it.y == nullptr)) || it.cols == 0 ||
         it.cols % 128u != 0 || uint64_t(it.rows) * it.cols > wc::kMaxElems)
         return WC_ERR_INVALID_ARG;
+    if (escape && it.cols % it.block != 0) return WC_ERR_INVALID_ARG;  // rows of whole blocks
     if (!aligned16(it.stream) || !aligned16(it.x) || (reinterpret_cast<uintptr_t>(it.y) & 3u) != 0)
         return WC_ERR_INVALID_ARG;
     if (it.stream_bytes < wc::make_layout(uint64_t(it.rows) * it.cols, it.block).off_exp)
@@ -504,9 +619,16 @@ int wc_gemm(const void* d_stream, uint64_t stream_bytes, uint32_t rows, uint32_t
 
 int wc_gemm_batch(const wc_gemv_item* h_items, uint32_t count, uint32_t tokens, int32_t* d_status,
                   void* stream) {
+    return wc_gemm_batch_flags(h_items, count, tokens, 0, d_status, stream);
+}
+
+int wc_gemm_batch_flags(const wc_gemv_item* h_items, uint32_t count, uint32_t tokens,
+                        uint32_t flags, int32_t* d_status, void* stream) {
     if (h_items == nullptr && count > 0) return WC_ERR_INVALID_ARG;
+    if (flags != 0 && flags != WC_FLAG_ESCAPE) return WC_ERR_INVALID_ARG;
+    const bool escape = flags == WC_FLAG_ESCAPE;
     for (uint32_t i = 0; i < count; ++i) {  // check everything before launching anything
-        const int rc = check_gemm_item(h_items[i], tokens);
+        const int rc = check_gemm_item(h_items[i], tokens, escape);
         if (rc != WC_OK) return rc;
     }
     constexpr uint32_t kChunk = wc::kGemmBatchMax;
@@ -515,7 +637,7 @@ int wc_gemm_batch(const wc_gemv_item* h_items, uint32_t count, uint32_t tokens, 
         const uint32_t c = (count - base < kChunk) ? count - base : kChunk;
         for (uint32_t i = 0; i < c; ++i) chunk[i] = to_gemv_item(h_items[base + i]);
         const cudaError_t err =
-            wc::launch_gemm(chunk, c, tokens, d_status, static_cast<cudaStream_t>(stream));
+            wc::launch_gemm(chunk, c, tokens, escape, d_status, static_cast<cudaStream_t>(stream));
         if (err != cudaSuccess) return WC_ERR_CUDA;
     }
     return WC_OK;
@@ -529,8 +651,24 @@ int wc_stream_info(const void* h_header, uint64_t header_bytes, uint64_t* n, uin
     const uint32_t B = uint32_t(get_le(p + 8, 4));
     const uint64_t flags = get_le(p + 12, 4);
     if (get_le(p, 4) != wc::kMagic || get_le(p + 4, 2) != wc::kVersion ||
-        get_le(p + 6, 2) != wc::kHeaderBytes || flags > 2 || !args_ok(nn, B))
+        get_le(p + 6, 2) != wc::kHeaderBytes)
         return WC_ERR_CORRUPT_STREAM;
+    if (flags == 4) {  // tANS-coded: chunk size in the block field, table log at 88
+        const uint64_t R = get_le(p + 88, 4);
+        const uint64_t E = get_le(p + 64, 8), total = get_le(p + 72, 8);
+        if (!wc::tans_chunk_ok(B) || nn > wc::kMaxElems || R < 8 || R > 12 ||
+            get_le(p + 24, 8) != (nn + B - 1) / B || get_le(p + 32, 8) != WC_HEADER_BYTES ||
+            total != wc::tans_fixed_bytes(nn, B) + E || get_le(p + 56, 8) != wc::tans_fixed_bytes(nn, B) ||
+            get_le(p + 80, 8) != 0)
+            return WC_ERR_CORRUPT_STREAM;
+        for (int k = 92; k < 128; ++k)
+            if (p[k] != 0) return WC_ERR_CORRUPT_STREAM;
+        if (n) *n = nn;
+        if (block) *block = B;
+        if (total_bytes) *total_bytes = total;
+        return WC_OK;
+    }
+    if (flags > 2 || !args_ok(nn, B)) return WC_ERR_CORRUPT_STREAM;
     const wc::Layout L = wc::make_layout(nn, B, flags == 1);  // escape-coded: the BF16 layout
     const uint64_t E = get_le(p + 64, 8), total = get_le(p + 72, 8);
     if (get_le(p + 24, 8) != L.nb || get_le(p + 32, 8) != L.off_hdr ||

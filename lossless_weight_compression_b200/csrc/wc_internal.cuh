@@ -303,8 +303,25 @@ cudaError_t launch_gemv(const GemvItem* items, uint32_t count, uint32_t n_vec, i
 // activation rows (wc_gemm.cu); one launch per kGemmBatchMax matrices.
 constexpr uint32_t kMaxGemmTokens = 128;
 constexpr uint32_t kGemmBatchMax = 64;
-cudaError_t launch_gemm(const GemvItem* items, uint32_t count, uint32_t tokens, int32_t* status,
-                        cudaStream_t stream);
+// escape: the streams are escape-coded (then every row is whole blocks).
+cudaError_t launch_gemm(const GemvItem* items, uint32_t count, uint32_t tokens, bool escape,
+                        int32_t* status, cudaStream_t stream);
+
+// tANS-coded streams (wc_tans.cu): chunk sizes 1024..8192, the bytes of the
+// fixed sections (header, counts, chunk offsets, mantissa plane), and the
+// decoder (one launch per 256 tensors; DecodeItem::block is the chunk size).
+bool tans_chunk_ok(uint32_t C);
+uint64_t tans_fixed_bytes(uint64_t n, uint32_t C);
+cudaError_t launch_decode_tans(const DecodeItem* items, uint32_t count, int32_t* status,
+                               cudaStream_t stream);
+// The encoder: the largest stream of n elements (chunk C, table log R), the
+// workspace of a batch (2 KB per tensor + 4 bytes per chunk, per 256 tensors),
+// and five launches per 256 tensors (EncodeItem::block is the chunk size,
+// logs[i] the table log of tensor i).
+uint64_t tans_bound_bytes(uint64_t n, uint32_t C, uint32_t R);
+uint64_t tans_workspace_bytes(const EncodeItem* items, uint32_t count);
+cudaError_t launch_encode_tans(const EncodeItem* items, const uint32_t* logs, uint32_t count,
+                               void* workspace, cudaStream_t stream);
 
 // The allocation-free encoder's fixed scratch array (wc_encode.cu).
 uint64_t noalloc_max_elems();

@@ -116,6 +116,19 @@ def lib() -> ctypes.CDLL:
     L.wc_gemm.restype = i
     L.wc_gemm_batch.argtypes = [ctypes.POINTER(wc_gemv_item), u32, u32, vp, vp]
     L.wc_gemm_batch.restype = i
+    L.wc_gemm_batch_flags.argtypes = [ctypes.POINTER(wc_gemv_item), u32, u32, u32, vp, vp]
+    L.wc_gemm_batch_flags.restype = i
+    L.wc_bound_tans.argtypes, L.wc_bound_tans.restype = [u64, u32, u32], u64
+    L.wc_compress_tans_batch_workspace_size.argtypes = [ctypes.POINTER(wc_compress_item), u32]
+    L.wc_compress_tans_batch_workspace_size.restype = u64
+    L.wc_compress_tans.argtypes = [vp, u64, u32, u32, vp, u64, vp, vp, u64, vp]
+    L.wc_compress_tans.restype = i
+    L.wc_compress_tans_batch.argtypes = [ctypes.POINTER(wc_compress_item), u32, u32, vp, u64, vp]
+    L.wc_compress_tans_batch.restype = i
+    L.wc_decompress_tans.argtypes = [vp, u64, vp, u64, u32, vp, vp]
+    L.wc_decompress_tans.restype = i
+    L.wc_decompress_tans_batch.argtypes = [ctypes.POINTER(wc_batch_item), u32, vp, vp]
+    L.wc_decompress_tans_batch.restype = i
     L.wc_compress_noalloc.argtypes = [vp, u64, u32, vp, u64, vp, vp, vp]
     L.wc_compress_noalloc.restype = i
     L.wc_debug_compress_stalled.argtypes = [vp, u64, u32, vp, u64, vp, vp, u64, vp, u64, vp]
@@ -207,6 +220,36 @@ def wc_decompress_fp32(d_stream, stream_bytes, d_out, n, block, d_status, stream
 def wc_gemm(d_stream, stream_bytes, rows, cols, block, d_x, tokens, d_y, d_status, stream) -> int:
     return lib().wc_gemm(d_stream, stream_bytes, rows, cols, block, d_x, tokens, d_y, d_status,
                          stream)
+
+
+def wc_bound_tans(n, chunk, table_log) -> int:
+    return lib().wc_bound_tans(n, chunk, table_log)
+
+
+def wc_compress_tans_batch_workspace_size(items, count) -> int:
+    return lib().wc_compress_tans_batch_workspace_size(items, count)
+
+
+def wc_compress_tans(d_in, n, chunk, table_log, d_out, out_capacity, d_out_bytes, d_ws, ws_bytes,
+                     stream) -> int:
+    return lib().wc_compress_tans(d_in, n, chunk, table_log, d_out, out_capacity, d_out_bytes,
+                                  d_ws, ws_bytes, stream)
+
+
+def wc_compress_tans_batch(items, count, table_log, d_ws, ws_bytes, stream) -> int:
+    return lib().wc_compress_tans_batch(items, count, table_log, d_ws, ws_bytes, stream)
+
+
+def wc_decompress_tans(d_stream, stream_bytes, d_out, n, chunk, d_status, stream) -> int:
+    return lib().wc_decompress_tans(d_stream, stream_bytes, d_out, n, chunk, d_status, stream)
+
+
+def wc_decompress_tans_batch(items, count, d_status, stream) -> int:
+    return lib().wc_decompress_tans_batch(items, count, d_status, stream)
+
+
+def wc_gemm_batch_flags(items, count, tokens, flags, d_status, stream) -> int:
+    return lib().wc_gemm_batch_flags(items, count, tokens, flags, d_status, stream)
 
 
 def wc_gemm_batch(items, count, tokens, d_status, stream) -> int:
@@ -376,11 +419,17 @@ def decompress_compressed(c: Compressed, out: torch.Tensor | None = None, status
 class CompressBatch:
     """Reusable buffers and descriptors for compressing a fixed list of tensors
     in one call: ``run()`` enqueues one encoder launch per 512 tensors (five for
-    escape-coded streams, ``escape=True``)."""
+    escape-coded streams, ``escape=True``; five per 512 for tANS-coded streams,
+    ``tans_log=R``, whose ``block`` is then the chunk size)."""
 
-    def __init__(self, tensors, block=1024, escape=False):
+    def __init__(self, tensors, block=1024, escape=False, tans_log=None):
         self.escape = escape
-        bound = wc_bound_escape if escape else wc_bound
+        self.tans_log = tans_log
+        if tans_log is not None:
+            def bound(n, b):
+                return wc_bound_tans(n, b, tans_log)
+        else:
+            bound = wc_bound_escape if escape else wc_bound
         self.words = [as_words(t) for t in tensors]
         dev = self.words[0].device if self.words else torch.device("cuda")
         k = len(self.words)
@@ -400,14 +449,23 @@ class CompressBatch:
             it.out = self.buffers[j].data_ptr()
             it.out_capacity = self.buffers[j].numel()
             it.out_bytes = self.nbytes[j:].data_ptr()
-        ws = (wc_compress_escape_batch_workspace_size if escape
-              else wc_compress_batch_workspace_size)(self.items, k)
+        if tans_log is not None:
+            ws = wc_compress_tans_batch_workspace_size(self.items, k)
+        else:
+            ws = (wc_compress_escape_batch_workspace_size if escape
+                  else wc_compress_batch_workspace_size)(self.items, k)
         if k and ws == 0:
             raise WcodecError(WC_ERR_INVALID_ARG, "workspace size")
         self.workspace = torch.empty(max(16, (ws + 15) // 16 * 16), dtype=torch.uint8, device=dev)
         self.count = k
 
     def run(self, stream=None):
+        if self.tans_log is not None:
+            rc = wc_compress_tans_batch(self.items, self.count, self.tans_log,
+                                        self.workspace.data_ptr(), self.workspace.numel(),
+                                        _stream_handle(stream))
+            _check(rc, "wc_compress_tans_batch")
+            return
         entry = wc_compress_escape_batch if self.escape else wc_compress_batch
         rc = entry(self.items, self.count, self.workspace.data_ptr(), self.workspace.numel(),
                    self.status.data_ptr(), _stream_handle(stream))
@@ -502,11 +560,13 @@ def gemm(stream_bytes: torch.Tensor, rows: int, cols: int, block: int, x: torch.
     return y
 
 
-def gemm_batch(batch, tokens: int, status: torch.Tensor, stream=None):
-    """batch from make_gemv_batch (x (tokens, cols), y (tokens, rows) per item)."""
+def gemm_batch(batch, tokens: int, status: torch.Tensor, stream=None, escape: bool = False):
+    """batch from make_gemv_batch (x (tokens, cols), y (tokens, rows) per item);
+    escape: the streams are escape-coded (every row whole blocks)."""
     arr, count = batch
-    rc = wc_gemm_batch(arr, count, tokens, status.data_ptr(), _stream_handle(stream))
-    _check(rc, "wc_gemm_batch")
+    rc = wc_gemm_batch_flags(arr, count, tokens, WC_FLAG_ESCAPE if escape else 0,
+                             status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_gemm_batch_flags")
 
 
 def compress_fp32(x: torch.Tensor, block: int = 1024, *, workspace: torch.Tensor | None = None,
@@ -607,3 +667,29 @@ def decompress_host_batch(batch, status: torch.Tensor, escape: bool = False, str
     rc = wc_decompress_host_batch(arr, count, WC_FLAG_ESCAPE if escape else 0,
                                   status.data_ptr(), _stream_handle(stream))
     _check(rc, "wc_decompress_host_batch")
+
+
+def decompress_tans_batch(batch, status: torch.Tensor, stream=None):
+    """Decode tANS-coded streams (a batch from ``make_batch``, block = the chunk
+    size), one launch per 256."""
+    arr, count = batch
+    rc = wc_decompress_tans_batch(arr, count, status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_decompress_tans_batch")
+
+
+def decompress_tans(stream_bytes: torch.Tensor, n: int, chunk: int, *,
+                    out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                    nbytes: int | None = None, stream=None) -> torch.Tensor:
+    """Decode a tANS-coded stream into n 16-bit values (``out`` if given)."""
+    if out is None:
+        out = torch.empty(n, dtype=torch.bfloat16, device=stream_bytes.device)
+    words = out.view(-1)
+    if words.numel() != n or not words.is_contiguous() or out.element_size() != 2:
+        raise ValueError("out must be a contiguous 16-bit tensor of %d elements" % n)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=stream_bytes.device)
+    size = stream_bytes.numel() if nbytes is None else nbytes
+    rc = wc_decompress_tans(stream_bytes.data_ptr(), size, words.data_ptr() if n else None, n,
+                            chunk, status.data_ptr(), _stream_handle(stream))
+    _check(rc, "wc_decompress_tans")
+    return out

@@ -12,7 +12,9 @@ rows.
 
 Shapes: the ragged ones of the bound tests (row tails, blocks shorter and
 longer than a row, every 128-column slice) and a full Llama-3-8B-shaped layer
-(cols 4096 and 14336, the widths of the benchmark).
+(cols 4096 and 14336, the widths of the benchmark). The tensor-core product is
+also run on escape-coded streams (wc_gemm_batch_flags), whose expected weights
+are the oracle's decode of its own escape-coded stream.
 """
 import numpy as np
 import pytest
@@ -29,10 +31,14 @@ GEMM_SHAPES = [(1, 128, 128), (7, 1024, 512), (130, 384, 128), (256, 4096, 1024)
                (33, 9216, 2048)]
 GEMV_SHAPES = [(1, 128, 128), (7, 1024, 512), (64, 4096, 1024), (33, 14336, 1024),
                (5, 9216, 1024), (3, 16384, 4096), (129, 256, 128), (1000, 2048, 2048)]
+# escape-coded streams: rows of whole blocks
+ESC_SHAPES = [(1, 128, 128), (7, 1024, 512), (130, 384, 128), (256, 4096, 1024),
+              (300, 1280, 256), (129, 14336, 1024), (64, 4096, 4096), (200, 512, 256)]
 
 
-def decoded_f32(orc, stream, rows, cols, B):
-    w = orc.decompress(stream, rows * cols, B).reshape(rows, cols)
+def decoded_f32(orc, stream, rows, cols, B, escape=False):
+    dec = orc.decompress_escape if escape else orc.decompress
+    w = dec(stream, rows * cols, B).reshape(rows, cols)
     return (w.astype(np.uint32) << 16).view(np.float32)
 
 
@@ -42,7 +48,8 @@ def one_hot(cols, device):
     return x
 
 
-def run_one_hot(wc, kind, s_dev, size, rows, cols, B, device, per_call, columns=None):
+def run_one_hot(wc, kind, s_dev, size, rows, cols, B, device, per_call, columns=None,
+                escape=False):
     """Y (len(columns) x rows) with row j the product of e_{columns[j]}."""
     cols_idx = np.arange(cols) if columns is None else np.asarray(columns)
     eye = one_hot(cols, device)
@@ -55,7 +62,11 @@ def run_one_hot(wc, kind, s_dev, size, rows, cols, B, device, per_call, columns=
     status = torch.zeros(1, dtype=torch.int32, device=device)
     full = [it for k, it in items if k == per_call]
     tail = [it for k, it in items if k != per_call]
-    batch_fn = wc.gemm_batch if kind == "gemm" else wc.gemv_batch
+    if kind == "gemm":
+        def batch_fn(batch, n, st):
+            wc.gemm_batch(batch, n, st, escape=escape)
+    else:
+        batch_fn = wc.gemv_batch
     if full:
         batch_fn(wc.make_gemv_batch(full), per_call, status)
     for s_, sz, x, y, r, c, b in tail:
@@ -128,6 +139,42 @@ def test_gemm_one_hot_special_weights(orc, wclib, cuda):
         assert np.array_equal(Y.T, expect), kind
 
 
+@pytest.mark.parametrize("rows,cols,B", ESC_SHAPES)
+def test_gemm_one_hot_every_column_escape_coded(orc, wclib, cuda, rows, cols, B):
+    rng = np.random.default_rng(rows * 13 + cols + B)
+    W = rand_bf16(rng, (rows, cols), 0.02)
+    stream = orc.compress_escape(W.reshape(-1), B)
+    expect = decoded_f32(orc, stream, rows, cols, B, escape=True)
+    s = torch.from_numpy(stream).to(cuda)
+    Y, _ = run_one_hot(wclib, "gemm", s, stream.size, rows, cols, B, cuda, 128, escape=True)
+    assert np.array_equal(Y.T, expect)
+
+
+def test_gemm_one_hot_escape_coded_many_exceptions(orc, wclib, cuda):
+    """Blocks of every kind in an escape-coded stream: long exception lists
+    (exponents spread over the whole range in one element of ten, so that a
+    block's list outgrows the bytes staged per row), constant rows (w = 0),
+    raw rows (w = 8), zeros and denormals."""
+    rng = np.random.default_rng(61)
+    rows, cols, B = 256, 2048, 512
+    W = rand_bf16(rng, (rows, cols), 0.02)
+    pick = rng.random((64, cols)) < 0.1
+    e = rng.integers(0, 255, size=(64, cols))
+    sm = rng.integers(0, 256, size=(64, cols))
+    W[:64] = np.where(pick, ((sm & 0x80) << 8) | (e << 7) | (sm & 0x7F), W[:64])
+    e = rng.integers(0, 255, size=(16, cols))
+    sm = rng.integers(0, 256, size=(16, cols))
+    W[64:80] = ((sm & 0x80) << 8) | (e << 7) | (sm & 0x7F)    # raw blocks
+    W[80:96] = 0x3F80
+    W[96:112] = 0x8000
+    W[112:128] = rng.integers(0, 128, size=(16, cols))
+    stream = orc.compress_escape(W.reshape(-1), B)
+    expect = decoded_f32(orc, stream, rows, cols, B, escape=True)
+    s = torch.from_numpy(stream).to(cuda)
+    Y, _ = run_one_hot(wclib, "gemm", s, stream.size, rows, cols, B, cuda, 128, escape=True)
+    assert np.array_equal(Y.T, expect)
+
+
 @pytest.fixture(scope="module")
 def layer(orc, cuda):
     """A full Llama-3-8B-shaped layer, its oracle streams on the device and the
@@ -149,4 +196,18 @@ def test_fused_one_hot_full_layer_every_weight(wclib, cuda, layer, kind, per_cal
     B, mats = layer
     for name, rows, cols, s, size, expect in mats:
         Y, _ = run_one_hot(wclib, kind, s, size, rows, cols, B, cuda, per_call)
+        assert np.array_equal(Y.T, expect), name
+
+
+def test_gemm_one_hot_full_layer_escape_coded(orc, wclib, cuda):
+    """The same layer as escape-coded streams, every weight through the tensor cores."""
+    from lossless_weight_compression_b200 import synth
+    B = 1024
+    for name, t in synth.layer_tensors(4, "cpu"):
+        rows, cols = t.shape
+        W = t.view(torch.int16).numpy().view(np.uint16).reshape(-1)
+        stream = orc.compress_escape(W, B)
+        expect = decoded_f32(orc, stream, rows, cols, B, escape=True)
+        s = torch.from_numpy(stream).to(cuda)
+        Y, _ = run_one_hot(wclib, "gemm", s, stream.size, rows, cols, B, cuda, 128, escape=True)
         assert np.array_equal(Y.T, expect), name

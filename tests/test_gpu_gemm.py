@@ -203,3 +203,111 @@ def test_gemm_refuses_escape_coded_stream(orc, wclib, cuda):
     y, status = run_gpu(wclib, stream, rows, cols, B, x, cuda)
     assert status == 0
     check_bound(y, y_ref, absum, cols)
+
+
+# ---------------------------------------------------------------------------
+# escape-coded streams through wc_gemm_batch_flags
+# ---------------------------------------------------------------------------
+def esc_reference(orc, stream, rows, cols, B, x):
+    """float64 product of the oracle's decode of an escape-coded stream."""
+    from oracle import bf16_to_f64
+    W = bf16_to_f64(orc.decompress_escape(stream, rows * cols, B)).reshape(rows, cols)
+    xf = bf16_to_f64(np.asarray(x, dtype=np.uint16).reshape(-1, cols))
+    with np.errstate(invalid="ignore", over="ignore"):
+        return xf @ W.T, np.abs(xf) @ np.abs(W).T
+
+
+def run_gpu_escape(wc, stream_np, rows, cols, B, x_np, device, nbytes=None):
+    s = torch.from_numpy(stream_np).to(device)
+    x = torch.from_numpy(x_np.view(np.int16)).to(device)
+    y = torch.empty((x_np.shape[0], rows), dtype=torch.float32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    batch = wc.make_gemv_batch([(s, stream_np.size if nbytes is None else nbytes, x, y, rows, cols,
+                                 B)])
+    wc.gemm_batch(batch, x_np.shape[0], status, escape=True)
+    torch.cuda.synchronize()
+    return y.cpu().numpy().astype(np.float64), int(status.item())
+
+
+@pytest.mark.parametrize("rows,cols,B", [(7, 1024, 512), (130, 384, 128), (256, 4096, 1024),
+                                         (129, 14336, 1024), (64, 4096, 4096)])
+@pytest.mark.parametrize("tokens", [1, 16, 64, 128])
+def test_gemm_escape_coded_matches_oracle(orc, wclib, cuda, rows, cols, B, tokens):
+    rng = np.random.default_rng(rows * 17 + cols + tokens)
+    W = rand_bf16(rng, (rows, cols), 0.02)
+    W[rng.random((rows, cols)) < 0.002] = 0x4580  # outliers: exceptions in most blocks
+    x = rand_bf16(rng, (tokens, cols), 1.0)
+    stream = orc.compress_escape(W.reshape(-1), B)
+    y_ref, absum = esc_reference(orc, stream, rows, cols, B, x)
+    y, status = run_gpu_escape(wclib, stream, rows, cols, B, x, cuda)
+    assert status == 0
+    check_bound(y, y_ref, absum, cols)
+    y2, _ = run_gpu_escape(wclib, stream, rows, cols, B, x, cuda)
+    assert np.array_equal(y, y2)
+
+
+def test_gemm_escape_coded_arguments_and_kinds(orc, wclib, cuda):
+    """Rows that are not whole blocks and unknown flags are refused on the host;
+    a plain stream multiplied as escape-coded (and the reverse) is corrupt."""
+    rng = np.random.default_rng(62)
+    rows, cols, B = 64, 1024, 512
+    W = rand_bf16(rng, (rows, cols), 0.02)
+    x = rand_bf16(rng, (16, cols), 1.0)
+    esc = orc.compress_escape(W.reshape(-1), B)
+    s = torch.from_numpy(esc).to(cuda)
+    xt = torch.from_numpy(x.view(np.int16)).to(cuda)
+    y = torch.empty((16, rows), dtype=torch.float32, device=cuda)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda)
+    arr, n = wclib.make_gemv_batch([(s, esc.size, xt, y, rows, cols, 2048)])  # 1024 % 2048 != 0
+    assert wclib.wc_gemm_batch_flags(arr, n, 16, 2, status.data_ptr(), None) == wclib.WC_ERR_INVALID_ARG
+    arr, n = wclib.make_gemv_batch([(s, esc.size, xt, y, rows, cols, B)])
+    assert wclib.wc_gemm_batch_flags(arr, n, 16, 1, status.data_ptr(), None) == wclib.WC_ERR_INVALID_ARG
+    _, st = run_gpu_escape(wclib, orc.compress(W, B), rows, cols, B, x, cuda)
+    assert st == 3
+    _, st = run_gpu(wclib, esc, rows, cols, B, x, cuda)
+    assert st == 3
+    y_ref, absum = esc_reference(orc, esc, rows, cols, B, x)
+    yy, st = run_gpu_escape(wclib, esc, rows, cols, B, x, cuda)
+    assert st == 0
+    check_bound(yy, y_ref, absum, cols)
+
+
+def test_gemm_escape_coded_reports_corruption(orc, wclib, cuda):
+    """Corrupt escape-coded streams are reported and every read stays inside
+    the stream; the device stays usable."""
+    rng = np.random.default_rng(63)
+    rows, cols, B = 128, 1024, 256
+    W = rand_bf16(rng, (rows, cols), 0.02)
+    W[rng.random((rows, cols)) < 0.01] = 0x4580
+    x = rand_bf16(rng, (16, cols), 1.0)
+    esc = orc.compress_escape(W.reshape(-1), B)
+    nb = rows * cols // B
+    hdr = esc[128:128 + 2 * nb].view(np.uint16)
+    off_offs = 128 + (2 * nb + 127) // 128 * 128
+    off_exp = off_offs + (4 * nb + 127) // 128 * 128 + rows * cols
+    offs = esc[off_offs:off_offs + 4 * nb].view(np.uint32)
+    psize = 16 * np.diff(offs.astype(np.int64))
+    b = int(np.flatnonzero(((hdr[:-1] >> 8) == 3) & (psize > (B // 8) * 3))[0])  # w = 3, K >= 1
+    cases = []
+    bad = esc.copy()
+    bad[128 + 2 * b] = 255                      # base above 255 - (2^w - 1)
+    cases.append(bad)
+    bad = esc.copy()
+    bad[128 + 2 * b + 1] = 9                    # w = 9
+    cases.append(bad)
+    bad = esc.copy()
+    start = off_exp + 16 * int(offs[b]) + (B // 8) * 3
+    bad[start] = hdr[b] & 0xFF                  # an exception inside the window
+    cases.append(bad)
+    bad = esc.copy()
+    bad[off_offs + 4 * 1: off_offs + 8] = np.frombuffer(np.uint32(1 << 28).tobytes(), np.uint8)
+    cases.append(bad)                           # offset far past the end
+    for k, bad in enumerate(cases):
+        _, st = run_gpu_escape(wclib, bad, rows, cols, B, x, cuda)
+        assert st == 3, k
+    _, st = run_gpu_escape(wclib, esc, rows, cols, B, x, cuda, nbytes=esc.size - 32)
+    assert st == 3
+    y_ref, absum = esc_reference(orc, esc, rows, cols, B, x)
+    y, st = run_gpu_escape(wclib, esc, rows, cols, B, x, cuda)
+    assert st == 0
+    check_bound(y, y_ref, absum, cols)
