@@ -43,7 +43,7 @@
 #include <algorithm>
 #include <mutex>
 
-#include "wc_decode_core.cuh"
+#include "wc_escape_core.cuh"
 
 namespace wc {
 namespace {
@@ -632,6 +632,20 @@ __device__ __forceinline__ uint32_t quad_bytes(uint32_t q, uint32_t w, uint32_t 
     return (prmt(t1, t2, 0x7610u) & m1x4) + base4;
 }
 
+// Octet of width W (compile time, at most 5) starting at byte q of a staged row:
+// its eight values as bytes, value t in byte t % 4 of word t / 4. 8W <= 40
+// bits starting at most 24 bits into a word lie in two words.
+template <int W>
+__device__ __forceinline__ void octet_bytes(const uint8_t* raw, uint32_t q, uint32_t& a,
+                                            uint32_t& b) {
+    const uint32_t* s32 = reinterpret_cast<const uint32_t*>(raw);
+    const uint32_t i = q >> 2;
+    const uint64_t v = ((uint64_t(s32[i + 1]) << 32) | s32[i]) >> ((q & 3u) * 8u);
+    constexpr uint32_t kQuad = (1u << (4 * W)) - 1u;
+    a = quad_to_bytes<W>(uint32_t(v) & kQuad);
+    b = quad_to_bytes<W>(uint32_t(v >> (4 * W)) & kQuad);
+}
+
 // Bit 7 of each byte of c whose value is m4's (m4 = the byte m in all four).
 __device__ __forceinline__ uint32_t bytes_equal(uint32_t c, uint32_t m4) {
     const uint32_t z = c ^ m4;
@@ -688,13 +702,19 @@ __device__ void gemm_transcode(const GemmParams<MAXI>& P, const GemmSmem& S, int
             const uint32_t w = mw[k] & 0xFFu, base = (mw[k] >> 8) & 0xFFu;
             const uint32_t base4 = ESC ? 0u : base * 0x01010101u;  // ESC: added after the escapes
             uint32_t e[4];
-            if (__all_sync(0xFFFFFFFFu, w == 4u)) {
+            // one width for the whole step (the common case): a path for it
+            const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, w, 0);
+            const bool same = __all_sync(0xFFFFFFFFu, w == w0);
+            if (same && w0 == 4u) {
 #pragma unroll
                 for (uint32_t h = 0; h < 2; ++h) {
                     const uint32_t ev = f[k][h] & 0x0F0F0F0Fu, od = (f[k][h] >> 4) & 0x0F0F0F0Fu;
                     e[2 * h] = prmt(ev, od, 0x5140u) + base4;
                     e[2 * h + 1] = prmt(ev, od, 0x7362u) + base4;
                 }
+            } else if (ESC && same && w0 == 3u) {  // escape-coded Gaussian blocks: width 3
+                octet_bytes<3>(raw, rr * kExpPitch + 3u * o0, e[0], e[1]);
+                octet_bytes<3>(raw, rr * kExpPitch + 3u * o1, e[2], e[3]);
             } else {
                 const uint32_t* s32 = reinterpret_cast<const uint32_t*>(raw);
                 const uint32_t m1x4 = ((1u << w) - 1u) * 0x01010101u;

@@ -159,3 +159,48 @@ def test_corrupt_streams_are_reported(orc, wclib, cuda):
         assert st in (0, 3)
     back, st = gpu_decode(wclib, [s], [n], C, cuda)             # the device is still usable
     assert st == 0 and np.array_equal(back[0], w)
+
+
+def test_corruption_verdict_matches_the_oracle(orc, wclib, cuda):
+    """Byte flips anywhere, and many in the header, counts, offsets and chunk
+    payloads: the GPU decoder reports a corrupt stream exactly when the oracle
+    does (a flip in the mantissa plane corrupts nothing; one in an unused
+    padding byte or a word does)."""
+    rng = np.random.default_rng(12)
+    n, C = 5000, 1024
+    w = gauss_words(rng, n)
+    s = orc.compress_tans(w, C, 11)
+    nb = -(-n // C)
+    off_man = 128 + 512 + (4 * nb + 127) // 128 * 128
+    off_exp = off_man + (n + 127) // 128 * 128
+    where = np.concatenate([rng.integers(0, s.size, 150), rng.integers(0, off_man, 100),
+                            rng.integers(off_man + n, off_exp, 20),
+                            rng.integers(off_exp, s.size, 250)])
+    corrupt = 0
+    for k, pos in enumerate(where):
+        b = s.copy()
+        b[int(pos)] ^= int(rng.integers(1, 256))
+        rc, ref = orc.decompress_tans_status(b, n, C)
+        got, st = gpu_decode(wclib, [b], [n], C, cuda)
+        assert st == (0 if rc == 0 else 3), (k, int(pos), rc, st)
+        if rc == 0:
+            assert np.array_equal(got[0], ref), (k, int(pos))
+        corrupt += rc != 0
+    assert corrupt > 300
+
+
+@pytest.mark.parametrize("C", CHUNKS)
+def test_staged_and_unstaged_chunks_in_one_tensor(orc, wclib, cuda, C):
+    """Chunks of Gaussian weights (payload about C/3 bytes, staged in shared
+    memory) next to chunks of uniformly spread exponents (payload near C bytes,
+    read from global memory), in one tensor and one launch."""
+    rng = np.random.default_rng(C + 3)
+    n = 9 * C + 123
+    w = gauss_words(rng, n)
+    for c in range(1, 10, 3):
+        w[c * C:(c + 1) * C] = rng.integers(0, 65536, C)
+    ref = orc.compress_tans(w, C, 12)
+    got = gpu_encode(wclib, [w], C, 12, cuda)[0]
+    assert np.array_equal(got, ref)
+    back, st = gpu_decode(wclib, [ref], [n], C, cuda)
+    assert st == 0 and np.array_equal(back[0], w)
