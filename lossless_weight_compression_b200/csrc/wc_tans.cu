@@ -20,10 +20,11 @@
 // block (8 warps) works through a contiguous range of 8-chunk tiles; it builds
 // the tensor's decoding table in shared memory whenever its tiles move to a
 // new tensor, and each warp stages its chunk's payload and mantissa bytes with
-// one bulk copy (payloads larger than C + 512 bytes, which only
-// incompressible chunks reach, are read from global memory instead). Every
-// read of the stream is checked against its bounds; a stream that breaks the
-// format writes WC_ERR_CORRUPT_STREAM to the status word.
+// one bulk copy (payloads larger than C/2 + 512 bytes, which only poorly
+// compressible chunks reach, are read from global memory instead). A full
+// chunk runs a step loop without per-element bounds tests: word indices are
+// clamped into the payload and the chunk is checked once at its end. A stream
+// that breaks the format writes WC_ERR_CORRUPT_STREAM to the status word.
 #include <mutex>
 
 #include "wc_decode_core.cuh"
@@ -36,7 +37,24 @@ constexpr int kTansThreads = 32 * kTansWarps;
 constexpr uint32_t kTansMaxLog = 12;
 constexpr uint32_t kTansMinLog = 8;
 constexpr uint32_t kTansTable = 1u << kTansMaxLog;  // entries
-constexpr uint32_t kTansSlack = 512;                // staged payload: C + 512 bytes
+constexpr uint32_t kTansSlack = 512;
+
+// Staged payload bytes per warp for chunk size C: a payload of Gaussian
+// weights takes about C/3 bytes; larger ones are read from global memory.
+__host__ __device__ constexpr uint32_t tans_pay_stage(uint32_t C) { return C / 2 + kTansSlack; }
+// per warp: the payload stage, then the chunk's mantissa bytes
+__host__ __device__ constexpr uint32_t tans_stage_bytes(uint32_t C) { return tans_pay_stage(C) + C; }
+// A full chunk takes at most one word per lane every other step (a word
+// leaves at least 32 - 12 bits after the step that takes it): 16 words per
+// step, C/2 words in all. A lane reads word index at most C/2 (a lane that
+// takes none reads the index after the pair's last), i.e. below 68 + 2C bytes
+// past the start of the warp's payload stage. The allocation extends that far
+// past the last warp's stage, so word reads of the staged path need no clamp:
+// a corrupt chunk reads stale bytes inside the block's shared memory and fails
+// its end checks.
+__host__ __device__ constexpr uint32_t tans_read_slack(uint32_t C) {
+    return 80u + 2u * C > tans_stage_bytes(C) ? 80u + 2u * C - tans_stage_bytes(C) : 0u;
+}
 
 template <int MAXI>
 struct TansParams {
@@ -82,12 +100,12 @@ __device__ __forceinline__ uint32_t tans_find_item(const TansParams<MAXI>& P, ui
 }
 
 struct TansShared {
-    uint32_t* table;   // kTansTable entries: exponent | bits << 8 | next << 16
+    uint32_t* table;   // kTansTable entries: bits | exponent << 7 | 4 next << 18
     uint32_t* cum;     // 257 cumulative counts
     uint32_t* seen;    // 256 running occurrence counts (table build)
     uint32_t* info;    // [0] R, [1] the tensor is usable (1) or not (0)
     unsigned long long* bar;  // one per warp
-    uint8_t* stage;    // per warp: payload (C + kTansSlack) then mantissa (C)
+    uint8_t* stage;    // per warp: tans_stage_bytes(max chunk)
 };
 
 // The container header and the counts of item I: checks, then the decoding
@@ -124,7 +142,15 @@ __device__ void tans_build(const TansParams<MAXI>& P, const DecodeItem& I, TansS
         if (lane >= d) incl += y;
     }
     if (lane == 31) S.seen[warp] = incl;  // warp totals, briefly
-    __syncthreads();
+    // the zero padding after the chunk offsets and after the mantissa plane
+    // (each under 128 bytes; inside the stream once the header is valid)
+    bool pad_bad = false;
+    if (S.info[1]) {
+        const uint64_t o1 = L.off_offs + 4 * L.nb, o2 = L.off_man + I.n;
+        if (uint64_t(tid) < L.off_man - o1) pad_bad |= st[o1 + tid] != 0;
+        if (uint64_t(tid) < L.off_exp - o2) pad_bad |= st[o2 + tid] != 0;
+    }
+    const bool any_pad_bad = __syncthreads_or(pad_bad) != 0;
     uint32_t before = 0;
     for (int k = 0; k < warp; ++k) before += S.seen[k];
     __syncthreads();
@@ -133,7 +159,7 @@ __device__ void tans_build(const TansParams<MAXI>& P, const DecodeItem& I, TansS
         S.seen[tid] = f;  // occurrence counters start at f
         if (tid == 255) {
             S.cum[256] = before + incl;
-            if (before + incl != Lst || S.info[1] == 0) {
+            if (before + incl != Lst || S.info[1] == 0 || any_pad_bad) {
                 if (S.info[1]) report(P.status, kStatusCorrupt);
                 S.info[1] = 0;
             }
@@ -165,11 +191,106 @@ __device__ void tans_build(const TansParams<MAXI>& P, const DecodeItem& I, TansS
             __syncwarp();
             if ((grp >> lane) == 1u) S.seen[e] = v + 1u;  // the group's highest lane
             const uint32_t nb = R - (31u - __clz(v));
-            S.table[X] = e | (nb << 8) | (((v << nb) - Lst) << 16);
+            S.table[X] = nb | (e << 7) | ((((v << nb) - Lst) * 4u) << 18);
             __syncwarp();
         }
     }
     __syncthreads();
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u8(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+// the low n bits set (n <= 32)
+__device__ __forceinline__ uint32_t low_mask(uint32_t n) {
+    uint32_t m;
+    asm("bmsk.clamp.b32 %0, 0, %1;" : "=r"(m) : "r"(n));
+    return m;
+}
+
+// One lane's decoder: the shared-memory address of its state's table entry,
+// its bit buffer (hi:lo, cnt bits, nothing above them) and the number of words
+// the warp has taken. At a refill cnt < R <= 12, so hi is zero then.
+struct TansLane {
+    uint32_t xa, lo, hi, cnt, p;
+};
+
+// A word taken while fewer than 32 bits are held (hi is zero then) goes above them.
+__device__ __forceinline__ void tans_insert(TansLane& d, uint32_t w) {
+    d.lo |= w << d.cnt;
+    d.hi = __funnelshift_l(w, 0u, d.cnt);  // w >> (32 - cnt), 0 for cnt = 0
+    d.cnt += 32u;
+}
+
+// The element of table entry t: read its bits, move to the next state, write
+// the BF16 word (sign and mantissa bits from the staged byte at ma, exponent
+// bits from the entry, in one select).
+__device__ __forceinline__ void tans_decode(TansLane& d, uint32_t t, uint32_t tbase, uint32_t ma,
+                                            uint16_t* o) {
+    const uint32_t nb = t & 15u;
+    d.xa = tbase + (t >> 18) + ((d.lo & low_mask(nb)) << 2);
+    d.lo = __funnelshift_r(d.lo, d.hi, nb);
+    d.hi >>= nb;
+    d.cnt -= nb;
+    const uint32_t x = lds_u8(ma) * 0x101u;  // the byte twice: sign at bit 15
+    *o = uint16_t((x & 0x807Fu) | (t & 0x7F80u));
+}
+
+// One step of lane `lane` for element i: refill (words in lane order among the
+// lanes holding fewer than R bits; the index is clamped into the payload, so a
+// corrupt stream reads stale words and is caught by the word count at the end),
+// then one table lookup: exponent, bits to read, next state. A table entry is
+// nb | e << 7 | 4 next << 18; the output takes the sign and mantissa bits of s
+// and the exponent bits of the entry in one select.
+template <bool STAGED, bool ACTIVE_CHECK>
+__device__ __forceinline__ void tans_step(TansLane& d, bool active, uint32_t tbase,
+                                          const uint32_t* wg, uint32_t ws, uint32_t last,
+                                          uint32_t R, uint32_t lt, uint32_t ma, uint16_t* o) {
+    const bool need = (!ACTIVE_CHECK || active) && d.cnt < R;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
+    const uint32_t q = min(d.p + __popc(m & lt), last);
+    const uint32_t w = STAGED ? lds_u32(ws + 4u * q) : __ldg(wg + q);
+    if (need) tans_insert(d, w);
+    d.p += __popc(m);
+    if (!ACTIVE_CHECK || active) tans_decode(d, lds_u32(d.xa), tbase, ma, o);
+}
+
+// Two steps of a full chunk with one word load: a lane that takes a word at a
+// step holds at least 32 - 12 bits at the next one, so it takes at most one
+// word per pair of steps. Its need at the second step follows from the first
+// step's bit count (table entry already read), and a word it takes there may
+// enter the buffer a step early: it goes above the bits the first step reads,
+// and with fewer than R + 12 <= 24 bits held it fits in the 64-bit buffer. The
+// second step's words follow the first step's in the shared stream. STAGED:
+// no clamp; the shared-memory allocation extends far enough past the payload
+// for the most words any chunk can take (16 per step).
+template <bool STAGED>
+__device__ __forceinline__ void tans_pair(TansLane& d, uint32_t tbase, const uint32_t* wg,
+                                          uint32_t ws, uint32_t last, uint32_t R, uint32_t lt,
+                                          uint32_t ma, uint16_t* o) {
+    const uint32_t t0 = lds_u32(d.xa);
+    const bool need0 = d.cnt < R;
+    const bool need1 = !need0 && d.cnt - (t0 & 15u) < R;
+    const uint32_t m0 = __ballot_sync(0xFFFFFFFFu, need0);
+    const uint32_t m1 = __ballot_sync(0xFFFFFFFFu, need1);
+    const uint32_t c0 = __popc(m0);
+    uint32_t q = d.p + (need0 ? __popc(m0 & lt) : c0 + __popc(m1 & lt));
+    if (!STAGED) q = min(q, last);
+    const uint32_t w = STAGED ? lds_u32(ws + 4u * q) : __ldg(wg + q);
+    if (need0 || need1) tans_insert(d, w);
+    d.p += c0 + __popc(m1);
+    tans_decode(d, t0, tbase, ma, o);
+    tans_decode(d, lds_u32(d.xa), tbase, ma + 32u, o + 32);
 }
 
 // Decode chunk c of item I with warp `warp` (all 32 lanes).
@@ -181,21 +302,23 @@ __device__ void tans_chunk(const TansParams<MAXI>& P, const DecodeItem& I, uint6
     const TansLayout L = tans_layout(I.n, C);
     const uint32_t R = S.info[0], Lst = 1u << R;
     const uint64_t E = ld_u64(st + 64);
-    const uint64_t start = 16ull * reinterpret_cast<const uint32_t*>(st + L.off_offs)[c];
-    const uint64_t end = c + 1 < L.nb ? 16ull * reinterpret_cast<const uint32_t*>(st + L.off_offs)[c + 1] : E;
+    const uint32_t* offs = reinterpret_cast<const uint32_t*>(st + L.off_offs);
+    const uint64_t start = 16ull * offs[c];
+    const uint64_t end = c + 1 < L.nb ? 16ull * offs[c + 1] : E;
     const uint32_t len = uint32_t(min(uint64_t(C), I.n - c * C));
-    // E lies inside the stream (header check); a chunk payload is a whole number
-    // of 16-byte units of at least 64 bytes (the states)
-    if (start > end || end > E || end - start < 64u || (end & 15u) != 0u) {
+    // E lies inside the stream (header check); the chunks follow one another
+    // from offset 0; a chunk payload is a whole number of 16-byte units holding
+    // the 64 bytes of states and at least one word (lane 0 takes one at step 0)
+    if ((c == 0 && start != 0) || start > end || end > E || end - start < 80u ||
+        (end & 15u) != 0u) {
         if (lane == 0) report(P.status, kStatusCorrupt);
         return;
     }
-    bool bad = false;
     const uint64_t psize = end - start;
     const uint8_t* pay_g = st + L.off_exp + start;
-    uint8_t* pay_s = S.stage + size_t(warp) * (2u * P.max_chunk + kTansSlack);
-    uint8_t* man_s = pay_s + P.max_chunk + kTansSlack;
-    const bool staged = psize <= C + kTansSlack;
+    uint8_t* pay_s = S.stage + size_t(warp) * tans_stage_bytes(P.max_chunk);
+    uint8_t* man_s = pay_s + tans_pay_stage(P.max_chunk);
+    const bool staged = psize <= tans_pay_stage(C);
     const uint32_t man16 = len & ~15u;
     // stage: the payload (if it fits) and the chunk's mantissa bytes. The
     // previous chunk's reads are done and its plain stores of mantissa bytes
@@ -221,41 +344,41 @@ __device__ void tans_chunk(const TansParams<MAXI>& P, const DecodeItem& I, uint6
         return;
     }
     const uint8_t* pay = staged ? pay_s : pay_g;
-    const uint32_t* words = reinterpret_cast<const uint32_t*>(pay + 64);
     const uint32_t avail = uint32_t((psize - 64u) / 4u);
-    uint32_t X = reinterpret_cast<const uint16_t*>(pay)[lane];
-    if (X >= Lst || (uint32_t(lane) >= len && X != 0u)) bad = true;
-    X &= Lst - 1u;
-    uint64_t buf = 0;
-    uint32_t cnt = 0, p = 0;
-    uint16_t* out = I.out + c * C;
+    const uint32_t X0 = reinterpret_cast<const uint16_t*>(pay)[lane];
+    bool bad = X0 >= Lst || (uint32_t(lane) >= len && X0 != 0u);
+    const uint32_t tbase = smem_addr(S.table);
+    TansLane d{tbase + 4u * (X0 & (Lst - 1u)), 0u, 0u, 0u, 0u};
+    const uint32_t* wg = reinterpret_cast<const uint32_t*>(pay_g + 64);
+    const uint32_t ws = smem_addr(pay_s + 64);
+    const uint32_t lt = lanemask_lt();
+    uint32_t ma = smem_addr(man_s) + uint32_t(lane);
+    uint16_t* o = I.out + c * C + lane;
     const uint32_t steps = (len + 31u) >> 5;
-    for (uint32_t k = 0; k < steps; ++k) {
-        const uint32_t i = 32u * k + uint32_t(lane);
-        const bool active = i < len;
-        const bool need = active && cnt < R;
-        const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
-        if (need) {
-            const uint32_t q = p + __popc(m & lanemask_lt());
-            uint32_t w = 0;
-            if (q < avail) w = words[q]; else bad = true;
-            buf |= uint64_t(w) << cnt;
-            cnt += 32u;
+    if (len == C) {  // a full chunk: every lane active at every step, steps even
+        if (staged) {
+#pragma unroll 2
+            for (uint32_t k = 0; k < steps; k += 2, ma += 64u, o += 64)
+                tans_pair<true>(d, tbase, wg, ws, avail - 1u, R, lt, ma, o);
+        } else {
+#pragma unroll 2
+            for (uint32_t k = 0; k < steps; k += 2, ma += 64u, o += 64)
+                tans_pair<false>(d, tbase, wg, ws, avail - 1u, R, lt, ma, o);
         }
-        p += __popc(m);
-        if (active) {
-            const uint32_t t = S.table[X];
-            const uint32_t nb = (t >> 8) & 0xFFu;
-            X = (t >> 16) + uint32_t(buf & ((1ull << nb) - 1ull));
-            buf >>= nb;
-            cnt -= nb;
-            const uint32_t s = man_s[i];
-            out[i] = uint16_t(((s & 0x80u) << 8) | ((t & 0xFFu) << 7) | (s & 0x7Fu));
+    } else {
+        for (uint32_t k = 0; k < steps; ++k, ma += 32u, o += 32) {
+            const bool active = 32u * k + uint32_t(lane) < len;
+            if (staged)
+                tans_step<true, true>(d, active, tbase, wg, ws, avail - 1u, R, lt, ma, o);
+            else
+                tans_step<false, true>(d, active, tbase, wg, ws, avail - 1u, R, lt, ma, o);
         }
     }
-    // a valid chunk: every lane back at state 0 with no bits left, fewer than 4
-    // unused words
-    bad |= X != 0u || buf != 0u || p > avail || avail - p > 3u;
+    // a valid chunk: every lane back at state 0 with no bits left, every word
+    // read inside the payload, fewer than 4 unused words and those zero
+    bad |= d.xa != tbase || (d.lo | d.hi) != 0u || d.p > avail || avail - d.p > 3u;
+    if (!bad && d.p + uint32_t(lane) < avail)
+        bad = reinterpret_cast<const uint32_t*>(pay + 64)[d.p + lane] != 0u;
     if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) report(P.status, kStatusCorrupt);
 }
 
@@ -311,7 +434,7 @@ cudaError_t tans_launch(const DecodeItem* items, uint32_t count, int32_t* status
     p.tile_begin[count] = tiles;
     if (tiles == 0) return cudaSuccess;
     const size_t smem = 4u * (kTansTable + 260u + 256u + 4u) + 8u * kTansWarps +
-                        size_t(kTansWarps) * (2u * p.max_chunk + kTansSlack);
+                        size_t(kTansWarps) * tans_stage_bytes(p.max_chunk) + tans_read_slack(p.max_chunk);
     static std::mutex mu;
     static int sms_of[64];
     static size_t smem_set[64];
