@@ -37,7 +37,7 @@
 // escapes before it (segmented by block for B < 1024, carried across the
 // segment's two steps for B >= 1024, and, for B > 1024, offset by the escape
 // totals of the block's earlier segments, which their warps post to shared
-// memory).
+// memory; a warp waits only for those warps).
 #include <mutex>
 #include <type_traits>
 
@@ -86,12 +86,14 @@ struct __align__(16) Stage {
 };
 
 // Escape-coded tiles with blocks longer than a consumer warp's segment: each
-// warp's escape total for the stage's tile, and a barrier per stage on which
-// all eight consumer warps arrive for every such tile (each warp keeps the
-// barriers' phases: the warps see the same tiles in the same order).
+// warp's escape total for the stage's tile and the tile's sequence number
+// (its round-robin index + 1), posted once the total is known. A warp waits
+// only for the warps of the earlier segments of its block. A slot cannot be
+// overwritten before its readers are done: stage s takes a new tile only
+// after all eight consumer warps released it.
 struct EscSegments {
     uint32_t count[stages_of<kKindEscape>()][kConsumerWarps];
-    unsigned long long done[stages_of<kKindEscape>()];
+    uint32_t seq[stages_of<kKindEscape>()][kConsumerWarps];
 };
 struct NoEscSegments {};
 
@@ -426,12 +428,23 @@ __device__ __forceinline__ bool finish_esc_chunk(const Stage<kKindEscape>& st, E
     return bad;
 }
 
+// Wait (bounded by the device timer, like every wait of the kernel) until a
+// warp's posted sequence number in shared memory reaches `tag`.
+__device__ __forceinline__ bool wait_tag(const uint32_t* p, uint32_t tag, volatile int* abort) {
+    const volatile uint32_t* v = p;
+    if (*v == tag) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (*v != tag) {
+        if (*abort || global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
 template <int MAXI>
 __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEscape>& sm, int tid,
                                int lane, int warp) {
     constexpr int kStages = DecodeSmem<kKindEscape>::kStages;
     (void)tid;
-    uint32_t seg_phase = 0;  // bit s: parity of stage s's next segment-total phase
     for (uint64_t i = 0;; ++i) {
         const uint64_t t = blockIdx.x + i * gridDim.x;
         if (t >= P.total_tiles) break;
@@ -477,25 +490,34 @@ __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEsca
             }
         }
         // Blocks longer than a segment: the escapes of the block's earlier
-        // segments, from the other warps' totals.
+        // segments, from the totals their warps post.
         const uint32_t last = B >= uint32_t(kSegment) ? __shfl_sync(0xFFFFFFFFu, incl, 31) : 0u;
         uint32_t carry = 0;
         if (B > uint32_t(kSegment)) {
+            const uint32_t tag = uint32_t(i) + 1u;
             if (lane == 0) {
                 sm.seg.count[s][warp] = (last & 0xFFFFu) + (last >> 16);
-                mbar_arrive(&sm.seg.done[s]);
+                __threadfence_block();
+                *reinterpret_cast<volatile uint32_t*>(&sm.seg.seq[s][warp]) = tag;
             }
-            const uint32_t parity = (seg_phase >> s) & 1u;
-            seg_phase ^= 1u << s;
-            if (!mbar_wait(&sm.seg.done[s], parity, &sm.abort)) {
+            // lane k waits for the warp of the block's k-th segment, if earlier
+            const uint32_t w0 = (seg & ~(B - 1u)) / uint32_t(kSegment);
+            const uint32_t wk = w0 + uint32_t(lane);
+            uint32_t c = 0;
+            bool ok = true;
+            if (wk < uint32_t(warp)) {
+                ok = wait_tag(&sm.seg.seq[s][wk], tag, &sm.abort);
+                __threadfence_block();
+                c = sm.seg.count[s][wk];
+            }
+            if (!__all_sync(0xFFFFFFFFu, ok)) {
                 if (lane == 0) {
                     report(P.status, kStatusTimeout);
                     sm.abort = 1;
                 }
                 return;
             }
-            for (uint32_t w = (seg & ~(B - 1u)) / uint32_t(kSegment); w < uint32_t(warp); ++w)
-                carry += sm.seg.count[s][w];
+            carry = __reduce_add_sync(0xFFFFFFFFu, c);
         }
         if (active) {
             const uint32_t excl = incl - v;
@@ -526,7 +548,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
             mbar_init(&sm.empty[s], kConsumerWarps);  // one arrive per consumer warp
         }
         if constexpr (KIND == kKindEscape)
-            for (int s = 0; s < kStages; ++s) mbar_init(&sm.seg.done[s], kConsumerWarps);
+            for (int s = 0; s < kStages; ++s)
+                for (int w = 0; w < kConsumerWarps; ++w) sm.seg.seq[s][w] = 0;
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }

@@ -347,18 +347,21 @@ __device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem<F32>& sm, in
             }
             if (nv)
                 st_stream_v4(I.out + man_base + el, make_uint4(S[0], S[1], S[2], S[3]));
-            // key = largest magnitude << 16 | (0x7FFF - smallest magnitude): one
-            // 16-bit lane maximum reduces both across the lanes of a block
+            // key = largest doubled magnitude << 16 | (0xFFFF - smallest): one
+            // 16-bit lane maximum reduces both across the lanes of a block. x + x
+            // doubles both halves' magnitudes at once: the low half's sign bit
+            // moves into bit 0 of the high half, below its exponent (bits 8..15
+            // of a doubled half), and the high half's sign bit leaves the word.
             uint32_t key = 0u;
             if (nv) {
-                uint32_t mn = x[k][0] & 0x7FFF7FFFu, mx = mn;
+                uint32_t mn = x[k][0] + x[k][0], mx = mn;
 #pragma unroll
                 for (int j = 1; j < 8; ++j) {
-                    const uint32_t m = x[k][j] & 0x7FFF7FFFu;
+                    const uint32_t m = x[k][j] + x[k][j];
                     mn = min_u16x2(mn, m);
                     mx = max_u16x2(mx, m);
                 }
-                key = (max(mx & 0xFFFFu, mx >> 16) << 16) | (0x7FFFu - min(mn & 0xFFFFu, mn >> 16));
+                key = (max(mx & 0xFFFFu, mx >> 16) << 16) | (0xFFFFu - min(mn & 0xFFFFu, mn >> 16));
             }
             if (group == 32) {  // B >= 512: the warp's 32 chunks are one block
                 key = (__reduce_max_sync(0xFFFFFFFFu, key >> 16) << 16) |
@@ -367,7 +370,7 @@ __device__ void encode_work(const EncodeParams<MAXI>& P, EncodeSmem<F32>& sm, in
                 for (uint32_t off = 1; off < group; off <<= 1)
                     key = max_u16x2(key, __shfl_xor_sync(0xFFFFFFFFu, key, off));
             }
-            const uint32_t lo = (0x7FFFu - (key & 0xFFFFu)) >> 7, hi = key >> (16 + 7);
+            const uint32_t lo = (0xFFFFu - (key & 0xFFFFu)) >> 8, hi = key >> (16 + 8);
             if ((lane & (group - 1)) == 0 && nv) {
                 atomicMin(&lo_of[el >> log2B], int(lo));
                 atomicMax(&hi_of[el >> log2B], int(hi));

@@ -36,6 +36,14 @@ template <uint32_t W>
 __device__ __forceinline__ void pack_chunk(const uint32_t V[4], uint8_t* dst) {
     if constexpr (W == 0) {
         return;
+    } else if constexpr (W == 4) {
+        // values below 16: v | v >> 4 holds pair 0 (v0 | v1 << 4) in byte 0 and
+        // pair 1 in byte 2 (the shifted copies land only in bytes 1 and 3), and
+        // the four pairs of two words are their octet's bytes in order
+        uint32_t p[4];
+#pragma unroll
+        for (uint32_t j = 0; j < 4; ++j) p[j] = V[j] | (V[j] >> 4);
+        *reinterpret_cast<uint2*>(dst) = make_uint2(prmt(p[0], p[1], 0x6420u), prmt(p[2], p[3], 0x6420u));
     } else {
         uint32_t F[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
