@@ -389,12 +389,12 @@ def escape_phase(args, wc, wcodec, inputs, outs, stream, dist, dev, world, mats=
 
 
 TANS_CHUNK = 4096
-TANS_LOG = 11
+TANS_LOG = 10
 
 
 def tans_phase(args, wc, wcodec, inputs, outs, stream, dist, dev, world):
     """The same tensors as tANS-coded streams (exponents entropy-coded, chunks
-    of 4096 elements as 32 interleaved lane streams, 2^11 states): one
+    of 4096 elements as 32 interleaved lane streams, 2^10 states): one
     wc_compress_tans_batch call (five launches) and one wc_decompress_tans_batch
     launch, each timed over the step count; every decoded tensor checked
     against its input."""
