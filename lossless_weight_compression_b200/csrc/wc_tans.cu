@@ -28,6 +28,7 @@
 #include <mutex>
 
 #include "wc_decode_core.cuh"
+#include "wc_pack_core.cuh"
 
 namespace wc {
 namespace {
@@ -546,23 +547,30 @@ __global__ void __launch_bounds__(256) tans_hist(const __grid_constant__ TansEnc
         // 32 elements per thread: their exponents counted, their sign+mantissa
         // bytes stored as two 16-byte words
         const uint32_t el = 32u * threadIdx.x;
-        if (el < len) {
-            uint8_t sb[32];
+        if (el + 32u <= len) {  // four 16-byte loads (a tile starts 16-byte aligned)
+            const uint4* src = reinterpret_cast<const uint4*>(I.in + first + el);
+            uint32_t sw[8];
 #pragma unroll
-            for (uint32_t j = 0; j < 32; ++j) {
-                const uint32_t x = el + j < len ? uint32_t(I.in[first + el + j]) : 0u;
-                if (el + j < len) atomicAdd(&h[(x >> 7) & 0xFFu], 1u);
-                sb[j] = uint8_t(((x >> 8) & 0x80u) | (x & 0x7Fu));
+            for (uint32_t v = 0; v < 4; ++v) {
+                const uint4 a = src[v];
+                uint32_t e0, e1;
+                split_quad(a.x, a.y, sw[2 * v], e0);
+                split_quad(a.z, a.w, sw[2 * v + 1], e1);
+#pragma unroll
+                for (uint32_t b = 0; b < 4; ++b) {
+                    atomicAdd(&h[(e0 >> (8u * b)) & 0xFFu], 1u);
+                    atomicAdd(&h[(e1 >> (8u * b)) & 0xFFu], 1u);
+                }
             }
             uint8_t* dst = I.out + L.off_man + first + el;
-            if (el + 32 <= len) {
-                uint4 a, b;
-                memcpy(&a, sb, 16);
-                memcpy(&b, sb + 16, 16);
-                *reinterpret_cast<uint4*>(dst) = a;
-                *reinterpret_cast<uint4*>(dst + 16) = b;
-            } else {
-                for (uint32_t j = 0; el + j < len; ++j) dst[j] = sb[j];
+            *reinterpret_cast<uint4*>(dst) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+            *reinterpret_cast<uint4*>(dst + 16) = make_uint4(sw[4], sw[5], sw[6], sw[7]);
+        } else if (el < len) {  // the ragged end of a tensor
+            uint8_t* dst = I.out + L.off_man + first + el;
+            for (uint32_t j = 0; el + j < len; ++j) {
+                const uint32_t x = uint32_t(I.in[first + el + j]);
+                atomicAdd(&h[(x >> 7) & 0xFFu], 1u);
+                dst[j] = uint8_t(((x >> 8) & 0x80u) | (x & 0x7Fu));
             }
         }
         __syncthreads();
@@ -751,12 +759,36 @@ __global__ void __launch_bounds__(kEncThreads) tans_encode(const __grid_constant
             const uint32_t C = I.chunk, R = I.log, Lst = 1u << R;
             const uint32_t len = uint32_t(min(uint64_t(C), I.n - c * C));
             const uint16_t* x = I.in + c * C;
-            // 1. backwards: each element's bits (value | count << 12)
+            // 0. the chunk's exponents into the element area (16-byte loads of eight
+            //    words each; a chunk starts 16-byte aligned), so that the serial
+            //    loop below waits on shared memory, not on global loads
+            for (uint32_t v = uint32_t(lane); 8u * v < len; v += 32u) {
+                const uint32_t i0 = 8u * v;
+                uint32_t wd[4];
+                if (i0 + 8u <= len) {
+                    const uint4 a = *reinterpret_cast<const uint4*>(x + i0);
+                    wd[0] = a.x; wd[1] = a.y; wd[2] = a.z; wd[3] = a.w;
+                } else {
+#pragma unroll
+                    for (uint32_t h = 0; h < 4; ++h) {
+                        const uint32_t lo = i0 + 2u * h < len ? uint32_t(x[i0 + 2u * h]) : 0u;
+                        const uint32_t hi = i0 + 2u * h + 1u < len ? uint32_t(x[i0 + 2u * h + 1u]) : 0u;
+                        wd[h] = lo | (hi << 16);
+                    }
+                }
+                // two words' exponents (bits 14..7 of each half) as two 16-bit lanes
+                *reinterpret_cast<uint4*>(elem + i0) =
+                    make_uint4((wd[0] >> 7) & 0x00FF00FFu, (wd[1] >> 7) & 0x00FF00FFu,
+                               (wd[2] >> 7) & 0x00FF00FFu, (wd[3] >> 7) & 0x00FF00FFu);
+            }
+            __syncwarp();
+            // 1. backwards: each element's bits (value | count << 12), in place of its exponent
             uint32_t st = Lst;
             const uint32_t steps = len > uint32_t(lane) ? (len - lane + 31u) >> 5 : 0u;
+#pragma unroll 4
             for (uint32_t k = steps; k-- > 0;) {
                 const uint32_t i = uint32_t(lane) + 32u * k;
-                const uint32_t e = (uint32_t(x[i]) >> 7) & 0xFFu;
+                const uint32_t e = elem[i];
                 const uint32_t f = S.freq[e];
                 uint32_t nb = R - (31u - __clz(f));     // (st >> nb) < 2f
                 if (nb > 0 && (st >> (nb - 1u)) < 2u * f) --nb;
