@@ -229,7 +229,7 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// 2-D tiled TMA load (no multicast) of the box at (c0, c1), completing on `bar`.
+// 2-D tiled TMA load of the box at (c0, c1) into this block's shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int32_t c0,
                                             int32_t c1, unsigned long long* bar) {
     asm volatile(
