@@ -66,7 +66,18 @@ struct TansParams {
     uint32_t max_chunk;               // the largest C of the batch (staging size)
 };
 
-__host__ __device__ inline uint64_t tans_chunks(uint64_t n, uint32_t C) { return (n + C - 1) / C; }
+// C is a power of two (1024..8192): chunk counts by a shift, not a 64-bit division
+// (which the decoder would otherwise run for every chunk).
+__host__ __device__ inline uint32_t tans_log2(uint32_t C) {
+#ifdef __CUDA_ARCH__
+    return uint32_t(__ffs(int(C))) - 1u;
+#else
+    return uint32_t(__builtin_ctz(C));
+#endif
+}
+__host__ __device__ inline uint64_t tans_chunks(uint64_t n, uint32_t C) {
+    return (n + C - 1) >> tans_log2(C);
+}
 __host__ __device__ inline uint64_t tans_tiles(uint64_t n, uint32_t C) {
     return (tans_chunks(n, C) + kTansWarps - 1) / kTansWarps;
 }
