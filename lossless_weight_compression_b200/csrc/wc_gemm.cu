@@ -646,12 +646,6 @@ __device__ __forceinline__ void octet_bytes(const uint8_t* raw, uint32_t q, uint
     b = quad_to_bytes<W>(uint32_t(v >> (4 * W)) & kQuad);
 }
 
-// Bit 7 of each byte of c whose value is m4's (m4 = the byte m in all four).
-__device__ __forceinline__ uint32_t bytes_equal(uint32_t c, uint32_t m4) {
-    const uint32_t z = c ^ m4;
-    return ~(((z & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | z) & 0x80808080u;
-}
-
 // Transcoding warps: warp t owns rows 16t .. 16t+15 of every slice, eight
 // lanes per row and four rows per step: step k takes rows 16t + k + 4*slot
 // (slot = lane / 8), so the two rows of a half-warp are four apart and their
@@ -730,11 +724,15 @@ __device__ void gemm_transcode(const GemmParams<MAXI>& P, const GemmSmem& S, int
             if (ESC) {
                 // e holds codes: flag the escapes, count them in element order
                 const uint32_t m = (1u << w) - 1u;
+                // a code equals 2^w - 1 exactly when adding 0x80 - (2^w - 1) sets its
+                // byte's top bit (codes are at most 2^w - 1: no carry leaves a byte)
                 const bool windowed = w >= 1u && w <= 7u;
+                const uint32_t esc_add = windowed ? (0x80u - m) * 0x01010101u : 0u;
+                const uint32_t esc_det = windowed ? 0x80808080u : 0u;
                 uint32_t fl[4], cnt = 0;
 #pragma unroll
                 for (uint32_t j = 0; j < 4; ++j) {
-                    fl[j] = windowed ? bytes_equal(e[j], m * 0x01010101u) : 0u;
+                    fl[j] = (e[j] + esc_add) & esc_det;
                     cnt += __popc(fl[j]);
                 }
                 uint32_t incl = cnt;
