@@ -315,10 +315,12 @@ struct EscChunk {
     bool active;
 };
 
+// FULL: a full tile (every chunk active), without the tail's selects and checks.
+template <bool FULL>
 __device__ __forceinline__ void load_esc_meta(const Stage<kKindEscape>& st, uint32_t el,
                                               uint32_t tile_n, uint32_t log2B, EscChunk& c) {
     c.el = el;
-    c.active = el < tile_n;
+    c.active = FULL || el < tile_n;
     c.count = 0;
     // an inactive chunk (past the end of the tile) decodes staged byte 0 as
     // width 3 and is never stored
@@ -332,9 +334,10 @@ __device__ __forceinline__ void load_esc_meta(const Stage<kKindEscape>& st, uint
 
 // The last chunk of a stream: bits past the block's codes are not codes (they
 // hold its exceptions and padding).
+template <bool FULL>
 __device__ __forceinline__ void finish_esc_codes(uint32_t tile_n, EscChunk& c) {
     const uint32_t nv = tile_n - c.el;
-    if (nv < uint32_t(kChunk)) {
+    if (!FULL && nv < uint32_t(kChunk)) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int valid = int(nv) - 4 * j;
@@ -350,14 +353,15 @@ __device__ __forceinline__ void finish_esc_codes(uint32_t tile_n, EscChunk& c) {
 // Both chunks are first decoded as 3-bit codes without a branch (so that their
 // shared-memory loads can be scheduled together); a chunk of another width is
 // then decoded again through the run-time path.
+template <bool FULL>
 __device__ __forceinline__ void decode_esc_pair(const Stage<kKindEscape>& st, uint32_t tile_n,
                                                 EscChunk& c0, EscChunk& c1) {
     chunk_exponents<3>(st.exp, c0.q, c0.t1.x, c0.t1.y, c0.E, c0.esc);
     chunk_exponents<3>(st.exp, c1.q, c1.t1.x, c1.t1.y, c1.E, c1.esc);
     if (c0.t0.y != 3u) chunk_exponents_rt(st.exp, c0.q, c0.t0.y, c0.t1.x, c0.t1.y, c0.E, c0.esc);
     if (c1.t0.y != 3u) chunk_exponents_rt(st.exp, c1.q, c1.t0.y, c1.t1.x, c1.t1.y, c1.E, c1.esc);
-    if (c0.active) finish_esc_codes(tile_n, c0);
-    if (c1.active) finish_esc_codes(tile_n, c1);
+    if (FULL || c0.active) finish_esc_codes<FULL>(tile_n, c0);
+    if (FULL || c1.active) finish_esc_codes<FULL>(tile_n, c1);
 }
 
 // Put the chunk's exceptions -- staged bytes [p, p + count), in element order --
@@ -396,6 +400,7 @@ __device__ __forceinline__ void patch_esc_chunk(const uint8_t* exp, uint32_t p, 
 // Patch the chunk's escaped elements with their exceptions (the `before`-th
 // exception of its block onwards), check the block's payload size if the
 // chunk holds the block's last element, and store the 16 BF16 words.
+template <bool FULL>
 __device__ __forceinline__ bool finish_esc_chunk(const Stage<kKindEscape>& st, EscChunk& c,
                                                  uint32_t before, uint32_t tile_n, uint32_t log2B,
                                                  uint16_t* out) {
@@ -408,7 +413,8 @@ __device__ __forceinline__ bool finish_esc_chunk(const Stage<kKindEscape>& st, E
             patch_esc_chunk(st.exp, p, c);
     }
     const uint32_t next = c.el + uint32_t(kChunk);
-    if (((next & ((1u << log2B) - 1u)) == 0u || next >= tile_n) &&
+    // (a full tile ends on a block boundary)
+    if (((next & ((1u << log2B) - 1u)) == 0u || (!FULL && next >= tile_n)) &&
         ((c.t0.z + before + c.count + 15u) & ~15u) != c.t0.w - c.t0.x)
         bad = true;
     uint4 r0, r1;
@@ -417,7 +423,7 @@ __device__ __forceinline__ bool finish_esc_chunk(const Stage<kKindEscape>& st, E
     merge_quad(c.E[2], c.M.z, r1.x, r1.y);
     merge_quad(c.E[3], c.M.w, r1.z, r1.w);
     uint16_t* dst = out + c.el;
-    if (tile_n - c.el >= uint32_t(kChunk)) {
+    if (FULL || tile_n - c.el >= uint32_t(kChunk)) {
         st_stream_v4(dst, r0);
         st_stream_v4(dst + 8, r1);
     } else {
@@ -463,14 +469,21 @@ __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEsca
         const uint32_t seg = uint32_t(warp) * kSegment;
         bool bad = false;
         const bool active = seg < info.tile_n;  // the same for the whole warp
+        const bool full = info.tile_n == uint32_t(kTile);
         // both 512-element steps of the segment at once: chunk k of this lane
         // starts at seg + 512k + 16 lane
         EscChunk c0, c1;
         uint32_t incl = 0, v = 0;
         if (active) {
-            load_esc_meta(st, seg + 16u * uint32_t(lane), info.tile_n, log2B, c0);
-            load_esc_meta(st, seg + 512u + 16u * uint32_t(lane), info.tile_n, log2B, c1);
-            decode_esc_pair(st, info.tile_n, c0, c1);
+            if (full) {
+                load_esc_meta<true>(st, seg + 16u * uint32_t(lane), kTile, log2B, c0);
+                load_esc_meta<true>(st, seg + 512u + 16u * uint32_t(lane), kTile, log2B, c1);
+                decode_esc_pair<true>(st, kTile, c0, c1);
+            } else {
+                load_esc_meta<false>(st, seg + 16u * uint32_t(lane), info.tile_n, log2B, c0);
+                load_esc_meta<false>(st, seg + 512u + 16u * uint32_t(lane), info.tile_n, log2B, c1);
+                decode_esc_pair<false>(st, info.tile_n, c0, c1);
+            }
             // one prefix count for both steps (step k's counts in bits [16k, 16k + 16)),
             // segmented by block: B/16 lanes hold one block of a step when B < 512
             v = c0.count | (c1.count << 16);
@@ -526,8 +539,13 @@ __device__ void consume_escape(const DecodeParams<MAXI>& P, DecodeSmem<kKindEsca
                 before0 += carry;
                 before1 += carry + (last & 0xFFFFu);
             }
-            if (c0.active) bad |= finish_esc_chunk(st, c0, before0, info.tile_n, log2B, info.out);
-            if (c1.active) bad |= finish_esc_chunk(st, c1, before1, info.tile_n, log2B, info.out);
+            if (full) {
+                bad |= finish_esc_chunk<true>(st, c0, before0, kTile, log2B, info.out);
+                bad |= finish_esc_chunk<true>(st, c1, before1, kTile, log2B, info.out);
+            } else {
+                if (c0.active) bad |= finish_esc_chunk<false>(st, c0, before0, info.tile_n, log2B, info.out);
+                if (c1.active) bad |= finish_esc_chunk<false>(st, c1, before1, info.tile_n, log2B, info.out);
+            }
         }
         if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) report(P.status, kStatusCorrupt);
         __syncwarp();
