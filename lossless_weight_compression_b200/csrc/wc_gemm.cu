@@ -21,17 +21,20 @@
 //     contiguous bytes; 16-byte cp.async pieces);
 //   - eight transcoding warps unpack those bits into one exponent byte per
 //     weight (base + v), eight lanes per row; a step of four rows whose widths
-//     are all 4 takes a nibble path, any other step a path for every width;
+//     are all 4 takes a nibble path (escape-coded streams: also a width-3
+//     path), any other step a path for every width; escape-coded streams
+//     (header flags bit 1) also have their escapes ranked and replaced by the
+//     block's exception bytes here;
 //   - eight writing warps, one lane per row (a warp's lanes are the 32 tensor
 //     memory lanes its rank in the warpgroup may access), merge each exponent
 //     byte with its sign+mantissa byte into BF16 and store the slice's A
 //     operand into tensor memory with tcgen05.st: the same few instructions
 //     for every width;
 //   - one thread issues tcgen05.mma (A from tensor memory, activations from
-//     shared memory; BF16 x BF16 -> FP32, M = 128, K = 16) into one of two
-//     accumulators in tensor memory;
-//   - four epilogue warps move a finished accumulator out with tcgen05.ld and
-//     write Y while the next unit accumulates in the other one.
+//     shared memory; BF16 x BF16 -> FP32, M = 128, K = 16), spreading
+//     consecutive MMAs over several accumulators in tensor memory;
+//   - four epilogue warps sum a finished unit's accumulators (tcgen05.ld) in a
+//     fixed order and write Y while the next unit accumulates.
 // Every wait is bounded by the device timer, after which the block stops and
 // reports WC_ERR_TIMEOUT. Each unit sums its row in the same order on every
 // run, so Y is reproducible bit for bit.
