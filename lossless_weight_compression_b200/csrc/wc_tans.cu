@@ -671,6 +671,7 @@ struct EncShared {
     uint16_t* freq;      // 256
     uint32_t* pbase;     // 256: first pos entry of each exponent
     uint32_t* seen;      // 256
+    uint2* dof;          // 256: {delta, pbase - f}, see tans_enc_tables
     uint16_t* pos;       // L: state of each (exponent, occurrence)
     uint8_t* warp_area;  // per warp: C u16 (value | bits << 12), then 32 x cap words
 };
@@ -700,6 +701,16 @@ __device__ void tans_enc_tables(const TansEncItem& I, EncShared& S) {
         }
     }
     __syncthreads();
+    // Per exponent, the encoder's bit count by one add and shift: from a state
+    // x in [L, 2L) it emits nb0 = R - floor(log2 f) bits, or one fewer when
+    // x < f << nb0 (then x >> (nb0 - 1) < 2f already); with delta =
+    // (nb0 << 16) - (f << nb0), (x + delta) >> 16 is that count (|x - (f << nb0)|
+    // < L <= 2^12, mod 2^32). The next state's slot is (x >> nb) + pbase - f.
+    for (int e = tid; e < 256; e += kEncThreads) {
+        const uint32_t f = S.freq[e];
+        const uint32_t nb0 = f ? R - (31u - __clz(f)) : 0u;
+        S.dof[e] = make_uint2(f ? (nb0 << 16) - (f << nb0) : 0u, S.pbase[e] - f);
+    }
     // the spread into pos (as a temporary state -> exponent map)
     const uint32_t step = (Lst >> 1) + (Lst >> 3) + 3u;
     for (uint32_t k = tid; k < Lst; k += kEncThreads) {
@@ -738,8 +749,9 @@ __global__ void __launch_bounds__(kEncThreads) tans_encode(const __grid_constant
     S.freq = reinterpret_cast<uint16_t*>(smem);
     S.pbase = reinterpret_cast<uint32_t*>(smem + 512);
     S.seen = S.pbase + 256;
-    S.pos = reinterpret_cast<uint16_t*>(smem + 2560);
-    S.warp_area = smem + 2560 + 2 * (1u << P.max_log);
+    S.dof = reinterpret_cast<uint2*>(smem + 2560);
+    S.pos = reinterpret_cast<uint16_t*>(smem + 4608);
+    S.warp_area = smem + 4608 + 2 * (1u << P.max_log);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t cap = tans_lane_cap(P.max_chunk, P.max_log);
     const size_t area = 2ull * P.max_chunk + 128ull * cap;
@@ -800,11 +812,10 @@ __global__ void __launch_bounds__(kEncThreads) tans_encode(const __grid_constant
             for (uint32_t k = steps; k-- > 0;) {
                 const uint32_t i = uint32_t(lane) + 32u * k;
                 const uint32_t e = elem[i];
-                const uint32_t f = S.freq[e];
-                uint32_t nb = R - (31u - __clz(f));     // (st >> nb) < 2f
-                if (nb > 0 && (st >> (nb - 1u)) < 2u * f) --nb;
-                elem[i] = uint16_t((st & ((1u << nb) - 1u)) | (nb << 12));
-                st = Lst + S.pos[S.pbase[e] + (st >> nb) - f];
+                const uint2 d = S.dof[e];
+                const uint32_t nb = (st + d.x) >> 16;  // the smallest nb with (st >> nb) < 2f
+                elem[i] = uint16_t((st & low_mask(nb)) | (nb << 12));
+                st = Lst + S.pos[(st >> nb) + d.y];
             }
             // 2. forwards: the lane's bits packed 32 to a word
             uint32_t nw = 0, acc_bits = 0;
@@ -932,7 +943,7 @@ cudaError_t tans_encode_batch(const EncodeItem* items, const uint32_t* logs, uin
     tans_plan<MAXI><<<count, 256, 0, stream>>>(p);
     if (chunks) {
         const uint32_t cap = tans_lane_cap(p.max_chunk, p.max_log);
-        const size_t smem = 2560 + 2ull * (1u << p.max_log) +
+        const size_t smem = 4608 + 2ull * (1u << p.max_log) +
                             size_t(kEncWarps) * (2ull * p.max_chunk + 128ull * cap);
         if ((err = cudaFuncSetAttribute(tans_encode<MAXI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         int(smem))) != cudaSuccess)
