@@ -693,23 +693,49 @@ __device__ void gemm_transcode(const GemmParams<MAXI>& P, const GemmSmem& S, int
             f[k][1] = *reinterpret_cast<const uint32_t*>(ep + 4u * o1);
         }
         bool bad = false;
+        // One path per step of four rows, all four steps decided by one warp
+        // reduction: bit k of all4 (all3) is set when every row of step k has
+        // width 4 (3).
+        uint32_t w4bits = 0, w3bits = 0;
 #pragma unroll
         for (uint32_t k = 0; k < 4; ++k) {
-            const uint32_t rr = row_base + k;
-            const uint32_t w = mw[k] & 0xFFu, base = (mw[k] >> 8) & 0xFFu;
-            const uint32_t base4 = ESC ? 0u : base * 0x01010101u;  // ESC: added after the escapes
-            uint32_t e[4];
-            // one width for the whole step (the common case): a path for it
-            const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, w, 0);
-            const bool same = __all_sync(0xFFFFFFFFu, w == w0);
-            if (same && w0 == 4u) {
+            w4bits |= ((mw[k] & 0xFFu) == 4u ? 1u : 0u) << k;
+            if (ESC) w3bits |= ((mw[k] & 0xFFu) == 3u ? 1u : 0u) << k;
+        }
+        const uint32_t all4 = __reduce_and_sync(0xFFFFFFFFu, w4bits);
+        const uint32_t all3 = ESC ? __reduce_and_sync(0xFFFFFFFFu, w3bits) : 0u;
+        if (!ESC && all4 == 0xFu) {
+            // the common case: every row of the four steps at width 4, in
+            // straight-line code (the four steps' work interleaves)
+#pragma unroll
+            for (uint32_t k = 0; k < 4; ++k) {
+                const uint32_t rr = row_base + k;
+                const uint32_t base4 = ((mw[k] >> 8) & 0xFFu) * 0x01010101u;
+                uint32_t e[4];
 #pragma unroll
                 for (uint32_t h = 0; h < 2; ++h) {
                     const uint32_t ev = f[k][h] & 0x0F0F0F0Fu, od = (f[k][h] >> 4) & 0x0F0F0F0Fu;
                     e[2 * h] = prmt(ev, od, 0x5140u) + base4;
                     e[2 * h + 1] = prmt(ev, od, 0x7362u) + base4;
                 }
-            } else if (ESC && same && w0 == 3u) {  // escape-coded Gaussian blocks: width 3
+                sts64(e_stage + rr * kExpPitch + 8u * o0, e[0], e[1]);
+                sts64(e_stage + rr * kExpPitch + 8u * o1, e[2], e[3]);
+            }
+        } else {
+#pragma unroll
+        for (uint32_t k = 0; k < 4; ++k) {
+            const uint32_t rr = row_base + k;
+            const uint32_t w = mw[k] & 0xFFu, base = (mw[k] >> 8) & 0xFFu;
+            const uint32_t base4 = ESC ? 0u : base * 0x01010101u;  // ESC: added after the escapes
+            uint32_t e[4];
+            if ((all4 >> k) & 1u) {
+#pragma unroll
+                for (uint32_t h = 0; h < 2; ++h) {
+                    const uint32_t ev = f[k][h] & 0x0F0F0F0Fu, od = (f[k][h] >> 4) & 0x0F0F0F0Fu;
+                    e[2 * h] = prmt(ev, od, 0x5140u) + base4;
+                    e[2 * h + 1] = prmt(ev, od, 0x7362u) + base4;
+                }
+            } else if (ESC && ((all3 >> k) & 1u)) {  // escape-coded Gaussian blocks: width 3
                 octet_bytes<3>(raw, rr * kExpPitch + 3u * o0, e[0], e[1]);
                 octet_bytes<3>(raw, rr * kExpPitch + 3u * o1, e[2], e[3]);
             } else {
@@ -781,6 +807,7 @@ __device__ void gemm_transcode(const GemmParams<MAXI>& P, const GemmSmem& S, int
             }
             sts64(e_stage + rr * kExpPitch + 8u * o0, e[0], e[1]);
             sts64(e_stage + rr * kExpPitch + 8u * o1, e[2], e[3]);
+        }
         }
         if (ESC && bad) report(P.status, kStatusCorrupt);
         __syncwarp();
