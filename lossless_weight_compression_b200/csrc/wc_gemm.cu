@@ -272,6 +272,10 @@ __device__ __forceinline__ void sts64(uint32_t saddr, uint32_t a, uint32_t b) {
     asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(saddr), "r"(a), "r"(b) : "memory");
 }
 
+__device__ __forceinline__ void sts8(uint32_t saddr, uint32_t v) {
+    asm volatile("st.shared.u8 [%0], %1;" ::"r"(saddr), "r"(v) : "memory");
+}
+
 template <int MAXI>
 __device__ __forceinline__ uint32_t find_item(const GemmParams<MAXI>& P, uint64_t u, uint32_t from) {
     while (u >= P.unit_begin[from + 1]) ++from;
@@ -774,12 +778,17 @@ __device__ void gemm_transcode(const GemmParams<MAXI>& P, const GemmSmem& S, int
                 const bool windowed = w >= 1u && w <= 7u;
                 const uint32_t esc_add = windowed ? (0x80u - m) * 0x01010101u : 0u;
                 const uint32_t esc_det = windowed ? 0x80808080u : 0u;
-                uint32_t fl[4], cnt = 0;
+                // bit 4j + t of fm: byte t of e[j] is an escape, so the lane's 16
+                // elements are in bit order. A word's four flags (bits 7, 15, 23,
+                // 31) gather into bits 24..27 of (flags >> 7) * 0x01020408: every
+                // partial product lands on a bit of its own, so nothing carries.
+                uint32_t fm = 0;
 #pragma unroll
                 for (uint32_t j = 0; j < 4; ++j) {
-                    fl[j] = (e[j] + esc_add) & esc_det;
-                    cnt += __popc(fl[j]);
+                    const uint32_t fl = (e[j] + esc_add) & esc_det;
+                    fm |= (((fl >> 7) * 0x01020408u) >> 24) << (4u * j);
                 }
+                const uint32_t cnt = __popc(fm);
                 uint32_t incl = cnt;
 #pragma unroll
                 for (uint32_t d = 1; d < 8; d <<= 1) {
@@ -792,27 +801,28 @@ __device__ void gemm_transcode(const GemmParams<MAXI>& P, const GemmSmem& S, int
 #pragma unroll
                 for (uint32_t j = 0; j < 4; ++j) e[j] += b4;
                 const bool last = (mw[k] & kMetaLast) != 0u;
+                // the row's sixteen exponent bytes of the lane, escapes still as
+                // base + 2^w - 1; the loop below overwrites those bytes
+                const uint32_t row_at = e_stage + rr * kExpPitch + 16u * c8;
+                sts128(row_at, e[0], e[1], e[2], e[3]);
                 if (__any_sync(0xFFFFFFFFu, cnt != 0u || last)) {
                     const uint4 em = S.emeta[rs * kTileRows + rr];
                     const uint8_t* xg = reinterpret_cast<const uint8_t*>(
                         (uint64_t(em.z) << 32) | uint64_t(em.y));
                     const uint8_t* xs = S.exc + rs * kExcStage + rr * kExcBytes;
                     uint32_t idx = run[k] + incl - cnt;  // the lane's first exception
-                    // element order: octet 2c, then 2c + 1 (o1 first where c >= 4)
-#pragma unroll
-                    for (uint32_t q = 0; q < 4; ++q) {
-                        const uint32_t j = pp ? (q ^ 2u) : q;
-                        uint32_t fm = fl[j];
-                        while (fm) {
-                            const uint32_t bit = __ffs(int(fm)) - 1u;  // 7, 15, 23 or 31
-                            uint32_t x = 0;
-                            if (idx < em.x) x = idx < kExcBytes ? xs[idx] : xg[idx];
-                            else bad = true;
-                            bad |= ((x - base) & 0xFFu) < m;  // an exception inside the window
-                            e[j] = (e[j] & ~(0xFFu << (bit - 7u))) | (x << (bit - 7u));
-                            ++idx;
-                            fm &= fm - 1u;
-                        }
+                    // one pass over the lane's escapes in element order (one loop
+                    // for all sixteen elements: a warp runs as many rounds as its
+                    // lane with the most escapes has)
+                    while (fm) {
+                        const uint32_t t = __ffs(int(fm)) - 1u;
+                        uint32_t x = 0;
+                        if (idx < em.x) x = idx < kExcBytes ? xs[idx] : xg[idx];
+                        else bad = true;
+                        bad |= ((x - base) & 0xFFu) < m;  // an exception inside the window
+                        sts8(row_at + t, x);
+                        ++idx;
+                        fm &= fm - 1u;
                     }
                     // the block's last slice: the list holds exactly its escapes
                     // (up to the payload's 15 bytes of padding)
@@ -821,9 +831,7 @@ __device__ void gemm_transcode(const GemmParams<MAXI>& P, const GemmSmem& S, int
                 }
                 run[k] += row_total;
             }
-            if (ESC) {
-                sts128(e_stage + rr * kExpPitch + 16u * c8, e[0], e[1], e[2], e[3]);
-            } else {
+            if (!ESC) {  // ESC: stored above, before the escapes' bytes
                 sts64(e_stage + rr * kExpPitch + 8u * o0, e[0], e[1]);
                 sts64(e_stage + rr * kExpPitch + 8u * o1, e[2], e[3]);
             }
