@@ -713,6 +713,7 @@ __device__ void gemm_transcode(const GemmParams<MAXI>& P, const GemmSmem& S, int
             }
         }
         bool bad = false;
+        uint32_t fm[4] = {0u, 0u, 0u, 0u}, cnt4 = 0;  // ESC: escape flags and counts per step
         // One path per step of four rows, all four steps decided by one warp
         // reduction: bit k of all4 (all3) is set when every row of step k has
         // width 4 (3).
@@ -771,58 +772,78 @@ __device__ void gemm_transcode(const GemmParams<MAXI>& P, const GemmSmem& S, int
                 }
             }
             if (ESC) {
-                // e holds codes: flag the escapes, count them in element order
+                // e holds codes: flag the escapes (counted below for all four
+                // steps at once), add the base and store the bytes
                 const uint32_t m = (1u << w) - 1u;
                 // a code equals 2^w - 1 exactly when adding 0x80 - (2^w - 1) sets its
                 // byte's top bit (codes are at most 2^w - 1: no carry leaves a byte)
                 const bool windowed = w >= 1u && w <= 7u;
                 const uint32_t esc_add = windowed ? (0x80u - m) * 0x01010101u : 0u;
                 const uint32_t esc_det = windowed ? 0x80808080u : 0u;
-                // bit 4j + t of fm: byte t of e[j] is an escape, so the lane's 16
+                // bit 4j + t of fm[k]: byte t of e[j] is an escape, so the lane's 16
                 // elements are in bit order. A word's four flags (bits 7, 15, 23,
                 // 31) gather into bits 24..27 of (flags >> 7) * 0x01020408: every
                 // partial product lands on a bit of its own, so nothing carries.
-                uint32_t fm = 0;
+                uint32_t f16 = 0;
 #pragma unroll
                 for (uint32_t j = 0; j < 4; ++j) {
                     const uint32_t fl = (e[j] + esc_add) & esc_det;
-                    fm |= (((fl >> 7) * 0x01020408u) >> 24) << (4u * j);
+                    f16 |= (((fl >> 7) * 0x01020408u) >> 24) << (4u * j);
                 }
-                const uint32_t cnt = __popc(fm);
-                uint32_t incl = cnt;
-#pragma unroll
-                for (uint32_t d = 1; d < 8; d <<= 1) {
-                    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d, 8);
-                    if (c8 >= d) incl += y;
-                }
-                const uint32_t row_total = __shfl_sync(0xFFFFFFFFu, incl, 7, 8);
-                if (mw[k] & kMetaFirst) run[k] = 0;
+                fm[k] = f16;
+                cnt4 |= uint32_t(__popc(f16)) << (8u * k);
                 const uint32_t b4 = base * 0x01010101u;  // base + code <= 255: no carries
 #pragma unroll
                 for (uint32_t j = 0; j < 4; ++j) e[j] += b4;
+                // escapes still as base + 2^w - 1: the patch below overwrites them
+                sts128(e_stage + rr * kExpPitch + 16u * c8, e[0], e[1], e[2], e[3]);
+            } else {
+                sts64(e_stage + rr * kExpPitch + 8u * o0, e[0], e[1]);
+                sts64(e_stage + rr * kExpPitch + 8u * o1, e[2], e[3]);
+            }
+        }
+        }
+        if (ESC) {
+            // The four steps' escape counts, one byte per step, scanned over the
+            // row's eight lanes at once (a row has at most 128 escapes in a
+            // slice: no byte carries into the next).
+            uint32_t incl4 = cnt4;
+#pragma unroll
+            for (uint32_t d = 1; d < 8; d <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl4, d, 8);
+                if (c8 >= d) incl4 += y;
+            }
+            const uint32_t tot4 = __shfl_sync(0xFFFFFFFFu, incl4, 7, 8);
+#pragma unroll
+            for (uint32_t k = 0; k < 4; ++k) {
+                const uint32_t rr = row_base + k;
+                const uint32_t w = mw[k] & 0xFFu, base = (mw[k] >> 8) & 0xFFu;
+                const uint32_t m = (1u << w) - 1u;
+                const uint32_t cnt = (cnt4 >> (8u * k)) & 0xFFu;
+                const uint32_t incl = (incl4 >> (8u * k)) & 0xFFu;
+                const uint32_t row_total = (tot4 >> (8u * k)) & 0xFFu;
+                if (mw[k] & kMetaFirst) run[k] = 0;
                 const bool last = (mw[k] & kMetaLast) != 0u;
-                // the row's sixteen exponent bytes of the lane, escapes still as
-                // base + 2^w - 1; the loop below overwrites those bytes
-                const uint32_t row_at = e_stage + rr * kExpPitch + 16u * c8;
-                sts128(row_at, e[0], e[1], e[2], e[3]);
-                if (__any_sync(0xFFFFFFFFu, cnt != 0u || last)) {
+                uint32_t f16 = fm[k];
+                if (__any_sync(0xFFFFFFFFu, f16 != 0u || last)) {
                     const uint4 em = S.emeta[rs * kTileRows + rr];
                     const uint8_t* xg = reinterpret_cast<const uint8_t*>(
                         (uint64_t(em.z) << 32) | uint64_t(em.y));
                     const uint8_t* xs = S.exc + rs * kExcStage + rr * kExcBytes;
+                    const uint32_t row_at = e_stage + rr * kExpPitch + 16u * c8;
                     uint32_t idx = run[k] + incl - cnt;  // the lane's first exception
                     // one pass over the lane's escapes in element order (one loop
                     // for all sixteen elements: a warp runs as many rounds as its
                     // lane with the most escapes has)
-                    while (fm) {
-                        const uint32_t t = __ffs(int(fm)) - 1u;
+                    while (f16) {
+                        const uint32_t t = __ffs(int(f16)) - 1u;
                         uint32_t x = 0;
                         if (idx < em.x) x = idx < kExcBytes ? xs[idx] : xg[idx];
                         else bad = true;
                         bad |= ((x - base) & 0xFFu) < m;  // an exception inside the window
                         sts8(row_at + t, x);
                         ++idx;
-                        fm &= fm - 1u;
+                        f16 &= f16 - 1u;
                     }
                     // the block's last slice: the list holds exactly its escapes
                     // (up to the payload's 15 bytes of padding)
@@ -831,11 +852,6 @@ __device__ void gemm_transcode(const GemmParams<MAXI>& P, const GemmSmem& S, int
                 }
                 run[k] += row_total;
             }
-            if (!ESC) {  // ESC: stored above, before the escapes' bytes
-                sts64(e_stage + rr * kExpPitch + 8u * o0, e[0], e[1]);
-                sts64(e_stage + rr * kExpPitch + 8u * o1, e[2], e[3]);
-            }
-        }
         }
         if (ESC && bad) report(P.status, kStatusCorrupt);
         __syncwarp();
